@@ -1,0 +1,215 @@
+/*
+ * recis.h -- C ABI of the B200 dynamic-hash embedding engine.
+ *
+ * The library implements the hot path of the RecIS Embedding Engine as the
+ * RecIS README describes it (page "RecIS (Recommendation Intelligence
+ * System)", codehub.bot mirror of github.com/alibaba/RecIS v1.1.0):
+ *   - Core architecture > Feature Engine: Hash / Mod / Bucketize feature ops,
+ *     fused into one operator;
+ *   - Key optimisations > Efficient dynamic embedding: a two-level store, the
+ *     IDMap (feature ID -> offset) and the EmbeddingBlocks (contiguous chunked
+ *     memory holding the embedding parameters and the optimiser state,
+ *     growing on demand);
+ *   - Key optimisations > Distributed optimisation: same-attribute tables merged
+ *     into one logical table; requests merged and deduplicated before lookup;
+ *   - Key optimisations > Efficient use of hardware > Operator implementation:
+ *     vectorised memory access, and reductions merged at warp level instead of
+ *     per-element atomics.
+ *
+ * Conventions (all entry points):
+ *   - Every call returns a recis_status and never aborts the process.  Kernels
+ *     never trap: device-detected problems set a status word in the table.
+ *   - Calls are asynchronous and ordered on the cudaStream_t they are given,
+ *     unless marked "synchronous".  Calls on one table (or one batch) must be
+ *     issued on one stream, or otherwise serialised by the caller.
+ *   - Device pointers are raw CUDA device addresses owned by the caller; they
+ *     must stay valid until the work of the call has finished on the stream.
+ *     Host pointers are plain host memory, read before the call returns.
+ *   - Device-detected errors (reserved key, table full, value too wide for its
+ *     tag) are reported by recis_table_status_sync(), and by the first later
+ *     call on the same table that finds the earlier work finished.
+ *   - Keys are int64.  The value -1 (all bits set) is reserved as the IDMap's
+ *     empty marker and is rejected (RECIS_ERR_RESERVED_KEY).
+ *   - recis_last_error_string() returns a description of the last error of the
+ *     calling thread.
+ */
+#ifndef RECIS_H
+#define RECIS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* recis_stream_t; /* == cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  RECIS_OK = 0,
+  RECIS_ERR_INVALID_ARG = 1,  /* bad argument, or a value wider than its tag field */
+  RECIS_ERR_OOM = 2,          /* device or host allocation failed */
+  RECIS_ERR_TABLE_FULL = 3,   /* IDMap probe sequence exhausted or row space exhausted */
+  RECIS_ERR_RESERVED_KEY = 4, /* an input key equals -1 */
+  RECIS_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed */
+  RECIS_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up */
+  RECIS_ERR_NO_DEVICE = 7     /* no usable sm_100 device */
+} recis_status;
+
+/* ------------------------------------------------------------------ features */
+/* Feature-op flags (README, Core architecture > Feature Engine: "Hash / Mod /
+ * Bucketize").  Per value x of a feature, in this order:
+ *   BUCKETIZE: v = number of boundaries <= x (boundaries sorted ascending);
+ *   otherwise: v = (uint64)x; HASH: v = H(v ^ hash_seed); MOD: v = v % mod;
+ *   TAG      : v must be < 2^tag_shift, key = (tag << tag_shift) | v.
+ * H is the SplitMix64 finaliser (Steele, Lea & Flood, OOPSLA 2014).
+ * BUCKETIZE cannot be combined with HASH or MOD. */
+#define RECIS_BUCKETIZE 1u
+#define RECIS_HASH 2u
+#define RECIS_MOD 4u
+#define RECIS_TAG 8u
+
+typedef struct {
+  uint32_t flags;
+  int32_t n_bound;            /* number of boundaries (BUCKETIZE) */
+  uint64_t hash_seed;
+  uint64_t mod;               /* > 0 when MOD is set */
+  uint64_t tag;               /* < 2^(63 - tag_shift) */
+  int32_t tag_shift;          /* 1..62 */
+  int32_t reserved_;
+  const int64_t* boundaries;  /* DEVICE pointer, n_bound int64, sorted ascending */
+} recis_feature_op;
+
+/* Fused feature transform of F features in one launch.
+ * values   : device int64[N], feature-major (feature f occupies
+ *            [feat_offsets[f], feat_offsets[f+1]));
+ * feat_offsets: HOST int64[F+1], non-decreasing, feat_offsets[0] = 0;
+ * keys_out : device int64[N] (may alias values).
+ * A transformed value wider than 2^tag_shift is a device-detected error
+ * (RECIS_ERR_INVALID_ARG via recis_feature_status_sync); its key is written
+ * as -1.  Up to 4096 features per call. */
+recis_status recis_feature_hash(const recis_feature_op* ops, int32_t F, const int64_t* values,
+                                const int64_t* feat_offsets, int64_t* keys_out,
+                                recis_stream_t stream);
+/* Synchronous: waits for `stream`, returns and clears the device-detected
+ * status of earlier recis_feature_hash calls on the current device. */
+recis_status recis_feature_status_sync(recis_stream_t stream);
+
+/* ------------------------------------------------------------------ tables */
+#define RECIS_ADAGRAD 0
+#define RECIS_ADAM 1
+#define RECIS_SUM 0
+#define RECIS_MEAN 1
+
+typedef struct {
+  int32_t dim;               /* D: multiple of 4, 4..1024 */
+  int32_t optimizer;         /* RECIS_ADAGRAD (state: acc) or RECIS_ADAM (state: m, v) */
+  double lr;
+  double beta1, beta2;       /* Adam */
+  double eps;                /* Adagrad 1e-10, Adam 1e-8 are the usual values */
+  double adagrad_init_acc;   /* initial accumulator */
+  double init_scale;         /* rows start uniform in [-init_scale, init_scale); <= 0: 1/sqrt(D) */
+  uint64_t init_seed;
+  int64_t initial_capacity;  /* expected live keys; the IDMap starts at >= 2x this */
+  int64_t block_rows;        /* rows per EmbeddingBlock (growth unit); 0 = 65536 */
+  int64_t max_rows;          /* upper bound on live rows (address space reserved); 0 = 2^28 */
+} recis_table_config;
+
+typedef struct recis_table* recis_table_t;
+typedef struct recis_batch* recis_batch_t;
+
+/* Create a table on the current device (README, Efficient dynamic embedding:
+ * IDMap + EmbeddingBlocks).  Rows are [emb D][state s*D] fp32 (s = 1 Adagrad,
+ * 2 Adam), kept side by side in EmbeddingBlocks that are physically separate
+ * allocations mapped into one contiguous virtual range, so a row is addressed
+ * as base + row * stride and growth never copies.  *out receives the handle. */
+recis_status recis_table_create(const recis_table_config* cfg, recis_stream_t stream,
+                                recis_table_t* out);
+recis_status recis_table_destroy(recis_table_t t);
+
+/* A batch holds the per-step scratch of one lookup (sorted keys, unique keys,
+ * inverse index, row offsets, per-occurrence bag ids) until the matching
+ * backward; it grows on demand and is reused across steps. */
+recis_status recis_batch_create(recis_batch_t* out);
+recis_status recis_batch_destroy(recis_batch_t b);
+
+/* Forward (README, Distributed optimisation: merged requests deduplicated; Efficient
+ * dynamic embedding: IDMap lookup, then the EmbeddingBlocks rows).  One call =
+ * one logical table:
+ *   1. dedup: uniq = distinct keys ascending (signed), inv[i] = index of keys[i];
+ *   2. IDMap find-or-insert: a missing key gets the next free row; new rows are
+ *      assigned in ascending key order and initialised from a seeded hash of
+ *      the key (emb) and the optimiser's initial state;
+ *   3. pooling: bag f*B+b covers keys[bag_offsets[f*B+b] .. bag_offsets[f*B+b+1]);
+ *      pooled_out[b][f][:] = sum of its rows (MEAN: / length; empty bag: 0);
+ *      unpooled_out[i][:] = row of keys[i].
+ * keys: device int64[N]; bag_offsets: device int64[F*B+1] (0 .. N, non-decreasing);
+ * pooled_out: device fp32 [B][F][D] or NULL; unpooled_out: device fp32 [N][D]
+ * or NULL.  keys and bag_offsets must stay unchanged until the matching
+ * recis_backward_update has run.  N <= 2^31 - 1. */
+recis_status recis_lookup_pooled(recis_table_t t, recis_batch_t b, const int64_t* keys,
+                                 int64_t N, const int64_t* bag_offsets, int32_t F, int64_t B,
+                                 int32_t combiner, float* pooled_out, float* unpooled_out,
+                                 recis_stream_t stream);
+
+/* Backward + optimiser for the batch's last lookup (README, Operator
+ * implementation: reduction merged at warp level; Efficient dynamic embedding:
+ * optimiser state beside the parameters).  g(u) = sum over occurrences of
+ * key u of grad_pooled[b][f] (x 1/length for MEAN) + grad_unpooled[i], then one
+ * Adagrad or Adam step on every row touched by the lookup (Adam: the table's
+ * step counter advances by one per call).  grad_pooled: device [B][F][D] or
+ * NULL; grad_unpooled: device [N][D] or NULL (NULL = zero gradient). */
+recis_status recis_backward_update(recis_table_t t, recis_batch_t b, const float* grad_pooled,
+                                   const float* grad_unpooled, recis_stream_t stream);
+
+/* Find-or-insert only (no pooling): used to pre-load a table.  keys: device
+ * int64[N].  rows_out: device int64[N] (row of each key) or NULL. */
+recis_status recis_table_insert(recis_table_t t, recis_batch_t b, const int64_t* keys, int64_t N,
+                                int64_t* rows_out, recis_stream_t stream);
+
+/* Synchronous.  Number of live rows and the Adam step counter. */
+recis_status recis_table_size(recis_table_t t, int64_t* n_out, int64_t* step_out,
+                              recis_stream_t stream);
+
+/* Synchronous (README, Core architecture > Saver: sparse parameters saved for
+ * delivery).  Copies the first min(n, capacity) rows, in ascending row order,
+ * to HOST buffers: keys int64[capacity] (or NULL), emb fp32 [capacity][D] (or
+ * NULL), state fp32 [capacity][s*D] (or NULL; Adam: m then v).  *n_out = live
+ * rows, *step_out = Adam step. */
+recis_status recis_table_export(recis_table_t t, int64_t* keys, float* emb, float* state,
+                                int64_t capacity, int64_t* n_out, int64_t* step_out,
+                                recis_stream_t stream);
+
+/* Synchronous.  Appends n rows from HOST buffers after the live rows (keys must
+ * not be present; state NULL = initial state) and sets the step counter. */
+recis_status recis_table_import(recis_table_t t, const int64_t* keys, const float* emb,
+                                const float* state, int64_t n, int64_t step,
+                                recis_stream_t stream);
+
+/* Synchronous: waits for `stream`; returns and clears the table's device status. */
+recis_status recis_table_status_sync(recis_table_t t, recis_stream_t stream);
+
+/* Synchronous.  Copies the last lookup's dedup into caller DEVICE buffers (each
+ * may be NULL): uniq_out int64[capacity] (the min(U, capacity) unique keys,
+ * ascending), rows_out int64[capacity] (their row offsets), inv_out int32[N]
+ * (index into uniq of every key).  *U_out = U, *n_new_out = keys inserted. */
+recis_status recis_batch_get_unique(recis_batch_t b, int64_t* uniq_out, int32_t* inv_out,
+                                    int64_t* rows_out, int64_t capacity, int64_t* U_out,
+                                    int64_t* n_new_out, recis_stream_t stream);
+
+/* ------------------------------------------------------------------ tracing */
+/* Kernel timing: while enabled, every kernel launch is bracketed by CUDA
+ * events on its stream.  recis_profile_collect (synchronous) returns per kernel
+ * name: launches and total milliseconds, clears the record, and returns the
+ * number of names (<= max).  recis_launch_count counts all kernel launches of
+ * the library since load. */
+recis_status recis_profile_enable(int32_t on);
+int32_t recis_profile_collect(const char** names, int64_t* launches, double* total_ms,
+                              int32_t max);
+int64_t recis_launch_count(void);
+
+const char* recis_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -2,7 +2,7 @@
  * oracle.h -- plain, slow, single-threaded CPU oracle of the RecIS dynamic-hash
  * embedding step.  TEST INFRASTRUCTURE ONLY: only the tests, the smoke check and
  * the benchmark's CPU-baseline leg may load it.  It shares no code, header,
- * constant or helper with the CUDA library under recommender_sparse_embedding_b200/.
+ * constant or helper with the CUDA library.
  *
  * What it follows (RecIS README, "Core architecture" and "Key optimisations"):
  *   - Feature Engine: Hash / Mod / Bucketize feature transforms.

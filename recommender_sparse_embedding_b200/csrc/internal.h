@@ -1,0 +1,168 @@
+// internal.h -- host-side structures and kernel launchers of the embedding engine.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "../../include/recis.h"
+#include "common.cuh"
+
+namespace recis {
+
+// ---------------------------------------------------------------- sort
+constexpr int kSortBits = 8;
+constexpr int kSortPasses = 64 / kSortBits;
+constexpr int kSortBlock = 256;
+constexpr int kSortItems = 8;
+constexpr int kSortTile = kSortBlock * kSortItems;  // 2048 keys per tile
+
+// Per-call control block of the sort and of the unique pass.  The first
+// kCtlZeroBytes bytes are cleared before every lookup.
+struct SortCtl {
+  unsigned int hist[kSortPasses][256];
+  unsigned int tile_counter[kSortPasses];
+  unsigned int ticket;
+  unsigned int seg_tile_counter;
+  unsigned int pad0[6];
+  // written by the last CTA of the histogram kernel
+  unsigned int active[kSortPasses];   // pass p moves keys (its digit is not constant)
+  unsigned int ordinal[kSortPasses];  // number of active passes before p
+  unsigned int n_active;
+  unsigned int pad1[15];
+  unsigned int base[kSortPasses][256];  // first output position of each digit
+};
+constexpr size_t kCtlZeroBytes = offsetof(SortCtl, active);
+
+// Per-batch device scalars.
+struct BatchDev {
+  unsigned long long row_base;  // table's next_free when the lookup started
+  unsigned int U;               // unique keys of the last lookup
+  unsigned int n_new;           // new keys of the last lookup
+};
+
+// ---------------------------------------------------------------- table
+struct VmmArray {
+  CUdeviceptr va = 0;
+  size_t reserved = 0;   // bytes of address space
+  size_t mapped = 0;     // bytes backed by physical blocks
+  std::vector<CUmemGenericAllocationHandle> handles;
+  std::vector<size_t> sizes;
+};
+
+}  // namespace recis
+
+struct recis_table {
+  int dev = 0;
+  recis_table_config cfg{};
+  int D = 0, s = 0, row_floats = 0;
+  size_t row_bytes = 0;
+  float init_two_s = 0.f;
+  size_t gran = 0;              // VMM granularity
+  int64_t block_rows = 0;
+  int64_t max_rows = 0;
+  int64_t mapped_rows = 0;
+  recis::VmmArray rows;         // [row][emb D | state s*D] fp32
+  recis::VmmArray keys;         // [row] int64, key of each row
+  recis::Slot* slots = nullptr; // IDMap
+  int64_t capacity = 0;         // slots, power of two
+  recis::DevState* dstate = nullptr;
+  recis::HostMirror* mirror = nullptr;  // host-mapped
+  recis::HostMirror* mirror_dev = nullptr;
+  // progress events: ring[k] recorded after a call, when cum_issued was ring_cum[k]
+  static constexpr int kRing = 8;
+  cudaEvent_t ring[kRing] = {};
+  int64_t ring_cum[kRing] = {};
+  int ring_next = 0;
+  int ring_live = 0;            // recorded events not yet consumed (newest first)
+  int64_t cum_issued = 0;       // sum of N over all lookups issued
+  int64_t rows_upper = 0;       // upper bound on live rows
+  int64_t step = 0;             // Adam step counter
+};
+
+struct recis_batch {
+  int dev = -1;
+  int64_t capN = 0;             // occurrence capacity of the N-sized buffers
+  int64_t capBags = 0;
+  int64_t capPartials = 0;      // floats
+  uint64_t* kbuf[2] = {nullptr, nullptr};
+  uint32_t* vbuf[2] = {nullptr, nullptr};
+  unsigned long long* sort_lookback = nullptr;  // [tiles][256], epoch-tagged
+  int64_t sort_lookback_tiles = 0;
+  recis::SortCtl* ctl = nullptr;
+  unsigned long long* seg_lookback = nullptr;   // [tiles], cleared per call (follows ctl)
+  int64_t seg_lookback_tiles = 0;
+  int64_t* uniq = nullptr;
+  int64_t* rows = nullptr;
+  int32_t* inv = nullptr;
+  int32_t* seg_of = nullptr;    // segment (unique index) of each sorted position
+  int32_t* seg_start = nullptr; // [U+1] first sorted position of each unique
+  int32_t* occ_bag = nullptr;   // bag of each occurrence
+  int32_t* seg_counter = nullptr;  // [capN] last-arrival counters (self-resetting)
+  int32_t* bag_counter = nullptr;  // [capBags]
+  float* partials = nullptr;
+  recis::BatchDev* bdev = nullptr;
+  uint32_t epoch = 0;
+  // the last lookup, for the backward
+  recis_table* table = nullptr;
+  int64_t N = 0;
+  int32_t F = 0;
+  int64_t B = 0;
+  int32_t combiner = 0;
+  const int64_t* keys = nullptr;
+  const int64_t* bag_offsets = nullptr;
+  bool have_lookup = false;
+  bool backward_done = true;
+};
+
+namespace recis {
+
+void set_error(const std::string& msg);
+recis_status cuda_fail(cudaError_t e, const char* what);
+
+// launch bookkeeping (tracing)
+struct LaunchScope {
+  LaunchScope(const char* name, cudaStream_t s);
+  ~LaunchScope();
+  const char* name;
+  cudaStream_t stream;
+  int slot;
+};
+
+// ---- launchers (each returns the CUDA error of the launch)
+cudaError_t launch_feature_hash(const recis_feature_op* ops, int F, const int64_t* values,
+                                const int64_t* feat_offsets, int64_t* keys_out, int* dev_status,
+                                cudaStream_t s);
+
+struct LookupArgs {
+  recis_table* t;
+  recis_batch* b;
+  const int64_t* keys;
+  int64_t N;
+  const int64_t* bag_offsets;
+  int32_t F;
+  int64_t B;
+  int32_t combiner;
+  float* pooled_out;
+  float* unpooled_out;
+  int64_t* rows_out;  // insert path: row per occurrence
+};
+
+cudaError_t launch_sort(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
+                        cudaStream_t s);
+cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cudaStream_t s);
+cudaError_t launch_pool(const LookupArgs& a, int64_t chunk, cudaStream_t s);
+cudaError_t launch_rows_per_key(recis_batch* b, int64_t N, int64_t* rows_out, cudaStream_t s);
+cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pooled,
+                          const float* grad_unpooled, int64_t chunk, float lr_t, float inv_sqrt_bc2,
+                          cudaStream_t s);
+cudaError_t launch_import(recis_table* t, const int64_t* keys, int64_t n, int64_t row0,
+                          cudaStream_t s);
+cudaError_t launch_rehash(recis_table* t, const Slot* old_slots, int64_t old_cap, cudaStream_t s);
+
+int64_t pool_chunk_for(int64_t N, int D);
+int64_t update_chunk_for(int64_t N, int D);
+
+}  // namespace recis

@@ -1,0 +1,85 @@
+// segreduce.cuh -- shared machinery of the two segmented reductions (bag
+// pooling in the forward, per-unique gradient reduction in the backward).
+//
+// The positions [0, N) are cut into fixed chunks of C positions; one group of
+// G lanes walks one chunk in order, 16 bytes (one float4 column) per lane, so
+// the work is balanced whatever the bag or segment lengths are.  A segment
+// that lies inside one chunk is finished by that group.  A segment cut by
+// chunk boundaries leaves one partial sum per chunk it touches (slot 0 when it
+// is the chunk's first segment, slot 1 otherwise); the group that arrives last
+// (atomic ticket per segment, reset by that group) adds the partials in chunk
+// order, so results are deterministic and no per-element atomics are used.
+#pragma once
+#include "internal.h"
+
+namespace recis {
+
+template <int G>
+struct GroupCtx {
+  int lane;        // lane within the group
+  unsigned mask;   // lanes of this group within the warp
+  int shift;       // first lane of the group within the warp
+  __device__ __forceinline__ GroupCtx() {
+    const int wl = threadIdx.x & 31;
+    lane = wl & (G - 1);
+    shift = wl & ~(G - 1);
+    mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << shift);
+  }
+  template <typename T>
+  __device__ __forceinline__ T bcast(T v, int src) const {
+    return __shfl_sync(mask, v, src, G);
+  }
+  __device__ __forceinline__ unsigned ballot(bool pr) const {
+    return (__ballot_sync(mask, pr) >> shift) & ((G == 32) ? 0xffffffffu : ((1u << G) - 1u));
+  }
+};
+
+__device__ __forceinline__ float4 f4_zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+__device__ __forceinline__ void f4_add(float4& a, const float4& b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+
+// Last-arrival combine of a split segment.  Every group that touched the
+// segment calls this once with its partial; returns true in the group that
+// must finish the segment, with the full sum in acc.
+template <int G, int VPL>
+__device__ __forceinline__ bool combine_split(const GroupCtx<G>& g, float4 (&acc)[VPL],
+                                              float* partials, int32_t* counters, int64_t seg,
+                                              int64_t chunk, bool first_of_chunk,
+                                              int64_t seg_start, int64_t seg_end, int64_t C,
+                                              int ncol) {
+  const int slot = first_of_chunk ? 0 : 1;
+  const int64_t D = (int64_t)ncol * 4;
+  float* mine = partials + (chunk * 2 + slot) * D;
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const int col = g.lane + v * G;
+    if (col < ncol) __stcg(reinterpret_cast<float4*>(mine) + col, acc[v]);
+  }
+  __threadfence();
+  __syncwarp(g.mask);
+  int ticket = 0;
+  if (g.lane == 0) ticket = atomicAdd(&counters[seg], 1);
+  ticket = g.bcast(ticket, 0);
+  const int64_t c0 = seg_start / C, c1 = (seg_end - 1) / C;
+  if (ticket != (int)(c1 - c0)) return false;
+  __threadfence();
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) acc[v] = f4_zero();
+  for (int64_t cc = c0; cc <= c1; ++cc) {
+    const int sl = (cc == c0 && seg_start != c0 * C) ? 1 : 0;
+    const float* src = partials + (cc * 2 + sl) * D;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const int col = g.lane + v * G;
+      if (col < ncol) f4_add(acc[v], __ldcg(reinterpret_cast<const float4*>(src) + col));
+    }
+  }
+  if (g.lane == 0) counters[seg] = 0;
+  return true;
+}
+
+}  // namespace recis

@@ -1,0 +1,398 @@
+// unique.cu -- the second half of the dedup step fused with the IDMap
+// find-or-insert and the initialisation of new rows (RecIS README, Key
+// optimisations > Efficient dynamic embedding: IDMap = first-level store,
+// feature ID -> offset; EmbeddingBlocks = second-level store of parameters and
+// optimiser state).
+//
+// One pass over the sorted (key, occurrence) pairs, 1024 positions per tile:
+//   1. head flags (first position of each distinct key);
+//   2. each head probes the IDMap (open addressing, linear probing, 16-byte
+//      slots {key, row}); a missing key is claimed with a 64-bit CAS;
+//   3. the tile publishes (heads, new keys) and resolves its prefix by
+//      decoupled look-back, which numbers the unique keys in ascending order
+//      and gives new keys consecutive rows in ascending key order after the
+//      table's live rows;
+//   4. writes uniq / rows / segment starts / inverse index, the row of each
+//      new slot and the key of each new row, and initialises the new rows
+//      (seeded hash of the key; optimiser state at its initial value).
+// The last tile publishes U, the new-key count and the table's next free row.
+#include "internal.h"
+
+namespace recis {
+
+namespace {
+
+constexpr int kUqBlock = 256, kUqItems = 4, kUqTile = kUqBlock * kUqItems;
+constexpr int kMaxProbes = 1 << 16;
+constexpr unsigned long long kUqAgg = 1ULL << 62, kUqIncl = 2ULL << 62;
+
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// IDMap find-or-insert.  Returns true when the key was inserted by this call
+// (slot index in *slot); otherwise *row holds the existing row.  *slot = -1
+// when the probe limit is reached.
+__device__ __forceinline__ bool idmap_find_or_insert(Slot* slots, uint64_t mask, int64_t key,
+                                                     int64_t* slot, int64_t* row) {
+  uint64_t h = mix64((uint64_t)key ^ kSlotSalt) & mask;
+  const int64_t limit = (int64_t)mask + 1 < kMaxProbes ? (int64_t)mask + 1 : kMaxProbes;
+  for (int64_t n = 0; n < limit; ++n) {
+    const longlong2 sv = __ldcg(reinterpret_cast<const longlong2*>(slots + h));
+    if (sv.x == key) {
+      *slot = (int64_t)h;
+      *row = sv.y;
+      return false;
+    }
+    if (sv.x == kEmptyKey) {
+      const unsigned long long old = atomicCAS(reinterpret_cast<unsigned long long*>(&slots[h].key),
+                                               (unsigned long long)kEmptyKey,
+                                               (unsigned long long)key);
+      if ((int64_t)old == kEmptyKey) {
+        *slot = (int64_t)h;
+        *row = -1;
+        return true;
+      }
+      if ((int64_t)old == key) {
+        *slot = (int64_t)h;
+        *row = __ldcg(&slots[h].row);
+        return false;
+      }
+    }
+    h = (h + 1) & mask;
+  }
+  *slot = -1;
+  *row = -1;
+  return false;
+}
+
+}  // namespace
+
+struct UniqueParams {
+  const int64_t* in_keys;
+  const uint64_t* kb0;
+  const uint64_t* kb1;
+  const uint32_t* vb0;
+  const uint32_t* vb1;
+  int64_t N;
+  SortCtl* ctl;
+  unsigned long long* lookback;
+  Slot* slots;
+  uint64_t slot_mask;
+  float* row_data;
+  int64_t* row_keys;
+  int64_t mapped_rows;
+  int row_floats;
+  int D;
+  int adagrad;
+  float acc0;
+  float two_s;
+  uint64_t init_seed;
+  int64_t* uniq;
+  int64_t* rows;
+  int32_t* inv;
+  int32_t* seg_of;
+  int32_t* seg_start;
+  BatchDev* bdev;
+  DevState* st;
+  HostMirror* mirror;
+};
+
+__global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_constant__ UniqueParams p) {
+  __shared__ uint64_t s_last[kUqBlock];
+  __shared__ unsigned s_scan[kUqBlock / 32];
+  __shared__ unsigned s_tile;
+  __shared__ unsigned long long s_prefix;
+  __shared__ int s_ninit;
+  __shared__ int64_t s_init_key[kUqTile];
+  __shared__ int64_t s_init_row[kUqTile];
+
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  if (tid == 0) {
+    s_tile = atomicAdd(&p.ctl->seg_tile_counter, 1u);
+    s_ninit = 0;
+  }
+  __syncthreads();
+  const unsigned tile = s_tile;
+  const int64_t N = p.N;
+  const unsigned na = p.ctl->n_active;
+  const uint64_t* ks = na == 0 ? nullptr : (((na - 1) & 1) ? p.kb1 : p.kb0);
+  const uint32_t* vs = na == 0 ? nullptr : (((na - 1) & 1) ? p.vb1 : p.vb0);
+  const int64_t tbase = (int64_t)tile * kUqTile;
+  const int64_t pos0 = tbase + (int64_t)tid * kUqItems;
+
+  uint64_t k[kUqItems];
+  uint32_t v[kUqItems];
+#pragma unroll
+  for (int j = 0; j < kUqItems; ++j) {
+    const int64_t pos = pos0 + j;
+    if (pos < N) {
+      k[j] = ks ? ks[pos] : to_ukey(p.in_keys[pos]);
+      v[j] = vs ? vs[pos] : (uint32_t)pos;
+    } else {
+      k[j] = 0;
+      v[j] = 0;
+    }
+  }
+  s_last[tid] = k[kUqItems - 1];
+  __syncthreads();
+  uint64_t prev;
+  bool have_prev;
+  if (tid > 0) {
+    prev = s_last[tid - 1];
+    have_prev = true;
+  } else if (tbase > 0) {
+    prev = ks ? ks[tbase - 1] : to_ukey(p.in_keys[tbase - 1]);
+    have_prev = true;
+  } else {
+    prev = 0;
+    have_prev = false;
+  }
+
+  bool head[kUqItems], isnew[kUqItems];
+  int64_t slot[kUqItems], row[kUqItems];
+  unsigned nh = 0, nn = 0;
+#pragma unroll
+  for (int j = 0; j < kUqItems; ++j) {
+    const int64_t pos = pos0 + j;
+    const uint64_t pk = j == 0 ? prev : k[j - 1];
+    head[j] = pos < N && (!(j == 0 ? have_prev : true) || pk != k[j]);
+    isnew[j] = false;
+    slot[j] = -1;
+    row[j] = -1;
+    if (head[j] && from_ukey(k[j]) != kEmptyKey) {  // the reserved key is reported by the sort
+      isnew[j] = idmap_find_or_insert(p.slots, p.slot_mask, from_ukey(k[j]), &slot[j], &row[j]);
+      if (slot[j] < 0) raise_error(p.st, p.mirror, kErrTableFull);
+    }
+    if (head[j]) {
+      ++nh;
+      nn += isnew[j];
+    }
+  }
+  // block exclusive scan of (heads, new) packed as heads | new << 16
+  const unsigned mine = nh | (nn << 16);
+  unsigned x = mine;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) s_scan[w] = x;
+  __syncthreads();
+  unsigned wpre = 0, tot = 0;
+#pragma unroll
+  for (int ww = 0; ww < kUqBlock / 32; ++ww) {
+    const unsigned c = s_scan[ww];
+    if (ww < w) wpre += c;
+    tot += c;
+  }
+  const unsigned excl_thread = wpre + x - mine;
+  const unsigned long long tH = tot & 0xffffu, tN = tot >> 16;
+
+  if (tid == 0) {
+    unsigned long long* my = p.lookback + tile;
+    unsigned long long hx = 0, nx = 0;
+    if (tile == 0) {
+      st_relaxed(my, kUqIncl | (tH << 31) | tN);
+    } else {
+      st_relaxed(my, kUqAgg | (tH << 31) | tN);
+      int64_t t = (int64_t)tile - 1;
+      int spins = 0;
+      while (t >= 0) {
+        const unsigned long long e = ld_relaxed(p.lookback + t);
+        const unsigned long long flag = e >> 62;
+        if (flag == 0) {
+          if (++spins > kSpinLimit) {
+            raise_error(p.st, p.mirror, kErrTimeout);
+            break;
+          }
+          __nanosleep(32);
+          continue;
+        }
+        hx += (e >> 31) & 0x7fffffffULL;
+        nx += e & 0x7fffffffULL;
+        if (flag == 2) break;
+        --t;
+      }
+      st_relaxed(my, kUqIncl | ((hx + tH) << 31) | (nx + tN));
+    }
+    s_prefix = (hx << 32) | nx;
+  }
+  __syncthreads();
+  const unsigned long long Hx = s_prefix >> 32, Nx = s_prefix & 0xffffffffULL;
+  const unsigned long long row_base = p.bdev->row_base;
+
+  unsigned hrun = Hx + (excl_thread & 0xffffu);
+  unsigned nrun = (unsigned)Nx + (excl_thread >> 16);
+#pragma unroll
+  for (int j = 0; j < kUqItems; ++j) {
+    const int64_t pos = pos0 + j;
+    if (pos >= N) break;
+    if (head[j]) {
+      const unsigned seg = hrun;
+      int64_t r = row[j];
+      if (isnew[j]) {
+        r = (int64_t)(row_base + nrun);
+        ++nrun;
+        if (r >= p.mapped_rows) {
+          raise_error(p.st, p.mirror, kErrTableFull);
+          r = -1;
+        } else {
+          p.slots[slot[j]].row = r;
+          p.row_keys[r] = from_ukey(k[j]);
+          const int q = atomicAdd(&s_ninit, 1);
+          s_init_key[q] = from_ukey(k[j]);
+          s_init_row[q] = r;
+        }
+      }
+      p.uniq[seg] = from_ukey(k[j]);
+      p.rows[seg] = r;
+      p.seg_start[seg] = (int32_t)pos;
+      ++hrun;
+    }
+    const int32_t seg = (int32_t)(hrun - 1);
+    p.seg_of[pos] = seg;
+    if (v[j] < (uint64_t)N) p.inv[v[j]] = seg;
+  }
+  if (tile == gridDim.x - 1 && tid == 0) {
+    const unsigned long long U = Hx + tH, nnew = Nx + tN;
+    p.bdev->U = (unsigned)U;
+    p.bdev->n_new = (unsigned)nnew;
+    unsigned long long nf = row_base + nnew;
+    if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
+    p.st->next_free = nf;
+    if (p.mirror) {
+      p.mirror->next_free = nf;
+      __threadfence_system();
+    }
+    p.seg_start[U] = (int32_t)N;
+  }
+  __syncthreads();
+  // initialise this tile's new rows, 16 bytes per thread per step
+  const int nf4 = p.row_floats >> 2;
+  const int total = s_ninit * nf4;
+  for (int idx = tid; idx < total; idx += kUqBlock) {
+    const int r = idx / nf4;
+    const int c = (idx - r * nf4) * 4;
+    const int64_t key = s_init_key[r];
+    const uint64_t base = mix64((uint64_t)key ^ p.init_seed);
+    float o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int col = c + e;
+      o[e] = col < p.D ? init_value(base, col, p.two_s) : (p.adagrad ? p.acc0 : 0.0f);
+    }
+    float4* dst = reinterpret_cast<float4*>(p.row_data + s_init_row[r] * (int64_t)p.row_floats + c);
+    *dst = make_float4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+__global__ void rows_per_key_kernel(const int32_t* __restrict__ inv, const int64_t* __restrict__ rows,
+                                    int64_t N, int64_t* __restrict__ out) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < N; i += stride)
+    out[i] = rows[inv[i]];
+}
+
+cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cudaStream_t s) {
+  UniqueParams p;
+  p.in_keys = b->keys;
+  p.kb0 = b->kbuf[0];
+  p.kb1 = b->kbuf[1];
+  p.vb0 = b->vbuf[0];
+  p.vb1 = b->vbuf[1];
+  p.N = N;
+  p.ctl = b->ctl;
+  p.lookback = b->seg_lookback;
+  p.slots = t->slots;
+  p.slot_mask = (uint64_t)t->capacity - 1;
+  p.row_data = reinterpret_cast<float*>(t->rows.va);
+  p.row_keys = reinterpret_cast<int64_t*>(t->keys.va);
+  p.mapped_rows = t->mapped_rows;
+  p.row_floats = t->row_floats;
+  p.D = t->D;
+  p.adagrad = t->cfg.optimizer == RECIS_ADAGRAD;
+  p.acc0 = (float)t->cfg.adagrad_init_acc;
+  p.two_s = t->init_two_s;
+  p.init_seed = t->cfg.init_seed;
+  p.uniq = b->uniq;
+  p.rows = b->rows;
+  p.inv = b->inv;
+  p.seg_of = b->seg_of;
+  p.seg_start = b->seg_start;
+  p.bdev = b->bdev;
+  p.st = t->dstate;
+  p.mirror = t->mirror_dev;
+  const int64_t tiles = (N + kUqTile - 1) / kUqTile;
+  LaunchScope ls("unique_insert", s);
+  unique_insert_kernel<<<(unsigned)tiles, kUqBlock, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rows_per_key(recis_batch* b, int64_t N, int64_t* rows_out, cudaStream_t s) {
+  int64_t blocks = (N + 255) / 256;
+  if (blocks > 8 * kSMs) blocks = 8 * kSMs;
+  LaunchScope ls("rows_per_key", s);
+  rows_per_key_kernel<<<(unsigned)blocks, 256, 0, s>>>(b->inv, b->rows, N, rows_out);
+  return cudaGetLastError();
+}
+
+__global__ void rehash_kernel(const Slot* __restrict__ old_slots, int64_t old_cap, Slot* slots,
+                              uint64_t mask, DevState* st, HostMirror* mirror) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < old_cap; i += stride) {
+    const Slot sl = old_slots[i];
+    if (sl.key == kEmptyKey) continue;
+    int64_t slot, row;
+    if (idmap_find_or_insert(slots, mask, sl.key, &slot, &row))
+      slots[slot].row = sl.row;
+    else
+      raise_error(st, mirror, slot < 0 ? kErrTableFull : kErrDuplicateImport);
+  }
+}
+
+__global__ void import_kernel(const int64_t* __restrict__ keys, int64_t n, int64_t row0,
+                              Slot* slots, uint64_t mask, int64_t* row_keys, DevState* st,
+                              HostMirror* mirror) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    int64_t slot, row;
+    if (idmap_find_or_insert(slots, mask, keys[i], &slot, &row)) {
+      slots[slot].row = row0 + i;
+      row_keys[row0 + i] = keys[i];
+    } else {
+      raise_error(st, mirror, slot < 0 ? kErrTableFull : kErrDuplicateImport);
+    }
+  }
+}
+
+cudaError_t launch_rehash(recis_table* t, const Slot* old_slots, int64_t old_cap, cudaStream_t s) {
+  int64_t blocks = (old_cap + 255) / 256;
+  if (blocks > 16 * kSMs) blocks = 16 * kSMs;
+  LaunchScope ls("idmap_rehash", s);
+  rehash_kernel<<<(unsigned)blocks, 256, 0, s>>>(old_slots, old_cap, t->slots,
+                                                 (uint64_t)t->capacity - 1, t->dstate,
+                                                 t->mirror_dev);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_import(recis_table* t, const int64_t* keys, int64_t n, int64_t row0,
+                          cudaStream_t s) {
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 16 * kSMs) blocks = 16 * kSMs;
+  if (blocks < 1) return cudaSuccess;
+  LaunchScope ls("idmap_import", s);
+  import_kernel<<<(unsigned)blocks, 256, 0, s>>>(keys, n, row0, t->slots, (uint64_t)t->capacity - 1,
+                                                 reinterpret_cast<int64_t*>(t->keys.va), t->dstate,
+                                                 t->mirror_dev);
+  return cudaGetLastError();
+}
+
+int64_t unique_tiles_for(int64_t N) { return (N + kUqTile - 1) / kUqTile; }
+
+}  // namespace recis
