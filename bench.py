@@ -196,7 +196,8 @@ def run_gpu(args):
                      torch.from_numpy(b.bag_offsets).to(dev), torch.from_numpy(g).to(dev),
                      len(b.values)))
     opt = R.ADAM if spec.optimizer == "adam" else R.ADAGRAD
-    table = R.Table(D, opt, spec.lr, init_seed=spec.init_seed, initial_capacity=8_000_000)
+    table = R.Table(D, opt, spec.lr, init_seed=spec.init_seed,
+                    initial_capacity=1_000_000 if args.small else 8_000_000)
     batch = R.Batch()
     keys = torch.empty(max(x[4] for x in devb), dtype=torch.int64, device=dev)
     pooled = torch.empty((w.B, w.F, D), dtype=torch.float32, device=dev)
@@ -355,6 +356,8 @@ def main():
     ap.add_argument("--batches", type=int, default=32, help="distinct batches generated")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--small", action="store_true",
+                    help="smaller table reservation (for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "own":
         args.warmup = 3

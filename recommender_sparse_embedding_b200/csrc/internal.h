@@ -86,7 +86,7 @@ struct recis_batch {
   int dev = -1;
   int64_t capN = 0;             // occurrence capacity of the N-sized buffers
   int64_t capBags = 0;
-  int64_t capPartials = 0;      // floats
+  int64_t capPartials = 0;      // doubles
   uint64_t* kbuf[2] = {nullptr, nullptr};
   uint32_t* vbuf[2] = {nullptr, nullptr};
   unsigned long long* sort_lookback = nullptr;  // [tiles][256], epoch-tagged
@@ -102,7 +102,7 @@ struct recis_batch {
   int32_t* occ_bag = nullptr;   // bag of each occurrence
   int32_t* seg_counter = nullptr;  // [capN] last-arrival counters (self-resetting)
   int32_t* bag_counter = nullptr;  // [capBags]
-  float* partials = nullptr;
+  double* partials = nullptr;
   recis::BatchDev* bdev = nullptr;
   uint32_t epoch = 0;
   // the last lookup, for the backward

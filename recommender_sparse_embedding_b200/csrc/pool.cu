@@ -35,7 +35,7 @@ struct PoolParams {
   float* pooled;         // [B][F][D] or null
   float* unpooled;       // [N][D] or null
   int32_t* occ_bag;      // [N]
-  float* partials;
+  double* partials;
   int32_t* counters;     // [nbags]
   DevState* st;
   HostMirror* mirror;
@@ -82,28 +82,28 @@ __global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolP
   int64_t wend = (wbase + g.lane < p.nbags) ? p.offs[wbase + g.lane + 1] : INT64_MAX;
   int64_t cur_end = g.bcast(wend, 0);
 
-  float4 acc[VPL];
+  Acc4 acc[VPL];
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) acc[v] = f4_zero();
+  for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
   bool has = false;
 
   auto epilogue = [&](int64_t bag, int64_t len) {
     if (!p.pooled) return;
     const int64_t f = bag / p.B, b = bag - f * p.B;
     float4* o = reinterpret_cast<float4*>(p.pooled + (b * p.F + f) * D);
-    const float flen = (float)len;
+    const double dlen = (double)len;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       const int col = g.lane + v * G;
       if (col < p.ncol) {
-        float4 r = acc[v];
+        Acc4 r = acc[v];
         if (p.mean) {
-          r.x = __fdiv_rn(r.x, flen);
-          r.y = __fdiv_rn(r.y, flen);
-          r.z = __fdiv_rn(r.z, flen);
-          r.w = __fdiv_rn(r.w, flen);
+          r.x /= dlen;
+          r.y /= dlen;
+          r.z /= dlen;
+          r.w /= dlen;
         }
-        o[col] = r;
+        o[col] = acc_round(r);
       }
     }
   };
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolP
     if (!(cur_start >= 0 && cur_start < cur_end && cur_end <= p.N)) {  // malformed bag offsets
       if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
 #pragma unroll
-      for (int v = 0; v < VPL; ++v) acc[v] = f4_zero();
+      for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
       has = false;
       return;
     }
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolP
       epilogue(cur, cur_end - cur_start);
     }
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) acc[v] = f4_zero();
+    for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
     has = false;
   };
 
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolP
         cur_end = g.bcast(wend, (int)(cur - wbase));
       }
 #pragma unroll
-      for (int v = 0; v < VPL; ++v) f4_add(acc[v], val[k][v]);
+      for (int v = 0; v < VPL; ++v) acc_add(acc[v], val[k][v]);
       has = true;
       if (p.unpooled) {
 #pragma unroll

@@ -35,29 +35,52 @@ struct GroupCtx {
 };
 
 __device__ __forceinline__ float4 f4_zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
-__device__ __forceinline__ void f4_add(float4& a, const float4& b) {
+
+// fp64 accumulator of one 16-byte column (4 floats).  Bags of thousands of
+// rows and hot keys with tens of thousands of occurrences are summed in double
+// and rounded once, so the fp32 result does not depend on the length of the
+// sum.
+struct Acc4 {
+  double x, y, z, w;
+};
+__device__ __forceinline__ Acc4 acc_zero() { return Acc4{0.0, 0.0, 0.0, 0.0}; }
+__device__ __forceinline__ void acc_add(Acc4& a, const float4& b) {
+  a.x += (double)b.x;
+  a.y += (double)b.y;
+  a.z += (double)b.z;
+  a.w += (double)b.w;
+}
+__device__ __forceinline__ void acc_add(Acc4& a, const Acc4& b) {
   a.x += b.x;
   a.y += b.y;
   a.z += b.z;
   a.w += b.w;
 }
+__device__ __forceinline__ float4 acc_round(const Acc4& a) {
+  return make_float4((float)a.x, (float)a.y, (float)a.z, (float)a.w);
+}
 
 // Last-arrival combine of a split segment.  Every group that touched the
 // segment calls this once with its partial; returns true in the group that
-// must finish the segment, with the full sum in acc.
+// must finish the segment, with the full sum in acc.  Partials are fp64,
+// 32 bytes per column, two slots of D doubles per chunk.
 template <int G, int VPL>
-__device__ __forceinline__ bool combine_split(const GroupCtx<G>& g, float4 (&acc)[VPL],
-                                              float* partials, int32_t* counters, int64_t seg,
+__device__ __forceinline__ bool combine_split(const GroupCtx<G>& g, Acc4 (&acc)[VPL],
+                                              double* partials, int32_t* counters, int64_t seg,
                                               int64_t chunk, bool first_of_chunk,
                                               int64_t seg_start, int64_t seg_end, int64_t C,
                                               int ncol) {
   const int slot = first_of_chunk ? 0 : 1;
   const int64_t D = (int64_t)ncol * 4;
-  float* mine = partials + (chunk * 2 + slot) * D;
+  double* mine = partials + (chunk * 2 + slot) * D;
 #pragma unroll
   for (int v = 0; v < VPL; ++v) {
     const int col = g.lane + v * G;
-    if (col < ncol) __stcg(reinterpret_cast<float4*>(mine) + col, acc[v]);
+    if (col < ncol) {
+      double2* d = reinterpret_cast<double2*>(mine) + 2 * col;
+      __stcg(d, make_double2(acc[v].x, acc[v].y));
+      __stcg(d + 1, make_double2(acc[v].z, acc[v].w));
+    }
   }
   __threadfence();
   __syncwarp(g.mask);
@@ -68,14 +91,18 @@ __device__ __forceinline__ bool combine_split(const GroupCtx<G>& g, float4 (&acc
   if (ticket != (int)(c1 - c0)) return false;
   __threadfence();
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) acc[v] = f4_zero();
+  for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
   for (int64_t cc = c0; cc <= c1; ++cc) {
     const int sl = (cc == c0 && seg_start != c0 * C) ? 1 : 0;
-    const float* src = partials + (cc * 2 + sl) * D;
+    const double* src = partials + (cc * 2 + sl) * D;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       const int col = g.lane + v * G;
-      if (col < ncol) f4_add(acc[v], __ldcg(reinterpret_cast<const float4*>(src) + col));
+      if (col < ncol) {
+        const double2 a = __ldcg(reinterpret_cast<const double2*>(src) + 2 * col);
+        const double2 b = __ldcg(reinterpret_cast<const double2*>(src) + 2 * col + 1);
+        acc_add(acc[v], Acc4{a.x, a.y, b.x, b.y});
+      }
     }
   }
   if (g.lane == 0) counters[seg] = 0;

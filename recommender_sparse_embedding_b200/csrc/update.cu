@@ -35,7 +35,7 @@ struct UpdateParams {
   const float* gp;          // grad_pooled [B][F][D] or null
   const float* gu;          // grad_unpooled [N][D] or null
   float* row_data;
-  float* partials;
+  double* partials;
   int32_t* counters;        // [U]
   const SortCtl* ctl;
   const uint32_t* vb0;
@@ -44,12 +44,13 @@ struct UpdateParams {
   float lr;        // Adagrad: lr; Adam: lr / (1 - beta1^t)
   float eps;
   float beta1, beta2;
+  float omb1, omb2;  // 1 - beta1, 1 - beta2 (formed in double, rounded once)
   float sqrt_bc2;  // Adam: sqrt(1 - beta2^t)
 };
 
 template <int G, int VPL, bool ADAM>
 __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateParams& p,
-                                             int64_t row, const float4 (&grad)[VPL]) {
+                                             int64_t row, const Acc4 (&grad)[VPL]) {
   if (row < 0) return;
   float* base = p.row_data + row * p.row_floats;
   const int D = p.ncol * 4;
@@ -60,7 +61,7 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
     float4* wp = reinterpret_cast<float4*>(base) + col;
     float4* s1p = reinterpret_cast<float4*>(base + D) + col;
     float4 w = *wp, s1 = *s1p;
-    const float gg[4] = {grad[v].x, grad[v].y, grad[v].z, grad[v].w};
+    const float gg[4] = {(float)grad[v].x, (float)grad[v].y, (float)grad[v].z, (float)grad[v].w};
     float ww[4] = {w.x, w.y, w.z, w.w};
     float a1[4] = {s1.x, s1.y, s1.z, s1.w};
     if (!ADAM) {
@@ -76,8 +77,8 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
       float a2[4] = {s2.x, s2.y, s2.z, s2.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float m = p.beta1 * a1[e] + (1.0f - p.beta1) * gg[e];
-        const float vv = p.beta2 * a2[e] + (1.0f - p.beta2) * gg[e] * gg[e];
+        const float m = p.beta1 * a1[e] + p.omb1 * gg[e];
+        const float vv = p.beta2 * a2[e] + p.omb2 * (gg[e] * gg[e]);
         ww[e] = ww[e] - p.lr * m / (sqrtf(vv) / p.sqrt_bc2 + p.eps);
         a1[e] = m;
         a2[e] = vv;
@@ -106,9 +107,9 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
 
   int32_t cur = s0;
   bool cur_starts_here = s0_starts_here;
-  float4 acc[VPL];
+  Acc4 acc[VPL];
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) acc[v] = f4_zero();
+  for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
 
   auto finish = [&](bool ends_here) {
     const int64_t row = p.rows[cur];
@@ -121,13 +122,13 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
         apply_update<G, VPL, ADAM>(g, p, row, acc);
     }
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) acc[v] = f4_zero();
+    for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
   };
 
   for (int64_t pb = p0; pb < p1; pb += K) {
     int32_t sg[K];
     int64_t occ[K];
-    float scale[K];
+    double scale[K];
     int64_t gprow[K];
 #pragma unroll
     for (int k = 0; k < K; ++k) {
@@ -138,33 +139,27 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
     }
 #pragma unroll
     for (int k = 0; k < K; ++k) {
-      scale[k] = 1.0f;
+      scale[k] = 1.0;
       gprow[k] = -1;
       if (occ[k] >= 0 && p.gp) {
         const int64_t bag = p.occ_bag[occ[k]];
         const int64_t f = bag / p.B, b = bag - f * p.B;
         gprow[k] = b * p.F + f;
-        if (p.mean) scale[k] = 1.0f / (float)(p.offs[bag + 1] - p.offs[bag]);
+        if (p.mean) scale[k] = 1.0 / (double)(p.offs[bag + 1] - p.offs[bag]);
       }
     }
-    float4 term[K][VPL];
+    float4 tp[K][VPL], tu[K][VPL];
 #pragma unroll
     for (int k = 0; k < K; ++k) {
 #pragma unroll
       for (int v = 0; v < VPL; ++v) {
         const int col = g.lane + v * G;
-        float4 t = f4_zero();
-        if (col < p.ncol) {
-          if (gprow[k] >= 0) {
-            const float4 a = __ldg(reinterpret_cast<const float4*>(p.gp + gprow[k] * D) + col);
-            t = make_float4(a.x * scale[k], a.y * scale[k], a.z * scale[k], a.w * scale[k]);
-          }
-          if (p.gu && occ[k] >= 0) {
-            const float4 b = __ldg(reinterpret_cast<const float4*>(p.gu + occ[k] * D) + col);
-            f4_add(t, b);
-          }
-        }
-        term[k][v] = t;
+        tp[k][v] = (col < p.ncol && gprow[k] >= 0)
+                       ? __ldg(reinterpret_cast<const float4*>(p.gp + gprow[k] * D) + col)
+                       : f4_zero();
+        tu[k][v] = (col < p.ncol && p.gu && occ[k] >= 0)
+                       ? __ldg(reinterpret_cast<const float4*>(p.gu + occ[k] * D) + col)
+                       : f4_zero();
       }
     }
 #pragma unroll
@@ -176,7 +171,12 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
         cur_starts_here = true;
       }
 #pragma unroll
-      for (int v = 0; v < VPL; ++v) f4_add(acc[v], term[k][v]);
+      for (int v = 0; v < VPL; ++v) {
+        acc[v].x += (double)tp[k][v].x * scale[k] + (double)tu[k][v].x;
+        acc[v].y += (double)tp[k][v].y * scale[k] + (double)tu[k][v].y;
+        acc[v].z += (double)tp[k][v].z * scale[k] + (double)tu[k][v].z;
+        acc[v].w += (double)tp[k][v].w * scale[k] + (double)tu[k][v].w;
+      }
     }
   }
   finish(after != cur);
@@ -234,6 +234,8 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.eps = (float)t->cfg.eps;
   p.beta1 = (float)t->cfg.beta1;
   p.beta2 = (float)t->cfg.beta2;
+  p.omb1 = (float)(1.0 - t->cfg.beta1);
+  p.omb2 = (float)(1.0 - t->cfg.beta2);
   p.sqrt_bc2 = sqrt_bc2;
   if (p.nchunks == 0) return cudaSuccess;
   const bool adam = t->cfg.optimizer == RECIS_ADAM;
