@@ -196,6 +196,29 @@ recis_status recis_batch_get_unique(recis_batch_t b, int64_t* uniq_out, int32_t*
                                     int64_t* rows_out, int64_t capacity, int64_t* U_out,
                                     int64_t* n_new_out, recis_stream_t stream);
 
+/* Dedup without any allocation.  The pages have no counterpart: this exists for
+ * callers that cannot allocate device memory (code inside a framework whose
+ * memory pool forbids foreign cudaMalloc calls, work recorded into a graph
+ * with allocation disabled, or a process that budgets its device memory up
+ * front), which cannot use recis_lookup_pooled because a recis_batch_t grows
+ * its scratch with cudaMalloc.  Computes the same dedup as the first step of
+ * recis_lookup_pooled: uniq_out = distinct keys ascending (signed), inv_out[i]
+ * = index of keys[i] in uniq_out, *U_out = number of unique keys (-1 if a
+ * bounded device-side wait gave up).  Any int64 key is allowed, -1 included
+ * (no IDMap is involved).
+ *   keys: device int64[N], 0 <= N <= 262144 (larger N: RECIS_ERR_INVALID_ARG);
+ *   uniq_out: device int64[N]; inv_out: device int32[N]; U_out: device int64[1].
+ * Asynchronous on `stream`; no cudaMalloc, cudaFree or allocating library call.
+ * Its scratch is one fixed __device__ array of about 6.3 MB that every GPU
+ * which loads the library holds until the process exits.  The first call on a
+ * device looks up that array's device address (cudaGetSymbolAddress); make
+ * that first call before any stream capture.  All calls share the array and
+ * clear what must start at zero themselves; calls that overlap on the GPU
+ * (different streams, or several host threads) race and must be serialised by
+ * the caller. */
+recis_status recis_unique_static(const int64_t* keys, int64_t N, int64_t* uniq_out,
+                                 int32_t* inv_out, int64_t* U_out, recis_stream_t stream);
+
 /* ------------------------------------------------------------------ tracing */
 /* Kernel timing: while enabled, every kernel launch is bracketed by CUDA
  * events on its stream.  recis_profile_collect (synchronous) returns per kernel

@@ -31,7 +31,7 @@ EXPORTS = (
     "recis_backward_update", "recis_table_insert", "recis_table_size", "recis_table_export",
     "recis_table_import", "recis_table_status_sync", "recis_batch_get_unique",
     "recis_profile_enable", "recis_profile_collect", "recis_launch_count",
-    "recis_last_error_string",
+    "recis_last_error_string", "recis_unique_static",
 )
 
 
@@ -104,6 +104,7 @@ def load(path: str = LIB_PATH):
             "recis_profile_collect": [_vp, _vp, _vp, _i32],
             "recis_launch_count": [],
             "recis_last_error_string": [],
+            "recis_unique_static": [_vp, _i64, _vp, _vp, _vp, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -295,6 +296,21 @@ class Table:
         _check(load().recis_table_import(self.handle, keys.ctypes.data, emb.ctypes.data,
                                          None if st is None else st.ctypes.data, len(keys), step,
                                          _stream(stream)), "recis_table_import")
+
+
+def unique_static(keys: torch.Tensor, stream=None):
+    """recis_unique_static: allocation-free dedup (N <= 262144).
+
+    Returns (uniq int64[N] buffer, inv int32[N], U int64[1]) on the device; the
+    first U entries of uniq are the unique keys.  The output tensors are
+    allocated here by torch, not by the library."""
+    n = keys.numel()
+    uniq = torch.empty(max(n, 1), dtype=torch.int64, device=keys.device)
+    inv = torch.empty(max(n, 1), dtype=torch.int32, device=keys.device)
+    U = torch.empty(1, dtype=torch.int64, device=keys.device)
+    _check(load().recis_unique_static(_dev(keys, torch.int64), n, uniq.data_ptr(), inv.data_ptr(),
+                                      U.data_ptr(), _stream(stream)), "recis_unique_static")
+    return uniq, inv, U
 
 
 def profile_enable(on: bool = True):
