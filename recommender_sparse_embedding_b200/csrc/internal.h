@@ -36,6 +36,23 @@ struct SortCtl {
 };
 constexpr size_t kCtlZeroBytes = offsetof(SortCtl, active);
 
+// Control block of the sample-sort dedup (samplesort.cu); the first
+// kSsCtlZeroBytes bytes are cleared before every lookup.
+struct SsCtl {
+  unsigned int hist[512];             // keys per bucket
+  unsigned int ticket;
+  unsigned int tile_counter;
+  unsigned int bucket_counter;
+  unsigned int pad0;
+  unsigned long long blb[512];        // bucket look-back (heads, new keys)
+  unsigned int nsplit;                // written by the plan kernel
+  unsigned int pad1[3];
+  unsigned int base[512];             // first sorted position of each bucket
+  unsigned long long split[256];      // distinct splitters, ascending (ukey order)
+};
+constexpr size_t kSsCtlZeroBytes = offsetof(SsCtl, nsplit);
+constexpr int64_t kSampleSortMaxN = (int64_t)400 * 1024;  // larger batches use the radix sort
+
 // Per-batch device scalars.
 struct BatchDev {
   unsigned long long row_base;  // table's next_free when the lookup started
@@ -93,13 +110,20 @@ struct recis_batch {
   int64_t sort_lookback_tiles = 0;
   recis::SortCtl* ctl = nullptr;
   unsigned long long* seg_lookback = nullptr;   // [tiles], cleared per call (follows ctl)
+  recis::SsCtl* ss = nullptr;                    // sample-sort control
+  unsigned long long* ss_lookback = nullptr;     // [tiles][512], epoch-tagged
   int64_t seg_lookback_tiles = 0;
   int64_t* uniq = nullptr;
   int64_t* rows = nullptr;
   int32_t* inv = nullptr;
   int32_t* seg_of = nullptr;    // segment (unique index) of each sorted position
+  uint32_t* svals = nullptr;    // occurrence index of each sorted position
   int32_t* seg_start = nullptr; // [U+1] first sorted position of each unique
-  int32_t* occ_bag = nullptr;   // bag of each occurrence
+  int2* occ_info = nullptr;     // per occurrence: {gradient row b*F+f, bag length}
+  int32_t* chunk_bag = nullptr; // bag of each pool chunk's first occurrence
+  int64_t capChunks = 0;
+  cudaStream_t side = nullptr;  // bag preparation runs here, beside the dedup
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   int32_t* seg_counter = nullptr;  // [capN] last-arrival counters (self-resetting)
   int32_t* bag_counter = nullptr;  // [capBags]
   double* partials = nullptr;
@@ -153,7 +177,10 @@ struct LookupArgs {
 cudaError_t launch_sort(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
                         cudaStream_t s);
 cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cudaStream_t s);
+cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
+                                cudaStream_t s);
 cudaError_t launch_pool(const LookupArgs& a, int64_t chunk, cudaStream_t s);
+cudaError_t launch_bag_prep(const LookupArgs& a, int64_t chunk, cudaStream_t s);
 cudaError_t launch_rows_per_key(recis_batch* b, int64_t N, int64_t* rows_out, cudaStream_t s);
 cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pooled,
                           const float* grad_unpooled, int64_t chunk, float lr_t, float inv_sqrt_bc2,

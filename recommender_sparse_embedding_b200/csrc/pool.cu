@@ -14,6 +14,8 @@
 // Outputs: pooled rows [B][F][D] (sum, or mean = sum / length), optional
 // unpooled rows [N][D], and the bag of every occurrence for the backward.
 // Empty bags are written as zeros by a grid-stride prologue.
+#include <climits>
+
 #include "segreduce.cuh"
 
 namespace recis {
@@ -34,68 +36,82 @@ struct PoolParams {
   const float* row_data;
   float* pooled;         // [B][F][D] or null
   float* unpooled;       // [N][D] or null
-  int32_t* occ_bag;      // [N]
+  int2* occ_info;        // [N] {gradient row b*F+f, bag length} per occurrence
+  int32_t* chunk_bag;    // [nchunks] bag of each chunk's first occurrence
   double* partials;
   int32_t* counters;     // [nbags]
   DevState* st;
   HostMirror* mirror;
 };
 
-template <int G, int VPL>
-__global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolParams p) {
-  constexpr int K = VPL >= 8 ? 1 : 8 / VPL;
+// Bag preparation, one thread per bag (runs beside the dedup on a side
+// stream): checks the offsets, writes the bag of every chunk's first
+// occurrence, and zeroes the pooled output of empty bags.
+__global__ void __launch_bounds__(256) bag_prep_kernel(const __grid_constant__ PoolParams p) {
   const int64_t D = (int64_t)p.ncol * 4;
-  // prologue: zero the output of empty bags
-  if (p.pooled) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < p.nbags; j += stride) {
-      if (p.offs[j] == p.offs[j + 1]) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  if (blockIdx.x == 0 && threadIdx.x == 0 &&
+      (p.offs[0] != 0 || p.offs[p.nbags] != p.N))
+    raise_error(p.st, p.mirror, kErrBadOffsets);
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < p.nbags; j += stride) {
+    const int64_t lo = p.offs[j], hi = p.offs[j + 1];
+    if (lo < 0 || hi < lo || hi > p.N) {
+      raise_error(p.st, p.mirror, kErrBadOffsets);
+      continue;
+    }
+    if (hi == lo) {
+      if (p.pooled) {
         const int64_t f = j / p.B, b = j - f * p.B;
         float4* o = reinterpret_cast<float4*>(p.pooled + (b * p.F + f) * D);
         for (int c = 0; c < p.ncol; ++c) o[c] = f4_zero();
       }
+      continue;
     }
+    for (int64_t c = (lo + p.C - 1) / p.C; c * p.C < hi; ++c) p.chunk_bag[c] = (int32_t)j;
   }
+}
+
+template <int G, int VPL>
+__global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
+    pool_kernel(const __grid_constant__ PoolParams p) {
+  constexpr int K = VPL >= 4 ? 1 : 4 / VPL;  // rows in flight per lane
+  // all positions, bags and rows fit in 32 bits (N < 2^30, F*B < 2^31,
+  // rows < 2^31), so the walk runs on 32-bit integers
+  const int ncol = p.ncol;
+  const int D = ncol * 4;
   const GroupCtx<G> g;
   const int64_t chunk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
   if (chunk >= p.nchunks) return;
-  const int64_t p0 = chunk * p.C;
-  const int64_t p1 = p0 + p.C < p.N ? p0 + p.C : p.N;
+  const int N = (int)p.N, nbags = (int)p.nbags, C = (int)p.C, B = (int)p.B, F = p.F;
+  const int p0 = (int)chunk * C;
+  const int p1 = p0 + C < N ? p0 + C : N;
 
-  // bag containing p0: last j with offs[j] <= p0 (offs[nbags] = N > p0)
-  int64_t lo = 0, hi = p.nbags;
-  while (hi - lo > 1) {
-    const int64_t span = hi - lo;
-    const int64_t piv = lo + ((int64_t)(g.lane + 1) * span) / (G + 1);
-    const bool pr = p.offs[piv] <= p0;
-    const int cnt = __popc(g.ballot(pr));
-    const int64_t nlo = cnt > 0 ? g.bcast(piv, cnt - 1) : lo;
-    const int64_t nhi = cnt < G ? g.bcast(piv, cnt < G ? cnt : 0) : hi;
-    lo = nlo;
-    hi = nhi;
+  // bag containing p0 (precomputed), its start, and a window of G bag ends
+  int j0 = p.chunk_bag[chunk];
+  if (j0 < 0 || j0 >= nbags) {  // only with malformed offsets
+    if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
+    j0 = 0;
   }
-  const int64_t j0 = lo;
-  int64_t cur = j0;
-  int64_t cur_start = p.offs[j0];
-  // window: lane l holds the end of bag wbase + l
-  int64_t wbase = j0;
-  int64_t wend = (wbase + g.lane < p.nbags) ? p.offs[wbase + g.lane + 1] : INT64_MAX;
-  int64_t cur_end = g.bcast(wend, 0);
+  int cur = j0;
+  int cf = cur / B, cb = cur - cf * B;  // feature and sample of the current bag
+  int cur_start = (int)p.offs[j0];
+  int wbase = j0;
+  int wend = (wbase + g.lane < nbags) ? (int)p.offs[wbase + g.lane + 1] : INT_MAX;
+  int cur_end = g.bcast(wend, 0);
 
   Acc4 acc[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
   bool has = false;
 
-  auto epilogue = [&](int64_t bag, int64_t len) {
+  auto epilogue = [&]() {
     if (!p.pooled) return;
-    const int64_t f = bag / p.B, b = bag - f * p.B;
-    float4* o = reinterpret_cast<float4*>(p.pooled + (b * p.F + f) * D);
-    const double dlen = (double)len;
+    float4* o = reinterpret_cast<float4*>(p.pooled + (int64_t)(cb * F + cf) * D);
+    const double dlen = (double)(cur_end - cur_start);
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       const int col = g.lane + v * G;
-      if (col < p.ncol) {
+      if (col < ncol) {
         Acc4 r = acc[v];
         if (p.mean) {
           r.x /= dlen;
@@ -103,78 +119,81 @@ __global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolP
           r.z /= dlen;
           r.w /= dlen;
         }
-        o[col] = acc_round(r);
+        __stcs(o + col, acc_round(r));
       }
     }
   };
   auto flush = [&]() {
     if (!has) return;
-    if (!(cur_start >= 0 && cur_start < cur_end && cur_end <= p.N)) {  // malformed bag offsets
+    if (!(cur_start >= 0 && cur_start < cur_end && cur_end <= N)) {  // malformed bag offsets
       if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
-      has = false;
-      return;
-    }
-    const bool complete = cur_start >= p0 && cur_end <= p1;
-    if (complete) {
-      epilogue(cur, cur_end - cur_start);
+    } else if (cur_start >= p0 && cur_end <= p1) {
+      epilogue();
     } else if (combine_split<G, VPL>(g, acc, p.partials, p.counters, cur, chunk, cur == j0,
-                                     cur_start, cur_end, p.C, p.ncol)) {
-      epilogue(cur, cur_end - cur_start);
+                                     cur_start, cur_end, C, ncol)) {
+      epilogue();
     }
 #pragma unroll
     for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
     has = false;
   };
 
-  for (int64_t pb = p0; pb < p1; pb += K) {
-    int64_t r[K];
+  for (int sub = p0; sub < p1; sub += G) {
+    // lane-parallel: the row of position sub + lane
+    const int q = sub + g.lane;
+    int my_row = -1;
+    if (q < p1) my_row = (int)__ldg(p.rows + __ldg(p.inv + q));
+    const int m = (p1 - sub) < G ? (p1 - sub) : G;
+    for (int kb = 0; kb < m; kb += K) {
+      float4 val[K][VPL];
 #pragma unroll
-    for (int k = 0; k < K; ++k) r[k] = (pb + k < p1) ? (int64_t)p.inv[pb + k] : -1;
-#pragma unroll
-    for (int k = 0; k < K; ++k) r[k] = r[k] >= 0 ? p.rows[r[k]] : -1;
-    float4 val[K][VPL];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) {
-        const int col = g.lane + v * G;
-        val[k][v] = (r[k] >= 0 && col < p.ncol)
-                        ? __ldg(reinterpret_cast<const float4*>(p.row_data + r[k] * p.row_floats) + col)
-                        : f4_zero();
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int64_t pos = pb + k;
-      if (pos >= p1) break;
-      while (pos >= cur_end) {  // leave the current bag (and any empty ones)
-        flush();
-        if (cur + 1 >= p.nbags) {  // only reachable with malformed bag offsets
-          if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
-          cur_end = INT64_MAX;
-          break;
-        }
-        ++cur;
-        cur_start = cur_end;
-        if (cur - wbase >= G) {
-          wbase = cur;
-          wend = (wbase + g.lane < p.nbags) ? p.offs[wbase + g.lane + 1] : INT64_MAX;
-        }
-        cur_end = g.bcast(wend, (int)(cur - wbase));
-      }
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) acc_add(acc[v], val[k][v]);
-      has = true;
-      if (p.unpooled) {
+      for (int k = 0; k < K; ++k) {
+        const int r = g.bcast(my_row, kb + k < m ? kb + k : 0);
+        const bool valid = kb + k < m && r >= 0;
+        const float4* src = reinterpret_cast<const float4*>(p.row_data + (int64_t)r * p.row_floats);
 #pragma unroll
         for (int v = 0; v < VPL; ++v) {
           const int col = g.lane + v * G;
-          if (col < p.ncol) __stcs(reinterpret_cast<float4*>(p.unpooled + pos * D) + col, val[k][v]);
+          val[k][v] = (valid && col < ncol) ? __ldg(src + col) : f4_zero();
         }
       }
-      if (g.lane == 0) p.occ_bag[pos] = (int32_t)cur;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        if (kb + k >= m) break;
+        const int pos = sub + kb + k;
+        while (pos >= cur_end) {  // leave the current bag (and any empty ones)
+          flush();
+          if (cur + 1 >= nbags) {  // only reachable with malformed bag offsets
+            if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
+            cur_end = INT_MAX;
+            break;
+          }
+          ++cur;
+          if (++cb == B) {
+            cb = 0;
+            ++cf;
+          }
+          cur_start = cur_end;
+          if (cur - wbase >= G) {
+            wbase = cur;
+            wend = (wbase + g.lane < nbags) ? (int)p.offs[wbase + g.lane + 1] : INT_MAX;
+          }
+          cur_end = g.bcast(wend, cur - wbase);
+        }
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) acc_add(acc[v], val[k][v]);
+        has = true;
+        if (p.unpooled) {
+          float4* dst = reinterpret_cast<float4*>(p.unpooled + (int64_t)pos * D);
+#pragma unroll
+          for (int v = 0; v < VPL; ++v) {
+            const int col = g.lane + v * G;
+            if (col < ncol) __stcs(dst + col, val[k][v]);
+          }
+        }
+        // for the backward: this occurrence's gradient row and bag length
+        if (g.lane == 0) p.occ_info[pos] = make_int2(cb * F + cf, cur_end - cur_start);
+      }
     }
   }
   flush();
@@ -205,7 +224,7 @@ int64_t pool_chunk_for(int64_t N, int D) {
   return C;
 }
 
-cudaError_t launch_pool(const LookupArgs& a, int64_t chunk, cudaStream_t s) {
+static PoolParams pool_params(const LookupArgs& a, int64_t chunk) {
   recis_table* t = a.t;
   recis_batch* b = a.b;
   PoolParams p;
@@ -224,12 +243,28 @@ cudaError_t launch_pool(const LookupArgs& a, int64_t chunk, cudaStream_t s) {
   p.row_data = reinterpret_cast<const float*>(t->rows.va);
   p.pooled = a.pooled_out;
   p.unpooled = a.unpooled_out;
-  p.occ_bag = b->occ_bag;
+  p.occ_info = b->occ_info;
+  p.chunk_bag = b->chunk_bag;
   p.partials = b->partials;
   p.counters = b->bag_counter;
   p.st = t->dstate;
   p.mirror = t->mirror_dev;
-  if (p.nchunks == 0 && !(p.pooled && p.nbags > 0)) return cudaSuccess;
+  return p;
+}
+
+cudaError_t launch_bag_prep(const LookupArgs& a, int64_t chunk, cudaStream_t s) {
+  const PoolParams p = pool_params(a, chunk);
+  if (p.nbags == 0) return cudaSuccess;
+  int64_t blocks = (p.nbags + 255) / 256;
+  if (blocks > 16 * kSMs) blocks = 16 * kSMs;
+  LaunchScope ls("bag_prep", s);
+  bag_prep_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool(const LookupArgs& a, int64_t chunk, cudaStream_t s) {
+  const PoolParams p = pool_params(a, chunk);
+  if (p.nchunks == 0) return cudaSuccess;
   const int ncol = p.ncol;
   if (ncol <= 1) return launch_pool_t<1, 1>(p, s);
   if (ncol <= 2) return launch_pool_t<2, 1>(p, s);

@@ -36,27 +36,35 @@ __device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long 
 __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restrict__ keys,
                                                         int64_t N, SortCtl* ctl, DevState* st,
                                                         HostMirror* mirror, BatchDev* bdev) {
+  constexpr int kPer = 4;  // keys per thread per round, loaded before they are counted
   __shared__ unsigned int sh[kSortPasses][256];
   __shared__ bool s_last;
   for (int i = threadIdx.x; i < kSortPasses * 256; i += blockDim.x) (&sh[0][0])[i] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   bool reserved = false;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x * kPer;
   // warp-uniform trip count so that match/ballot see the whole warp
-  const int64_t base0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  const int64_t base0 = ((int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31)) * kPer;
   for (int64_t wb = base0; wb < N; wb += stride) {
-    const int64_t i = wb + lane;
-    const bool valid = i < N;
-    const int64_t k = valid ? keys[i] : 0;
-    reserved |= valid && (k == kEmptyKey);
-    const uint64_t u = to_ukey(k);
-    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    int64_t k[kPer];
 #pragma unroll
-    for (int p = 0; p < kSortPasses; ++p) {
-      const unsigned d = (unsigned)(u >> (p * kSortBits)) & 255u;
-      const unsigned peers = __match_any_sync(0xffffffffu, valid ? d : 256u) & vmask;
-      if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh[p][d], (unsigned)__popc(peers));
+    for (int j = 0; j < kPer; ++j) {
+      const int64_t i = wb + j * 32 + lane;
+      k[j] = i < N ? keys[i] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const bool valid = wb + j * 32 + lane < N;
+      reserved |= valid && (k[j] == kEmptyKey);
+      const uint64_t u = to_ukey(k[j]);
+      const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+      for (int p = 0; p < kSortPasses; ++p) {
+        const unsigned d = (unsigned)(u >> (p * kSortBits)) & 255u;
+        const unsigned peers = __match_any_sync(0xffffffffu, valid ? d : 256u) & vmask;
+        if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh[p][d], (unsigned)__popc(peers));
+      }
     }
   }
   if (__any_sync(0xffffffffu, reserved) && lane == 0) raise_error(st, mirror, kErrReservedKey);
@@ -71,27 +79,34 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restric
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // last CTA: plan the passes
+  // last CTA plans the passes: warp p scans the 256 digit counts of pass p
   __shared__ unsigned int s_active[kSortPasses];
-  const int d = threadIdx.x;  // blockDim == 256
-  for (int p = 0; p < kSortPasses; ++p) {
-    const unsigned c = __ldcg(&ctl->hist[p][d]);
-    const int all_one_bucket = __syncthreads_or(c == (unsigned)N);
-    if (d == 0) s_active[p] = all_one_bucket ? 0u : 1u;
-    // exclusive scan of the 256 counts
-    __shared__ unsigned int s_scan[256];
-    s_scan[d] = c;
-    __syncthreads();
-    for (int off = 1; off < 256; off <<= 1) {
-      const unsigned v = d >= off ? s_scan[d - off] : 0u;
-      __syncthreads();
-      s_scan[d] += v;
-      __syncthreads();
-    }
-    ctl->base[p][d] = s_scan[d] - c;
-    __syncthreads();
+  const int wp = threadIdx.x >> 5;  // blockDim == 256: one warp per pass
+  unsigned c[8];
+  unsigned run = 0;
+  bool one_bucket = false;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    c[q] = __ldcg(&ctl->hist[wp][lane * 8 + q]);
+    one_bucket |= c[q] == (unsigned)N;
+    run += c[q];
   }
-  if (d == 0) {
+  unsigned x = run;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  unsigned base = x - run;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    ctl->base[wp][lane * 8 + q] = base;
+    base += c[q];
+  }
+  one_bucket = __any_sync(0xffffffffu, one_bucket);
+  if (lane == 0) s_active[wp] = one_bucket ? 0u : 1u;
+  __syncthreads();
+  if (threadIdx.x == 0) {
     bdev->row_base = *(volatile unsigned long long*)&st->next_free;
     unsigned n = 0;
     for (int p = 0; p < kSortPasses; ++p) {
@@ -198,24 +213,41 @@ __global__ void __launch_bounds__(kSortBlock) sort_pass_kernel(
       if (ww < w) pre += s_wsum[ww];
     s_doff[d] = pre + x - total;
   }
-  // decoupled look-back for digit d
+  // decoupled look-back for digit d: kWin predecessor entries are loaded at
+  // once, then consumed nearest first until an inclusive one is met
   unsigned excl = 0;
   if (tile > 0) {
+    constexpr int kWin = 16;
     int64_t t = (int64_t)tile - 1;
     int spins = 0;
-    while (t >= 0) {
-      const unsigned long long e = ld_relaxed(lookback + (size_t)t * 256 + d);
-      if ((uint32_t)(e >> 32) != epoch || ((e >> 30) & 3u) == 0) {
-        if (++spins > kSpinLimit) {
-          raise_error(st, mirror, kErrTimeout);
+    bool done = false;
+    while (!done) {
+      unsigned long long e[kWin];
+#pragma unroll
+      for (int w = 0; w < kWin; ++w)
+        e[w] = (t - w >= 0) ? ld_relaxed(lookback + (size_t)(t - w) * 256 + d) : 0ULL;
+#pragma unroll
+      for (int w = 0; w < kWin; ++w) {
+        if (done) break;
+        if (t - w < 0) {  // unreachable: tile 0 publishes an inclusive count
+          done = true;
           break;
         }
-        __nanosleep(32);
-        continue;
+        unsigned long long v = e[w];
+        while ((uint32_t)(v >> 32) != epoch || ((v >> 30) & 3u) == 0) {
+          if (++spins > kSpinLimit) {
+            raise_error(st, mirror, kErrTimeout);
+            done = true;
+            break;
+          }
+          __nanosleep(32);
+          v = ld_relaxed(lookback + (size_t)(t - w) * 256 + d);
+        }
+        if (done) break;
+        excl += (unsigned)(v & 0x3fffffffu);
+        if (((v >> 30) & 3u) == kFlagIncl) done = true;
       }
-      excl += (unsigned)(e & 0x3fffffffu);
-      if (((e >> 30) & 3u) == kFlagIncl) break;
-      --t;
+      t -= kWin;
     }
     st_relaxed(my, tag | ((unsigned long long)kFlagIncl << 30) | (excl + total));
   }
@@ -253,8 +285,8 @@ cudaError_t launch_sort(recis_batch* b, recis_table* t, const int64_t* keys, int
     if (e != cudaSuccess) return e;
   }
   {
-    int64_t blocks = (N + 4095) / 4096;
-    if (blocks > 2 * kSMs) blocks = 2 * kSMs;
+    int64_t blocks = (N + 1023) / 1024;  // 4 keys per thread
+    if (blocks > 8 * kSMs) blocks = 8 * kSMs;
     if (blocks < 1) blocks = 1;
     LaunchScope ls("sort_hist", s);
     sort_hist_kernel<<<(unsigned)blocks, 256, 0, s>>>(keys, N, b->ctl, t->dstate, t->mirror_dev,

@@ -353,6 +353,7 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
   if (!b->ctl) {
     if ((e = realloc_dev(b->ctl, 1, true)) != cudaSuccess) return cuda_fail(e, "batch alloc");
     if ((e = realloc_dev(b->bdev, 1, true)) != cudaSuccess) return cuda_fail(e, "batch alloc");
+    if ((e = realloc_dev(b->ss, 1, true)) != cudaSuccess) return cuda_fail(e, "batch alloc");
   }
   if (N > b->capN) {
     const int64_t cap = std::max<int64_t>(N + N / 4, 1 << 12);
@@ -366,14 +367,17 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
         (e = realloc_dev(b->rows, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->inv, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_of, cap, true)) != cudaSuccess ||
+        (e = realloc_dev(b->svals, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_start, cap + 1, true)) != cudaSuccess ||
-        (e = realloc_dev(b->occ_bag, cap, true)) != cudaSuccess ||
+        (e = realloc_dev(b->occ_info, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_counter, cap, true)) != cudaSuccess)
       return cuda_fail(e, "batch alloc");
     const int64_t st = (cap + kSortTile - 1) / kSortTile;
     if ((e = realloc_dev(b->sort_lookback, (size_t)st * 256, true)) != cudaSuccess)
       return cuda_fail(e, "batch alloc");
     b->sort_lookback_tiles = st;
+    if ((e = realloc_dev(b->ss_lookback, (size_t)st * 512, true)) != cudaSuccess)
+      return cuda_fail(e, "batch alloc");
     const int64_t ut = unique_tiles_for(cap);
     if ((e = realloc_dev(b->seg_lookback, (size_t)ut, true)) != cudaSuccess)
       return cuda_fail(e, "batch alloc");
@@ -385,7 +389,18 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
     if ((e = realloc_dev(b->bag_counter, cap, true)) != cudaSuccess) return cuda_fail(e, "batch alloc");
     b->capBags = cap;
   }
+  if (!b->side) {
+    if ((e = cudaStreamCreateWithFlags(&b->side, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&b->ev_fork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&b->ev_join, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail(e, "batch stream");
+  }
   const int64_t cf = pool_chunk_for(N, D), cu = update_chunk_for(N, D);
+  if ((N + cf - 1) / cf + 1 > b->capChunks) {
+    const int64_t cap = (N + cf - 1) / cf + 1 + 1024;
+    if ((e = realloc_dev(b->chunk_bag, cap, true)) != cudaSuccess) return cuda_fail(e, "batch alloc");
+    b->capChunks = cap;
+  }
   const int64_t nch = std::max((N + cf - 1) / cf, (N + cu - 1) / cu);
   const int64_t need = nch * 2 * D;
   if (need > b->capPartials) {
@@ -403,17 +418,24 @@ static void batch_free(recis_batch* b) {
   }
   cudaFree(b->sort_lookback);
   cudaFree(b->ctl);
+  cudaFree(b->ss);
+  cudaFree(b->ss_lookback);
   cudaFree(b->seg_lookback);
   cudaFree(b->uniq);
   cudaFree(b->rows);
   cudaFree(b->inv);
   cudaFree(b->seg_of);
+  cudaFree(b->svals);
   cudaFree(b->seg_start);
-  cudaFree(b->occ_bag);
+  cudaFree(b->occ_info);
   cudaFree(b->seg_counter);
   cudaFree(b->bag_counter);
   cudaFree(b->partials);
   cudaFree(b->bdev);
+  cudaFree(b->chunk_bag);
+  if (b->side) cudaStreamDestroy(b->side);
+  if (b->ev_fork) cudaEventDestroy(b->ev_fork);
+  if (b->ev_join) cudaEventDestroy(b->ev_join);
 }
 
 static recis_status check_device() {
@@ -449,18 +471,34 @@ static recis_status lookup_impl(const LookupArgs& a, cudaStream_t s) {
   b->bag_offsets = a.bag_offsets;
   b->have_lookup = true;
   cudaError_t e;
+  const bool pool = a.pooled_out || a.unpooled_out;
+  const int64_t cf = pool_chunk_for(a.N, t->D);
+  if (pool) {
+    // bag preparation on the side stream, overlapping the dedup
+    if ((e = cudaEventRecord(b->ev_fork, s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(b->side, b->ev_fork, 0)) != cudaSuccess ||
+        (e = launch_bag_prep(a, cf, b->side)) != cudaSuccess ||
+        (e = cudaEventRecord(b->ev_join, b->side)) != cudaSuccess)
+      return cuda_fail(e, "bag preparation");
+  }
   if (a.N > 0) {
-    if ((e = launch_sort(b, t, a.keys, a.N, s)) != cudaSuccess) return cuda_fail(e, "sort launch");
-    if ((e = launch_unique_insert(b, t, a.N, s)) != cudaSuccess) return cuda_fail(e, "unique launch");
+    if (a.N <= kSampleSortMaxN) {
+      if ((e = launch_sample_dedup(b, t, a.keys, a.N, s)) != cudaSuccess)
+        return cuda_fail(e, "dedup launch");
+    } else {
+      if ((e = launch_sort(b, t, a.keys, a.N, s)) != cudaSuccess) return cuda_fail(e, "sort launch");
+      if ((e = launch_unique_insert(b, t, a.N, s)) != cudaSuccess)
+        return cuda_fail(e, "unique launch");
+    }
     if (a.rows_out && (e = launch_rows_per_key(b, a.N, a.rows_out, s)) != cudaSuccess)
       return cuda_fail(e, "rows launch");
   } else {
     if ((e = cudaMemsetAsync(b->bdev, 0, sizeof(BatchDev), s)) != cudaSuccess)
       return cuda_fail(e, "memset");
   }
-  if (a.pooled_out || a.unpooled_out) {
-    if ((e = launch_pool(a, pool_chunk_for(a.N, t->D), s)) != cudaSuccess)
-      return cuda_fail(e, "pool launch");
+  if (pool) {
+    if ((e = cudaStreamWaitEvent(s, b->ev_join, 0)) != cudaSuccess) return cuda_fail(e, "join");
+    if ((e = launch_pool(a, cf, s)) != cudaSuccess) return cuda_fail(e, "pool launch");
   }
   after_call(t, a.N, s);
   return RECIS_OK;
@@ -611,6 +649,7 @@ recis_status recis_table_create(const recis_table_config* cfg, recis_stream_t st
   t->init_two_s = 2.0f * (float)scale;
   t->block_rows = cfg->block_rows > 0 ? cfg->block_rows : 65536;
   t->max_rows = cfg->max_rows > 0 ? cfg->max_rows : (int64_t)1 << 28;
+  if (t->max_rows > INT32_MAX) t->max_rows = INT32_MAX;  // row offsets are 31-bit in the kernels
 
   CUmemAllocationProp prop = {};
   prop.type = CU_MEM_ALLOCATION_TYPE_PINNED;

@@ -97,6 +97,7 @@ struct UniqueParams {
   int64_t* rows;
   int32_t* inv;
   int32_t* seg_of;
+  uint32_t* svals;
   int32_t* seg_start;
   BatchDev* bdev;
   DevState* st;
@@ -194,34 +195,46 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
   const unsigned excl_thread = wpre + x - mine;
   const unsigned long long tH = tot & 0xffffu, tN = tot >> 16;
 
-  if (tid == 0) {
+  if (w == 0) {
+    // decoupled look-back by warp 0: 32 predecessor tiles per step
     unsigned long long* my = p.lookback + tile;
     unsigned long long hx = 0, nx = 0;
     if (tile == 0) {
-      st_relaxed(my, kUqIncl | (tH << 31) | tN);
+      if (lane == 0) st_relaxed(my, kUqIncl | (tH << 31) | tN);
     } else {
-      st_relaxed(my, kUqAgg | (tH << 31) | tN);
+      if (lane == 0) st_relaxed(my, kUqAgg | (tH << 31) | tN);
       int64_t t = (int64_t)tile - 1;
       int spins = 0;
-      while (t >= 0) {
-        const unsigned long long e = ld_relaxed(p.lookback + t);
-        const unsigned long long flag = e >> 62;
-        if (flag == 0) {
-          if (++spins > kSpinLimit) {
-            raise_error(p.st, p.mirror, kErrTimeout);
-            break;
-          }
+      bool done = false;
+      while (!done) {
+        const int64_t idx = t - lane;
+        unsigned long long e = idx >= 0 ? ld_relaxed(p.lookback + idx) : kUqIncl;
+        while (!__all_sync(0xffffffffu, (e >> 62) != 0)) {
+          if (++spins > kSpinLimit) break;
           __nanosleep(32);
-          continue;
+          if ((e >> 62) == 0) e = ld_relaxed(p.lookback + idx);
         }
-        hx += (e >> 31) & 0x7fffffffULL;
-        nx += e & 0x7fffffffULL;
-        if (flag == 2) break;
-        --t;
+        if (spins > kSpinLimit) {
+          if (lane == 0) raise_error(p.st, p.mirror, kErrTimeout);
+          break;
+        }
+        const unsigned incl = __ballot_sync(0xffffffffu, (e >> 62) == 2);
+        const int stop = incl ? __ffs(incl) - 1 : 31;  // nearest inclusive entry
+        unsigned long long h = lane <= stop ? (e >> 31) & 0x7fffffffULL : 0;
+        unsigned long long n = lane <= stop ? e & 0x7fffffffULL : 0;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          h += __shfl_xor_sync(0xffffffffu, h, off);
+          n += __shfl_xor_sync(0xffffffffu, n, off);
+        }
+        hx += h;
+        nx += n;
+        done = incl != 0;
+        t -= 32;
       }
-      st_relaxed(my, kUqIncl | ((hx + tH) << 31) | (nx + tN));
+      if (lane == 0) st_relaxed(my, kUqIncl | ((hx + tH) << 31) | (nx + tN));
     }
-    s_prefix = (hx << 32) | nx;
+    if (lane == 0) s_prefix = (hx << 32) | nx;
   }
   __syncthreads();
   const unsigned long long Hx = s_prefix >> 32, Nx = s_prefix & 0xffffffffULL;
@@ -257,6 +270,7 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
     }
     const int32_t seg = (int32_t)(hrun - 1);
     p.seg_of[pos] = seg;
+    p.svals[pos] = v[j];
     if (v[j] < (uint64_t)N) p.inv[v[j]] = seg;
   }
   if (tile == gridDim.x - 1 && tid == 0) {
@@ -273,22 +287,26 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
     p.seg_start[U] = (int32_t)N;
   }
   __syncthreads();
-  // initialise this tile's new rows, 16 bytes per thread per step
+  // initialise this tile's new rows: one warp per row, 16 bytes per lane per
+  // step; the key's base hash is formed once per row
   const int nf4 = p.row_floats >> 2;
-  const int total = s_ninit * nf4;
-  for (int idx = tid; idx < total; idx += kUqBlock) {
-    const int r = idx / nf4;
-    const int c = (idx - r * nf4) * 4;
-    const int64_t key = s_init_key[r];
-    const uint64_t base = mix64((uint64_t)key ^ p.init_seed);
-    float o[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int col = c + e;
-      o[e] = col < p.D ? init_value(base, col, p.two_s) : (p.adagrad ? p.acc0 : 0.0f);
+  const int ncol = p.D >> 2;
+  const float sv = p.adagrad ? p.acc0 : 0.0f;
+  for (int r = w; r < s_ninit; r += kUqBlock / 32) {
+    const uint64_t base = mix64((uint64_t)s_init_key[r] ^ p.init_seed);
+    float4* dst = reinterpret_cast<float4*>(p.row_data + s_init_row[r] * (int64_t)p.row_floats);
+    for (int c = lane; c < nf4; c += 32) {
+      float4 o;
+      if (c < ncol) {
+        o.x = init_value(base, 4 * c + 0, p.two_s);
+        o.y = init_value(base, 4 * c + 1, p.two_s);
+        o.z = init_value(base, 4 * c + 2, p.two_s);
+        o.w = init_value(base, 4 * c + 3, p.two_s);
+      } else {
+        o = make_float4(sv, sv, sv, sv);
+      }
+      dst[c] = o;
     }
-    float4* dst = reinterpret_cast<float4*>(p.row_data + s_init_row[r] * (int64_t)p.row_floats + c);
-    *dst = make_float4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -324,6 +342,7 @@ cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cuda
   p.rows = b->rows;
   p.inv = b->inv;
   p.seg_of = b->seg_of;
+  p.svals = b->svals;
   p.seg_start = b->seg_start;
   p.bdev = b->bdev;
   p.st = t->dstate;

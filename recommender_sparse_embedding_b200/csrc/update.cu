@@ -6,7 +6,7 @@
 //
 // The sorted positions of the dedup are already grouped by unique key, so the
 // backward is a segmented reduction over sorted order (segreduce.cuh).  For
-// sorted position q (occurrence i = vals[q], bag = occ_bag[i]) the term is
+// sorted position q (occurrence i = vals[q], its bag from the forward) the term is
 //   grad_pooled[b][f] * (1 or 1/length) + grad_unpooled[i];
 // a group sums the terms of each unique key in its chunk in position order and
 // then applies Adagrad or Adam to that key's row [emb | state] in place.  Keys
@@ -29,7 +29,7 @@ struct UpdateParams {
   const uint32_t* vals;     // sorted occurrence indices
   const int32_t* seg_of;    // [N] sorted position -> unique index
   const int32_t* seg_start; // [U+1]
-  const int32_t* occ_bag;   // [N]
+  const int2* occ_info;     // [N] {gradient row, bag length}
   const int64_t* offs;      // bag offsets
   const int64_t* rows;      // [U]
   const float* gp;          // grad_pooled [B][F][D] or null
@@ -37,9 +37,6 @@ struct UpdateParams {
   float* row_data;
   double* partials;
   int32_t* counters;        // [U]
-  const SortCtl* ctl;
-  const uint32_t* vb0;
-  const uint32_t* vb1;
   // optimiser
   float lr;        // Adagrad: lr; Adam: lr / (1 - beta1^t)
   float eps;
@@ -48,9 +45,33 @@ struct UpdateParams {
   float sqrt_bc2;  // Adam: sqrt(1 - beta2^t)
 };
 
+// Row data of one unique key: emb and the optimiser state, VPL 16-byte
+// columns per lane.
+template <int VPL, bool ADAM>
+struct RowRegs {
+  float4 w[VPL], s1[VPL], s2[ADAM ? VPL : 1];
+};
+
+template <int G, int VPL, bool ADAM>
+__device__ __forceinline__ void load_row(const GroupCtx<G>& g, const UpdateParams& p, int64_t row,
+                                         RowRegs<VPL, ADAM>& r) {
+  const int D = p.ncol * 4;
+  const float* base = p.row_data + (row < 0 ? 0 : row) * (int64_t)p.row_floats;
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const int col = g.lane + v * G;
+    if (row >= 0 && col < p.ncol) {
+      r.w[v] = __ldcg(reinterpret_cast<const float4*>(base) + col);
+      r.s1[v] = __ldcg(reinterpret_cast<const float4*>(base + D) + col);
+      if (ADAM) r.s2[v] = __ldcg(reinterpret_cast<const float4*>(base + 2 * D) + col);
+    }
+  }
+}
+
 template <int G, int VPL, bool ADAM>
 __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateParams& p,
-                                             int64_t row, const Acc4 (&grad)[VPL]) {
+                                             int64_t row, const RowRegs<VPL, ADAM>& r,
+                                             const Acc4 (&grad)[VPL]) {
   if (row < 0) return;
   float* base = p.row_data + row * p.row_floats;
   const int D = p.ncol * 4;
@@ -58,12 +79,9 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
   for (int v = 0; v < VPL; ++v) {
     const int col = g.lane + v * G;
     if (col >= p.ncol) continue;
-    float4* wp = reinterpret_cast<float4*>(base) + col;
-    float4* s1p = reinterpret_cast<float4*>(base + D) + col;
-    float4 w = *wp, s1 = *s1p;
     const float gg[4] = {(float)grad[v].x, (float)grad[v].y, (float)grad[v].z, (float)grad[v].w};
-    float ww[4] = {w.x, w.y, w.z, w.w};
-    float a1[4] = {s1.x, s1.y, s1.z, s1.w};
+    float ww[4] = {r.w[v].x, r.w[v].y, r.w[v].z, r.w[v].w};
+    float a1[4] = {r.s1[v].x, r.s1[v].y, r.s1[v].z, r.s1[v].w};
     if (!ADAM) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -72,9 +90,7 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
         a1[e] = acc;
       }
     } else {
-      float4* s2p = reinterpret_cast<float4*>(base + 2 * D) + col;
-      const float4 s2 = *s2p;
-      float a2[4] = {s2.x, s2.y, s2.z, s2.w};
+      float a2[4] = {r.s2[v].x, r.s2[v].y, r.s2[v].z, r.s2[v].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float m = p.beta1 * a1[e] + p.omb1 * gg[e];
@@ -83,99 +99,127 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
         a1[e] = m;
         a2[e] = vv;
       }
-      *s2p = make_float4(a2[0], a2[1], a2[2], a2[3]);
+      __stcg(reinterpret_cast<float4*>(base + 2 * D) + col, make_float4(a2[0], a2[1], a2[2], a2[3]));
     }
-    *s1p = make_float4(a1[0], a1[1], a1[2], a1[3]);
-    *wp = make_float4(ww[0], ww[1], ww[2], ww[3]);
+    __stcg(reinterpret_cast<float4*>(base + D) + col, make_float4(a1[0], a1[1], a1[2], a1[3]));
+    __stcg(reinterpret_cast<float4*>(base) + col, make_float4(ww[0], ww[1], ww[2], ww[3]));
   }
 }
 
+// One group per chunk of C sorted positions.  Index work is lane-parallel:
+// for G positions at a time each lane resolves one position (sorted position
+// -> occurrence -> bag -> gradient row), then the group streams the gradient
+// rows RB at a time, every lane loading its 16-byte column of each.  The
+// chunk's unique keys are consecutive segment ids s0..s_last; their row
+// offsets are fetched one per lane, and the row of the next key is loaded
+// while the current key's terms are summed, so the epilogue rarely waits.
 template <int G, int VPL, bool ADAM>
-__global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ UpdateParams p) {
-  constexpr int K = VPL >= 4 ? 1 : 4 / VPL;
+__global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
+    update_kernel(const __grid_constant__ UpdateParams p) {
+  constexpr int RB = VPL >= 2 ? 1 : 2;  // gradient rows in flight per lane
   const GroupCtx<G> g;
   const int64_t chunk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
   if (chunk >= p.nchunks) return;
   const int64_t D = (int64_t)p.ncol * 4;
-  const unsigned na = p.ctl->n_active;
-  const uint32_t* vals = na == 0 ? nullptr : (((na - 1) & 1) ? p.vb1 : p.vb0);
+  const uint32_t* vals = p.vals;
   const int64_t p0 = chunk * p.C;
   const int64_t p1 = p0 + p.C < p.N ? p0 + p.C : p.N;
-  const int32_t s0 = p.seg_of[p0];
-  const bool s0_starts_here = p.seg_start[s0] == p0;
-  const int32_t after = p1 < p.N ? p.seg_of[p1] : -1;
+  const int32_t s0 = __ldg(p.seg_of + p0);
+  const int32_t s_last = __ldg(p.seg_of + p1 - 1);
+  const bool s0_starts_here = __ldg(p.seg_start + s0) == p0;
+  const int32_t after = p1 < p.N ? __ldg(p.seg_of + p1) : -1;
+  int32_t wbase = s0;
+  int64_t wrow = (s0 + g.lane <= s_last) ? __ldg(p.rows + s0 + g.lane) : -1;
 
   int32_t cur = s0;
   bool cur_starts_here = s0_starts_here;
+  int64_t cur_row = g.bcast(wrow, 0);
+  RowRegs<VPL, ADAM> rcur, rnext;
+  load_row<G, VPL, ADAM>(g, p, cur_row, rcur);
+  int64_t next_row = -1;
+  auto fetch_next = [&]() {  // row of cur + 1, if it belongs to this chunk
+    next_row = -1;
+    if (cur + 1 <= s_last) {
+      if (cur + 1 - wbase >= G) {
+        wbase = cur + 1;
+        wrow = (wbase + g.lane <= s_last) ? __ldg(p.rows + wbase + g.lane) : -1;
+      }
+      next_row = g.bcast(wrow, cur + 1 - wbase);
+      load_row<G, VPL, ADAM>(g, p, next_row, rnext);
+    }
+  };
+  fetch_next();
+
   Acc4 acc[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
 
   auto finish = [&](bool ends_here) {
-    const int64_t row = p.rows[cur];
     if (cur_starts_here && ends_here) {
-      apply_update<G, VPL, ADAM>(g, p, row, acc);
+      apply_update<G, VPL, ADAM>(g, p, cur_row, rcur, acc);
     } else {
       const int64_t st = p.seg_start[cur], en = p.seg_start[cur + 1];
       if (combine_split<G, VPL>(g, acc, p.partials, p.counters, cur, chunk, cur == s0, st, en,
                                 p.C, p.ncol))
-        apply_update<G, VPL, ADAM>(g, p, row, acc);
+        apply_update<G, VPL, ADAM>(g, p, cur_row, rcur, acc);
     }
 #pragma unroll
     for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
   };
 
-  for (int64_t pb = p0; pb < p1; pb += K) {
-    int32_t sg[K];
-    int64_t occ[K];
-    double scale[K];
-    int64_t gprow[K];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int64_t q = pb + k;
-      const bool ok = q < p1;
-      sg[k] = ok ? p.seg_of[q] : -1;
-      occ[k] = ok ? (vals ? (int64_t)vals[q] : q) : -1;
+  for (int64_t sub = p0; sub < p1; sub += G) {
+    // lane-parallel resolution of positions sub .. sub+G-1
+    const int64_t q = sub + g.lane;
+    const bool ok = q < p1;
+    const int32_t my_seg = ok ? __ldg(p.seg_of + q) : -1;
+    const int32_t my_occ = ok ? (int32_t)__ldg(vals + q) : -1;
+    int32_t my_gprow = -1;
+    double my_scale = 1.0;
+    if (ok && p.gp) {
+      const int2 oi = __ldg(p.occ_info + my_occ);
+      my_gprow = oi.x;
+      if (p.mean) my_scale = 1.0 / (double)oi.y;
     }
+    const int m = (int)((p1 - sub) < G ? (p1 - sub) : G);
+    for (int kb = 0; kb < m; kb += RB) {
+      float4 tp[RB][VPL], tu[RB][VPL];
+      int32_t sg[RB];
+      double sc[RB];
 #pragma unroll
-    for (int k = 0; k < K; ++k) {
-      scale[k] = 1.0;
-      gprow[k] = -1;
-      if (occ[k] >= 0 && p.gp) {
-        const int64_t bag = p.occ_bag[occ[k]];
-        const int64_t f = bag / p.B, b = bag - f * p.B;
-        gprow[k] = b * p.F + f;
-        if (p.mean) scale[k] = 1.0 / (double)(p.offs[bag + 1] - p.offs[bag]);
-      }
-    }
-    float4 tp[K][VPL], tu[K][VPL];
+      for (int k = 0; k < RB; ++k) {
+        const int src = kb + k < m ? kb + k : 0;
+        const int32_t gr = g.bcast(my_gprow, src);
+        const int32_t oc = g.bcast(my_occ, src);
+        sg[k] = g.bcast(my_seg, src);
+        sc[k] = p.mean ? g.bcast(my_scale, src) : 1.0;
+        const bool valid = kb + k < m;
+        const float4* gps = reinterpret_cast<const float4*>(p.gp + (int64_t)gr * D);
+        const float4* gus = reinterpret_cast<const float4*>(p.gu + (int64_t)oc * D);
 #pragma unroll
-    for (int k = 0; k < K; ++k) {
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) {
-        const int col = g.lane + v * G;
-        tp[k][v] = (col < p.ncol && gprow[k] >= 0)
-                       ? __ldg(reinterpret_cast<const float4*>(p.gp + gprow[k] * D) + col)
-                       : f4_zero();
-        tu[k][v] = (col < p.ncol && p.gu && occ[k] >= 0)
-                       ? __ldg(reinterpret_cast<const float4*>(p.gu + occ[k] * D) + col)
-                       : f4_zero();
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      if (pb + k >= p1) break;
-      if (sg[k] != cur) {
-        finish(true);
-        cur = sg[k];
-        cur_starts_here = true;
+        for (int v = 0; v < VPL; ++v) {
+          const int col = g.lane + v * G;
+          tp[k][v] = (valid && col < p.ncol && gr >= 0) ? __ldcs(gps + col) : f4_zero();
+          tu[k][v] = (valid && col < p.ncol && p.gu) ? __ldcs(gus + col) : f4_zero();
+        }
       }
 #pragma unroll
-      for (int v = 0; v < VPL; ++v) {
-        acc[v].x += (double)tp[k][v].x * scale[k] + (double)tu[k][v].x;
-        acc[v].y += (double)tp[k][v].y * scale[k] + (double)tu[k][v].y;
-        acc[v].z += (double)tp[k][v].z * scale[k] + (double)tu[k][v].z;
-        acc[v].w += (double)tp[k][v].w * scale[k] + (double)tu[k][v].w;
+      for (int k = 0; k < RB; ++k) {
+        if (kb + k >= m) break;
+        if (sg[k] != cur) {
+          finish(true);
+          cur = sg[k];
+          cur_starts_here = true;
+          cur_row = next_row;
+          rcur = rnext;
+          fetch_next();
+        }
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+          acc[v].x += (double)tp[k][v].x * sc[k] + (double)tu[k][v].x;
+          acc[v].y += (double)tp[k][v].y * sc[k] + (double)tu[k][v].y;
+          acc[v].z += (double)tp[k][v].z * sc[k] + (double)tu[k][v].z;
+          acc[v].w += (double)tp[k][v].w * sc[k] + (double)tu[k][v].w;
+        }
       }
     }
   }
@@ -216,10 +260,10 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.nchunks = (b->N + chunk - 1) / chunk;
   p.mean = b->combiner == RECIS_MEAN;
   p.row_floats = t->row_floats;
-  p.vals = nullptr;
+  p.vals = b->svals;
   p.seg_of = b->seg_of;
   p.seg_start = b->seg_start;
-  p.occ_bag = b->occ_bag;
+  p.occ_info = b->occ_info;
   p.offs = b->bag_offsets;
   p.rows = b->rows;
   p.gp = grad_pooled;
@@ -227,9 +271,6 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.row_data = reinterpret_cast<float*>(t->rows.va);
   p.partials = b->partials;
   p.counters = b->seg_counter;
-  p.ctl = b->ctl;
-  p.vb0 = b->vbuf[0];
-  p.vb1 = b->vbuf[1];
   p.lr = lr_t;
   p.eps = (float)t->cfg.eps;
   p.beta1 = (float)t->cfg.beta1;

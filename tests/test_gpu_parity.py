@@ -173,6 +173,27 @@ def test_all_occurrences_one_key(R):
     _single(R, np.full(70_000, 123456789), np.ones(70_000, np.int64), D=32, opt="adam")
 
 
+def test_adversarial_key_order_oversized_bucket(R):
+    # the dedup samples keys at fixed positions; put spread-out keys there and
+    # crowd every other key between two of them, so one bucket holds almost
+    # the whole batch and is sorted and streamed from global memory
+    N = 24_000
+    rng = np.random.default_rng(12)
+    keys = 500_000 + rng.permutation(400_000)[: N].astype(np.int64)
+    sampled = (np.arange(2048, dtype=np.int64) * N) // 2048
+    keys[sampled] = np.arange(len(sampled), dtype=np.int64) * 1000
+    _single(R, keys, np.ones(N, np.int64), D=8, steps=2)
+
+
+def test_hot_key_among_others(R):
+    # one key holds 40% of the batch: its equality bucket is streamed
+    N = 30_000
+    rng = np.random.default_rng(13)
+    keys = rng.integers(0, 1 << 40, size=N)
+    keys[rng.random(N) < 0.4] = 77
+    _single(R, keys, np.ones(N, np.int64), D=16, opt="adam", grad_signed=True)
+
+
 def test_all_new_then_all_old(R):
     keys = np.arange(50_000, dtype=np.int64) * 1_000_003
     _single(R, keys[::-1].copy(), np.ones(50_000, np.int64), D=8, steps=3)
