@@ -2,26 +2,30 @@
 """Benchmark of the dynamic-hash embedding step (RecIS Embedding Engine hot path).
 
 One step = recis_feature_hash + recis_lookup_pooled + recis_backward_update
-over one batch of the 26-feature one-hot workload (26 categorical features,
-batch 8192, int64 IDs Zipf(1.05) over 10^7 per feature, hashed then mod 2^40,
-tagged and merged into one dim-64 fp32 table with Adam state, sum pooling).
+over one batch of a synthetic workload.  The default workload is the
+26-feature one-hot one (26 categorical features, batch 8192, int64 IDs
+Zipf(1.05) over 10^7 per feature, hashed then mod 2^40, tagged and merged into
+one dim-64 fp32 table with Adam state, sum pooling); `--workload` selects the
+others (seq8, longseq, tiny) for profiling.
 
 Prints one JSON line: IDs/s (device time, inputs resident, L2 flushed between
 steps), the same through the API with host buffers (e2e), the roofline of the
-dominant kernel, and the CPU oracle's rate on this host as a baseline.
+dominant kernel, SM clocks sampled during the timed region, and the CPU
+oracle's rate on this host as a baseline.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
 Multi-GPU runs (torchrun, one rank per GPU) are independent replicas: each rank
 owns its own table and batches; only the timing is reduced (max over ranks).
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -33,8 +37,10 @@ import numpy as np  # noqa: E402
 import workloads as W  # noqa: E402
 
 METRIC = "lookups/sec (IDs/s) fwd+bwd+update per step; achieved HBM GB/s vs B200 peak"
-WORKLOAD = "criteo26"
+DEFAULT_WORKLOAD = "criteo26"
 FALLBACK_HBM_GBS = 6650.0
+CSRC = os.path.join(ROOT, "recommender_sparse_embedding_b200", "csrc")
+TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def _peaks():
@@ -46,12 +52,21 @@ def _peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def _describe(w: W.Workload) -> str:
+    tabs = ", ".join(f"dim-{t.dim} {t.optimizer} {t.combiner}"
+                     + (" pooled" if t.pooled else "") + (" +unpooled" if t.unpooled else "")
+                     for t in w.tables)
+    f0 = w.features[0]
+    tf = "hash->mod 2^40->tag" if f0.flags & W.HASH else "tag"
+    return (f"{w.name}: F={w.F} features, B={w.B}, bag length {w.length}, IDs Zipf({w.zipf_a}) "
+            f"over {w.n_ids:.0e} per feature, {tf}, fp32 tables [{tabs}]")
+
+
 def _config(w: W.Workload, extra=None):
-    t = w.tables[0]
-    c = {"workload": f"{w.name}: F={w.F} one-hot features, B={w.B}, IDs Zipf({w.zipf_a}) over "
-                     f"{w.n_ids:.0e} per feature, hash->mod 2^40->tag, one merged dim-{t.dim} fp32 "
-                     f"table, {t.optimizer}, {t.combiner} pooling",
-         "F": w.F, "B": w.B, "dim": t.dim, "optimizer": t.optimizer, "combiner": t.combiner,
+    c = {"workload": _describe(w), "F": w.F, "B": w.B,
+         "tables": [{"dim": t.dim, "features": len(t.features), "optimizer": t.optimizer,
+                     "combiner": t.combiner, "pooled": t.pooled, "unpooled": t.unpooled}
+                    for t in w.tables],
          "l2": "flushed (256 MiB write) between timed steps", "parallelism": "replicas"}
     if extra:
         c.update(extra)
@@ -62,18 +77,22 @@ def _config(w: W.Workload, extra=None):
 def _oracle_rate(w: W.Workload, budget_s: float, batches):
     """The CPU oracle (single thread) on full steps of the workload, ~budget_s."""
     import oracle as O
-    t = w.tables[0]
     ops = [O.FeatureOp(flags=f.flags, hash_seed=f.hash_seed, mod=f.mod, tag=f.tag,
-                       tag_shift=f.tag_shift) for f in w.features]
-    tab = O.Table(t.dim, O.ADAM if t.optimizer == "adam" else O.ADAGRAD, t.lr, init_seed=t.init_seed)
+                       tag_shift=f.tag_shift, boundaries=list(f.boundaries)) for f in w.features]
+    tabs = [O.Table(t.dim, O.ADAM if t.optimizer == "adam" else O.ADAGRAD, t.lr,
+                    init_seed=t.init_seed) for t in w.tables]
     n_ids, steps, t0 = 0, 0, time.perf_counter()
     times = []
     while True:
-        b, g = batches[steps % len(batches)]
+        b, grads = batches[steps % len(batches)]
         s0 = time.perf_counter()
         keys = O.feature_hash(ops, b.values, b.feat_offsets)
-        tab.lookup(keys, b.bag_offsets, w.F, w.B)
-        tab.backward_update(g)
+        for t, tab, (gp, gu) in zip(w.tables, tabs, grads):
+            lo, hi, bo = b.table_slice(t, w.B)
+            tab.lookup(keys[lo:hi], bo, len(t.features), w.B,
+                       O.SUM if t.combiner == "sum" else O.MEAN, pooled=t.pooled,
+                       unpooled=t.unpooled)
+            tab.backward_update(gp, gu)
         times.append(time.perf_counter() - s0)
         n_ids += len(b.values)
         steps += 1
@@ -81,21 +100,34 @@ def _oracle_rate(w: W.Workload, budget_s: float, batches):
             break
     el = sum(times)
     return {"value": n_ids / el, "unit": "IDs/s", "cores": 1, "kind": "oracle",
-            "sample": f"{steps} full {w.name} steps (feature hash + lookup + backward/Adam) "
-                      f"on the single-threaded CPU oracle, {el:.1f} s",
+            "sample": f"{steps} full {w.name} steps (feature hash + lookup + backward/"
+                      f"optimiser) on the single-threaded CPU oracle, {el:.1f} s",
             "ms_per_step": 1e3 * el / steps, "steps": steps}
+
+
+def _grads(w: W.Workload, b: W.Batch, seed: int):
+    """Upstream gradients of one batch: (grad_pooled, grad_unpooled) per table."""
+    out = []
+    for i, t in enumerate(w.tables):
+        lo, hi, _ = b.table_slice(t, w.B)
+        gp = W.make_grad((w.B, len(t.features), t.dim), seed + 17 * i) if t.pooled else None
+        gu = W.make_grad((hi - lo, t.dim), seed + 17 * i + 1) if t.unpooled else None
+        out.append((gp, gu))
+    return out
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = W.WORKLOADS[WORKLOAD]
-    t = w.tables[0]
-    batches = [(W.make_batch(w, i), W.make_grad((w.B, w.F, t.dim), 100 + i)) for i in range(2)]
-    warm = _oracle_rate(w, 0.0, batches) if args.warmup > 0 else None  # one untimed step
-    del warm
-    res = _oracle_rate(w, max(5.0, 2.0 * args.steps), batches)
+    w = W.WORKLOADS[args.workload]
+    batches = []
+    for i in range(2):
+        b = W.make_batch(w, i)
+        batches.append((b, _grads(w, b, 100 + i)))
+    if args.warmup > 0:
+        _oracle_rate(w, 0.0, batches)  # one untimed step
+    res = _oracle_rate(w, max(5.0, 2.0 * args.steps) if args.steps < 60 else 120.0, batches)
     line = {"impl": "reference", "metric": METRIC, "value": res["value"], "unit": "IDs/s",
             "n_gpus": args.gpus, "steps": res["steps"], "warmup": args.warmup,
             "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
@@ -109,49 +141,128 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ GPU arm
 class Clocks:
-    """nvidia-smi sampling during the timed region."""
+    """SM clock and clock-event reasons, sampled through NVML every few ms on a
+    background thread; only samples inside [t0, t1] (the timed region) count."""
 
-    def __init__(self, index: int):
-        self.proc = None
-        self.index = index
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(index), "--query-gpu=clocks.sm,clocks.max.sm,"
-                 "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-                 "clocks_event_reasons.sw_power_cap,utilization.gpu",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
+    def __init__(self, torch_index: int, period_s: float = 0.002):
+        self.samples = []
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
         try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
+            import pynvml as N
+            import torch
+            N.nvmlInit()
+            self.N = N
+            uuid = str(torch.cuda.get_device_properties(torch_index).uuid)
+            handle = None
+            for i in range(N.nvmlDeviceGetCount()):
+                h = N.nvmlDeviceGetHandleByIndex(i)
+                u = N.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    handle = h
+                    break
+            if handle is None:
+                handle = N.nvmlDeviceGetHandleByIndex(torch_index)
+            self.h = handle
+            self.max_mhz = float(N.nvmlDeviceGetMaxClockInfo(handle, N.NVML_CLOCK_SM))
+            self.masks = [(name, getattr(N, attr, 0)) for name, attr in self.REASONS]
+            self._thread = threading.Thread(target=self._run, args=(period_s,), daemon=True)
+            self._thread.start()
+        except Exception as e:  # NVML missing: report no clocks rather than fail the bench
+            self.error = f"{type(e).__name__}: {e}"
+
+    def _run(self, period_s):
+        N = self.N
+        while not self._stop.is_set():
             try:
-                clk, cmax, util = float(parts[0]), float(parts[1]), float(parts[7])
-            except ValueError:
-                continue
-            mx = max(mx, cmax)
-            if util > 0:
-                sm.append(clk)
-            for n, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
-                "reasons": sorted(reasons), "samples_under_load": len(sm)}
+                t = time.perf_counter()
+                clk = N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM)
+                rs = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((t, float(clk), int(rs)))
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(period_s)
+
+    def stop(self, t0: float, t1: float):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        reasons = set()
+        for _, _, rs in inside:
+            for name, m in getattr(self, "masks", []):
+                if m and rs & m:
+                    reasons.add(name)
+        out = {"sm_mhz": statistics.median(s[1] for s in inside) if inside else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+               "samples": len(inside), "source": "nvml, 2 ms period, timed region only"}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+def _files_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def _traffic(kernel: str, units: float):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, scaled
+    to `units` (occurrences) when it was captured on another size; None when the
+    kernel's sources changed since the capture."""
+    if not os.path.exists(TRAFFIC):
+        return None, "no capture"
+    with open(TRAFFIC) as fh:
+        d = json.load(fh)
+    e = d.get(kernel)
+    if not e:
+        return None, "no capture of this kernel"
+    try:
+        if _files_sha(e["files"]) != e["sha256"]:
+            return None, "kernel changed since the capture"
+    except OSError:
+        return None, "kernel sources missing"
+    scale = units / e["units"] if e.get("units") else 1.0
+    return e["dram_bytes_per_launch"] * scale, e.get("note", "")
+
+
+# kernels of the step, grouped by the row of the method they implement
+GROUPS = {
+    "feature_hash": ("feature_hash",),
+    "dedup": ("ss_rank", "ss_probe", "ss_count", "ss_tilescan", "ss_scatter", "ss_local", "ss_finish", "sort_hist",
+              "sort_pass", "unique_insert"),
+    "gather_pool": ("bag_prep", "gather_pool"),
+    "backward": ("seg_reduce", "row_update", "reduce_update"),
+}
+
+
+def _alg_bytes(w: W.Workload, stats):
+    """Algorithmic bytes per step of each group (what the method must move; the
+    dedup's sort scratch is not credited).  stats[i] = (N, U, n_new) of table i."""
+    total_N = sum(s[0] for s in stats)
+    out = {"feature_hash": 16.0 * total_N, "dedup": 0.0, "gather_pool": 0.0, "backward": 0.0}
+    for t, (N, U, n_new) in zip(w.tables, stats):
+        D, s = t.dim, (2 if t.optimizer == "adam" else 1)
+        bags = len(t.features) * w.B
+        out["dedup"] += 8 * N + 4 * N + 16 * U + 16 * U + 4 * D * (1 + s) * n_new
+        out["gather_pool"] += 4 * D * U + (4 * D * bags if t.pooled else 0) + \
+            (4 * D * N if t.unpooled else 0) + 8 * bags
+        out["backward"] += (4 * D * bags if t.pooled else 0) + (4 * D * N if t.unpooled else 0) \
+            + 2 * 4 * D * (1 + s) * U
+    return out
 
 
 def run_gpu(args):
@@ -177,162 +288,227 @@ def run_gpu(args):
     import recommender_sparse_embedding_b200 as R
     R.load()
 
-    w = W.WORKLOADS[WORKLOAD]
-    spec = w.tables[0]
-    D = spec.dim
+    w = W.WORKLOADS[args.workload]
     nb = args.warmup + args.steps
     n_distinct = min(nb, args.batches)
     seed = 2025 + w.index + 1000 * rank
     host = []
     for i in range(n_distinct):
         b = W.make_batch(w, i, seed=seed)
-        g = W.make_grad((w.B, w.F, D), seed + i)
-        host.append((b, g))
+        host.append((b, _grads(w, b, seed + i)))
     feats = [R.Feature(flags=f.flags, hash_seed=f.hash_seed, mod=f.mod, tag=f.tag,
-                       tag_shift=f.tag_shift) for f in w.features]
-    devb = []
-    for b, g in host:
-        devb.append((torch.from_numpy(b.values).to(dev), b.feat_offsets.tolist(),
-                     torch.from_numpy(b.bag_offsets).to(dev), torch.from_numpy(g).to(dev),
-                     len(b.values)))
-    opt = R.ADAM if spec.optimizer == "adam" else R.ADAGRAD
-    table = R.Table(D, opt, spec.lr, init_seed=spec.init_seed,
-                    initial_capacity=1_000_000 if args.small else 8_000_000)
-    batch = R.Batch()
-    keys = torch.empty(max(x[4] for x in devb), dtype=torch.int64, device=dev)
-    pooled = torch.empty((w.B, w.F, D), dtype=torch.float32, device=dev)
+                       tag_shift=f.tag_shift,
+                       boundaries=(torch.tensor(list(f.boundaries), dtype=torch.int64, device=dev)
+                                   if f.boundaries else None)) for f in w.features]
+
+    def dev_batch(b, grads, pin=False):
+        mv = (lambda a: torch.from_numpy(a).pin_memory()) if pin else \
+            (lambda a: torch.from_numpy(a).to(dev))
+        per_table = []
+        for t, (gp, gu) in zip(w.tables, grads):
+            lo, hi, bo = b.table_slice(t, w.B)
+            per_table.append((lo, hi, mv(bo), None if gp is None else mv(gp),
+                              None if gu is None else mv(gu)))
+        return mv(b.values), b.feat_offsets.tolist(), per_table, len(b.values)
+
+    devb = [dev_batch(b, g) for b, g in host]
+    tables = [R.Table(t.dim, R.ADAM if t.optimizer == "adam" else R.ADAGRAD, t.lr,
+                      init_seed=t.init_seed,
+                      initial_capacity=1_000_000 if args.small else 8_000_000) for t in w.tables]
+    batches = [R.Batch() for _ in w.tables]
+    maxN = max(x[3] for x in devb)
+    keys = torch.empty(maxN, dtype=torch.int64, device=dev)
+    pooled = [torch.empty((w.B, len(t.features), t.dim), dtype=torch.float32, device=dev)
+              if t.pooled else None for t in w.tables]
+    max_n = [max(x[2][i][1] - x[2][i][0] for x in devb) for i in range(len(w.tables))]
+    unpooled = [torch.empty((max_n[i], t.dim), dtype=torch.float32, device=dev)
+                if t.unpooled else None for i, t in enumerate(w.tables)]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    combiner = [R.SUM if t.combiner == "sum" else R.MEAN for t in w.tables]
 
-    def step(i):
-        vals, foffs, boffs, grad, n = devb[i % n_distinct]
-        k = keys[:n]
+    def run_step(vals, foffs, per_table, n, kbuf):
+        k = kbuf[:n]
         R.feature_hash(feats, vals, foffs, keys_out=k)
-        table.lookup_pooled(batch, k, boffs, w.F, w.B, R.SUM, pooled_out=pooled)
-        table.backward_update(batch, grad)
+        for i, t in enumerate(w.tables):
+            lo, hi, bo, gp, gu = per_table[i]
+            up = unpooled[i][: hi - lo] if unpooled[i] is not None else None
+            tables[i].lookup_pooled(batches[i], k[lo:hi], bo, len(t.features), w.B, combiner[i],
+                                    pooled_out=pooled[i], unpooled_out=up)
+            tables[i].backward_update(batches[i], gp, gu)
         return n
 
-    # unique keys per batch (for the algorithmic bytes), outside any timing
-    uniq_counts = []
-    for i in range(n_distinct):
-        vals, foffs, _, _, n = devb[i]
+    # unique keys per table and batch (for the algorithmic bytes), outside any timing
+    uniq = []
+    for vals, foffs, per_table, n in devb:
         k = R.feature_hash(feats, vals, foffs)
-        uniq_counts.append(int(torch.unique(k).numel()))
+        uniq.append([int(torch.unique(k[lo:hi]).numel()) for (lo, hi, *_r) in per_table])
 
     for i in range(args.warmup):
-        step(i)
+        run_step(*devb[i % n_distinct], keys)
     torch.cuda.synchronize()
-    table.status_sync()
+    for t in tables:
+        t.status_sync()
+    rows0 = [t.size()[0] for t in tables]
 
+    # ---- timed region: K steps, no tracing events between the kernels
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    R.profile_enable(True)
-    R.profile_collect()
     launches0 = R.launch_count()
     clocks = Clocks(torch.cuda.current_device()) if rank == 0 else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    h0 = time.perf_counter()
     ids = 0
     for j in range(args.steps):
         flush.zero_()
         ev[j][0].record(stream)
-        ids += step(args.warmup + j)
+        ids += run_step(*devb[(args.warmup + j) % n_distinct], keys)
         ev[j][1].record(stream)
     torch.cuda.synchronize()
+    h1 = time.perf_counter()
     if world > 1:
         dist.barrier()
     launches = R.launch_count() - launches0
-    clk = clocks.stop() if clocks else None
-    prof = R.profile_collect()
-    R.profile_enable(False)
-    table.status_sync()
+    clk = clocks.stop(h0, h1) if clocks else None
+    for t in tables:
+        t.status_sync()
+    new_rows = [(t.size()[0] - r0) / args.steps for t, r0 in zip(tables, rows0)]
     dev_ms = sum(a.elapsed_time(b) for a, b in ev)
 
+    # ---- traced region: the same steps again with CUDA events around every
+    # launch of the library (per-kernel durations for the roofline)
+    prof_steps = min(args.steps, 50)
+    R.profile_enable(True)
+    R.profile_collect()
+    torch.cuda.synchronize()
+    for j in range(prof_steps):
+        flush.zero_()
+        run_step(*devb[(args.warmup + j) % n_distinct], keys)
+    torch.cuda.synchronize()
+    prof = R.profile_collect()
+    R.profile_enable(False)
+    for t in tables:
+        t.status_sync()
+
     # ---- e2e through the API with host buffers (pinned), copies inside the timing
-    e2e_ids, e2e_ms, h2d, d2h = 0, 0.0, 0, 0
-    pin = []
-    for b, g in host[: min(4, n_distinct)]:
-        pin.append((torch.from_numpy(b.values).pin_memory(), b.feat_offsets.tolist(),
-                    torch.from_numpy(b.bag_offsets).pin_memory(), torch.from_numpy(g).pin_memory(),
-                    len(b.values)))
-    pooled_h = torch.empty((w.B, w.F, D), dtype=torch.float32).pin_memory()
-    dv = torch.empty(max(x[4] for x in pin), dtype=torch.int64, device=dev)
-    dbo = torch.empty(w.F * w.B + 1, dtype=torch.int64, device=dev)
-    dg = torch.empty((w.B, w.F, D), dtype=torch.float32, device=dev)
-    e2e_steps = max(3, args.steps // 2)
+    e2e_ids, h2d, d2h = 0, 0, 0
+    pin = [dev_batch(b, g, pin=True) for b, g in host[: min(4, n_distinct)]]
+    dv = torch.empty(maxN, dtype=torch.int64, device=dev)
+    dbo = [torch.empty(w.F * w.B + 1, dtype=torch.int64, device=dev) for _ in w.tables]
+    dgp = [torch.empty_like(p) if p is not None else None for p in pooled]
+    dgu = [torch.empty_like(u) if u is not None else None for u in unpooled]
+    pooled_h = [torch.empty(p.shape, dtype=p.dtype).pin_memory() if p is not None else None
+                for p in pooled]
+    e2e_steps = max(3, min(args.steps, 50) // 2)
     eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(e2e_steps)]
     torch.cuda.synchronize()
     for j in range(e2e_steps):
-        vals_h, foffs, bo_h, g_h, n = pin[j % len(pin)]
+        vals_h, foffs, per_h, n = pin[j % len(pin)]
         flush.zero_()
         eev[j][0].record(stream)
         v = dv[:n]
         v.copy_(vals_h, non_blocking=True)
-        dbo.copy_(bo_h, non_blocking=True)
-        dg.copy_(g_h, non_blocking=True)
-        k = keys[:n]
-        R.feature_hash(feats, v, foffs, keys_out=k)
-        table.lookup_pooled(batch, k, dbo, w.F, w.B, R.SUM, pooled_out=pooled)
-        table.backward_update(batch, dg)
-        pooled_h.copy_(pooled, non_blocking=True)
+        h2d = vals_h.numel() * 8
+        per_d = []
+        for i, (lo, hi, bo_h, gp_h, gu_h) in enumerate(per_h):
+            bo = dbo[i][: bo_h.numel()]
+            bo.copy_(bo_h, non_blocking=True)
+            h2d += bo_h.numel() * 8
+            gp = gu = None
+            if gp_h is not None:
+                gp = dgp[i]
+                gp.copy_(gp_h, non_blocking=True)
+                h2d += gp_h.numel() * 4
+            if gu_h is not None:
+                gu = dgu[i][: gu_h.shape[0]]
+                gu.copy_(gu_h, non_blocking=True)
+                h2d += gu_h.numel() * 4
+            per_d.append((lo, hi, bo, gp, gu))
+        run_step(v, foffs, per_d, n, keys)
+        d2h = 0
+        for i, ph in enumerate(pooled_h):
+            if ph is not None:
+                ph.copy_(pooled[i], non_blocking=True)
+                d2h += ph.numel() * 4
         eev[j][1].record(stream)
         e2e_ids += n
-        h2d = vals_h.numel() * 8 + bo_h.numel() * 8 + g_h.numel() * 4
-        d2h = pooled_h.numel() * 4
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
-    table.status_sync()
+    for t in tables:
+        t.status_sync()
 
     # ---- reduce over ranks: max time, summed work
-    t_dev = torch.tensor([dev_ms, e2e_ms, float(ids), float(e2e_ids)], dtype=torch.float64, device=dev)
+    t_dev = torch.tensor([dev_ms, e2e_ms, float(ids), float(e2e_ids)], dtype=torch.float64,
+                         device=dev)
     if world > 1:
         mx = t_dev.clone()
-        dist.all_reduce(mx[:2], op=dist.ReduceOp.MAX)
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
         sm = t_dev.clone()
-        dist.all_reduce(sm[2:], op=dist.ReduceOp.SUM)
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
         dev_ms, e2e_ms, ids, e2e_ids = float(mx[0]), float(mx[1]), float(sm[2]), float(sm[3])
     value = ids / (dev_ms / 1e3)
     e2e_value = e2e_ids / (e2e_ms / 1e3)
 
     if rank == 0:
         peak, peak_kind = _peaks()
-        # algorithmic bytes per launch of each kernel of the step
-        Nm = statistics.mean(x[4] for x in devb)
-        Um = statistics.mean(uniq_counts)
-        nb_ = w.F * w.B
-        s = 2 if spec.optimizer == "adam" else 1
-        alg = {
-            "reduce_update": 4 * D * nb_ + 2 * 4 * D * (1 + s) * Um,
-            "gather_pool": 4 * D * Um + 4 * D * nb_,
-            "feature_hash": 16 * Nm,
-            "unique_insert": 16 * Um,
-        }
+        Nm = statistics.mean(x[3] for x in devb)
+        stats = []
+        for i, t in enumerate(w.tables):
+            Ni = statistics.mean(x[2][i][1] - x[2][i][0] for x in devb)
+            Ui = statistics.mean(u[i] for u in uniq)
+            stats.append((Ni, Ui, new_rows[i]))
+        alg = _alg_bytes(w, stats)
         kern = {k: {"launches": v[0], "total_ms": v[1], "avg_us": 1e3 * v[1] / max(v[0], 1)}
                 for k, v in prof.items()}
-        top = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+        # the dominant kernel, and its row of the method
         roof = None
-        if top in alg:
-            avg_s = prof[top][1] / prof[top][0] / 1e3
-            achieved = alg[top] / avg_s / 1e9
-            roof = {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peak,
-                    "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": None, "alg_bytes_per_launch": alg[top]}
-        step_alg = (8 * Nm + 16 * Um + 4 * D * Um + 4 * D * nb_) + alg["reduce_update"]
+        if prof:
+            top = max(prof.items(), key=lambda kv: kv[1][1])[0]
+            grp = next((g for g, ks in GROUPS.items() if top in ks), None)
+            if grp is not None:
+                members = [k for k in GROUPS[grp] if k in prof]
+                # bytes of the row per step; time of the row's kernels per step
+                row_s = sum(prof[k][1] for k in members) / prof_steps / 1e3
+                top_launches_per_step = prof[top][0] / prof_steps
+                top_s = prof[top][1] / prof[top][0] / 1e3
+                if len(members) == 1:
+                    per_launch = alg[grp] / top_launches_per_step
+                    achieved = per_launch / top_s / 1e9
+                else:
+                    per_launch = alg[grp]
+                    achieved = alg[grp] / row_s / 1e9
+                traffic, tnote = _traffic(top, Nm)
+                roof = {"bound": "hbm", "kernel": top, "row": grp,
+                        "row_kernels": members, "achieved": achieved, "peak": peak,
+                        "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                        "traffic": traffic, "traffic_note": tnote,
+                        "alg_bytes_per_launch": per_launch,
+                        "note": ("algorithmic bytes of the row / its kernels' event time"
+                                 if len(members) > 1 else
+                                 "algorithmic bytes per launch / CUDA-event time per launch")}
+        step_alg = sum(alg.values()) - alg["feature_hash"] + 16 * Nm
         line = {
             "metric": METRIC, "value": value, "unit": "IDs/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dev_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": _config(w, {"ids_per_step": Nm, "unique_per_step": Um,
+            "config": _config(w, {"ids_per_step": Nm,
+                                  "unique_per_step": [s[1] for s in stats],
+                                  "new_rows_per_step": [s[2] for s in stats],
                                   "distinct_batches": n_distinct}),
             "roofline": roof,
+            "step_alg_bytes": step_alg,
             "step_alg_gbs": step_alg / (dev_ms / args.steps / 1e3) / 1e9,
+            "step_frac_of_peak": step_alg / (dev_ms / args.steps / 1e3) / 1e9 / peak,
             "e2e": {"value": e2e_value, "unit": "IDs/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "kernels": kern,
+            "kernels_note": f"CUDA events around every launch, {prof_steps} further steps after the "
+                            "timed region (the timed region itself runs without them)",
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -340,8 +516,10 @@ def run_gpu(args):
             line["cpu_baseline"] = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")}
         print(json.dumps(line), flush=True)
 
-    table.close()
-    batch.close()
+    for t in tables:
+        t.close()
+    for b in batches:
+        b.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -350,9 +528,10 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--batches", type=int, default=32, help="distinct batches generated")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -36,22 +36,25 @@ struct SortCtl {
 };
 constexpr size_t kCtlZeroBytes = offsetof(SortCtl, active);
 
-// Control block of the sample-sort dedup (samplesort.cu); the first
-// kSsCtlZeroBytes bytes are cleared before every lookup.
+// Control block of the sample-sort dedup (samplesort.cu).  Every field is
+// written by the kernels of each call before it is read; nothing is cleared
+// on the host.
+constexpr int kMaxSplitters = 1024;       // distinct splitters <= 1023
+constexpr int kMaxBucketSlots = 2048;     // buckets 0 .. 2 * nsplit (<= 2046)
+constexpr int kMaxSample = 8192;          // sample size of the largest batches
 struct SsCtl {
-  unsigned int hist[512];             // keys per bucket
-  unsigned int ticket;
-  unsigned int tile_counter;
-  unsigned int bucket_counter;
-  unsigned int pad0;
-  unsigned long long blb[512];        // bucket look-back (heads, new keys)
-  unsigned int nsplit;                // written by the plan kernel
-  unsigned int pad1[3];
-  unsigned int base[512];             // first sorted position of each bucket
-  unsigned long long split[256];      // distinct splitters, ascending (ukey order)
+  unsigned nsplit, nb, nbp, pad0;         // splitters, buckets, buckets rounded up to 32
+  unsigned ticket_scan, ticket_local, pad1, pad2;
+  uint64_t samp[kMaxSample];              // the sorted sample (ukey order)
+  uint64_t cand[2][kMaxSplitters];  // candidate splitters of this call and the next
+  unsigned tot[kMaxBucketSlots];          // keys per bucket
+  unsigned base[kMaxBucketSlots];         // first sorted position of each bucket
+  unsigned hcnt[kMaxBucketSlots];         // distinct keys (heads) per bucket
+  unsigned ncnt[kMaxBucketSlots];         // new keys per bucket
+  unsigned hpre[kMaxBucketSlots];         // heads in earlier buckets
+  unsigned npre[kMaxBucketSlots];         // new keys in earlier buckets
 };
-constexpr size_t kSsCtlZeroBytes = offsetof(SsCtl, nsplit);
-constexpr int64_t kSampleSortMaxN = (int64_t)400 * 1024;  // larger batches use the radix sort
+constexpr int64_t kSampleSortMaxN = (int64_t)1600 * 1000;  // larger batches use the radix sort
 
 // Per-batch device scalars.
 struct BatchDev {
@@ -111,7 +114,9 @@ struct recis_batch {
   recis::SortCtl* ctl = nullptr;
   unsigned long long* seg_lookback = nullptr;   // [tiles], cleared per call (follows ctl)
   recis::SsCtl* ss = nullptr;                    // sample-sort control
-  unsigned long long* ss_lookback = nullptr;     // [tiles][512], epoch-tagged
+  uint32_t* ss_th = nullptr;                     // [tiles][2048] tile histograms
+  uint64_t* ss_meta = nullptr;                   // [capN] per sorted position
+  int64_t ss_th_cap = 0;
   int64_t seg_lookback_tiles = 0;
   int64_t* uniq = nullptr;
   int64_t* rows = nullptr;
@@ -124,6 +129,9 @@ struct recis_batch {
   int64_t capChunks = 0;
   cudaStream_t side = nullptr;  // bag preparation runs here, beside the dedup
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaEvent_t ev_pfork = nullptr, ev_probe = nullptr;  // IDMap probes beside the sort
+  int cand_parity = 0;          // which candidate array the next call reads
+  int64_t cand_n = 0;           // batch size that wrote it (0: none yet)
   int32_t* seg_counter = nullptr;  // [capN] last-arrival counters (self-resetting)
   int32_t* bag_counter = nullptr;  // [capBags]
   double* partials = nullptr;
@@ -179,6 +187,8 @@ cudaError_t launch_sort(recis_batch* b, recis_table* t, const int64_t* keys, int
 cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cudaStream_t s);
 cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
                                 cudaStream_t s);
+int samplesort_splits_for(int64_t N);
+int64_t samplesort_tiles_for(int64_t N);
 cudaError_t launch_pool(const LookupArgs& a, int64_t chunk, cudaStream_t s);
 cudaError_t launch_bag_prep(const LookupArgs& a, int64_t chunk, cudaStream_t s);
 cudaError_t launch_rows_per_key(recis_batch* b, int64_t N, int64_t* rows_out, cudaStream_t s);

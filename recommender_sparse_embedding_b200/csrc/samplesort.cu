@@ -1,28 +1,37 @@
-// samplesort.cu -- dedup + IDMap find-or-insert for batches of up to 2^19
-// keys in three launches (RecIS README, Key optimisations > Distributed
+// samplesort.cu -- dedup + IDMap find-or-insert for batches of up to
+// kSampleSortMaxN keys (RecIS README, Key optimisations > Distributed
 // optimisation: merged requests deduplicated; > Efficient dynamic embedding:
 // IDMap first-level store, EmbeddingBlocks second-level store).
 //
-// It produces exactly what the radix-sort path (sort.cu + unique.cu) produces
-// -- unique keys ascending, inverse index, rows (new keys in ascending key
-// order), segment starts, segment of each sorted position, occurrence of each
-// sorted position, initialised new rows -- but replaces the eight digit
-// passes by one bucket pass:
-//   ss_plan     every CTA sorts the same 2048-key sample (bitonic network in
-//               shared memory) and takes up to 255 distinct splitters; key k
-//               goes to bucket 2r + [k == splitter r], r = #splitters < k, so
-//               buckets are ordered, and a key equal to a splitter (a hot key)
-//               gets a bucket of its own.  The CTAs then histogram their
-//               slice of the keys; the last CTA scans the histogram.
-//   ss_scatter  one stable pass moving (key, occurrence) into bucket order:
-//               warp match/ballot ranking, decoupled look-back over tiles.
-//   ss_local    one CTA per bucket: sorts the bucket in shared memory by
-//               (key, occurrence) (an ascending-only bitonic network), finds
-//               the heads, probes the IDMap, resolves its unique/new prefix by
-//               look-back over buckets, writes all outputs and initialises
-//               its new rows.  A bucket larger than shared memory (possible
-//               only for adversarial key orders) is sorted by the same
-//               network in global memory and streamed.
+// It produces exactly what the radix-sort path (sort.cu + unique.cu) produces:
+// unique keys ascending, inverse index, rows (new keys get rows in ascending
+// key order), segment starts, the segment and the occurrence of each sorted
+// position, and initialised new rows.  The digit passes are replaced by six
+// short launches, none of which waits on another CTA:
+//   ss_rank      a strided sample of the keys (2048 to 8192 by batch size) is
+//                sorted by ranking: every sample's rank is its count of
+//                smaller samples (ties by position), spread over many CTAs.
+//   ss_count     per tile of 2048 keys: up to 1023 distinct splitters from the
+//                sorted sample, the bucket of every key (key u goes to bucket
+//                2r + [u == split[r]], r = #splitters < u, so buckets are
+//                ordered by key and a key equal to a splitter -- a hot key --
+//                has a bucket of its own), the tile's bucket histogram, and
+//                the IDMap find-or-insert of every occurrence (a missing key
+//                claims a free slot by CAS; its row is assigned later).
+//   ss_tilescan  per bucket, the exclusive prefix of the tile histograms (so
+//                the scatter is stable); the last CTA scans the bucket totals
+//                into bucket starts.
+//   ss_scatter   moves (key, occurrence) into bucket order, stably.
+//   ss_local     sorts every key-range bucket by (key, occurrence): one warp
+//                per bucket of up to 512 keys, in registers; the whole CTA in
+//                shared memory for larger ones.  An equality bucket holds one
+//                key, already in occurrence order.  Heads (first position of
+//                each distinct key) and new keys are numbered within the
+//                bucket; the last CTA scans the per-bucket counts.
+//   ss_finish    a flat pass over the sorted positions writes every output and
+//                initialises the new rows.
+// A key-range bucket larger than shared memory (only for adversarial key
+// orders) is sorted by the same network in global memory.
 #include <climits>
 
 #include "internal.h"
@@ -31,26 +40,19 @@ namespace recis {
 
 namespace {
 
-constexpr int kSsSample = 2048;
-constexpr int kSsSplit = 255;         // at most 255 distinct splitters
-constexpr int kSsDigits = 512;        // buckets 0 .. 2*nsplit (<= 510)
-constexpr int kSsBlock = 256;         // scatter CTA
-constexpr int kSsItems = 8;
-constexpr int kSsTile = kSsBlock * kSsItems;  // 2048 keys per scatter tile
-constexpr int kLocBlock = 512;        // local CTA
-constexpr int kLocCap = 3072;         // bucket elements held in shared memory
+constexpr int kRankThreads = 256;
+constexpr int kCountThreads = 256;
+constexpr int kCountItems = 8;
+constexpr int kTile = kCountThreads * kCountItems;  // 2048 keys per count/scatter tile
+constexpr int kFinThreads = 256;
+constexpr int kFinItems = 2;
+constexpr int kSub = kFinThreads * kFinItems;       // sorted positions per finish CTA
 constexpr int kMaxProbes = 1 << 16;
-constexpr unsigned long long kAgg = 1ULL << 62, kIncl = 2ULL << 62;
-constexpr unsigned kFlagAgg = 1u, kFlagIncl = 2u;
 
-__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
+// IDMap probe result of a head: row >= 0 for a key already present; -2 - slot
+// for a new key whose slot this call claimed; -1 when there is no row
+// (reserved key, or the IDMap was exhausted).
+__device__ __forceinline__ int64_t encode_new(int64_t slot) { return -2 - slot; }
 
 // bucket of ukey u: 2r + [u == split[r]], r = number of splitters < u
 __device__ __forceinline__ unsigned bucket_of(const uint64_t* split, int nsplit, uint64_t u) {
@@ -62,70 +64,132 @@ __device__ __forceinline__ unsigned bucket_of(const uint64_t* split, int nsplit,
   return 2u * (unsigned)lo + ((lo < nsplit && split[lo] == u) ? 1u : 0u);
 }
 
-// Ascending bitonic network on n elements (any n): for each merge size k the
-// first stage compares i with its mirror i ^ (k-1), later stages compare i
-// with i ^ d; every comparator puts the smaller (key, idx) at the lower index,
-// so a partner past the end behaves as +infinity and is skipped.  All threads
-// of the block must call it.
-template <typename KeyPtr, typename IdxPtr>
-__device__ void bitonic_sort(KeyPtr key, IdxPtr idx, int n) {
-  int n2 = 1;
+// Ascending bitonic network (mirror form) on n elements in shared memory: for
+// merge size k the first stage compares i with i ^ (k-1), later stages i with
+// i | d; every comparator puts the smaller element at the lower index, so a
+// partner past the end behaves as +infinity and is skipped.  Comparator t acts
+// on i = 2t - (t mod d) and its partner; the comparators of one 64-element
+// block are t in [32a, 32a+32), so warp a mod (NT/32) owns block a in every
+// stage whose partners stay inside a block (k <= 64, or d <= 32) and those
+// stages need only __syncwarp; the others end with __syncthreads.  PAIRS
+// orders by (key, idx), otherwise by key alone (idx unused).  All threads of
+// the block call it; it returns after a final __syncthreads.
+template <int NT, bool PAIRS, typename KeyPtr, typename IdxPtr>
+__device__ void staged_sort(KeyPtr key, IdxPtr idx, int n) {
+  int n2 = 64;
   while (n2 < n) n2 <<= 1;
+  const int half = n2 >> 1;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  bool prev_local = false;
   for (int k = 2; k <= n2; k <<= 1) {
     for (int d = k >> 1; d > 0; d >>= 1) {
       const bool mirror = d == (k >> 1);
-      for (int t = threadIdx.x; t < (n2 >> 1); t += blockDim.x) {
-        // t-th pair: lower index i has bit d clear
+      const bool local = mirror ? k <= 64 : d <= 32;
+      if (!local && prev_local) __syncthreads();
+      const int t0 = local ? lane + 32 * w : (int)threadIdx.x;
+      for (int t = t0; t < half; t += NT) {
         const int i = ((t & ~(d - 1)) << 1) | (t & (d - 1));
         const int j = mirror ? (i ^ (k - 1)) : (i | d);
         if (j < n) {
           const uint64_t ki = key[i], kj = key[j];
-          const uint32_t ii = idx[i], ij = idx[j];
-          if (kj < ki || (kj == ki && ij < ii)) {
+          if (PAIRS) {
+            const uint32_t ii = idx[i], ij = idx[j];
+            if (kj < ki || (kj == ki && ij < ii)) {
+              key[i] = kj;
+              key[j] = ki;
+              idx[i] = ij;
+              idx[j] = ii;
+            }
+          } else if (kj < ki) {
             key[i] = kj;
             key[j] = ki;
-            idx[i] = ij;
-            idx[j] = ii;
           }
         }
       }
-      __syncthreads();
+      if (local) __syncwarp(); else __syncthreads();
+      prev_local = local;
     }
   }
+  __syncthreads();
 }
 
-// IDMap find-or-insert (the same protocol as the radix path).
-__device__ __forceinline__ bool idmap_probe(Slot* slots, uint64_t mask, int64_t key,
-                                            int64_t* slot, int64_t* row) {
-  uint64_t h = mix64((uint64_t)key ^ kSlotSalt) & mask;
+// IDMap find-or-insert: linear probing from slot h = H(key ^ salt); a free
+// slot is claimed by a 64-bit CAS on its key.  Returns the row of a key
+// already present, -2 - slot for a key claimed in this call (its row is -1
+// until the call assigns it, whichever occurrence claimed it), or -1 when
+// the probe limit was reached.
+__device__ __forceinline__ int64_t idmap_resolve(Slot* slots, uint64_t mask, int64_t key, uint64_t h,
+                                                 longlong2 sv) {
   const int64_t limit = (int64_t)mask + 1 < kMaxProbes ? (int64_t)mask + 1 : kMaxProbes;
   for (int64_t n = 0; n < limit; ++n) {
-    const longlong2 sv = __ldcg(reinterpret_cast<const longlong2*>(slots + h));
+    if (n > 0) sv = __ldcg(reinterpret_cast<const longlong2*>(slots + h));
     if (sv.x == key) {
-      *slot = (int64_t)h;
-      *row = sv.y;
-      return false;
+      const int64_t row = sv.y >= 0 ? sv.y : __ldcg(&slots[h].row);
+      return row >= 0 ? row : encode_new((int64_t)h);
     }
     if (sv.x == kEmptyKey) {
       const unsigned long long old = atomicCAS(reinterpret_cast<unsigned long long*>(&slots[h].key),
                                                (unsigned long long)kEmptyKey,
                                                (unsigned long long)key);
-      if ((int64_t)old == kEmptyKey) {
-        *slot = (int64_t)h;
-        *row = -1;
-        return true;
-      }
+      if ((int64_t)old == kEmptyKey) return encode_new((int64_t)h);
       if ((int64_t)old == key) {
-        *slot = (int64_t)h;
-        *row = __ldcg(&slots[h].row);
-        return false;
+        const int64_t row = __ldcg(&slots[h].row);
+        return row >= 0 ? row : encode_new((int64_t)h);
       }
     }
     h = (h + 1) & mask;
   }
-  *slot = -1;
-  *row = -1;
-  return false;
+  return -1;
+}
+
+// exclusive block scan of one value per thread; *total gets the block sum
+template <int NT>
+__device__ __forceinline__ unsigned block_excl_scan(unsigned x, unsigned* s_warp, unsigned* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  unsigned y = x;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned z = __shfl_up_sync(0xffffffffu, y, off);
+    if (lane >= off) y += z;
+  }
+  __syncthreads();
+  if (lane == 31) s_warp[w] = y;
+  __syncthreads();
+  unsigned pre = 0, tot = 0;
+#pragma unroll
+  for (int ww = 0; ww < NT / 32; ++ww) {
+    const unsigned c = s_warp[ww];
+    pre += ww < w ? c : 0u;
+    tot += c;
+  }
+  *total = tot;
+  return pre + y - x;
+}
+
+// exclusive block scan of two values per thread at once (low and high 32 bits)
+template <int NT>
+__device__ __forceinline__ unsigned long long block_excl_scan2(unsigned long long x,
+                                                               unsigned long long* s_warp,
+                                                               unsigned long long* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  unsigned long long y = x;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long z = __shfl_up_sync(0xffffffffu, y, off);
+    if (lane >= off) y += z;
+  }
+  __syncthreads();
+  if (lane == 31) s_warp[w] = y;
+  __syncthreads();
+  unsigned long long pre = 0, tot = 0;
+#pragma unroll
+  for (int ww = 0; ww < NT / 32; ++ww) {
+    const unsigned long long c = s_warp[ww];
+    pre += ww < w ? c : 0ull;
+    tot += c;
+  }
+  *total = tot;
+  return pre + y - x;
 }
 
 }  // namespace
@@ -133,13 +197,20 @@ __device__ __forceinline__ bool idmap_probe(Slot* slots, uint64_t mask, int64_t 
 struct SsParams {
   const int64_t* keys;
   int64_t N;
+  int splits;               // splitter slots S + 1
+  int nsample;              // sample size
+  int tiles;                // count/scatter tiles
+  int max_buckets;          // 2S + 1
   SsCtl* ctl;
-  uint64_t* kb0;
-  uint32_t* vb0;
-  uint64_t* kb1;            // scratch for oversized buckets
-  uint32_t* vb1;
-  unsigned long long* lookback;  // scatter look-back [tiles][512], epoch-tagged
-  uint32_t epoch;
+  const uint64_t* cand;     // candidate splitters: cand[(i+1)*cand_step - 1], i < S, ascending
+  int cand_step;
+  uint64_t* cand_next;      // [S] quantiles of this call's sorted keys, for the next call
+  uint32_t* th;             // [tiles][nbp] tile histograms, then their column prefix
+  uint16_t* bkt;            // [N] bucket of each key
+  uint64_t* kb;             // [N] ukeys in bucket order, then sorted
+  uint32_t* vb;             // [N] occurrence of each position
+  int64_t* pocc;            // [N] IDMap result of each occurrence (see idmap_resolve)
+  uint64_t* meta;           // [N] per sorted position, see pack_meta
   // table
   Slot* slots;
   uint64_t slot_mask;
@@ -164,372 +235,460 @@ struct SsParams {
   HostMirror* mirror;
 };
 
-// ------------------------------------------------------------------ plan
-__global__ void __launch_bounds__(512) ss_plan_kernel(const __grid_constant__ SsParams p) {
-  __shared__ uint64_t s_samp[kSsSample];
-  __shared__ uint32_t s_sidx[kSsSample];
-  __shared__ uint64_t s_split[kSsSplit];
-  __shared__ unsigned s_hist[kSsDigits];
-  __shared__ int s_nsplit;
+// Per sorted position, written by ss_local: the bucket, the position's
+// segment within the bucket (1-based count of heads up to it), and for a head
+// whether its key is new and the 1-based count of new heads up to it.
+__device__ __forceinline__ uint64_t pack_meta(unsigned b, unsigned lh, unsigned lnew, bool head,
+                                              bool isnew) {
+  return ((uint64_t)b << 44) | ((uint64_t)head << 43) | ((uint64_t)isnew << 42) |
+         ((uint64_t)lnew << 21) | (uint64_t)lh;
+}
+
+// ------------------------------------------------------------------ rank
+// Sample k is the key at position floor(k N / ns).  CTA c ranks samples
+// [32c, 32c+32): 8 threads per sample each count the smaller samples (ties
+// broken by sample index) in one eighth of the sample, and the sum is the
+// sample's place in ctl->samp.
+__global__ void __launch_bounds__(kRankThreads) ss_rank_kernel(const __grid_constant__ SsParams p) {
+  extern __shared__ __align__(16) uint64_t s_samp[];  // [nsample]
+  const int tid = threadIdx.x;
+  const int ns = p.nsample;
+  const unsigned long long N = (unsigned long long)p.N;
+  const int lg = 31 - __clz(ns);  // ns is a power of two
+  for (int k = tid; k < ns; k += kRankThreads)
+    s_samp[k] = to_ukey(__ldg(p.keys + (int64_t)(((unsigned long long)k * N) >> lg)));
+  __syncthreads();
+  const int i = (int)blockIdx.x * 32 + (tid >> 3);
+  const int part = tid & 7;
+  const uint64_t v = s_samp[i];
+  unsigned cnt = 0;
+#pragma unroll 8
+  for (int j = part; j < ns; j += 8) {
+    const uint64_t sj = s_samp[j];
+    cnt += (sj < v || (sj == v && j < i)) ? 1u : 0u;
+  }
+  cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
+  cnt += __shfl_xor_sync(0xffffffffu, cnt, 2);
+  cnt += __shfl_xor_sync(0xffffffffu, cnt, 4);
+  if (part == 0) p.ctl->samp[cnt] = v;
+}
+
+// ------------------------------------------------------------------ count
+// Per tile of 2048 keys: the splitters (the S candidates, ascending; a run of
+// equal candidates keeps its first), the bucket of each key (kept for the
+// scatter) and the tile's bucket histogram (row `tile` of th).  CTA 0 resets
+// the call's tickets and records where this call's new rows start.
+__global__ void __launch_bounds__(kCountThreads) ss_count_kernel(const __grid_constant__ SsParams p) {
+  __shared__ uint64_t s_split[kMaxSplitters];
+  __shared__ unsigned s_hist[kMaxBucketSlots];
+  __shared__ unsigned s_warp[kCountThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int64_t pos0 = (int64_t)blockIdx.x * kTile + w * (kCountItems * 32) + lane;
+  int64_t k[kCountItems];
+#pragma unroll
+  for (int j = 0; j < kCountItems; ++j) {
+    const int64_t pos = pos0 + j * 32;
+    k[j] = pos < p.N ? __ldcs(p.keys + pos) : 0;
+  }
+  // splitters: 4 candidates per thread, in order
+  const int S = p.splits - 1, step = p.cand_step;
+  constexpr int kCand = kMaxSplitters / kCountThreads;  // 4
+  uint64_t c[kCand];
+  unsigned keepm = 0, nkeep = 0;
+#pragma unroll
+  for (int q = 0; q < kCand; ++q) {
+    const int ci = tid * kCand + q;
+    if (ci < S) {
+      c[q] = __ldcg(p.cand + (ci + 1) * step - 1);
+      const bool keep = ci == 0 || c[q] != __ldcg(p.cand + ci * step - 1);
+      keepm |= keep ? (1u << q) : 0u;
+      nkeep += keep ? 1u : 0u;
+    }
+  }
+  unsigned nsplit;
+  unsigned at = block_excl_scan<kCountThreads>(nkeep, s_warp, &nsplit);
+#pragma unroll
+  for (int q = 0; q < kCand; ++q)
+    if (keepm & (1u << q)) s_split[at++] = c[q];
+  const int nb = 2 * (int)nsplit + 1;
+  const int nbp = (nb + 31) & ~31;
+  for (int i = tid; i < nbp; i += kCountThreads) s_hist[i] = 0;
+  if (blockIdx.x == 0 && tid == 0) {
+    p.ctl->nsplit = nsplit;
+    p.ctl->nb = (unsigned)nb;
+    p.ctl->nbp = (unsigned)nbp;
+    p.ctl->ticket_scan = 0;
+    p.ctl->ticket_local = 0;
+    p.bdev->row_base = *(volatile unsigned long long*)&p.st->next_free;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kCountItems; ++j) {
+    const int64_t pos = pos0 + j * 32;
+    if (pos < p.N) {
+      const unsigned b = bucket_of(s_split, (int)nsplit, to_ukey(k[j]));
+      p.bkt[pos] = (uint16_t)b;
+      atomicAdd(&s_hist[b], 1u);
+    }
+  }
+  __syncthreads();
+  uint32_t* row = p.th + (size_t)blockIdx.x * nbp;
+  for (int i = tid; i < nbp; i += kCountThreads) row[i] = s_hist[i];
+}
+
+// ------------------------------------------------------------------ probe
+// IDMap find-or-insert of every occurrence (runs on a second stream beside
+// count, tile scan and scatter): two keys per thread, both first slots loaded
+// before either is resolved.  A missing key claims a free slot by CAS; every
+// occurrence of it then sees the slot with row -1 and records -2 - slot.
+constexpr int kProbeThreads = 256;
+constexpr int kProbeItems = 2;
+__global__ void __launch_bounds__(kProbeThreads) ss_probe_kernel(const __grid_constant__ SsParams p) {
+  const int64_t pos0 = (int64_t)blockIdx.x * (kProbeThreads * kProbeItems) + threadIdx.x;
+  int64_t k[kProbeItems];
+  uint64_t h[kProbeItems];
+  longlong2 sv[kProbeItems];
+#pragma unroll
+  for (int j = 0; j < kProbeItems; ++j) {
+    const int64_t pos = pos0 + j * kProbeThreads;
+    k[j] = pos < p.N ? __ldcs(p.keys + pos) : kEmptyKey;
+    h[j] = mix64((uint64_t)k[j] ^ kSlotSalt) & p.slot_mask;
+    if (k[j] != kEmptyKey) sv[j] = __ldcg(reinterpret_cast<const longlong2*>(p.slots + h[j]));
+  }
+  bool reserved = false;
+#pragma unroll
+  for (int j = 0; j < kProbeItems; ++j) {
+    const int64_t pos = pos0 + j * kProbeThreads;
+    if (pos >= p.N) continue;
+    int64_t r = -1;
+    if (k[j] == kEmptyKey) {
+      reserved = true;
+    } else {
+      r = idmap_resolve(p.slots, p.slot_mask, k[j], h[j], sv[j]);
+      if (r == -1) raise_error(p.st, p.mirror, kErrTableFull);
+    }
+    p.pocc[pos] = r;
+  }
+  if (reserved) raise_error(p.st, p.mirror, kErrReservedKey);
+}
+
+// ------------------------------------------------------------------ tile scan
+// CTA c owns buckets 32c .. 32c+31 (one per lane); warp w owns a contiguous
+// range of tiles.  Turns th[t][b] into the exclusive prefix over tiles and
+// writes the bucket totals; the last CTA scans the totals into bucket starts.
+__global__ void __launch_bounds__(1024) ss_tilescan_kernel(const __grid_constant__ SsParams p) {
+  __shared__ unsigned s_part[32][33];
+  __shared__ unsigned s_warp[32];
   __shared__ bool s_last;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int64_t N = p.N;
-  for (int k = tid; k < kSsSample; k += blockDim.x) {
-    const int64_t pos = (int64_t)(((unsigned long long)k * (unsigned long long)N) / kSsSample);
-    s_samp[k] = to_ukey(p.keys[pos]);
-    s_sidx[k] = (uint32_t)k;
-  }
-  for (int k = tid; k < kSsDigits; k += blockDim.x) s_hist[k] = 0;
-  __syncthreads();
-  bitonic_sort(s_samp, s_sidx, kSsSample);
-  // candidates: every 8th sample; keep the distinct ones (warp 0 compacts)
-  if (w == 0) {
-    int n = 0;
-    uint64_t prev = 0;
-    bool have = false;
-    for (int base = 0; base < kSsSplit; base += 32) {
-      const int i = base + lane;
-      const uint64_t c = i < kSsSplit ? s_samp[(i + 1) * (kSsSample / (kSsSplit + 1)) - 1] : 0;
-      const uint64_t pc = __shfl_up_sync(0xffffffffu, c, 1);
-      const bool first = i < kSsSplit && (lane == 0 ? (!have || c != prev) : c != pc);
-      const unsigned bal = __ballot_sync(0xffffffffu, first);
-      if (first) s_split[n + __popc(bal & ((1u << lane) - 1u))] = c;
-      n += __popc(bal);
-      prev = __shfl_sync(0xffffffffu, c, 31);
-      have = true;
+  const int nbp = (int)p.ctl->nbp;
+  const int T = p.tiles;
+  const int per = (T + 31) / 32;
+  const int ta = w * per, tb = ta + per < T ? ta + per : T;
+  if ((int)blockIdx.x * 32 < nbp) {
+    const int b = (int)blockIdx.x * 32 + lane;
+    unsigned sum = 0;
+#pragma unroll 4
+    for (int t = ta; t < tb; ++t) sum += __ldcg(p.th + (size_t)t * nbp + b);
+    s_part[w][lane] = sum;
+    __syncthreads();
+    if (w == 0) {
+      unsigned run = 0;
+      for (int ww = 0; ww < 32; ++ww) {
+        const unsigned c = s_part[ww][lane];
+        s_part[ww][lane] = run;
+        run += c;
+      }
+      p.ctl->tot[b] = run;
     }
-    if (lane == 0) s_nsplit = n;
+    __syncthreads();
+    unsigned run = s_part[w][lane];
+    for (int t = ta; t < tb; ++t) {
+      uint32_t* q = p.th + (size_t)t * nbp + b;
+      const unsigned c = __ldcg(q);
+      *q = run;
+      run += c;
+    }
   }
-  __syncthreads();
-  const int nsplit = s_nsplit;
-  if (blockIdx.x == 0) {
-    for (int i = tid; i < nsplit; i += blockDim.x) p.ctl->split[i] = s_split[i];
-    if (tid == 0) p.ctl->nsplit = (unsigned)nsplit;
-  }
-  // histogram of this CTA's slice
-  bool reserved = false;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < N; i += stride) {
-    const int64_t k = p.keys[i];
-    reserved |= k == kEmptyKey;
-    atomicAdd(&s_hist[bucket_of(s_split, nsplit, to_ukey(k))], 1u);
-  }
-  if (__any_sync(0xffffffffu, reserved) && lane == 0) raise_error(p.st, p.mirror, kErrReservedKey);
-  __syncthreads();
-  for (int k = tid; k < kSsDigits; k += blockDim.x)
-    if (s_hist[k]) atomicAdd(&p.ctl->hist[k], s_hist[k]);
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&p.ctl->ticket, 1u) == gridDim.x - 1;
+  if (tid == 0) s_last = atomicAdd(&p.ctl->ticket_scan, 1u) == gridDim.x - 1;
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // last CTA: exclusive scan of the bucket counts (warp 0, 16 per lane)
-  if (w == 0) {
-    unsigned c[16], run = 0;
+  // bucket starts: two consecutive buckets per thread
+  const int nb = (int)p.ctl->nb;
+  unsigned c[2];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      c[q] = __ldcg(&p.ctl->hist[lane * 16 + q]);
-      run += c[q];
-    }
-    unsigned x = run;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const unsigned y = __shfl_up_sync(0xffffffffu, x, off);
-      if (lane >= off) x += y;
-    }
-    unsigned b = x - run;
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      p.ctl->base[lane * 16 + q] = b;
-      b += c[q];
-    }
-    if (lane == 0) p.bdev->row_base = *(volatile unsigned long long*)&p.st->next_free;
+  for (int h = 0; h < 2; ++h) {
+    const int b = 2 * tid + h;
+    c[h] = b < nb ? __ldcg(&p.ctl->tot[b]) : 0u;
   }
+  unsigned total;
+  const unsigned ex = block_excl_scan<1024>(c[0] + c[1], s_warp, &total);
+  if (2 * tid < nb) p.ctl->base[2 * tid] = ex;
+  if (2 * tid + 1 < nb) p.ctl->base[2 * tid + 1] = ex + c[0];
 }
 
 // ------------------------------------------------------------------ scatter
-__global__ void __launch_bounds__(kSsBlock) ss_scatter_kernel(const __grid_constant__ SsParams p) {
-  __shared__ uint64_t s_keys[kSsTile];
-  __shared__ uint32_t s_vals[kSsTile];
-  __shared__ unsigned s_whist[kSsBlock / 32][kSsDigits];
-  __shared__ unsigned s_doff[kSsDigits];
-  __shared__ int s_glob[kSsDigits];
-  __shared__ uint64_t s_split[kSsSplit];
-  __shared__ unsigned s_wsum[kSsBlock / 32];
-  __shared__ unsigned s_tile;
+// Stable move of (ukey, occurrence) into bucket order.  Within a tile, warp w
+// holds keys w*256 .. w*256+255 (item j of lane l is key w*256 + 32j + l);
+// ranks within a warp come from match_any over the items in order, ranks
+// across warps from a prefix over per-warp bucket counters.
+__global__ void __launch_bounds__(kCountThreads) ss_scatter_kernel(const __grid_constant__ SsParams p) {
+  extern __shared__ unsigned s_wc[];  // [8][nbp] per-warp counters, then destinations
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int nsplit = (int)p.ctl->nsplit;
-  for (int i = tid; i < nsplit; i += kSsBlock) s_split[i] = p.ctl->split[i];
-  for (int i = tid; i < (kSsBlock / 32) * kSsDigits; i += kSsBlock) (&s_whist[0][0])[i] = 0;
-  if (tid == 0) s_tile = atomicAdd(&p.ctl->tile_counter, 1u);
+  const int nbp = (int)p.ctl->nbp;
+  const int64_t pos0 = (int64_t)blockIdx.x * kTile + w * (kCountItems * 32) + lane;
+  uint64_t k[kCountItems];
+  unsigned b[kCountItems], rank[kCountItems];
+#pragma unroll
+  for (int j = 0; j < kCountItems; ++j) {
+    const int64_t pos = pos0 + j * 32;
+    const bool ok = pos < p.N;
+    k[j] = ok ? to_ukey(__ldcs(p.keys + pos)) : 0;
+    b[j] = ok ? (unsigned)p.bkt[pos] : 0xffffffffu;
+  }
+  for (int i = tid; i < (kCountThreads / 32) * nbp; i += kCountThreads) s_wc[i] = 0;
   __syncthreads();
-  const unsigned tile = s_tile;
-  const int64_t tbase = (int64_t)tile * kSsTile;
-  const int64_t N = p.N;
-
-  uint64_t k[kSsItems];
-  uint32_t v[kSsItems];
-  unsigned d[kSsItems], rank[kSsItems];
-#pragma unroll
-  for (int j = 0; j < kSsItems; ++j) {
-    const int64_t pos = tbase + w * (kSsItems * 32) + j * 32 + lane;
-    if (pos < N) {
-      k[j] = to_ukey(p.keys[pos]);
-      v[j] = (uint32_t)pos;
-    } else {
-      k[j] = ~0ULL;
-      v[j] = 0xffffffffu;
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < kSsItems; ++j) {
-    const int64_t pos = tbase + w * (kSsItems * 32) + j * 32 + lane;
-    // padding goes to digit 511, after every real bucket
-    d[j] = pos < N ? bucket_of(s_split, nsplit, k[j]) : (unsigned)(kSsDigits - 1);
-  }
+  unsigned* mine = s_wc + w * nbp;
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int j = 0; j < kSsItems; ++j) {
-    const unsigned peers = __match_any_sync(0xffffffffu, d[j]);
+  for (int j = 0; j < kCountItems; ++j) {
+    const unsigned peers = __match_any_sync(0xffffffffu, b[j]);
     const int leader = __ffs(peers) - 1;
-    unsigned old = 0;
-    if (lane == leader) {
-      old = s_whist[w][d[j]];
-      s_whist[w][d[j]] = old + __popc(peers);
-    }
-    old = __shfl_sync(0xffffffffu, old, leader);
-    rank[j] = old + __popc(peers & lt);
+    const unsigned before = b[j] != 0xffffffffu ? mine[b[j]] : 0u;
+    rank[j] = before + __popc(peers & lt);
+    __syncwarp();
+    if (lane == leader && b[j] != 0xffffffffu) mine[b[j]] = before + __popc(peers);
     __syncwarp();
   }
   __syncthreads();
-  // two digits per thread: totals over warps, prefix per warp
-  unsigned total[2];
+  const uint32_t* th_row = p.th + (size_t)blockIdx.x * nbp;
+  const int nb = (int)p.ctl->nb;
+  for (int i = tid; i < nbp; i += kCountThreads) {
+    unsigned run = __ldcg(th_row + i) + (i < nb ? __ldcg(&p.ctl->base[i]) : 0u);
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int dd = tid + h * kSsBlock;
-    unsigned t = 0;
-#pragma unroll
-    for (int ww = 0; ww < kSsBlock / 32; ++ww) {
-      const unsigned c = s_whist[ww][dd];
-      s_whist[ww][dd] = t;
-      t += c;
+    for (int ww = 0; ww < kCountThreads / 32; ++ww) {
+      const unsigned c = s_wc[ww * nbp + i];
+      s_wc[ww * nbp + i] = run;
+      run += c;
     }
-    total[h] = t;
-    unsigned long long* my = p.lookback + (size_t)tile * kSsDigits + dd;
-    const unsigned long long tag = (unsigned long long)p.epoch << 32;
-    st_relaxed(my, tag | ((unsigned long long)(tile == 0 ? kFlagIncl : kFlagAgg) << 30) | t);
-  }
-  {
-    // low half: digits 0..255 in thread order
-    unsigned x = total[0];
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const unsigned y = __shfl_up_sync(0xffffffffu, x, off);
-      if (lane >= off) x += y;
-    }
-    if (lane == 31) s_wsum[w] = x;
-    __syncthreads();
-    unsigned pre = 0, lowsum = 0;
-#pragma unroll
-    for (int ww = 0; ww < kSsBlock / 32; ++ww) {
-      if (ww < w) pre += s_wsum[ww];
-      lowsum += s_wsum[ww];
-    }
-    s_doff[tid] = pre + x - total[0];
-    __syncthreads();
-    // high half: digits 256..511
-    unsigned y2 = total[1];
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const unsigned y = __shfl_up_sync(0xffffffffu, y2, off);
-      if (lane >= off) y2 += y;
-    }
-    if (lane == 31) s_wsum[w] = y2;
-    __syncthreads();
-    unsigned pre2 = 0;
-#pragma unroll
-    for (int ww = 0; ww < kSsBlock / 32; ++ww)
-      if (ww < w) pre2 += s_wsum[ww];
-    s_doff[tid + kSsBlock] = lowsum + pre2 + y2 - total[1];
-  }
-  // decoupled look-back, two digits per thread
-  int spins = 0;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int dd = tid + h * kSsBlock;
-    unsigned excl = 0;
-    if (tile > 0) {
-      constexpr int kWin = 8;
-      int64_t t = (int64_t)tile - 1;
-      bool done = false;
-      while (!done) {
-        unsigned long long e[kWin];
-#pragma unroll
-        for (int q = 0; q < kWin; ++q)
-          e[q] = (t - q >= 0) ? ld_relaxed(p.lookback + (size_t)(t - q) * kSsDigits + dd) : 0ULL;
-#pragma unroll
-        for (int q = 0; q < kWin; ++q) {
-          if (done) break;
-          if (t - q < 0) {
-            done = true;
-            break;
-          }
-          unsigned long long val = e[q];
-          while ((uint32_t)(val >> 32) != p.epoch || ((val >> 30) & 3u) == 0) {
-            if (++spins > kSpinLimit) {
-              raise_error(p.st, p.mirror, kErrTimeout);
-              done = true;
-              break;
-            }
-            __nanosleep(32);
-            val = ld_relaxed(p.lookback + (size_t)(t - q) * kSsDigits + dd);
-          }
-          if (done) break;
-          excl += (unsigned)(val & 0x3fffffffu);
-          if (((val >> 30) & 3u) == kFlagIncl) done = true;
-        }
-        t -= kWin;
-      }
-      const unsigned long long tag = (unsigned long long)p.epoch << 32;
-      st_relaxed(p.lookback + (size_t)tile * kSsDigits + dd,
-                 tag | ((unsigned long long)kFlagIncl << 30) | (excl + total[h]));
-    }
-    s_glob[dd] = (int)(p.ctl->base[dd] + excl) - (int)s_doff[dd];
   }
   __syncthreads();
 #pragma unroll
-  for (int j = 0; j < kSsItems; ++j) {
-    const unsigned sp = s_doff[d[j]] + s_whist[w][d[j]] + rank[j];
-    s_keys[sp] = k[j];
-    s_vals[sp] = v[j];
-  }
-  __syncthreads();
-  const int64_t valid = N - tbase < kSsTile ? N - tbase : kSsTile;
-  for (int sidx = tid; sidx < valid; sidx += kSsBlock) {
-    const int g = s_glob[bucket_of(s_split, nsplit, s_keys[sidx])] + sidx;
-    if ((unsigned)g < (unsigned)N) {
-      p.kb0[g] = s_keys[sidx];
-      p.vb0[g] = s_vals[sidx];
+  for (int j = 0; j < kCountItems; ++j) {
+    if (b[j] == 0xffffffffu) continue;
+    const unsigned dst = mine[b[j]] + rank[j];
+    if (dst < (unsigned)p.N) {
+      p.kb[dst] = k[j];
+      p.vb[dst] = (uint32_t)(pos0 + j * 32);
     }
   }
 }
 
 // ------------------------------------------------------------------ local
+template <int NT, int CAP>
 struct LocalShared {
-  uint64_t key[kLocCap];
-  uint32_t idx[kLocCap];
-  int32_t init_pos[kLocCap];  // sorted position of each new head (its key is kb0[pos])
-  int32_t init_row[kLocCap];
-  unsigned scan[kLocBlock / 32];
-  unsigned long long prefix;
-  unsigned bucket;
+  uint64_t key[CAP];
+  uint32_t idx[CAP];
+  unsigned long long warp[NT / 32];
+  bool last;
+};
+
+// Number heads and new keys of a sorted bucket (in shared memory, or in
+// global memory for an oversized one) in rounds of NT positions, write the
+// sorted keys and occurrences (from shared memory) and every position's meta.
+template <int NT, int CAP>
+__device__ void block_number(const SsParams& p, LocalShared<NT, CAP>& sh, unsigned b, int64_t m,
+                             int64_t off, bool in_smem) {
+  const int tid = threadIdx.x;
+  unsigned long long carry = 0;
+  for (int64_t c0 = 0; c0 < m; c0 += NT) {
+    const int64_t i = c0 + tid;
+    unsigned f = 0;
+    uint64_t u = 0;
+    uint32_t occ = 0;
+    if (i < m) {
+      u = in_smem ? sh.key[i] : __ldcg(p.kb + off + i);
+      occ = in_smem ? sh.idx[i] : __ldcg(p.vb + off + i);
+      const uint64_t before = i == 0 ? 0 : (in_smem ? sh.key[i - 1] : __ldcg(p.kb + off + i - 1));
+      if (i == 0 || u != before) f = 1u | (__ldcg(p.pocc + occ) <= -2 ? 2u : 0u);
+    }
+    unsigned long long tot;
+    const unsigned long long ex =
+        carry + block_excl_scan2<NT>(((unsigned long long)(f >> 1) << 32) | (f & 1u), sh.warp, &tot);
+    if (i < m) {
+      const unsigned lh = (unsigned)(ex & 0xffffffffULL) + (f & 1u);
+      const unsigned ln = (unsigned)(ex >> 32) + (f >> 1);
+      if (in_smem) {
+        p.kb[off + i] = u;
+        p.vb[off + i] = occ;
+      }
+      p.meta[off + i] = pack_meta(b, lh, ln, f & 1u, (f >> 1) != 0);
+    }
+    carry += tot;
+  }
+  if (tid == 0) {
+    p.ctl->hcnt[b] = (unsigned)(carry & 0xffffffffULL);
+    p.ctl->ncnt[b] = (unsigned)(carry >> 32);
+  }
+}
+
+// One CTA per bucket.  A key-range bucket is sorted by (key, occurrence) in
+// shared memory (oversized ones in global memory), then numbered; an
+// equality bucket holds one key, already in occurrence order (stable
+// scatter).  The last CTA scans the bucket counts into the call's segment and
+// new-row prefixes.
+template <int NT, int CAP>
+__global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ SsParams p) {
+  extern __shared__ __align__(16) unsigned char s_raw[];
+  LocalShared<NT, CAP>& sh = *reinterpret_cast<LocalShared<NT, CAP>*>(s_raw);
+  const int tid = threadIdx.x;
+  const unsigned b = blockIdx.x;
+  const unsigned nb = p.ctl->nb;
+  if (b < nb) {
+    const int64_t m = (int64_t)p.ctl->tot[b];
+    const int64_t off = (int64_t)p.ctl->base[b];
+    if (m == 0) {
+      if (tid == 0) {
+        p.ctl->hcnt[b] = 0;
+        p.ctl->ncnt[b] = 0;
+      }
+    } else if (b & 1u) {
+      const bool isnew = __ldcg(p.pocc + __ldcg(p.vb + off)) <= -2;
+      for (int64_t i = tid; i < m; i += NT)
+        p.meta[off + i] = pack_meta(b, 1u, isnew ? 1u : 0u, i == 0, i == 0 && isnew);
+      if (tid == 0) {
+        p.ctl->hcnt[b] = 1;
+        p.ctl->ncnt[b] = isnew ? 1u : 0u;
+      }
+    } else if (m <= CAP) {
+      for (int i = tid; i < m; i += NT) {
+        sh.key[i] = __ldcg(p.kb + off + i);
+        sh.idx[i] = __ldcg(p.vb + off + i);
+      }
+      __syncthreads();
+      staged_sort<NT, true>(sh.key, sh.idx, (int)m);
+      block_number<NT, CAP>(p, sh, b, m, off, true);
+    } else {
+      staged_sort<NT, true>(p.kb + off, p.vb + off, (int)m);
+      __threadfence_block();
+      block_number<NT, CAP>(p, sh, b, m, off, false);
+    }
+  }
+  // the last CTA scans the bucket counts and publishes the call's totals
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(&p.ctl->ticket_local, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!sh.last) return;
+  __threadfence();
+  unsigned long long carry = 0;
+  for (unsigned c0 = 0; c0 < nb; c0 += NT) {
+    const unsigned i = c0 + tid;
+    unsigned long long v = 0;
+    if (i < nb) v = ((unsigned long long)__ldcg(&p.ctl->ncnt[i]) << 32) | __ldcg(&p.ctl->hcnt[i]);
+    unsigned long long tot;
+    const unsigned long long ex = carry + block_excl_scan2<NT>(v, sh.warp, &tot);
+    if (i < nb) {
+      p.ctl->hpre[i] = (unsigned)(ex & 0xffffffffULL);
+      p.ctl->npre[i] = (unsigned)(ex >> 32);
+    }
+    carry += tot;
+  }
+  if (tid == 0) {
+    const unsigned long long U = carry & 0xffffffffULL, nnew = carry >> 32;
+    p.bdev->U = (unsigned)U;
+    p.bdev->n_new = (unsigned)nnew;
+    unsigned long long nf = p.bdev->row_base + nnew;
+    if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
+    p.st->next_free = nf;
+    if (p.mirror) {
+      p.mirror->next_free = nf;
+      __threadfence_system();
+    }
+    p.seg_start[U] = (int32_t)p.N;
+  }
+}
+
+// ------------------------------------------------------------------ finish
+struct FinishShared {
+  int64_t init_key[kFinThreads * kFinItems];
+  int32_t init_row[kFinThreads * kFinItems];
   int ninit;
 };
 
-__device__ __forceinline__ unsigned block_excl_scan(unsigned x, unsigned* s_scan, unsigned* total) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  unsigned y = x;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const unsigned z = __shfl_up_sync(0xffffffffu, y, off);
-    if (lane >= off) y += z;
-  }
+// Flat pass over the sorted positions, kSub per CTA (position blk*kSub +
+// j*256 + t for item j of thread t): segment of every position from its
+// bucket's prefix, all outputs, and the initialisation of the new rows.
+__global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_constant__ SsParams p) {
+  __shared__ FinishShared sh;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  if (tid == 0) sh.ninit = 0;
   __syncthreads();
-  if (lane == 31) s_scan[w] = y;
-  __syncthreads();
-  unsigned pre = 0, tot = 0;
-  for (int ww = 0; ww < (int)(blockDim.x >> 5); ++ww) {
-    const unsigned c = s_scan[ww];
-    if (ww < w) pre += c;
-    tot += c;
-  }
-  *total = tot;
-  return pre + y - x;
-}
-
-// look-back over buckets by warp 0: (heads, new) prefix of this bucket
-__device__ __forceinline__ void bucket_lookback(const SsParams& p, unsigned b, unsigned long long tH,
-                                                unsigned long long tN, LocalShared& sh) {
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x >= 32) return;
-  unsigned long long* lb = p.ctl->blb;
-  unsigned long long hx = 0, nx = 0;
-  if (b == 0) {
-    if (lane == 0) st_relaxed(lb, kIncl | (tH << 31) | tN);
-  } else {
-    if (lane == 0) st_relaxed(lb + b, kAgg | (tH << 31) | tN);
-    int64_t t = (int64_t)b - 1;
-    int spins = 0;
-    bool done = false;
-    while (!done) {
-      const int64_t idx = t - lane;
-      unsigned long long e = idx >= 0 ? ld_relaxed(lb + idx) : kIncl;
-      while (!__all_sync(0xffffffffu, (e >> 62) != 0)) {
-        if (++spins > kSpinLimit) break;
-        __nanosleep(32);
-        if ((e >> 62) == 0) e = ld_relaxed(lb + idx);
-      }
-      if (spins > kSpinLimit) {
-        if (lane == 0) raise_error(p.st, p.mirror, kErrTimeout);
-        break;
-      }
-      const unsigned incl = __ballot_sync(0xffffffffu, (e >> 62) == 2);
-      const int stop = incl ? __ffs(incl) - 1 : 31;
-      unsigned long long h = lane <= stop ? (e >> 31) & 0x7fffffffULL : 0;
-      unsigned long long n = lane <= stop ? e & 0x7fffffffULL : 0;
+  const int64_t q0 = (int64_t)blockIdx.x * kSub + tid;
+  const uint64_t row_base = p.bdev->row_base;
+  uint64_t mt[kFinItems];
+  uint32_t occ[kFinItems];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        h += __shfl_xor_sync(0xffffffffu, h, off);
-        n += __shfl_xor_sync(0xffffffffu, n, off);
-      }
-      hx += h;
-      nx += n;
-      done = incl != 0;
-      t -= 32;
-    }
-    if (lane == 0) st_relaxed(lb + b, kIncl | ((hx + tH) << 31) | (nx + tN));
-  }
-  if (lane == 0) sh.prefix = (hx << 32) | nx;
-}
-
-// outputs of one head / element (shared by the in-memory and streamed paths)
-__device__ __forceinline__ void write_head(const SsParams& p, LocalShared& sh, uint64_t ukey,
-                                           unsigned seg, int64_t pos, bool isnew, int64_t slot,
-                                           int64_t row, unsigned new_rank, int32_t key_at) {
-  const int64_t key = from_ukey(ukey);
-  int64_t r = row;
-  if (isnew) {
-    r = (int64_t)(p.bdev->row_base + new_rank);
-    if (r >= p.mapped_rows) {
-      raise_error(p.st, p.mirror, kErrTableFull);
-      r = -1;
-    } else {
-      p.slots[slot].row = r;
-      p.row_keys[r] = key;
-      const int q = atomicAdd(&sh.ninit, 1);
-      if (q < kLocCap) {
-        sh.init_pos[q] = key_at;
-        sh.init_row[q] = (int32_t)r;
-      }
+  for (int j = 0; j < kFinItems; ++j) {
+    const int64_t q = q0 + j * kFinThreads;
+    if (q < p.N) {
+      mt[j] = __ldcs(p.meta + q);
+      occ[j] = __ldcs(p.vb + q);
     }
   }
-  p.uniq[seg] = key;
-  p.rows[seg] = r;
-  p.seg_start[seg] = (int32_t)pos;
-}
-
-// keys: where init_pos points (the bucket in shared memory, or the sorted
-// keys in global memory for a streamed bucket)
-__device__ void init_rows(const SsParams& p, LocalShared& sh, const uint64_t* keys) {
+#pragma unroll
+  for (int j = 0; j < kFinItems; ++j) {
+    const int64_t q = q0 + j * kFinThreads;
+    if (q >= p.N) break;
+    const uint64_t m = mt[j];
+    const unsigned b = (unsigned)(m >> 44) & 0xfffu;
+    const unsigned lh = (unsigned)(m & 0x1fffffULL);
+    const unsigned seg = __ldg(&p.ctl->hpre[b]) + lh - 1u;
+    p.seg_of[q] = (int32_t)seg;
+    p.svals[q] = occ[j];
+    if (occ[j] < (uint32_t)p.N) p.inv[occ[j]] = (int32_t)seg;
+    if ((m >> 43) & 1u) {
+      const int64_t key = from_ukey(__ldcs(p.kb + q));
+      int64_t row = __ldcg(p.pocc + occ[j]);
+      if ((m >> 42) & 1u) {
+        const int64_t slot = -2 - row;
+        const unsigned ln = (unsigned)((m >> 21) & 0x1fffffULL);
+        row = (int64_t)(row_base + __ldg(&p.ctl->npre[b]) + ln - 1u);
+        if (row >= p.mapped_rows) {
+          raise_error(p.st, p.mirror, kErrTableFull);
+          row = -1;
+        } else {
+          p.slots[slot].row = row;
+          p.row_keys[row] = key;
+          const int at = atomicAdd(&sh.ninit, 1);
+          sh.init_key[at] = key;
+          sh.init_row[at] = (int32_t)row;
+        }
+      }
+      p.uniq[seg] = key;
+      p.rows[seg] = row;
+      p.seg_start[seg] = (int32_t)q;
+    }
+  }
+  // the next call's candidate splitters: quantiles of this call's sorted keys
+  if (blockIdx.x == 0) {
+    const unsigned long long N = (unsigned long long)p.N;
+    for (int i = tid; i < p.splits - 1; i += kFinThreads) {
+      const unsigned long long q = ((unsigned long long)(i + 1) * N) / (unsigned long long)p.splits;
+      p.cand_next[i] = __ldcg(p.kb + (q > 0 ? q - 1 : 0));
+    }
+  }
   __syncthreads();
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  // initialise the new rows: one warp per row, one 16-byte column per lane
+  const int n = sh.ninit;
   const int nf4 = p.row_floats >> 2, ncol = p.D >> 2;
   const float sv = p.adagrad ? p.acc0 : 0.0f;
-  const int n = sh.ninit < kLocCap ? sh.ninit : kLocCap;
-  for (int r = w; r < n; r += kLocBlock / 32) {
-    const uint64_t base = mix64((uint64_t)from_ukey(keys[sh.init_pos[r]]) ^ p.init_seed);
-    float4* dst = reinterpret_cast<float4*>(p.row_data + (int64_t)sh.init_row[r] * p.row_floats);
+  for (int rr = w; rr < n; rr += kFinThreads / 32) {
+    const uint64_t base = mix64((uint64_t)sh.init_key[rr] ^ p.init_seed);
+    float4* dst = reinterpret_cast<float4*>(p.row_data + (int64_t)sh.init_row[rr] * p.row_floats);
     for (int c = lane; c < nf4; c += 32) {
       float4 o;
       if (c < ncol) {
@@ -543,191 +702,53 @@ __device__ void init_rows(const SsParams& p, LocalShared& sh, const uint64_t* ke
       dst[c] = o;
     }
   }
-  __syncthreads();
-  if (threadIdx.x == 0) sh.ninit = 0;
-  __syncthreads();
 }
 
-__global__ void __launch_bounds__(kLocBlock) ss_local_kernel(const __grid_constant__ SsParams p) {
-  extern __shared__ __align__(16) unsigned char s_raw[];
-  LocalShared& sh = *reinterpret_cast<LocalShared*>(s_raw);
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    sh.bucket = atomicAdd(&p.ctl->bucket_counter, 1u);
-    sh.ninit = 0;
-  }
-  __syncthreads();
-  const unsigned b = sh.bucket;
-  const int nsplit = (int)p.ctl->nsplit;
-  const unsigned nb = 2u * (unsigned)nsplit + 1u;
-  const int64_t off = p.ctl->base[b];
-  const int64_t m = b < nb ? (int64_t)p.ctl->hist[b] : 0;
-  const bool eq_bucket = (b & 1u) != 0;
-  const int64_t N = p.N;
+// ------------------------------------------------------------------ host
+int samplesort_splits_for(int64_t) { return kMaxSplitters; }
 
-  if (m <= kLocCap) {
-    // ---- in shared memory: load, sort, heads, probes
-    for (int i = tid; i < m; i += kLocBlock) {
-      sh.key[i] = p.kb0[off + i];
-      sh.idx[i] = p.vb0[off + i];
-    }
-    __syncthreads();
-    if (!eq_bucket && m > 1) bitonic_sort(sh.key, sh.idx, (int)m);
-    // each thread: 8 consecutive sorted elements
-    constexpr int kPer = kLocCap / kLocBlock;
-    const int i0 = tid * kPer;
-    bool head[kPer], isnew[kPer];
-    int64_t slot[kPer], row[kPer];
-    unsigned nh = 0, nn = 0;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int i = i0 + j;
-      head[j] = i < m && (i == 0 || sh.key[i] != sh.key[i - 1]);
-      isnew[j] = false;
-      slot[j] = -1;
-      row[j] = -1;
-    }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      if (head[j] && from_ukey(sh.key[i0 + j]) != kEmptyKey) {
-        isnew[j] = idmap_probe(p.slots, p.slot_mask, from_ukey(sh.key[i0 + j]), &slot[j], &row[j]);
-        if (slot[j] < 0) raise_error(p.st, p.mirror, kErrTableFull);
-      }
-      nh += head[j];
-      nn += isnew[j];
-    }
-    unsigned totH, totN;
-    const unsigned exH = block_excl_scan(nh, sh.scan, &totH);
-    const unsigned exN = block_excl_scan(nn, sh.scan, &totN);
-    __syncthreads();
-    bucket_lookback(p, b, totH, totN, sh);
-    __syncthreads();
-    const unsigned Hx = (unsigned)(sh.prefix >> 32), Nx = (unsigned)(sh.prefix & 0xffffffffULL);
-    unsigned hrun = Hx + exH, nrun = Nx + exN;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int i = i0 + j;
-      if (i >= m) break;
-      const int64_t pos = off + i;
-      if (head[j]) {
-        write_head(p, sh, sh.key[i], hrun, pos, isnew[j], slot[j], row[j], nrun, i);
-        nrun += isnew[j];
-        ++hrun;
-      }
-      const unsigned seg = hrun - 1;
-      const uint32_t occ = sh.idx[i];
-      p.seg_of[pos] = (int32_t)seg;
-      p.svals[pos] = occ;
-      if (occ < (uint64_t)N) p.inv[occ] = (int32_t)seg;
-    }
-    if (b == gridDim.x - 1 && tid == 0) {
-      // the last bucket CTA knows the totals
-      const unsigned long long U = (unsigned long long)Hx + totH, nnew = (unsigned long long)Nx + totN;
-      p.bdev->U = (unsigned)U;
-      p.bdev->n_new = (unsigned)nnew;
-      unsigned long long nf = p.bdev->row_base + nnew;
-      if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
-      p.st->next_free = nf;
-      if (p.mirror) {
-        p.mirror->next_free = nf;
-        __threadfence_system();
-      }
-      p.seg_start[U] = (int32_t)N;
-    }
-    init_rows(p, sh, sh.key);
-    return;
-  }
+int64_t samplesort_tiles_for(int64_t N) { return (N + kTile - 1) / kTile; }
 
-  // ---- oversized bucket, streamed from global memory
-  if (!eq_bucket) bitonic_sort(p.kb0 + off, p.vb0 + off, (int)m);
-  __threadfence_block();
-  __syncthreads();
-  // sweep 1: heads, probes (kept in kb1/vb1 of the same range), counts
-  unsigned long long cH = 0, cN = 0;
-  for (int64_t c0 = 0; c0 < m; c0 += kLocBlock) {
-    const int64_t i = c0 + tid;
-    bool hd = false, nw = false;
-    if (i < m) {
-      const uint64_t u = p.kb0[off + i];
-      hd = i == 0 || u != p.kb0[off + i - 1];
-      int64_t slot = -1, row = -1;
-      if (hd && from_ukey(u) != kEmptyKey) {
-        nw = idmap_probe(p.slots, p.slot_mask, from_ukey(u), &slot, &row);
-        if (slot < 0) raise_error(p.st, p.mirror, kErrTableFull);
-      }
-      p.kb1[off + i] = (uint64_t)(nw ? slot : row);
-      p.vb1[off + i] = (hd ? 1u : 0u) | (nw ? 2u : 0u);
-    }
-    unsigned t1, t2;
-    block_excl_scan(hd ? 1u : 0u, sh.scan, &t1);
-    block_excl_scan(nw ? 1u : 0u, sh.scan, &t2);
-    cH += t1;
-    cN += t2;
-  }
-  __syncthreads();
-  bucket_lookback(p, b, cH, cN, sh);
-  __syncthreads();
-  const unsigned Hx = (unsigned)(sh.prefix >> 32), Nx = (unsigned)(sh.prefix & 0xffffffffULL);
-  // sweep 2: outputs
-  unsigned hcarry = Hx, ncarry = Nx;
-  for (int64_t c0 = 0; c0 < m; c0 += kLocBlock) {
-    const int64_t i = c0 + tid;
-    const uint32_t fl = i < m ? p.vb1[off + i] : 0u;
-    const bool hd = fl & 1u, nw = (fl & 2u) != 0;
-    unsigned t1, t2;
-    const unsigned eh = block_excl_scan(hd ? 1u : 0u, sh.scan, &t1);
-    const unsigned en = block_excl_scan(nw ? 1u : 0u, sh.scan, &t2);
-    if (i < m) {
-      const int64_t pos = off + i;
-      const uint64_t u = p.kb0[pos];
-      const int64_t sr = (int64_t)p.kb1[pos];
-      if (hd)
-        write_head(p, sh, u, hcarry + eh, pos, nw, nw ? sr : -1, nw ? -1 : sr, ncarry + en,
-                   (int32_t)pos);
-      // the segment of element i: heads up to and including i, minus one
-      const unsigned seg = hcarry + eh + (hd ? 1u : 0u) - 1u;
-      const uint32_t occ = p.vb0[pos];
-      p.seg_of[pos] = (int32_t)seg;
-      p.svals[pos] = occ;
-      if (occ < (uint64_t)N) p.inv[occ] = (int32_t)seg;
-    }
-    hcarry += t1;
-    ncarry += t2;
-    __syncthreads();
-    if (sh.ninit >= kLocCap - kLocBlock) init_rows(p, sh, p.kb0);
-  }
-  if (b == gridDim.x - 1 && tid == 0) {
-    const unsigned long long U = hcarry, nnew = ncarry;
-    p.bdev->U = (unsigned)U;
-    p.bdev->n_new = (unsigned)nnew;
-    unsigned long long nf = p.bdev->row_base + nnew;
-    if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
-    p.st->next_free = nf;
-    if (p.mirror) {
-      p.mirror->next_free = nf;
-      __threadfence_system();
-    }
-    p.seg_start[U] = (int32_t)N;
-  }
-  init_rows(p, sh, p.kb0);
+static int sample_size_for(int64_t N) {
+  if (N <= 262144) return 2048;
+  if (N <= 524288) return 4096;
+  return 8192;
+}
+
+template <typename K>
+static cudaError_t set_smem(K kernel, int bytes, bool* done, int dev) {
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  return e;
+}
+
+template <int NT, int CAP>
+static cudaError_t launch_local(const SsParams& p, int dev, cudaStream_t s) {
+  static bool attr[64] = {false};
+  cudaError_t e = set_smem(ss_local_kernel<NT, CAP>, (int)sizeof(LocalShared<NT, CAP>), attr, dev);
+  if (e != cudaSuccess) return e;
+  LaunchScope ls("ss_local", s);
+  ss_local_kernel<NT, CAP><<<(unsigned)p.max_buckets, NT, sizeof(LocalShared<NT, CAP>), s>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
                                 cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(b->ss, 0, kSsCtlZeroBytes, s);
-  if (e != cudaSuccess) return e;
-  b->epoch += 1;
-  if (b->epoch == 0) b->epoch = 1;
   SsParams p;
   p.keys = keys;
   p.N = N;
+  p.splits = samplesort_splits_for(N);
+  p.nsample = sample_size_for(N);
+  p.tiles = (int)samplesort_tiles_for(N);
+  p.max_buckets = 2 * (p.splits - 1) + 1;
   p.ctl = b->ss;
-  p.kb0 = b->kbuf[0];
-  p.vb0 = b->vbuf[0];
-  p.kb1 = b->kbuf[1];
-  p.vb1 = b->vbuf[1];
-  p.lookback = b->ss_lookback;
-  p.epoch = b->epoch;
+  p.th = b->ss_th;
+  p.bkt = reinterpret_cast<uint16_t*>(b->vbuf[1]);
+  p.kb = b->kbuf[0];
+  p.vb = b->vbuf[0];
+  p.pocc = reinterpret_cast<int64_t*>(b->kbuf[1]);
+  p.meta = b->ss_meta;
   p.slots = t->slots;
   p.slot_mask = (uint64_t)t->capacity - 1;
   p.row_data = reinterpret_cast<float*>(t->rows.va);
@@ -748,32 +769,68 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   p.bdev = b->bdev;
   p.st = t->dstate;
   p.mirror = t->mirror_dev;
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool rank_attr[64] = {false}, scatter_attr[64] = {false};
+  const int nbp_max = (p.max_buckets + 31) & ~31;
+  // splitters: quantiles of the previous call on this batch when its size was
+  // comparable, else a sorted sample of this call's keys
+  const int cur = b->cand_parity;
+  const bool reuse = b->cand_n > 0 && b->cand_n >= N / 2 && b->cand_n <= 2 * N;
+  p.cand_next = b->ss->cand[cur ^ 1];
+  if (reuse) {
+    p.cand = b->ss->cand[cur];
+    p.cand_step = 1;
+  } else {
+    p.cand = b->ss->samp;
+    p.cand_step = p.nsample / p.splits;
+    if ((e = set_smem(ss_rank_kernel, kMaxSample * (int)sizeof(uint64_t), rank_attr, dev)) != cudaSuccess)
+      return e;
+    LaunchScope ls("ss_rank", s);
+    ss_rank_kernel<<<(unsigned)(p.nsample / 32), kRankThreads, p.nsample * sizeof(uint64_t), s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  b->cand_parity = cur ^ 1;
+  b->cand_n = N;
+  // IDMap probes of every occurrence on the side stream, beside the sort
+  if ((e = cudaEventRecord(b->ev_pfork, s)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(b->side, b->ev_pfork, 0)) != cudaSuccess)
+    return e;
   {
-    int64_t blocks = (N + 4095) / 4096;
-    if (blocks > 2 * kSMs) blocks = 2 * kSMs;
-    if (blocks < 1) blocks = 1;
-    LaunchScope ls("ss_plan", s);
-    ss_plan_kernel<<<(unsigned)blocks, 512, 0, s>>>(p);
+    LaunchScope ls("ss_probe", b->side);
+    const int64_t per = kProbeThreads * kProbeItems;
+    ss_probe_kernel<<<(unsigned)((N + per - 1) / per), kProbeThreads, 0, b->side>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = cudaEventRecord(b->ev_probe, b->side)) != cudaSuccess) return e;
+  {
+    LaunchScope ls("ss_count", s);
+    ss_count_kernel<<<(unsigned)p.tiles, kCountThreads, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
-    const int64_t tiles = (N + kSsTile - 1) / kSsTile;
+    LaunchScope ls("ss_tilescan", s);
+    ss_tilescan_kernel<<<(unsigned)(nbp_max / 32), 1024, 0, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    const int smem = (kCountThreads / 32) * nbp_max * (int)sizeof(unsigned);
+    if ((e = set_smem(ss_scatter_kernel, smem, scatter_attr, dev)) != cudaSuccess) return e;
     LaunchScope ls("ss_scatter", s);
-    ss_scatter_kernel<<<(unsigned)tiles, kSsBlock, 0, s>>>(p);
+    ss_scatter_kernel<<<(unsigned)p.tiles, kCountThreads, smem, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if ((e = cudaStreamWaitEvent(s, b->ev_probe, 0)) != cudaSuccess) return e;
+  if (N <= 524288)
+    e = launch_local<128, 2048>(p, dev, s);
+  else
+    e = launch_local<512, 4096>(p, dev, s);
+  if (e != cudaSuccess) return e;
   {
-    static bool attr_set[128] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 128 && !attr_set[dev]) {
-      e = cudaFuncSetAttribute(ss_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)sizeof(LocalShared));
-      if (e != cudaSuccess) return e;
-      attr_set[dev] = true;
-    }
-    LaunchScope ls("ss_local", s);
-    ss_local_kernel<<<kSsDigits - 1, kLocBlock, sizeof(LocalShared), s>>>(p);
+    LaunchScope ls("ss_finish", s);
+    ss_finish_kernel<<<(unsigned)((N + kSub - 1) / kSub), kFinThreads, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -368,6 +368,7 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
         (e = realloc_dev(b->inv, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_of, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->svals, cap, true)) != cudaSuccess ||
+        (e = realloc_dev(b->ss_meta, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_start, cap + 1, true)) != cudaSuccess ||
         (e = realloc_dev(b->occ_info, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_counter, cap, true)) != cudaSuccess)
@@ -376,8 +377,6 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
     if ((e = realloc_dev(b->sort_lookback, (size_t)st * 256, true)) != cudaSuccess)
       return cuda_fail(e, "batch alloc");
     b->sort_lookback_tiles = st;
-    if ((e = realloc_dev(b->ss_lookback, (size_t)st * 512, true)) != cudaSuccess)
-      return cuda_fail(e, "batch alloc");
     const int64_t ut = unique_tiles_for(cap);
     if ((e = realloc_dev(b->seg_lookback, (size_t)ut, true)) != cudaSuccess)
       return cuda_fail(e, "batch alloc");
@@ -392,8 +391,18 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
   if (!b->side) {
     if ((e = cudaStreamCreateWithFlags(&b->side, cudaStreamNonBlocking)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&b->ev_fork, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&b->ev_join, cudaEventDisableTiming)) != cudaSuccess)
+        (e = cudaEventCreateWithFlags(&b->ev_join, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&b->ev_pfork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&b->ev_probe, cudaEventDisableTiming)) != cudaSuccess)
       return cuda_fail(e, "batch stream");
+  }
+  if (N <= kSampleSortMaxN) {
+    const int64_t th = samplesort_tiles_for(N) * kMaxBucketSlots;
+    if (th > b->ss_th_cap) {
+      const int64_t cap = th + th / 4;
+      if ((e = realloc_dev(b->ss_th, cap, true)) != cudaSuccess) return cuda_fail(e, "batch alloc");
+      b->ss_th_cap = cap;
+    }
   }
   const int64_t cf = pool_chunk_for(N, D), cu = update_chunk_for(N, D);
   if ((N + cf - 1) / cf + 1 > b->capChunks) {
@@ -419,7 +428,8 @@ static void batch_free(recis_batch* b) {
   cudaFree(b->sort_lookback);
   cudaFree(b->ctl);
   cudaFree(b->ss);
-  cudaFree(b->ss_lookback);
+  cudaFree(b->ss_th);
+  cudaFree(b->ss_meta);
   cudaFree(b->seg_lookback);
   cudaFree(b->uniq);
   cudaFree(b->rows);
@@ -436,6 +446,8 @@ static void batch_free(recis_batch* b) {
   if (b->side) cudaStreamDestroy(b->side);
   if (b->ev_fork) cudaEventDestroy(b->ev_fork);
   if (b->ev_join) cudaEventDestroy(b->ev_join);
+  if (b->ev_pfork) cudaEventDestroy(b->ev_pfork);
+  if (b->ev_probe) cudaEventDestroy(b->ev_probe);
 }
 
 static recis_status check_device() {
