@@ -245,7 +245,7 @@ GROUPS = {
     "dedup": ("ss_rank", "ss_probe", "ss_count", "ss_tilescan", "ss_scatter", "ss_local", "ss_finish", "sort_hist",
               "sort_pass", "unique_insert"),
     "gather_pool": ("bag_prep", "gather_pool"),
-    "backward": ("seg_reduce", "row_update", "reduce_update"),
+    "backward": ("seg_reduce", "row_update"),
 }
 
 

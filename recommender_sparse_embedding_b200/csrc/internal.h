@@ -42,6 +42,9 @@ constexpr size_t kCtlZeroBytes = offsetof(SortCtl, active);
 constexpr int kMaxSplitters = 1024;       // distinct splitters <= 1023
 constexpr int kMaxBucketSlots = 2048;     // buckets 0 .. 2 * nsplit (<= 2046)
 constexpr int kMaxSample = 8192;          // sample size of the largest batches
+// Segments (occurrences of one unique key) longer than this are summed by a
+// separate chunked reduction in the backward; the dedup marks their positions.
+constexpr int kShortSeg = 16;
 struct SsCtl {
   unsigned nsplit, nb, nbp, pad0;         // splitters, buckets, buckets rounded up to 32
   unsigned ticket_scan, ticket_local, pad1, pad2;
@@ -61,6 +64,8 @@ struct BatchDev {
   unsigned long long row_base;  // table's next_free when the lookup started
   unsigned int U;               // unique keys of the last lookup
   unsigned int n_new;           // new keys of the last lookup
+  unsigned int nlong;           // chunks of kShortSeg positions holding a long segment
+  unsigned int pad;
 };
 
 // ---------------------------------------------------------------- table
@@ -124,7 +129,9 @@ struct recis_batch {
   int32_t* seg_of = nullptr;    // segment (unique index) of each sorted position
   uint32_t* svals = nullptr;    // occurrence index of each sorted position
   int32_t* seg_start = nullptr; // [U+1] first sorted position of each unique
-  int2* occ_info = nullptr;     // per occurrence: {gradient row b*F+f, bag length}
+  uint32_t* spos = nullptr;     // [capN] sorted position of each occurrence
+  int4* gsrc = nullptr;         // [capN] per sorted position: {gradient row, bag length, occurrence, 0}
+  int4* gfirst = nullptr;       // [capN] per unique key: the same, of one of its occurrences
   int32_t* chunk_bag = nullptr; // bag of each pool chunk's first occurrence
   int64_t capChunks = 0;
   cudaStream_t side = nullptr;  // bag preparation runs here, beside the dedup
@@ -135,6 +142,9 @@ struct recis_batch {
   int32_t* seg_counter = nullptr;  // [capN] last-arrival counters (self-resetting)
   int32_t* bag_counter = nullptr;  // [capBags]
   double* partials = nullptr;
+  float* gbuf = nullptr;          // [chunks][D] reduced gradients of long segments
+  int32_t* long_chunks = nullptr; // [chunks] chunks holding a long segment (sample-sort path)
+  int64_t capGbuf = 0;            // floats
   recis::BatchDev* bdev = nullptr;
   uint32_t epoch = 0;
   // the last lookup, for the backward

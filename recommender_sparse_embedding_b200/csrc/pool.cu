@@ -12,7 +12,8 @@
 // occurrence is found by a G-ary search over the bag offsets; later bag
 // boundaries come from a window of G bag ends held one per lane.
 // Outputs: pooled rows [B][F][D] (sum, or mean = sum / length), optional
-// unpooled rows [N][D], and the bag of every occurrence for the backward.
+// unpooled rows [N][D], and the gradient source of every occurrence for the
+// backward.
 // Empty bags are written as zeros by a grid-stride prologue.
 #include <climits>
 
@@ -36,7 +37,9 @@ struct PoolParams {
   const float* row_data;
   float* pooled;         // [B][F][D] or null
   float* unpooled;       // [N][D] or null
-  int2* occ_info;        // [N] {gradient row b*F+f, bag length} per occurrence
+  const uint32_t* spos;  // [N] sorted position of each occurrence
+  int4* gsrc;            // [N] per sorted position: {gradient row b*F+f, bag length, occurrence, 0}
+  int4* gfirst;          // [U] per unique key: the same, of one of its occurrences
   int32_t* chunk_bag;    // [nchunks] bag of each chunk's first occurrence
   double* partials;
   int32_t* counters;     // [nbags]
@@ -191,8 +194,13 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
             if (col < ncol) __stcs(dst + col, val[k][v]);
           }
         }
-        // for the backward: this occurrence's gradient row and bag length
-        if (g.lane == 0) p.occ_info[pos] = make_int2(cb * F + cf, cur_end - cur_start);
+        // for the backward: this occurrence's gradient source, by sorted
+        // position and by unique key
+        if (g.lane == 0) {
+          const int4 src = make_int4(cb * F + cf, cur_end - cur_start, pos, 0);
+          p.gsrc[__ldg(p.spos + pos)] = src;
+          p.gfirst[__ldg(p.inv + pos)] = src;
+        }
       }
     }
   }
@@ -243,7 +251,9 @@ static PoolParams pool_params(const LookupArgs& a, int64_t chunk) {
   p.row_data = reinterpret_cast<const float*>(t->rows.va);
   p.pooled = a.pooled_out;
   p.unpooled = a.unpooled_out;
-  p.occ_info = b->occ_info;
+  p.spos = b->spos;
+  p.gsrc = b->gsrc;
+  p.gfirst = b->gfirst;
   p.chunk_bag = b->chunk_bag;
   p.partials = b->partials;
   p.counters = b->bag_counter;

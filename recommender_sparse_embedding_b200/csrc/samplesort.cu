@@ -227,17 +227,21 @@ struct SsParams {
   int64_t* uniq;
   int64_t* rows;
   int32_t* inv;
+  uint32_t* spos;
   int32_t* seg_of;
   uint32_t* svals;
   int32_t* seg_start;
   BatchDev* bdev;
+  int32_t* long_chunks;     // chunks (kShortSeg positions) holding a long segment
   DevState* st;
   HostMirror* mirror;
 };
 
 // Per sorted position, written by ss_local: the bucket, the position's
-// segment within the bucket (1-based count of heads up to it), and for a head
-// whether its key is new and the 1-based count of new heads up to it.
+// segment within the bucket (1-based count of heads up to it), for a head
+// whether its key is new and the 1-based count of new heads up to it, and in
+// bit 63 whether the position's segment is longer than kShortSeg.
+constexpr uint64_t kMetaLong = 1ULL << 63;
 __device__ __forceinline__ uint64_t pack_meta(unsigned b, unsigned lh, unsigned lnew, bool head,
                                               bool isnew) {
   return ((uint64_t)b << 44) | ((uint64_t)head << 43) | ((uint64_t)isnew << 42) |
@@ -492,6 +496,8 @@ template <int NT, int CAP>
 struct LocalShared {
   uint64_t key[CAP];
   uint32_t idx[CAP];
+  uint32_t loc[CAP];    // per position: lh | lnew << 13 | head << 26 | new << 27
+  uint8_t hlong[CAP];   // per bucket-local segment: longer than kShortSeg
   unsigned long long warp[NT / 32];
   bool last;
 };
@@ -499,6 +505,7 @@ struct LocalShared {
 // Number heads and new keys of a sorted bucket (in shared memory, or in
 // global memory for an oversized one) in rounds of NT positions, write the
 // sorted keys and occurrences (from shared memory) and every position's meta.
+// A segment is long when the key 16 positions after its head is the same.
 template <int NT, int CAP>
 __device__ void block_number(const SsParams& p, LocalShared<NT, CAP>& sh, unsigned b, int64_t m,
                              int64_t off, bool in_smem) {
@@ -509,11 +516,16 @@ __device__ void block_number(const SsParams& p, LocalShared<NT, CAP>& sh, unsign
     unsigned f = 0;
     uint64_t u = 0;
     uint32_t occ = 0;
+    bool lng = false;
     if (i < m) {
       u = in_smem ? sh.key[i] : __ldcg(p.kb + off + i);
       occ = in_smem ? sh.idx[i] : __ldcg(p.vb + off + i);
       const uint64_t before = i == 0 ? 0 : (in_smem ? sh.key[i - 1] : __ldcg(p.kb + off + i - 1));
-      if (i == 0 || u != before) f = 1u | (__ldcg(p.pocc + occ) <= -2 ? 2u : 0u);
+      if (i == 0 || u != before) {
+        f = 1u | (__ldcg(p.pocc + occ) <= -2 ? 2u : 0u);
+        const int64_t j = i + kShortSeg;
+        lng = j < m && (in_smem ? sh.key[j] : __ldcg(p.kb + off + j)) == u;
+      }
     }
     unsigned long long tot;
     const unsigned long long ex =
@@ -524,14 +536,37 @@ __device__ void block_number(const SsParams& p, LocalShared<NT, CAP>& sh, unsign
       if (in_smem) {
         p.kb[off + i] = u;
         p.vb[off + i] = occ;
+        sh.loc[i] = lh | (ln << 13) | ((f & 1u) << 26) | ((f >> 1) << 27);
+        if (f & 1u) sh.hlong[lh - 1] = lng ? 1 : 0;
+      } else {
+        p.meta[off + i] = pack_meta(b, lh, ln, f & 1u, (f >> 1) != 0);
       }
-      p.meta[off + i] = pack_meta(b, lh, ln, f & 1u, (f >> 1) != 0);
     }
     carry += tot;
   }
   if (tid == 0) {
     p.ctl->hcnt[b] = (unsigned)(carry & 0xffffffffULL);
     p.ctl->ncnt[b] = (unsigned)(carry >> 32);
+  }
+  __syncthreads();
+  if (in_smem) {
+    for (int i = tid; i < m; i += NT) {
+      const uint32_t v = sh.loc[i];
+      const unsigned lh = v & 0x1fffu;
+      const uint64_t mt = pack_meta(b, lh, (v >> 13) & 0x1fffu, (v >> 26) & 1u, (v >> 27) & 1u);
+      p.meta[off + i] = mt | (sh.hlong[lh - 1] ? kMetaLong : 0ULL);
+    }
+  } else {
+    // oversized bucket (adversarial key order): a head of a long segment marks
+    // its positions
+    __threadfence_block();
+    for (int64_t i = tid; i < m; i += NT) {
+      const uint64_t u = __ldcg(p.kb + off + i);
+      if ((i == 0 || u != __ldcg(p.kb + off + i - 1)) && i + kShortSeg < m &&
+          __ldcg(p.kb + off + i + kShortSeg) == u) {
+        for (int64_t j = i; j < m && __ldcg(p.kb + off + j) == u; ++j) p.meta[off + j] |= kMetaLong;
+      }
+    }
   }
 }
 
@@ -557,8 +592,9 @@ __global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ Ss
       }
     } else if (b & 1u) {
       const bool isnew = __ldcg(p.pocc + __ldcg(p.vb + off)) <= -2;
+      const uint64_t lng = m > kShortSeg ? kMetaLong : 0ULL;
       for (int64_t i = tid; i < m; i += NT)
-        p.meta[off + i] = pack_meta(b, 1u, isnew ? 1u : 0u, i == 0, i == 0 && isnew);
+        p.meta[off + i] = pack_meta(b, 1u, isnew ? 1u : 0u, i == 0, i == 0 && isnew) | lng;
       if (tid == 0) {
         p.ctl->hcnt[b] = 1;
         p.ctl->ncnt[b] = isnew ? 1u : 0u;
@@ -601,6 +637,7 @@ __global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ Ss
     const unsigned long long U = carry & 0xffffffffULL, nnew = carry >> 32;
     p.bdev->U = (unsigned)U;
     p.bdev->n_new = (unsigned)nnew;
+    p.bdev->nlong = 0;
     unsigned long long nf = p.bdev->row_base + nnew;
     if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
     p.st->next_free = nf;
@@ -616,8 +653,10 @@ __global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ Ss
 struct FinishShared {
   int64_t init_key[kFinThreads * kFinItems];
   int32_t init_row[kFinThreads * kFinItems];
+  unsigned chunk_long;  // bit c: chunk c (kShortSeg positions) of this CTA holds a long segment
   int ninit;
 };
+static_assert(kSub / kShortSeg <= 32, "one bit per chunk of a finish CTA");
 
 // Flat pass over the sorted positions, kSub per CTA (position blk*kSub +
 // j*256 + t for item j of thread t): segment of every position from its
@@ -625,7 +664,10 @@ struct FinishShared {
 __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_constant__ SsParams p) {
   __shared__ FinishShared sh;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  if (tid == 0) sh.ninit = 0;
+  if (tid == 0) {
+    sh.ninit = 0;
+    sh.chunk_long = 0;
+  }
   __syncthreads();
   const int64_t q0 = (int64_t)blockIdx.x * kSub + tid;
   const uint64_t row_base = p.bdev->row_base;
@@ -644,12 +686,16 @@ __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_con
     const int64_t q = q0 + j * kFinThreads;
     if (q >= p.N) break;
     const uint64_t m = mt[j];
+    if (m >> 63) atomicOr(&sh.chunk_long, 1u << ((tid + j * kFinThreads) / kShortSeg));
     const unsigned b = (unsigned)(m >> 44) & 0xfffu;
     const unsigned lh = (unsigned)(m & 0x1fffffULL);
     const unsigned seg = __ldg(&p.ctl->hpre[b]) + lh - 1u;
     p.seg_of[q] = (int32_t)seg;
     p.svals[q] = occ[j];
-    if (occ[j] < (uint32_t)p.N) p.inv[occ[j]] = (int32_t)seg;
+    if (occ[j] < (uint32_t)p.N) {
+      p.inv[occ[j]] = (int32_t)seg;
+      p.spos[occ[j]] = (uint32_t)q;
+    }
     if ((m >> 43) & 1u) {
       const int64_t key = from_ukey(__ldcs(p.kb + q));
       int64_t row = __ldcg(p.pocc + occ[j]);
@@ -672,6 +718,18 @@ __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_con
       p.rows[seg] = row;
       p.seg_start[seg] = (int32_t)q;
     }
+  }
+  // chunks of this CTA holding a long segment, for the backward's reduction
+  __syncthreads();
+  if (w == 0) {
+    const bool has = (sh.chunk_long >> lane) & 1u;
+    const unsigned bal = __ballot_sync(0xffffffffu, has);
+    unsigned at = 0;
+    if (lane == 0 && bal) at = atomicAdd(&p.bdev->nlong, (unsigned)__popc(bal));
+    at = __shfl_sync(0xffffffffu, at, 0);
+    if (has)
+      p.long_chunks[at + __popc(bal & ((1u << lane) - 1u))] =
+          (int32_t)(blockIdx.x * (kSub / kShortSeg) + lane);
   }
   // the next call's candidate splitters: quantiles of this call's sorted keys
   if (blockIdx.x == 0) {
@@ -763,10 +821,12 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   p.uniq = b->uniq;
   p.rows = b->rows;
   p.inv = b->inv;
+  p.spos = b->spos;
   p.seg_of = b->seg_of;
   p.svals = b->svals;
   p.seg_start = b->seg_start;
   p.bdev = b->bdev;
+  p.long_chunks = b->long_chunks;
   p.st = t->dstate;
   p.mirror = t->mirror_dev;
 

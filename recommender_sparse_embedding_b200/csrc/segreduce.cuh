@@ -64,7 +64,7 @@ __device__ __forceinline__ float4 acc_round(const Acc4& a) {
 // segment calls this once with its partial; returns true in the group that
 // must finish the segment, with the full sum in acc.  Partials are fp64,
 // 32 bytes per column, two slots of D doubles per chunk.
-template <int G, int VPL>
+template <int G, int VPL, int NB = 1>
 __device__ __forceinline__ bool combine_split(const GroupCtx<G>& g, Acc4 (&acc)[VPL],
                                               double* partials, int32_t* counters, int64_t seg,
                                               int64_t chunk, bool first_of_chunk,
@@ -92,17 +92,31 @@ __device__ __forceinline__ bool combine_split(const GroupCtx<G>& g, Acc4 (&acc)[
   __threadfence();
 #pragma unroll
   for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
-  for (int64_t cc = c0; cc <= c1; ++cc) {
-    const int sl = (cc == c0 && seg_start != c0 * C) ? 1 : 0;
-    const double* src = partials + (cc * 2 + sl) * D;
+  // the partials in chunk order, NB chunks' loads in flight at a time
+  for (int64_t cb = c0; cb <= c1; cb += NB) {
+    double2 pa[NB][VPL], pb[NB][VPL];
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      const int col = g.lane + v * G;
-      if (col < ncol) {
-        const double2 a = __ldcg(reinterpret_cast<const double2*>(src) + 2 * col);
-        const double2 b = __ldcg(reinterpret_cast<const double2*>(src) + 2 * col + 1);
-        acc_add(acc[v], Acc4{a.x, a.y, b.x, b.y});
+    for (int t = 0; t < NB; ++t) {
+      const int64_t cc = cb + t;
+      const int sl = (cc == c0 && seg_start != c0 * C) ? 1 : 0;
+      const double* src = partials + (cc * 2 + sl) * D;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int col = g.lane + v * G;
+        if (cc <= c1 && col < ncol) {
+          pa[t][v] = __ldcg(reinterpret_cast<const double2*>(src) + 2 * col);
+          pb[t][v] = __ldcg(reinterpret_cast<const double2*>(src) + 2 * col + 1);
+        } else {
+          pa[t][v] = make_double2(0.0, 0.0);
+          pb[t][v] = make_double2(0.0, 0.0);
+        }
       }
+    }
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      if (cb + t > c1) break;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) acc_add(acc[v], Acc4{pa[t][v].x, pa[t][v].y, pb[t][v].x, pb[t][v].y});
     }
   }
   if (g.lane == 0) counters[seg] = 0;

@@ -370,7 +370,9 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
         (e = realloc_dev(b->svals, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->ss_meta, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_start, cap + 1, true)) != cudaSuccess ||
-        (e = realloc_dev(b->occ_info, cap, true)) != cudaSuccess ||
+        (e = realloc_dev(b->spos, cap, true)) != cudaSuccess ||
+        (e = realloc_dev(b->gsrc, cap, true)) != cudaSuccess ||
+        (e = realloc_dev(b->gfirst, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_counter, cap, true)) != cudaSuccess)
       return cuda_fail(e, "batch alloc");
     const int64_t st = (cap + kSortTile - 1) / kSortTile;
@@ -417,6 +419,13 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
     if ((e = realloc_dev(b->partials, cap, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
     b->capPartials = cap;
   }
+  const int64_t gneed = ((N + cu - 1) / cu + 1) * (int64_t)D;
+  if (gneed > b->capGbuf) {
+    const int64_t cap = gneed + gneed / 4;
+    if ((e = realloc_dev(b->gbuf, cap, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
+    if ((e = realloc_dev(b->long_chunks, cap / D + 1, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
+    b->capGbuf = cap;
+  }
   return RECIS_OK;
 }
 
@@ -437,10 +446,14 @@ static void batch_free(recis_batch* b) {
   cudaFree(b->seg_of);
   cudaFree(b->svals);
   cudaFree(b->seg_start);
-  cudaFree(b->occ_info);
+  cudaFree(b->spos);
+  cudaFree(b->gsrc);
+  cudaFree(b->gfirst);
   cudaFree(b->seg_counter);
   cudaFree(b->bag_counter);
   cudaFree(b->partials);
+  cudaFree(b->gbuf);
+  cudaFree(b->long_chunks);
   cudaFree(b->bdev);
   cudaFree(b->chunk_bag);
   if (b->side) cudaStreamDestroy(b->side);

@@ -96,6 +96,7 @@ struct UniqueParams {
   int64_t* uniq;
   int64_t* rows;
   int32_t* inv;
+  uint32_t* spos;           // [N] sorted position of each occurrence
   int32_t* seg_of;
   uint32_t* svals;
   int32_t* seg_start;
@@ -271,7 +272,10 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
     const int32_t seg = (int32_t)(hrun - 1);
     p.seg_of[pos] = seg;
     p.svals[pos] = v[j];
-    if (v[j] < (uint64_t)N) p.inv[v[j]] = seg;
+    if (v[j] < (uint64_t)N) {
+      p.inv[v[j]] = seg;
+      p.spos[v[j]] = (uint32_t)pos;
+    }
   }
   if (tile == gridDim.x - 1 && tid == 0) {
     const unsigned long long U = Hx + tH, nnew = Nx + tN;
@@ -341,6 +345,7 @@ cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cuda
   p.uniq = b->uniq;
   p.rows = b->rows;
   p.inv = b->inv;
+  p.spos = b->spos;
   p.seg_of = b->seg_of;
   p.svals = b->svals;
   p.seg_start = b->seg_start;

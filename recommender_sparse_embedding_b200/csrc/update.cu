@@ -1,50 +1,203 @@
-// update.cu -- backward: per-unique gradient reduction fused with the sparse
+// update.cu -- backward: per-unique gradient reduction and the sparse
 // optimiser row update (RecIS README, Key optimisations > Operator
 // implementation: reductions merged at warp level rather than by per-element
 // atomics; > Efficient dynamic embedding: optimiser state stored beside the
 // parameters in the EmbeddingBlocks).
 //
-// The sorted positions of the dedup are already grouped by unique key, so the
-// backward is a segmented reduction over sorted order (segreduce.cuh).  For
-// sorted position q (occurrence i = vals[q], its bag from the forward) the term is
-//   grad_pooled[b][f] * (1 or 1/length) + grad_unpooled[i];
-// a group sums the terms of each unique key in its chunk in position order and
-// then applies Adagrad or Adam to that key's row [emb | state] in place.  Keys
-// whose occurrences cross chunk boundaries are combined by the last-arriving
-// group, which also applies the update, so every touched row is updated
-// exactly once.
+// The dedup left the sorted positions grouped by unique key: segment u spans
+// sorted positions seg_start[u] .. seg_start[u+1]-1, position q holds
+// occurrence vals[q].  The gradient of u is
+//   g(u) = sum over its positions of grad_pooled[bag] * (1 or 1/length)
+//          + grad_unpooled[occurrence],
+// summed in fp64 in position order and rounded once to fp32.  Two launches:
+//   seg_reduce  segments longer than kShortSeg (hot keys) are cut into
+//               chunks of kChunk positions; each lane group sums its chunk's
+//               part of a segment into an fp64 partial and the group that
+//               arrives last (ticket per segment) adds the partials in chunk
+//               order and stores g(u) in gbuf at row seg_start[u] / kChunk (a
+//               long segment is the only long one starting in its chunk).
+//   row_update  one lane group per unique key loads the row [emb | state],
+//               sums the key's gradient terms itself when the segment is
+//               short (all loads issued before the sum) or reads gbuf, and
+//               applies Adagrad or Adam in place.
+// No float atomics anywhere; the result does not depend on scheduling.
 #include "segreduce.cuh"
 
 namespace recis {
 
+constexpr int kChunk = 16;  // seg_reduce positions per group (<= kShortSeg + 1)
+static_assert(kChunk <= kShortSeg + 1, "a chunk must hold at most one long segment start");
+static_assert(kChunk == kShortSeg, "the dedup lists long chunks of kShortSeg positions");
+
 struct UpdateParams {
   int64_t N;
-  int64_t B;
-  int32_t F;
-  int32_t ncol;
-  int64_t C;
-  int64_t nchunks;
+  int32_t ncol;             // D / 4
   int32_t mean;
   int32_t row_floats;
-  const uint32_t* vals;     // sorted occurrence indices
+  int64_t nchunks;          // seg_reduce chunks
+  const int4* gsrc;         // [N] per sorted position: {gradient row, bag length, occurrence, 0}
+  const int4* gfirst;       // [U] per unique key: gsrc of one of its occurrences
+  const uint64_t* meta;     // [N] per sorted position, bit 63: long segment (null: use seg_start)
+  const int32_t* long_chunks;  // chunks holding a long segment, bdev->nlong of them (or null)
   const int32_t* seg_of;    // [N] sorted position -> unique index
   const int32_t* seg_start; // [U+1]
-  const int2* occ_info;     // [N] {gradient row, bag length}
-  const int64_t* offs;      // bag offsets
   const int64_t* rows;      // [U]
+  const BatchDev* bdev;     // U of the lookup
   const float* gp;          // grad_pooled [B][F][D] or null
   const float* gu;          // grad_unpooled [N][D] or null
+  float* gbuf;              // [nchunks][D] reduced gradients of long segments
   float* row_data;
-  double* partials;
-  int32_t* counters;        // [U]
+  double* partials;         // [nchunks][2][D]
+  int32_t* counters;        // [U] last-arrival tickets (self-resetting)
   // optimiser
   float lr;        // Adagrad: lr; Adam: lr / (1 - beta1^t)
   float eps;
   float beta1, beta2;
   float omb1, omb2;  // 1 - beta1, 1 - beta2 (formed in double, rounded once)
-  float sqrt_bc2;  // Adam: sqrt(1 - beta2^t)
+  float sqrt_bc2;    // Adam: sqrt(1 - beta2^t)
 };
 
+// gradient rows each lane loads before adding (fewer for wide rows: registers)
+template <int VPL>
+constexpr int kRowsInFlight = VPL >= 4 ? 1 : (VPL == 2 ? 2 : 4);
+
+// Gradient source of one position: row of grad_pooled, its scale (1, or
+// 1/length for mean pooling) and the occurrence (row of grad_unpooled).
+struct Src {
+  int32_t gr;
+  int32_t occ;
+  double scale;
+};
+
+__device__ __forceinline__ Src make_src(const UpdateParams& p, int4 v) {
+  Src s;
+  s.gr = v.x;
+  s.occ = v.z;
+  s.scale = p.mean ? 1.0 / (double)v.y : 1.0;
+  return s;
+}
+
+// Adds the terms of `count` (<= K) positions whose sources sit in lanes
+// first .. first+count-1 to acc; every lane loads its 16-byte columns of all
+// the rows before adding.  GP / GU: pooled / unpooled gradient present.
+template <int G, int VPL, int K, bool GP, bool GU>
+__device__ __forceinline__ void add_terms(const GroupCtx<G>& g, const UpdateParams& p, const Src& my,
+                                          int first, int count, Acc4 (&acc)[VPL]) {
+  const int64_t D = (int64_t)p.ncol * 4;
+  float4 tp[K][VPL], tu[K][VPL];
+  double sc[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const bool valid = k < count;
+    const int src = valid ? first + k : first;
+    const int32_t gr = GP ? g.bcast(my.gr, src) : 0;
+    const int32_t oc = GU ? g.bcast(my.occ, src) : 0;
+    sc[k] = (GP && p.mean) ? g.bcast(my.scale, src) : 1.0;
+    const float4* gps = reinterpret_cast<const float4*>(p.gp + (int64_t)gr * D);
+    const float4* gus = reinterpret_cast<const float4*>(p.gu + (int64_t)oc * D);
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const int col = g.lane + v * G;
+      const bool ok = valid && col < p.ncol;
+      tp[k][v] = (GP && ok) ? __ldcs(gps + col) : f4_zero();
+      tu[k][v] = (GU && ok) ? __ldcs(gus + col) : f4_zero();
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      // one term per position: pooled gradient * scale + unpooled gradient
+      acc[v].x += (GP ? (double)tp[k][v].x * sc[k] : 0.0) + (GU ? (double)tu[k][v].x : 0.0);
+      acc[v].y += (GP ? (double)tp[k][v].y * sc[k] : 0.0) + (GU ? (double)tu[k][v].y : 0.0);
+      acc[v].z += (GP ? (double)tp[k][v].z * sc[k] : 0.0) + (GU ? (double)tu[k][v].z : 0.0);
+      acc[v].w += (GP ? (double)tp[k][v].w * sc[k] : 0.0) + (GU ? (double)tu[k][v].w : 0.0);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ seg_reduce
+// One group per chunk of kChunk sorted positions.  Lanes resolve G positions
+// at a time: the long-segment mark (or, without marks, the segment's bounds),
+// the segment and the gradient source; positions of short segments are
+// skipped, so a chunk without a long segment ends after one load.  A chunk
+// meets at most two long segments (one ending, one starting); each gets one
+// partial per chunk, in slot 0 if it starts at or before the chunk's first
+// position, else slot 1.
+template <int G, int VPL, bool GP, bool GU>
+__device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateParams& p, int64_t chunk) {
+  const int64_t D = (int64_t)p.ncol * 4;
+  const int64_t p0 = chunk * kChunk;
+  const int64_t p1 = p0 + kChunk < p.N ? p0 + kChunk : p.N;
+  Acc4 acc[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
+  int32_t cur = -1;
+  int64_t cst = 0, cen = 0;
+  auto flush = [&]() {
+    if (combine_split<G, VPL, VPL >= 4 ? 1 : 4 / VPL>(g, acc, p.partials, p.counters, cur, chunk,
+                                                       cst <= p0, cst, cen, kChunk, p.ncol)) {
+      float4* dst = reinterpret_cast<float4*>(p.gbuf + (cst / kChunk) * D);
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int col = g.lane + v * G;
+        if (col < p.ncol) __stcg(dst + col, acc_round(acc[v]));
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
+  };
+  for (int64_t sub = p0; sub < p1; sub += G) {
+    const int64_t q = sub + g.lane;
+    bool maybe = q < p1;
+    if (maybe && p.meta) maybe = (__ldg(p.meta + q) >> 63) != 0;
+    if (!g.ballot(maybe)) continue;
+    int32_t seg = -1, st = 0, en = 0;
+    Src s{0, 0, 1.0};
+    if (maybe) {
+      seg = __ldg(p.seg_of + q);
+      s = make_src(p, __ldg(p.gsrc + q));
+      st = __ldg(p.seg_start + seg);
+      en = __ldg(p.seg_start + seg + 1);
+    }
+    const bool is_long = maybe && en - st > kShortSeg;
+    unsigned rest = g.ballot(is_long);
+    while (rest) {
+      const int a = __ffs(rest) - 1;
+      const int32_t sg = g.bcast(seg, a);
+      const unsigned same = g.ballot(is_long && seg == sg);  // lanes a .. a+cnt-1
+      const int cnt = __popc(same);
+      if (sg != cur) {
+        if (cur >= 0) flush();
+        cur = sg;
+        cst = g.bcast(st, a);
+        cen = g.bcast(en, a);
+      }
+      constexpr int K = kRowsInFlight<VPL>;
+      for (int k0 = 0; k0 < cnt; k0 += K)
+        add_terms<G, VPL, K, GP, GU>(g, p, s, a + k0, cnt - k0 < K ? cnt - k0 : K, acc);
+      rest &= ~same;
+    }
+  }
+  if (cur >= 0) flush();
+}
+
+// With the dedup's list of chunks holding a long segment, a persistent grid
+// of groups walks the list; without it, one group per chunk.
+template <int G, int VPL, bool GP, bool GU>
+__global__ void __launch_bounds__(256, 3) seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
+  const GroupCtx<G> g;
+  const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  if (p.long_chunks) {
+    const int64_t n = (int64_t)p.bdev->nlong;
+    const int64_t groups = (int64_t)gridDim.x * blockDim.x / G;
+    for (int64_t i = gid; i < n; i += groups) reduce_chunk<G, VPL, GP, GU>(g, p, __ldg(p.long_chunks + i));
+  } else if (gid < p.nchunks) {
+    reduce_chunk<G, VPL, GP, GU>(g, p, gid);
+  }
+}
+
+// ------------------------------------------------------------------ row_update
 // Row data of one unique key: emb and the optimiser state, VPL 16-byte
 // columns per lane.
 template <int VPL, bool ADAM>
@@ -61,17 +214,20 @@ __device__ __forceinline__ void load_row(const GroupCtx<G>& g, const UpdateParam
   for (int v = 0; v < VPL; ++v) {
     const int col = g.lane + v * G;
     if (row >= 0 && col < p.ncol) {
-      r.w[v] = __ldcg(reinterpret_cast<const float4*>(base) + col);
-      r.s1[v] = __ldcg(reinterpret_cast<const float4*>(base + D) + col);
-      if (ADAM) r.s2[v] = __ldcg(reinterpret_cast<const float4*>(base + 2 * D) + col);
+      r.w[v] = __ldcs(reinterpret_cast<const float4*>(base) + col);
+      r.s1[v] = __ldcs(reinterpret_cast<const float4*>(base + D) + col);
+      if (ADAM) r.s2[v] = __ldcs(reinterpret_cast<const float4*>(base + 2 * D) + col);
     }
   }
 }
 
+// g rounded once to fp32, then the optimiser in fp32 in the order written:
+//   Adagrad  acc += g^2;  w -= lr g / (sqrt(acc) + eps)
+//   Adam     m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;
+//            w -= (lr / (1-b1^t)) m / (sqrt(v) / sqrt(1-b2^t) + eps)
 template <int G, int VPL, bool ADAM>
-__device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateParams& p,
-                                             int64_t row, const RowRegs<VPL, ADAM>& r,
-                                             const Acc4 (&grad)[VPL]) {
+__device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateParams& p, int64_t row,
+                                             const RowRegs<VPL, ADAM>& r, const Acc4 (&grad)[VPL]) {
   if (row < 0) return;
   float* base = p.row_data + row * p.row_floats;
   const int D = p.ncol * 4;
@@ -99,175 +255,115 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
         a1[e] = m;
         a2[e] = vv;
       }
-      __stcg(reinterpret_cast<float4*>(base + 2 * D) + col, make_float4(a2[0], a2[1], a2[2], a2[3]));
+      __stcs(reinterpret_cast<float4*>(base + 2 * D) + col, make_float4(a2[0], a2[1], a2[2], a2[3]));
     }
-    __stcg(reinterpret_cast<float4*>(base + D) + col, make_float4(a1[0], a1[1], a1[2], a1[3]));
-    __stcg(reinterpret_cast<float4*>(base) + col, make_float4(ww[0], ww[1], ww[2], ww[3]));
+    __stcs(reinterpret_cast<float4*>(base + D) + col, make_float4(a1[0], a1[1], a1[2], a1[3]));
+    __stcs(reinterpret_cast<float4*>(base) + col, make_float4(ww[0], ww[1], ww[2], ww[3]));
   }
 }
 
-// One group per chunk of C sorted positions.  Index work is lane-parallel:
-// for G positions at a time each lane resolves one position (sorted position
-// -> occurrence -> bag -> gradient row), then the group streams the gradient
-// rows RB at a time, every lane loading its 16-byte column of each.  The
-// chunk's unique keys are consecutive segment ids s0..s_last; their row
-// offsets are fetched one per lane, and the row of the next key is loaded
-// while the current key's terms are summed, so the epilogue rarely waits.
-template <int G, int VPL, bool ADAM>
-__global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
-    update_kernel(const __grid_constant__ UpdateParams p) {
-  constexpr int RB = VPL >= 2 ? 1 : 2;  // gradient rows in flight per lane
+// One group of G lanes per unique key u (U from the lookup).  The first
+// loads (segment bounds, row offset, and the source of a singleton's one
+// occurrence) are independent; the row loads go out next, together with the
+// gradient rows of a singleton.  A longer short segment resolves its
+// positions' sources one per lane and loads several rows at a time; a long
+// segment's sum is read from gbuf.
+template <int G, int VPL, bool ADAM, bool GP, bool GU>
+__global__ void __launch_bounds__(256, VPL >= 2 ? 2 : 4) row_update_kernel(const __grid_constant__ UpdateParams p) {
   const GroupCtx<G> g;
-  const int64_t chunk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
-  if (chunk >= p.nchunks) return;
+  const int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  if (u >= (int64_t)p.bdev->U) return;
   const int64_t D = (int64_t)p.ncol * 4;
-  const uint32_t* vals = p.vals;
-  const int64_t p0 = chunk * p.C;
-  const int64_t p1 = p0 + p.C < p.N ? p0 + p.C : p.N;
-  const int32_t s0 = __ldg(p.seg_of + p0);
-  const int32_t s_last = __ldg(p.seg_of + p1 - 1);
-  const bool s0_starts_here = __ldg(p.seg_start + s0) == p0;
-  const int32_t after = p1 < p.N ? __ldg(p.seg_of + p1) : -1;
-  int32_t wbase = s0;
-  int64_t wrow = (s0 + g.lane <= s_last) ? __ldg(p.rows + s0 + g.lane) : -1;
-
-  int32_t cur = s0;
-  bool cur_starts_here = s0_starts_here;
-  int64_t cur_row = g.bcast(wrow, 0);
-  RowRegs<VPL, ADAM> rcur, rnext;
-  load_row<G, VPL, ADAM>(g, p, cur_row, rcur);
-  int64_t next_row = -1;
-  auto fetch_next = [&]() {  // row of cur + 1, if it belongs to this chunk
-    next_row = -1;
-    if (cur + 1 <= s_last) {
-      if (cur + 1 - wbase >= G) {
-        wbase = cur + 1;
-        wrow = (wbase + g.lane <= s_last) ? __ldg(p.rows + wbase + g.lane) : -1;
-      }
-      next_row = g.bcast(wrow, cur + 1 - wbase);
-      load_row<G, VPL, ADAM>(g, p, next_row, rnext);
-    }
-  };
-  fetch_next();
-
+  const int64_t s0 = __ldg(p.seg_start + u), s1 = __ldg(p.seg_start + u + 1);
+  const int64_t row = __ldg(p.rows + u);
+  const int4 first = __ldg(p.gfirst + u);
+  RowRegs<VPL, ADAM> r;
+  load_row<G, VPL, ADAM>(g, p, row, r);
   Acc4 acc[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
-
-  auto finish = [&](bool ends_here) {
-    if (cur_starts_here && ends_here) {
-      apply_update<G, VPL, ADAM>(g, p, cur_row, rcur, acc);
-    } else {
-      const int64_t st = p.seg_start[cur], en = p.seg_start[cur + 1];
-      if (combine_split<G, VPL>(g, acc, p.partials, p.counters, cur, chunk, cur == s0, st, en,
-                                p.C, p.ncol))
-        apply_update<G, VPL, ADAM>(g, p, cur_row, rcur, acc);
-    }
+  const int len = (int)(s1 - s0);
+  constexpr int K = kRowsInFlight<VPL>;
+  if (len == 1) {
+    // every lane holds the same source; lane 0's is broadcast
+    add_terms<G, VPL, 1, GP, GU>(g, p, make_src(p, first), 0, 1, acc);
+  } else if (len > kShortSeg) {
+    const float4* src = reinterpret_cast<const float4*>(p.gbuf + (s0 / kChunk) * D);
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
-  };
-
-  for (int64_t sub = p0; sub < p1; sub += G) {
-    // lane-parallel resolution of positions sub .. sub+G-1
-    const int64_t q = sub + g.lane;
-    const bool ok = q < p1;
-    const int32_t my_seg = ok ? __ldg(p.seg_of + q) : -1;
-    const int32_t my_occ = ok ? (int32_t)__ldg(vals + q) : -1;
-    int32_t my_gprow = -1;
-    double my_scale = 1.0;
-    if (ok && p.gp) {
-      const int2 oi = __ldg(p.occ_info + my_occ);
-      my_gprow = oi.x;
-      if (p.mean) my_scale = 1.0 / (double)oi.y;
-    }
-    const int m = (int)((p1 - sub) < G ? (p1 - sub) : G);
-    for (int kb = 0; kb < m; kb += RB) {
-      float4 tp[RB][VPL], tu[RB][VPL];
-      int32_t sg[RB];
-      double sc[RB];
-#pragma unroll
-      for (int k = 0; k < RB; ++k) {
-        const int src = kb + k < m ? kb + k : 0;
-        const int32_t gr = g.bcast(my_gprow, src);
-        const int32_t oc = g.bcast(my_occ, src);
-        sg[k] = g.bcast(my_seg, src);
-        sc[k] = p.mean ? g.bcast(my_scale, src) : 1.0;
-        const bool valid = kb + k < m;
-        const float4* gps = reinterpret_cast<const float4*>(p.gp + (int64_t)gr * D);
-        const float4* gus = reinterpret_cast<const float4*>(p.gu + (int64_t)oc * D);
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-          const int col = g.lane + v * G;
-          tp[k][v] = (valid && col < p.ncol && gr >= 0) ? __ldcs(gps + col) : f4_zero();
-          tu[k][v] = (valid && col < p.ncol && p.gu) ? __ldcs(gus + col) : f4_zero();
-        }
+    for (int v = 0; v < VPL; ++v) {
+      const int col = g.lane + v * G;
+      if (col < p.ncol) {
+        const float4 t = __ldcg(src + col);
+        acc[v] = Acc4{(double)t.x, (double)t.y, (double)t.z, (double)t.w};
       }
-#pragma unroll
-      for (int k = 0; k < RB; ++k) {
-        if (kb + k >= m) break;
-        if (sg[k] != cur) {
-          finish(true);
-          cur = sg[k];
-          cur_starts_here = true;
-          cur_row = next_row;
-          rcur = rnext;
-          fetch_next();
-        }
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-          acc[v].x += (double)tp[k][v].x * sc[k] + (double)tu[k][v].x;
-          acc[v].y += (double)tp[k][v].y * sc[k] + (double)tu[k][v].y;
-          acc[v].z += (double)tp[k][v].z * sc[k] + (double)tu[k][v].z;
-          acc[v].w += (double)tp[k][v].w * sc[k] + (double)tu[k][v].w;
-        }
-      }
+    }
+  } else {
+    for (int base = 0; base < len; base += G) {
+      const int m = len - base < G ? len - base : G;
+      Src s{0, 0, 1.0};
+      if (g.lane < m) s = make_src(p, __ldg(p.gsrc + s0 + base + g.lane));
+      for (int k0 = 0; k0 < m; k0 += K)
+        add_terms<G, VPL, K, GP, GU>(g, p, s, k0, m - k0 < K ? m - k0 : K, acc);
     }
   }
-  finish(after != cur);
+  apply_update<G, VPL, ADAM>(g, p, row, r, acc);
 }
 
-template <int G, int VPL>
-static cudaError_t launch_update_t(const UpdateParams& p, bool adam, cudaStream_t s) {
-  const int64_t threads = p.nchunks * G;
-  int64_t blocks = (threads + 255) / 256;
+// ------------------------------------------------------------------ host
+int group_lanes_for(int D);
+
+int64_t update_chunk_for(int64_t, int) { return kChunk; }
+
+template <int G, int VPL, bool GP, bool GU>
+static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t ucap, cudaStream_t s) {
+  {
+    int64_t blocks = (p.nchunks * G + 255) / 256;
+    if (p.long_chunks && blocks > 3 * kSMs) blocks = 3 * kSMs;
+    if (blocks < 1) blocks = 1;
+    LaunchScope ls("seg_reduce", s);
+    seg_reduce_kernel<G, VPL, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  int64_t blocks = (ucap * G + 255) / 256;
   if (blocks < 1) blocks = 1;
-  LaunchScope ls("reduce_update", s);
+  LaunchScope ls("row_update", s);
   if (adam)
-    update_kernel<G, VPL, true><<<(unsigned)blocks, 256, 0, s>>>(p);
+    row_update_kernel<G, VPL, true, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
   else
-    update_kernel<G, VPL, false><<<(unsigned)blocks, 256, 0, s>>>(p);
+    row_update_kernel<G, VPL, false, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
-int group_lanes_for(int D);
-
-int64_t update_chunk_for(int64_t N, int D) {
-  const int G = group_lanes_for(D);
-  int64_t C = 8;
-  while (C < 256 && (N / (C * 2)) * G >= (int64_t)kSMs * 2048) C *= 2;
-  return C;
+template <int G, int VPL>
+static cudaError_t launch_update_t(const UpdateParams& p, bool adam, int64_t ucap, cudaStream_t s) {
+  if (p.gp && p.gu) return launch_update_g<G, VPL, true, true>(p, adam, ucap, s);
+  if (p.gp) return launch_update_g<G, VPL, true, false>(p, adam, ucap, s);
+  if (p.gu) return launch_update_g<G, VPL, false, true>(p, adam, ucap, s);
+  return launch_update_g<G, VPL, false, false>(p, adam, ucap, s);  // touched rows, zero gradient
 }
 
 cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pooled,
-                          const float* grad_unpooled, int64_t chunk, float lr_t, float sqrt_bc2,
+                          const float* grad_unpooled, int64_t, float lr_t, float sqrt_bc2,
                           cudaStream_t s) {
   UpdateParams p;
   p.N = b->N;
-  p.B = b->B;
-  p.F = b->F;
   p.ncol = t->D / 4;
-  p.C = chunk;
-  p.nchunks = (b->N + chunk - 1) / chunk;
   p.mean = b->combiner == RECIS_MEAN;
   p.row_floats = t->row_floats;
-  p.vals = b->svals;
+  p.nchunks = (b->N + kChunk - 1) / kChunk;
+  p.gsrc = b->gsrc;
+  p.gfirst = b->gfirst;
+  // long-segment marks and the long-chunk list come from the sample-sort dedup
+  p.meta = b->N <= kSampleSortMaxN ? b->ss_meta : nullptr;
+  p.long_chunks = b->N <= kSampleSortMaxN ? b->long_chunks : nullptr;
   p.seg_of = b->seg_of;
   p.seg_start = b->seg_start;
-  p.occ_info = b->occ_info;
-  p.offs = b->bag_offsets;
   p.rows = b->rows;
+  p.bdev = b->bdev;
   p.gp = grad_pooled;
   p.gu = grad_unpooled;
+  p.gbuf = b->gbuf;
   p.row_data = reinterpret_cast<float*>(t->rows.va);
   p.partials = b->partials;
   p.counters = b->seg_counter;
@@ -278,18 +374,19 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.omb1 = (float)(1.0 - t->cfg.beta1);
   p.omb2 = (float)(1.0 - t->cfg.beta2);
   p.sqrt_bc2 = sqrt_bc2;
-  if (p.nchunks == 0) return cudaSuccess;
+  if (p.N == 0) return cudaSuccess;
   const bool adam = t->cfg.optimizer == RECIS_ADAM;
+  const int64_t ucap = b->N;  // U <= N; groups past U return at once
   const int ncol = p.ncol;
-  if (ncol <= 1) return launch_update_t<1, 1>(p, adam, s);
-  if (ncol <= 2) return launch_update_t<2, 1>(p, adam, s);
-  if (ncol <= 4) return launch_update_t<4, 1>(p, adam, s);
-  if (ncol <= 8) return launch_update_t<8, 1>(p, adam, s);
-  if (ncol <= 16) return launch_update_t<16, 1>(p, adam, s);
-  if (ncol <= 32) return launch_update_t<32, 1>(p, adam, s);
-  if (ncol <= 64) return launch_update_t<32, 2>(p, adam, s);
-  if (ncol <= 128) return launch_update_t<32, 4>(p, adam, s);
-  return launch_update_t<32, 8>(p, adam, s);
+  if (ncol <= 1) return launch_update_t<1, 1>(p, adam, ucap, s);
+  if (ncol <= 2) return launch_update_t<2, 1>(p, adam, ucap, s);
+  if (ncol <= 4) return launch_update_t<4, 1>(p, adam, ucap, s);
+  if (ncol <= 8) return launch_update_t<8, 1>(p, adam, ucap, s);
+  if (ncol <= 16) return launch_update_t<16, 1>(p, adam, ucap, s);
+  if (ncol <= 32) return launch_update_t<32, 1>(p, adam, ucap, s);
+  if (ncol <= 64) return launch_update_t<32, 2>(p, adam, ucap, s);
+  if (ncol <= 128) return launch_update_t<32, 4>(p, adam, ucap, s);
+  return launch_update_t<32, 8>(p, adam, ucap, s);
 }
 
 }  // namespace recis
