@@ -58,8 +58,8 @@ struct UpdateParams {
 };
 
 // gradient rows each lane loads before adding (fewer for wide rows: registers)
-template <int VPL>
-constexpr int kRowsInFlight = VPL >= 4 ? 1 : (VPL == 2 ? 2 : 4);
+template <int VPL, bool BOTH = false>
+constexpr int kRowsInFlight = VPL >= 4 ? 1 : ((VPL == 2 ? 2 : 4) / (BOTH ? 2 : 1));
 
 // Gradient source of one position: row of grad_pooled, its scale (1, or
 // 1/length for mean pooling) and the occurrence (row of grad_unpooled).
@@ -173,7 +173,7 @@ __device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateP
         cst = g.bcast(st, a);
         cen = g.bcast(en, a);
       }
-      constexpr int K = kRowsInFlight<VPL>;
+      constexpr int K = kRowsInFlight<VPL, GP && GU>;
       for (int k0 = 0; k0 < cnt; k0 += K)
         add_terms<G, VPL, K, GP, GU>(g, p, s, a + k0, cnt - k0 < K ? cnt - k0 : K, acc);
       rest &= ~same;
@@ -185,7 +185,7 @@ __device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateP
 // With the dedup's list of chunks holding a long segment, a persistent grid
 // of groups walks the list; without it, one group per chunk.
 template <int G, int VPL, bool GP, bool GU>
-__global__ void __launch_bounds__(256, 3) seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
+__global__ void __launch_bounds__(256, VPL >= 2 ? 2 : 3) seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
   const GroupCtx<G> g;
   const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
   if (p.long_chunks) {
@@ -268,27 +268,31 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
 // gradient rows of a singleton.  A longer short segment resolves its
 // positions' sources one per lane and loads several rows at a time; a long
 // segment's sum is read from gbuf.
-template <int G, int VPL, bool ADAM, bool GP, bool GU>
-__global__ void __launch_bounds__(256, VPL >= 2 ? 2 : 4) row_update_kernel(const __grid_constant__ UpdateParams p) {
-  const GroupCtx<G> g;
-  const int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
-  if (u >= (int64_t)p.bdev->U) return;
+// Gradient of key (s0, s1, first) into acc: a singleton's one term (its
+// pooled gradient row already staged in shared memory when staged != null),
+// a long segment's sum from gbuf, else the terms gathered here.
+template <int G, int VPL, bool GP, bool GU>
+__device__ __forceinline__ void key_grad(const GroupCtx<G>& g, const UpdateParams& p, int32_t s0,
+                                         int32_t s1, int4 first, const float4* staged, int stride,
+                                         Acc4 (&acc)[VPL]) {
   const int64_t D = (int64_t)p.ncol * 4;
-  const int64_t s0 = __ldg(p.seg_start + u), s1 = __ldg(p.seg_start + u + 1);
-  const int64_t row = __ldg(p.rows + u);
-  const int4 first = __ldg(p.gfirst + u);
-  RowRegs<VPL, ADAM> r;
-  load_row<G, VPL, ADAM>(g, p, row, r);
-  Acc4 acc[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
-  const int len = (int)(s1 - s0);
-  constexpr int K = kRowsInFlight<VPL>;
+  const int len = s1 - s0;
+  constexpr int K = kRowsInFlight<VPL, GP && GU>;
   if (len == 1) {
-    // every lane holds the same source; lane 0's is broadcast
-    add_terms<G, VPL, 1, GP, GU>(g, p, make_src(p, first), 0, 1, acc);
+    if (staged) {
+      const double sc = p.mean ? 1.0 / (double)first.y : 1.0;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const float4 t = staged[v * stride];
+        acc[v] = Acc4{(double)t.x * sc, (double)t.y * sc, (double)t.z * sc, (double)t.w * sc};
+      }
+    } else {
+      add_terms<G, VPL, 1, GP, GU>(g, p, make_src(p, first), 0, 1, acc);
+    }
   } else if (len > kShortSeg) {
-    const float4* src = reinterpret_cast<const float4*>(p.gbuf + (s0 / kChunk) * D);
+    const float4* src = reinterpret_cast<const float4*>(p.gbuf + (int64_t)(s0 / kChunk) * D);
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       const int col = g.lane + v * G;
@@ -306,7 +310,121 @@ __global__ void __launch_bounds__(256, VPL >= 2 ? 2 : 4) row_update_kernel(const
         add_terms<G, VPL, K, GP, GU>(g, p, s, k0, m - k0 < K ? m - k0 : K, acc);
     }
   }
-  apply_update<G, VPL, ADAM>(g, p, row, r, acc);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Indices of one key: segment bounds, row offset (positions and rows fit in
+// 32 bits: N < 2^31, rows < 2^31) and the source of one of its occurrences.
+struct KeyIdx {
+  int32_t s0, s1, row;
+  int4 first;
+};
+
+__device__ __forceinline__ KeyIdx key_idx(const UpdateParams& p, int64_t u) {
+  KeyIdx k;
+  k.s0 = __ldg(p.seg_start + u);
+  k.s1 = __ldg(p.seg_start + u + 1);
+  k.row = (int32_t)__ldg(p.rows + u);
+  k.first = __ldg(p.gfirst + u);
+  return k;
+}
+
+// A persistent grid of G-lane groups walks the unique keys u = gid, gid +
+// groups, ... (U from the lookup), two keys deep: while key u is updated, the
+// next key's row [emb | state] (and a singleton's pooled gradient row) are in
+// flight into shared memory by cp.async, and the key after that has its
+// indices loaded.  Each lane copies and reads back only its own 16-byte
+// columns, so no barrier is needed beyond the thread's own wait.  Other keys'
+// gradients (repeated keys, long segments, unpooled gradients) are gathered
+// while the key is updated.
+template <int G, int VPL, bool ADAM, bool GP, bool GU>
+__global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constant__ UpdateParams p) {
+  constexpr int NR = ADAM ? 3 : 2;             // row slices: emb, state(s)
+  constexpr int NS = NR * VPL + VPL;           // staged float4 per thread per stage
+  extern __shared__ float4 s_stage[];          // [2][NS][blockDim]
+  const GroupCtx<G> g;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int64_t groups = (int64_t)gridDim.x * blockDim.x / G;
+  const int64_t U = (int64_t)p.bdev->U;
+  const int D = p.ncol * 4;
+  int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  if (u >= U) return;
+  auto slot = [&](int stage, int sl) -> float4* { return s_stage + ((stage * NS + sl) * nt + tid); };
+  auto issue = [&](int stage, const KeyIdx& k) {
+    if (k.row < 0) return;
+    const float* base = p.row_data + (int64_t)k.row * p.row_floats;
+    const bool stage_grad = GP && !GU && k.s1 - k.s0 == 1;
+    const float* gsrc_row = p.gp + (int64_t)k.first.x * D;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const int col = g.lane + v * G;
+      if (col < p.ncol) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) cp_async16(slot(stage, r * VPL + v), base + r * D + 4 * col);
+        if (stage_grad) cp_async16(slot(stage, NR * VPL + v), gsrc_row + 4 * col);
+      }
+    }
+  };
+  KeyIdx cur = key_idx(p, u);
+  issue(0, cur);
+  cp_async_commit();
+  int64_t un = u + groups;
+  KeyIdx nxt{0, 1, -1, make_int4(0, 1, 0, 0)};
+  if (un < U) nxt = key_idx(p, un);
+  int stage = 0;
+  while (true) {
+    if (un < U) issue(stage ^ 1, nxt);
+    cp_async_commit();
+    const int64_t unn = un + groups;
+    KeyIdx nn{0, 1, -1, make_int4(0, 1, 0, 0)};
+    if (unn < U) nn = key_idx(p, unn);
+    // the gradient of the current key; its staged data then completes
+    const bool staged_grad = GP && !GU && cur.s1 - cur.s0 == 1;
+    Acc4 acc[VPL];
+    cp_async_wait_prev();
+    key_grad<G, VPL, GP, GU>(g, p, cur.s0, cur.s1, cur.first,
+                             staged_grad ? slot(stage, NR * VPL) : nullptr, nt, acc);
+    if (cur.row >= 0) {
+      RowRegs<VPL, ADAM> r;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        r.w[v] = *slot(stage, 0 * VPL + v);
+        r.s1[v] = *slot(stage, 1 * VPL + v);
+        if (ADAM) r.s2[v] = *slot(stage, 2 * VPL + v);
+      }
+      apply_update<G, VPL, ADAM>(g, p, cur.row, r, acc);
+    }
+    if (un >= U) break;
+    u = un;
+    cur = nxt;
+    un = unn;
+    nxt = nn;
+    stage ^= 1;
+  }
+}
+
+// Rows wider than one 16-byte column per lane (D > 128): the same walk over
+// keys with the row loaded into registers (staging would need too much
+// shared memory).
+template <int G, int VPL, bool ADAM, bool GP, bool GU>
+__global__ void __launch_bounds__(256, 2) row_update_wide_kernel(const __grid_constant__ UpdateParams p) {
+  const GroupCtx<G> g;
+  const int64_t groups = (int64_t)gridDim.x * blockDim.x / G;
+  const int64_t U = (int64_t)p.bdev->U;
+  for (int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G; u < U; u += groups) {
+    const KeyIdx k = key_idx(p, u);
+    RowRegs<VPL, ADAM> r;
+    load_row<G, VPL, ADAM>(g, p, k.row, r);
+    Acc4 acc[VPL];
+    key_grad<G, VPL, GP, GU>(g, p, k.s0, k.s1, k.first, nullptr, 0, acc);
+    apply_update<G, VPL, ADAM>(g, p, k.row, r, acc);
+  }
 }
 
 // ------------------------------------------------------------------ host
@@ -318,20 +436,40 @@ template <int G, int VPL, bool GP, bool GU>
 static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t ucap, cudaStream_t s) {
   {
     int64_t blocks = (p.nchunks * G + 255) / 256;
-    if (p.long_chunks && blocks > 3 * kSMs) blocks = 3 * kSMs;
+    if (p.long_chunks && blocks > (VPL >= 2 ? 2 : 3) * kSMs) blocks = (VPL >= 2 ? 2 : 3) * kSMs;
     if (blocks < 1) blocks = 1;
     LaunchScope ls("seg_reduce", s);
     seg_reduce_kernel<G, VPL, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  // persistent: as many CTAs as fit at once (U is known only on the device)
   int64_t blocks = (ucap * G + 255) / 256;
+  const int64_t resident = (int64_t)kSMs * (VPL == 1 ? 3 : 2);
+  if (blocks > resident) blocks = resident;
   if (blocks < 1) blocks = 1;
   LaunchScope ls("row_update", s);
-  if (adam)
-    row_update_kernel<G, VPL, true, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
-  else
-    row_update_kernel<G, VPL, false, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
+  if constexpr (VPL == 1) {
+    const int ns = ((adam ? 3 : 2) * VPL + VPL);
+    const size_t smem = (size_t)2 * ns * 256 * sizeof(float4);
+    cudaError_t e;
+    if (adam) {
+      if ((e = cudaFuncSetAttribute(row_update_kernel<G, VPL, true, GP, GU>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+      row_update_kernel<G, VPL, true, GP, GU><<<(unsigned)blocks, 256, smem, s>>>(p);
+    } else {
+      if ((e = cudaFuncSetAttribute(row_update_kernel<G, VPL, false, GP, GU>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+      row_update_kernel<G, VPL, false, GP, GU><<<(unsigned)blocks, 256, smem, s>>>(p);
+    }
+  } else {
+    if (adam)
+      row_update_wide_kernel<G, VPL, true, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
+    else
+      row_update_wide_kernel<G, VPL, false, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 
