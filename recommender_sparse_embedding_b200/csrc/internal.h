@@ -144,6 +144,7 @@ struct recis_batch {
   double* partials = nullptr;
   float* gbuf = nullptr;          // [chunks][D] reduced gradients of long segments
   int32_t* long_chunks = nullptr; // [chunks] chunks holding a long segment (sample-sort path)
+  int32_t* chunk_counter = nullptr;  // [chunks][2] block-level tickets of the backward
   int64_t capGbuf = 0;            // floats
   recis::BatchDev* bdev = nullptr;
   uint32_t epoch = 0;
@@ -190,13 +191,14 @@ struct LookupArgs {
   float* pooled_out;
   float* unpooled_out;
   int64_t* rows_out;  // insert path: row per occurrence
+  bool insert;        // bulk insert (keys may arrive sorted): fresh splitters, none kept
 };
 
 cudaError_t launch_sort(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
                         cudaStream_t s);
 cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cudaStream_t s);
 cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
-                                cudaStream_t s);
+                                bool insert, cudaStream_t s);
 int samplesort_splits_for(int64_t N);
 int64_t samplesort_tiles_for(int64_t N);
 cudaError_t launch_pool(const LookupArgs& a, int64_t chunk, cudaStream_t s);

@@ -38,6 +38,7 @@ struct PoolParams {
   float* pooled;         // [B][F][D] or null
   float* unpooled;       // [N][D] or null
   const uint32_t* spos;  // [N] sorted position of each occurrence
+  const int64_t* pocc;   // [N] IDMap result of each occurrence (row if >= 0), or null
   int4* gsrc;            // [N] per sorted position: {gradient row b*F+f, bag length, occurrence, 0}
   int4* gfirst;          // [U] per unique key: the same, of one of its occurrences
   int32_t* chunk_bag;    // [nchunks] bag of each chunk's first occurrence
@@ -74,10 +75,24 @@ __global__ void __launch_bounds__(256) bag_prep_kernel(const __grid_constant__ P
   }
 }
 
+// depth of the row ring: up to 8 rows, at most one sub-block (G) ahead
+template <int G, int VPL>
+__host__ __device__ constexpr int pool_ring() {
+  return (VPL >= 4 ? 2 : (VPL == 2 ? 4 : 8)) < G ? (VPL >= 4 ? 2 : (VPL == 2 ? 4 : 8)) : G;
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <int G, int VPL>
 __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     pool_kernel(const __grid_constant__ PoolParams p) {
-  constexpr int K = VPL >= 4 ? 1 : 4 / VPL;  // rows in flight per lane
+  constexpr int R = pool_ring<G, VPL>();  // rows in flight per group
   // all positions, bags and rows fit in 32 bits (N < 2^30, F*B < 2^31,
   // rows < 2^31), so the walk runs on 32-bit integers
   const int ncol = p.ncol;
@@ -141,67 +156,102 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     has = false;
   };
 
-  for (int sub = p0; sub < p1; sub += G) {
-    // lane-parallel: the row of position sub + lane
+  // Row, sorted position and unique index of the G positions of one
+  // sub-block, one position per lane.  The row of an occurrence whose key
+  // was already present comes straight from the IDMap result of the dedup.
+  struct Ids {
+    int row, spos, seg;
+  };
+  auto resolve = [&](int sub) {
+    Ids r{-1, 0, 0};
     const int q = sub + g.lane;
-    int my_row = -1;
-    if (q < p1) my_row = (int)__ldg(p.rows + __ldg(p.inv + q));
-    const int m = (p1 - sub) < G ? (p1 - sub) : G;
-    for (int kb = 0; kb < m; kb += K) {
-      float4 val[K][VPL];
+    if (q < p1) {
+      r.seg = __ldg(p.inv + q);
+      r.spos = (int)__ldg(p.spos + q);
+      const int64_t pr = p.pocc ? __ldcg(p.pocc + q) : -2;
+      r.row = pr >= 0 ? (int)pr : (int)__ldg(p.rows + r.seg);
+    }
+    return r;
+  };
+  // rows stream through a ring of R slots per lane in shared memory: row t+R
+  // is in flight (cp.async) while row t is added
+  extern __shared__ float4 s_ring[];  // [R][VPL][blockDim]
+  auto slot = [&](int r, int v) -> float4* {
+    return s_ring + ((r * VPL + v) * (int)blockDim.x + (int)threadIdx.x);
+  };
+  auto issue = [&](int t, int row) {
+    if (row >= 0) {
+      const float4* src = reinterpret_cast<const float4*>(p.row_data + (int64_t)row * p.row_floats);
 #pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int r = g.bcast(my_row, kb + k < m ? kb + k : 0);
-        const bool valid = kb + k < m && r >= 0;
-        const float4* src = reinterpret_cast<const float4*>(p.row_data + (int64_t)r * p.row_floats);
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-          const int col = g.lane + v * G;
-          val[k][v] = (valid && col < ncol) ? __ldg(src + col) : f4_zero();
-        }
+      for (int v = 0; v < VPL; ++v) {
+        const int col = g.lane + v * G;
+        if (col < ncol) cp_async16(slot(t % R, v), src + col);
       }
+    }
+    cp_async_commit();
+  };
+  const int m = p1 - p0;
+  Ids cur_ids = resolve(p0), nxt_ids = resolve(p0 + G);
 #pragma unroll
-      for (int k = 0; k < K; ++k) {
-        if (kb + k >= m) break;
-        const int pos = sub + kb + k;
-        while (pos >= cur_end) {  // leave the current bag (and any empty ones)
-          flush();
-          if (cur + 1 >= nbags) {  // only reachable with malformed bag offsets
-            if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
-            cur_end = INT_MAX;
-            break;
-          }
-          ++cur;
-          if (++cb == B) {
-            cb = 0;
-            ++cf;
-          }
-          cur_start = cur_end;
-          if (cur - wbase >= G) {
-            wbase = cur;
-            wend = (wbase + g.lane < nbags) ? (int)p.offs[wbase + g.lane + 1] : INT_MAX;
-          }
-          cur_end = g.bcast(wend, cur - wbase);
-        }
+  for (int t = 0; t < R; ++t) issue(t, t < m ? g.bcast(cur_ids.row, t) : -1);
+  for (int t = 0; t < m; ++t) {
+    const int pos = p0 + t;
+    const int ln = t % G;
+    const int row = g.bcast(cur_ids.row, ln);
+    const int spos = g.bcast(cur_ids.spos, ln);
+    const int seg = g.bcast(cur_ids.seg, ln);
+    cp_async_wait<R - 1>();
+    float4 val[VPL];
 #pragma unroll
-        for (int v = 0; v < VPL; ++v) acc_add(acc[v], val[k][v]);
-        has = true;
-        if (p.unpooled) {
-          float4* dst = reinterpret_cast<float4*>(p.unpooled + (int64_t)pos * D);
-#pragma unroll
-          for (int v = 0; v < VPL; ++v) {
-            const int col = g.lane + v * G;
-            if (col < ncol) __stcs(dst + col, val[k][v]);
-          }
-        }
-        // for the backward: this occurrence's gradient source, by sorted
-        // position and by unique key
-        if (g.lane == 0) {
-          const int4 src = make_int4(cb * F + cf, cur_end - cur_start, pos, 0);
-          p.gsrc[__ldg(p.spos + pos)] = src;
-          p.gfirst[__ldg(p.inv + pos)] = src;
-        }
+    for (int v = 0; v < VPL; ++v) {
+      const int col = g.lane + v * G;
+      val[v] = (row >= 0 && col < ncol) ? *slot(t % R, v) : f4_zero();
+    }
+    // the row R positions ahead (in this sub-block or the next) into the slot just read
+    const int ta = t + R;
+    int arow = -1;
+    if (ta < m) arow = (ta / G == t / G) ? g.bcast(cur_ids.row, ta % G) : g.bcast(nxt_ids.row, ta % G);
+    issue(ta, arow);
+    while (pos >= cur_end) {  // leave the current bag (and any empty ones)
+      flush();
+      if (cur + 1 >= nbags) {  // only reachable with malformed bag offsets
+        if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
+        cur_end = INT_MAX;
+        break;
       }
+      ++cur;
+      if (++cb == B) {
+        cb = 0;
+        ++cf;
+      }
+      cur_start = cur_end;
+      if (cur - wbase >= G) {
+        wbase = cur;
+        wend = (wbase + g.lane < nbags) ? (int)p.offs[wbase + g.lane + 1] : INT_MAX;
+      }
+      cur_end = g.bcast(wend, cur - wbase);
+    }
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) acc_add(acc[v], val[v]);
+    has = true;
+    if (p.unpooled) {
+      float4* dst = reinterpret_cast<float4*>(p.unpooled + (int64_t)pos * D);
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int col = g.lane + v * G;
+        if (col < ncol) __stcs(dst + col, val[v]);
+      }
+    }
+    // for the backward: this occurrence's gradient source, by sorted
+    // position and by unique key
+    if (g.lane == 0) {
+      const int4 src = make_int4(cb * F + cf, cur_end - cur_start, pos, 0);
+      p.gsrc[spos] = src;
+      p.gfirst[seg] = src;
+    }
+    if (ln == G - 1) {  // next sub-block
+      cur_ids = nxt_ids;
+      nxt_ids = resolve(p0 + t + 1 + G);
     }
   }
   flush();
@@ -212,8 +262,12 @@ static cudaError_t launch_pool_t(const PoolParams& p, cudaStream_t s) {
   const int64_t threads = p.nchunks * G;
   int64_t blocks = (threads + 255) / 256;
   if (blocks < 1) blocks = 1;
+  const size_t smem = (size_t)pool_ring<G, VPL>() * VPL * 256 * sizeof(float4);
+  const cudaError_t e =
+      cudaFuncSetAttribute(pool_kernel<G, VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   LaunchScope ls("gather_pool", s);
-  pool_kernel<G, VPL><<<(unsigned)blocks, 256, 0, s>>>(p);
+  pool_kernel<G, VPL><<<(unsigned)blocks, 256, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -252,6 +306,7 @@ static PoolParams pool_params(const LookupArgs& a, int64_t chunk) {
   p.pooled = a.pooled_out;
   p.unpooled = a.unpooled_out;
   p.spos = b->spos;
+  p.pocc = a.N <= kSampleSortMaxN ? reinterpret_cast<const int64_t*>(b->kbuf[1]) : nullptr;
   p.gsrc = b->gsrc;
   p.gfirst = b->gfirst;
   p.chunk_bag = b->chunk_bag;

@@ -792,7 +792,7 @@ static cudaError_t launch_local(const SsParams& p, int dev, cudaStream_t s) {
 }
 
 cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
-                                cudaStream_t s) {
+                                bool insert, cudaStream_t s) {
   SsParams p;
   p.keys = keys;
   p.N = N;
@@ -836,9 +836,13 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   static bool rank_attr[64] = {false}, scatter_attr[64] = {false};
   const int nbp_max = (p.max_buckets + 31) & ~31;
   // splitters: quantiles of the previous call on this batch when its size was
-  // comparable, else a sorted sample of this call's keys
+  // comparable (batches of one training stream share their key
+  // distribution), else a sorted sample of this call's keys.  A bulk insert
+  // never reuses and leaves nothing to reuse: its key chunks may arrive
+  // sorted, one key range after another, where old quantiles would put a
+  // whole call into one bucket.
   const int cur = b->cand_parity;
-  const bool reuse = b->cand_n > 0 && b->cand_n >= N / 2 && b->cand_n <= 2 * N;
+  const bool reuse = !insert && b->cand_n > 0 && b->cand_n >= N / 2 && b->cand_n <= 2 * N;
   p.cand_next = b->ss->cand[cur ^ 1];
   if (reuse) {
     p.cand = b->ss->cand[cur];
@@ -853,7 +857,7 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   b->cand_parity = cur ^ 1;
-  b->cand_n = N;
+  b->cand_n = insert ? 0 : N;
   // IDMap probes of every occurrence on the side stream, beside the sort
   if ((e = cudaEventRecord(b->ev_pfork, s)) != cudaSuccess ||
       (e = cudaStreamWaitEvent(b->side, b->ev_pfork, 0)) != cudaSuccess)

@@ -424,6 +424,8 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
     const int64_t cap = gneed + gneed / 4;
     if ((e = realloc_dev(b->gbuf, cap, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
     if ((e = realloc_dev(b->long_chunks, cap / D + 1, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
+    if ((e = realloc_dev(b->chunk_counter, 2 * (cap / D + 1), true)) != cudaSuccess)
+      return cuda_fail(e, "batch alloc");
     b->capGbuf = cap;
   }
   return RECIS_OK;
@@ -454,6 +456,7 @@ static void batch_free(recis_batch* b) {
   cudaFree(b->partials);
   cudaFree(b->gbuf);
   cudaFree(b->long_chunks);
+  cudaFree(b->chunk_counter);
   cudaFree(b->bdev);
   cudaFree(b->chunk_bag);
   if (b->side) cudaStreamDestroy(b->side);
@@ -508,7 +511,7 @@ static recis_status lookup_impl(const LookupArgs& a, cudaStream_t s) {
   }
   if (a.N > 0) {
     if (a.N <= kSampleSortMaxN) {
-      if ((e = launch_sample_dedup(b, t, a.keys, a.N, s)) != cudaSuccess)
+      if ((e = launch_sample_dedup(b, t, a.keys, a.N, a.insert, s)) != cudaSuccess)
         return cuda_fail(e, "dedup launch");
     } else {
       if ((e = launch_sort(b, t, a.keys, a.N, s)) != cudaSuccess) return cuda_fail(e, "sort launch");
@@ -802,7 +805,7 @@ recis_status recis_table_insert(recis_table_t t, recis_batch_t b, const int64_t*
                                 int64_t* rows_out, recis_stream_t stream) {
   recis_status st = check_lookup_args(t, b, keys, N, nullptr, 0, 0, RECIS_SUM, false);
   if (st != RECIS_OK) return st;
-  LookupArgs a{t, b, keys, N, nullptr, 0, 0, RECIS_SUM, nullptr, nullptr, rows_out};
+  LookupArgs a{t, b, keys, N, nullptr, 0, 0, RECIS_SUM, nullptr, nullptr, rows_out, true};
   st = lookup_impl(a, (cudaStream_t)stream);
   b->have_lookup = false;  // no bags: nothing to back-propagate
   return st;

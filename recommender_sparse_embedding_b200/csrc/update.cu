@@ -12,10 +12,12 @@
 // summed in fp64 in position order and rounded once to fp32.  Two launches:
 //   seg_reduce  segments longer than kShortSeg (hot keys) are cut into
 //               chunks of kChunk positions; each lane group sums its chunk's
-//               part of a segment into an fp64 partial and the group that
-//               arrives last (ticket per segment) adds the partials in chunk
-//               order and stores g(u) in gbuf at row seg_start[u] / kChunk (a
-//               long segment is the only long one starting in its chunk).
+//               part of a segment into an fp64 partial; the group that
+//               arrives last adds the partials in chunk order (for a segment
+//               of more than 64 chunks, in two levels: per block of 32
+//               chunks, then the block sums in block order) and stores g(u)
+//               in gbuf at row seg_start[u] / kChunk (a long segment is the
+//               only long one starting in its chunk).
 //   row_update  one lane group per unique key loads the row [emb | state],
 //               sums the key's gradient terms itself when the segment is
 //               short (all loads issued before the sum) or reads gbuf, and
@@ -28,6 +30,7 @@ namespace recis {
 constexpr int kChunk = 16;  // seg_reduce positions per group (<= kShortSeg + 1)
 static_assert(kChunk <= kShortSeg + 1, "a chunk must hold at most one long segment start");
 static_assert(kChunk == kShortSeg, "the dedup lists long chunks of kShortSeg positions");
+constexpr int kCombineBlock = 32;  // chunks per block of the two-level combine
 
 struct UpdateParams {
   int64_t N;
@@ -49,6 +52,7 @@ struct UpdateParams {
   float* row_data;
   double* partials;         // [nchunks][2][D]
   int32_t* counters;        // [U] last-arrival tickets (self-resetting)
+  int32_t* chunk_counters;  // [nchunks][2] block-level tickets (self-resetting)
   // optimiser
   float lr;        // Adagrad: lr; Adam: lr / (1 - beta1^t)
   float eps;
@@ -135,8 +139,14 @@ __device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateP
   int32_t cur = -1;
   int64_t cst = 0, cen = 0;
   auto flush = [&]() {
-    if (combine_split<G, VPL, VPL >= 4 ? 1 : 4 / VPL>(g, acc, p.partials, p.counters, cur, chunk,
-                                                       cst <= p0, cst, cen, kChunk, p.ncol)) {
+    // segments of up to two blocks of chunks: one last-arrival combine;
+    // longer ones (hot keys of long sequences): two levels
+    const bool two_level = (cen - 1) / kChunk - cst / kChunk >= 2 * kCombineBlock;
+    if (two_level ? combine_split2<G, VPL, VPL >= 4 ? 1 : 4 / VPL, kCombineBlock>(
+                        g, acc, p.partials, p.chunk_counters, p.counters, cur, chunk, cst <= p0, cst, cen,
+                        kChunk, p.ncol)
+                  : combine_split<G, VPL, VPL >= 4 ? 1 : 4 / VPL>(g, acc, p.partials, p.counters, cur, chunk,
+                                                                 cst <= p0, cst, cen, kChunk, p.ncol)) {
       float4* dst = reinterpret_cast<float4*>(p.gbuf + (cst / kChunk) * D);
 #pragma unroll
       for (int v = 0; v < VPL; ++v) {
@@ -185,7 +195,7 @@ __device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateP
 // With the dedup's list of chunks holding a long segment, a persistent grid
 // of groups walks the list; without it, one group per chunk.
 template <int G, int VPL, bool GP, bool GU>
-__global__ void __launch_bounds__(256, VPL >= 2 ? 2 : 3) seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
+__global__ void __launch_bounds__(256, 3) seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
   const GroupCtx<G> g;
   const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
   if (p.long_chunks) {
@@ -436,7 +446,7 @@ template <int G, int VPL, bool GP, bool GU>
 static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t ucap, cudaStream_t s) {
   {
     int64_t blocks = (p.nchunks * G + 255) / 256;
-    if (p.long_chunks && blocks > (VPL >= 2 ? 2 : 3) * kSMs) blocks = (VPL >= 2 ? 2 : 3) * kSMs;
+    if (p.long_chunks && blocks > 3 * kSMs) blocks = 3 * kSMs;
     if (blocks < 1) blocks = 1;
     LaunchScope ls("seg_reduce", s);
     seg_reduce_kernel<G, VPL, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
@@ -505,6 +515,7 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.row_data = reinterpret_cast<float*>(t->rows.va);
   p.partials = b->partials;
   p.counters = b->seg_counter;
+  p.chunk_counters = b->chunk_counter;
   p.lr = lr_t;
   p.eps = (float)t->cfg.eps;
   p.beta1 = (float)t->cfg.beta1;
