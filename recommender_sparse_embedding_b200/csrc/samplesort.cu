@@ -570,7 +570,8 @@ __device__ void block_number(const SsParams& p, LocalShared<NT, CAP>& sh, unsign
   }
 }
 
-// One CTA per bucket.  A key-range bucket is sorted by (key, occurrence) in
+// One CTA per key-range bucket and the equality bucket after it.  A
+// key-range bucket is sorted by (key, occurrence) in
 // shared memory (oversized ones in global memory), then numbered; an
 // equality bucket holds one key, already in occurrence order (stable
 // scatter).  The last CTA scans the bucket counts into the call's segment and
@@ -580,9 +581,9 @@ __global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ Ss
   extern __shared__ __align__(16) unsigned char s_raw[];
   LocalShared<NT, CAP>& sh = *reinterpret_cast<LocalShared<NT, CAP>*>(s_raw);
   const int tid = threadIdx.x;
-  const unsigned b = blockIdx.x;
   const unsigned nb = p.ctl->nb;
-  if (b < nb) {
+  // CTA c: key-range bucket 2c, then equality bucket 2c+1
+  for (unsigned b = 2 * blockIdx.x; b < 2 * blockIdx.x + 2 && b < nb; ++b) {
     const int64_t m = (int64_t)p.ctl->tot[b];
     const int64_t off = (int64_t)p.ctl->base[b];
     if (m == 0) {
@@ -612,6 +613,7 @@ __global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ Ss
       __threadfence_block();
       block_number<NT, CAP>(p, sh, b, m, off, false);
     }
+    __syncthreads();
   }
   // the last CTA scans the bucket counts and publishes the call's totals
   __threadfence();
@@ -620,18 +622,27 @@ __global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ Ss
   __syncthreads();
   if (!sh.last) return;
   __threadfence();
-  unsigned long long carry = 0;
-  for (unsigned c0 = 0; c0 < nb; c0 += NT) {
-    const unsigned i = c0 + tid;
-    unsigned long long v = 0;
-    if (i < nb) v = ((unsigned long long)__ldcg(&p.ctl->ncnt[i]) << 32) | __ldcg(&p.ctl->hcnt[i]);
-    unsigned long long tot;
-    const unsigned long long ex = carry + block_excl_scan2<NT>(v, sh.warp, &tot);
+  // thread t owns buckets PER*t .. PER*t+PER-1: all loads at once, a serial
+  // scan of its own, one block scan
+  constexpr int PER = (kMaxBucketSlots + NT - 1) / NT;
+  unsigned long long v[PER], own = 0;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const unsigned i = (unsigned)(tid * PER + q);
+    v[q] = i < nb ? ((unsigned long long)__ldcg(&p.ctl->ncnt[i]) << 32) | __ldcg(&p.ctl->hcnt[i]) : 0ULL;
+  }
+#pragma unroll
+  for (int q = 0; q < PER; ++q) own += v[q];
+  unsigned long long carry;
+  unsigned long long ex = block_excl_scan2<NT>(own, sh.warp, &carry);
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const unsigned i = (unsigned)(tid * PER + q);
     if (i < nb) {
       p.ctl->hpre[i] = (unsigned)(ex & 0xffffffffULL);
       p.ctl->npre[i] = (unsigned)(ex >> 32);
     }
-    carry += tot;
+    ex += v[q];
   }
   if (tid == 0) {
     const unsigned long long U = carry & 0xffffffffULL, nnew = carry >> 32;
@@ -787,7 +798,7 @@ static cudaError_t launch_local(const SsParams& p, int dev, cudaStream_t s) {
   cudaError_t e = set_smem(ss_local_kernel<NT, CAP>, (int)sizeof(LocalShared<NT, CAP>), attr, dev);
   if (e != cudaSuccess) return e;
   LaunchScope ls("ss_local", s);
-  ss_local_kernel<NT, CAP><<<(unsigned)p.max_buckets, NT, sizeof(LocalShared<NT, CAP>), s>>>(p);
+  ss_local_kernel<NT, CAP><<<(unsigned)((p.max_buckets + 1) / 2), NT, sizeof(LocalShared<NT, CAP>), s>>>(p);
   return cudaGetLastError();
 }
 
