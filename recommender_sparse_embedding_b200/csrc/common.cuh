@@ -81,4 +81,14 @@ __device__ __forceinline__ float init_value(uint64_t base, int j, float two_s) {
   return __fmul_rn(u - 0.5f, two_s);
 }
 
+// Programmatic dependent launch.  Kernels of the step are launched with the
+// programmatic-serialization attribute (launch_pdl): a kernel may be
+// scheduled while its predecessor in the stream is still running, so its
+// first statement waits for the predecessor's completion and memory
+// (griddepcontrol.wait), and a CTA whose stores are done lets the successor
+// start launching (griddepcontrol.launch_dependents).  Without the
+// attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace recis

@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(256) feature_hash_kernel(const __grid_constant
                                                            const int64_t* __restrict__ values,
                                                            int64_t* __restrict__ keys,
                                                            int* __restrict__ status) {
+  pdl_wait();
   const int64_t lo = p.offs[0], hi = p.offs[p.F];
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = lo + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < hi; i += stride) {
@@ -70,6 +71,7 @@ __global__ void __launch_bounds__(256) feature_hash_kernel(const __grid_constant
     }
     keys[i] = key;
   }
+  pdl_trigger();
 }
 
 cudaError_t launch_feature_hash(const recis_feature_op* ops, int F, const int64_t* values,
@@ -99,7 +101,9 @@ cudaError_t launch_feature_hash(const recis_feature_op* ops, int F, const int64_
     const int64_t cap = (int64_t)kSMs * 8;
     if (blocks > cap) blocks = cap;
     LaunchScope ls("feature_hash", s);
-    feature_hash_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, values, keys_out, dev_status);
+    const cudaError_t le = launch_pdl(feature_hash_kernel, (unsigned)blocks, 256, 0, s, p, values, keys_out,
+                                      dev_status);
+    if (le != cudaSuccess) return le;
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

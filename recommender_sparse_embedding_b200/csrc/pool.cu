@@ -92,6 +92,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 template <int G, int VPL>
 __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     pool_kernel(const __grid_constant__ PoolParams p) {
+  pdl_wait();
   constexpr int R = pool_ring<G, VPL>();  // rows in flight per group
   // all positions, bags and rows fit in 32 bits (N < 2^30, F*B < 2^31,
   // rows < 2^31), so the walk runs on 32-bit integers
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     }
   }
   flush();
+  pdl_trigger();
 }
 
 template <int G, int VPL>
@@ -267,8 +269,7 @@ static cudaError_t launch_pool_t(const PoolParams& p, cudaStream_t s) {
       cudaFuncSetAttribute(pool_kernel<G, VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   LaunchScope ls("gather_pool", s);
-  pool_kernel<G, VPL><<<(unsigned)blocks, 256, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(pool_kernel<G, VPL>, (unsigned)blocks, 256, smem, s, p);
 }
 
 int group_lanes_for(int D) {

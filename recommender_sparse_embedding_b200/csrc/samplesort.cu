@@ -283,6 +283,7 @@ __global__ void __launch_bounds__(kRankThreads) ss_rank_kernel(const __grid_cons
 // scatter) and the tile's bucket histogram (row `tile` of th).  CTA 0 resets
 // the call's tickets and records where this call's new rows start.
 __global__ void __launch_bounds__(kCountThreads) ss_count_kernel(const __grid_constant__ SsParams p) {
+  pdl_wait();
   __shared__ uint64_t s_split[kMaxSplitters];
   __shared__ unsigned s_hist[kMaxBucketSlots];
   __shared__ unsigned s_warp[kCountThreads / 32];
@@ -338,6 +339,7 @@ __global__ void __launch_bounds__(kCountThreads) ss_count_kernel(const __grid_co
   __syncthreads();
   uint32_t* row = p.th + (size_t)blockIdx.x * nbp;
   for (int i = tid; i < nbp; i += kCountThreads) row[i] = s_hist[i];
+  pdl_trigger();
 }
 
 // ------------------------------------------------------------------ probe
@@ -381,6 +383,7 @@ __global__ void __launch_bounds__(kProbeThreads) ss_probe_kernel(const __grid_co
 // range of tiles.  Turns th[t][b] into the exclusive prefix over tiles and
 // writes the bucket totals; the last CTA scans the totals into bucket starts.
 __global__ void __launch_bounds__(1024) ss_tilescan_kernel(const __grid_constant__ SsParams p) {
+  pdl_wait();
   __shared__ unsigned s_part[32][33];
   __shared__ unsigned s_warp[32];
   __shared__ bool s_last;
@@ -432,6 +435,7 @@ __global__ void __launch_bounds__(1024) ss_tilescan_kernel(const __grid_constant
   const unsigned ex = block_excl_scan<1024>(c[0] + c[1], s_warp, &total);
   if (2 * tid < nb) p.ctl->base[2 * tid] = ex;
   if (2 * tid + 1 < nb) p.ctl->base[2 * tid + 1] = ex + c[0];
+  pdl_trigger();
 }
 
 // ------------------------------------------------------------------ scatter
@@ -440,6 +444,7 @@ __global__ void __launch_bounds__(1024) ss_tilescan_kernel(const __grid_constant
 // ranks within a warp come from match_any over the items in order, ranks
 // across warps from a prefix over per-warp bucket counters.
 __global__ void __launch_bounds__(kCountThreads) ss_scatter_kernel(const __grid_constant__ SsParams p) {
+  pdl_wait();
   extern __shared__ unsigned s_wc[];  // [8][nbp] per-warp counters, then destinations
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int nbp = (int)p.ctl->nbp;
@@ -489,6 +494,7 @@ __global__ void __launch_bounds__(kCountThreads) ss_scatter_kernel(const __grid_
       p.vb[dst] = (uint32_t)(pos0 + j * 32);
     }
   }
+  pdl_trigger();
 }
 
 // ------------------------------------------------------------------ local
@@ -578,6 +584,7 @@ __device__ void block_number(const SsParams& p, LocalShared<NT, CAP>& sh, unsign
 // new-row prefixes.
 template <int NT, int CAP>
 __global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ SsParams p) {
+  pdl_wait();
   extern __shared__ __align__(16) unsigned char s_raw[];
   LocalShared<NT, CAP>& sh = *reinterpret_cast<LocalShared<NT, CAP>*>(s_raw);
   const int tid = threadIdx.x;
@@ -658,6 +665,7 @@ __global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ Ss
     }
     p.seg_start[U] = (int32_t)p.N;
   }
+  pdl_trigger();
 }
 
 // ------------------------------------------------------------------ finish
@@ -673,6 +681,7 @@ static_assert(kSub / kShortSeg <= 32, "one bit per chunk of a finish CTA");
 // j*256 + t for item j of thread t): segment of every position from its
 // bucket's prefix, all outputs, and the initialisation of the new rows.
 __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_constant__ SsParams p) {
+  pdl_wait();
   __shared__ FinishShared sh;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   if (tid == 0) {
@@ -771,6 +780,7 @@ __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_con
       dst[c] = o;
     }
   }
+  pdl_trigger();
 }
 
 // ------------------------------------------------------------------ host
@@ -798,8 +808,8 @@ static cudaError_t launch_local(const SsParams& p, int dev, cudaStream_t s) {
   cudaError_t e = set_smem(ss_local_kernel<NT, CAP>, (int)sizeof(LocalShared<NT, CAP>), attr, dev);
   if (e != cudaSuccess) return e;
   LaunchScope ls("ss_local", s);
-  ss_local_kernel<NT, CAP><<<(unsigned)((p.max_buckets + 1) / 2), NT, sizeof(LocalShared<NT, CAP>), s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(ss_local_kernel<NT, CAP>, (unsigned)((p.max_buckets + 1) / 2), NT,
+                    sizeof(LocalShared<NT, CAP>), s, p);
 }
 
 cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
@@ -882,20 +892,17 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   if ((e = cudaEventRecord(b->ev_probe, b->side)) != cudaSuccess) return e;
   {
     LaunchScope ls("ss_count", s);
-    ss_count_kernel<<<(unsigned)p.tiles, kCountThreads, 0, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(ss_count_kernel, (unsigned)p.tiles, kCountThreads, 0, s, p)) != cudaSuccess) return e;
   }
   {
     LaunchScope ls("ss_tilescan", s);
-    ss_tilescan_kernel<<<(unsigned)(nbp_max / 32), 1024, 0, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(ss_tilescan_kernel, (unsigned)(nbp_max / 32), 1024, 0, s, p)) != cudaSuccess) return e;
   }
   {
     const int smem = (kCountThreads / 32) * nbp_max * (int)sizeof(unsigned);
     if ((e = set_smem(ss_scatter_kernel, smem, scatter_attr, dev)) != cudaSuccess) return e;
     LaunchScope ls("ss_scatter", s);
-    ss_scatter_kernel<<<(unsigned)p.tiles, kCountThreads, smem, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(ss_scatter_kernel, (unsigned)p.tiles, kCountThreads, smem, s, p)) != cudaSuccess) return e;
   }
   if ((e = cudaStreamWaitEvent(s, b->ev_probe, 0)) != cudaSuccess) return e;
   if (N <= 524288)
@@ -905,8 +912,8 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   if (e != cudaSuccess) return e;
   {
     LaunchScope ls("ss_finish", s);
-    ss_finish_kernel<<<(unsigned)((N + kSub - 1) / kSub), kFinThreads, 0, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(ss_finish_kernel, (unsigned)((N + kSub - 1) / kSub), kFinThreads, 0, s, p)) != cudaSuccess)
+      return e;
   }
   return cudaSuccess;
 }

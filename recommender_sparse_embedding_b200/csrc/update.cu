@@ -196,6 +196,7 @@ __device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateP
 // of groups walks the list; without it, one group per chunk.
 template <int G, int VPL, bool GP, bool GU>
 __global__ void __launch_bounds__(256, 3) seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
+  pdl_wait();
   const GroupCtx<G> g;
   const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
   if (p.long_chunks) {
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(256, 3) seg_reduce_kernel(const __grid_constan
   } else if (gid < p.nchunks) {
     reduce_chunk<G, VPL, GP, GU>(g, p, gid);
   }
+  pdl_trigger();
 }
 
 // ------------------------------------------------------------------ row_update
@@ -327,17 +329,19 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Indices of one key: segment bounds, row offset (positions and rows fit in
 // 32 bits: N < 2^31, rows < 2^31) and the source of one of its occurrences.
-struct KeyIdx {
-  int32_t s0, s1, row;
+struct __align__(16) KeyIdx {
+  int32_t s0, s1, row, pad;
   int4 first;
 };
 
 __device__ __forceinline__ KeyIdx key_idx(const UpdateParams& p, int64_t u) {
   KeyIdx k;
+  k.pad = 0;
   k.s0 = __ldg(p.seg_start + u);
   k.s1 = __ldg(p.seg_start + u + 1);
   k.row = (int32_t)__ldg(p.rows + u);
@@ -346,27 +350,35 @@ __device__ __forceinline__ KeyIdx key_idx(const UpdateParams& p, int64_t u) {
 }
 
 // A persistent grid of G-lane groups walks the unique keys u = gid, gid +
-// groups, ... (U from the lookup), two keys deep: while key u is updated, the
-// next key's row [emb | state] (and a singleton's pooled gradient row) are in
-// flight into shared memory by cp.async, and the key after that has its
-// indices loaded.  Each lane copies and reads back only its own 16-byte
-// columns, so no barrier is needed beyond the thread's own wait.  Other keys'
-// gradients (repeated keys, long segments, unpooled gradients) are gathered
-// while the key is updated.
-template <int G, int VPL, bool ADAM, bool GP, bool GU>
+// groups, ... (U from the lookup), S keys deep: while key u is
+// updated, the next S-1 keys' rows [emb | state] (and a singleton's
+// pooled gradient row) are in flight into shared memory by cp.async, and the
+// key after those has its indices loaded.  Each lane copies and reads back
+// only its own 16-byte columns, so a lane's own wait is enough for the data;
+// a key's indices are shared by the group through shared memory (written by
+// its lane 0, read after __syncwarp).  Other keys' gradients (repeated keys,
+// long segments, unpooled gradients) are gathered while the key is updated.
+// Pipeline depth: 4 when each group walks many keys (long-sequence batches),
+// 2 otherwise (filling and draining a deep pipeline costs more than it hides).
+template <int G, int VPL, bool ADAM, bool GP, bool GU, int S>
 __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constant__ UpdateParams p) {
+  pdl_wait();
   constexpr int NR = ADAM ? 3 : 2;             // row slices: emb, state(s)
   constexpr int NS = NR * VPL + VPL;           // staged float4 per thread per stage
-  extern __shared__ float4 s_stage[];          // [2][NS][blockDim]
+  extern __shared__ float4 s_stage[];          // [S][NS][blockDim], then [S][groups] keys
   const GroupCtx<G> g;
   const int tid = threadIdx.x, nt = blockDim.x;
+  const int grp = tid / G, ngrp = nt / G;
   const int64_t groups = (int64_t)gridDim.x * blockDim.x / G;
   const int64_t U = (int64_t)p.bdev->U;
   const int D = p.ncol * 4;
-  int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
-  if (u >= U) return;
+  const int64_t u0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  if (u0 >= U) return;
+  KeyIdx* s_keys = reinterpret_cast<KeyIdx*>(s_stage + S * NS * nt);
+  auto key_slot = [&](int st) -> KeyIdx* { return s_keys + st * ngrp + grp; };
   auto slot = [&](int stage, int sl) -> float4* { return s_stage + ((stage * NS + sl) * nt + tid); };
   auto issue = [&](int stage, const KeyIdx& k) {
+    if (g.lane == 0) *key_slot(stage) = k;
     if (k.row < 0) return;
     const float* base = p.row_data + (int64_t)k.row * p.row_floats;
     const bool stage_grad = GP && !GU && k.s1 - k.s0 == 1;
@@ -381,23 +393,27 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
       }
     }
   };
-  KeyIdx cur = key_idx(p, u);
-  issue(0, cur);
-  cp_async_commit();
-  int64_t un = u + groups;
-  KeyIdx nxt{0, 1, -1, make_int4(0, 1, 0, 0)};
-  if (un < U) nxt = key_idx(p, un);
-  int stage = 0;
-  while (true) {
-    if (un < U) issue(stage ^ 1, nxt);
+  auto idx_of = [&](int64_t k) -> KeyIdx {
+    const int64_t uk = u0 + k * groups;
+    return uk < U ? key_idx(p, uk) : KeyIdx{0, 1, -1, 0, make_int4(0, 1, 0, 0)};
+  };
+#pragma unroll
+  for (int k = 0; k < S - 1; ++k) {
+    issue(k, idx_of(k));
     cp_async_commit();
-    const int64_t unn = un + groups;
-    KeyIdx nn{0, 1, -1, make_int4(0, 1, 0, 0)};
-    if (unn < U) nn = key_idx(p, unn);
-    // the gradient of the current key; its staged data then completes
+  }
+  KeyIdx pre = idx_of(S - 1);
+  for (int64_t k = 0; u0 + k * groups < U; ++k) {
+    __syncwarp(g.mask);  // every lane is done with the slot about to be reused
+    issue((int)((k + S - 1) % S), pre);
+    cp_async_commit();
+    pre = idx_of(k + S);
+    __syncwarp(g.mask);
+    const int stage = (int)(k % S);
+    const KeyIdx cur = *key_slot(stage);
     const bool staged_grad = GP && !GU && cur.s1 - cur.s0 == 1;
     Acc4 acc[VPL];
-    cp_async_wait_prev();
+    cp_async_wait<S - 1>();
     key_grad<G, VPL, GP, GU>(g, p, cur.s0, cur.s1, cur.first,
                              staged_grad ? slot(stage, NR * VPL) : nullptr, nt, acc);
     if (cur.row >= 0) {
@@ -410,13 +426,8 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
       }
       apply_update<G, VPL, ADAM>(g, p, cur.row, r, acc);
     }
-    if (un >= U) break;
-    u = un;
-    cur = nxt;
-    un = unn;
-    nxt = nn;
-    stage ^= 1;
   }
+  pdl_trigger();
 }
 
 // Rows wider than one 16-byte column per lane (D > 128): the same walk over
@@ -424,6 +435,7 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
 // shared memory).
 template <int G, int VPL, bool ADAM, bool GP, bool GU>
 __global__ void __launch_bounds__(256, 2) row_update_wide_kernel(const __grid_constant__ UpdateParams p) {
+  pdl_wait();
   const GroupCtx<G> g;
   const int64_t groups = (int64_t)gridDim.x * blockDim.x / G;
   const int64_t U = (int64_t)p.bdev->U;
@@ -435,6 +447,7 @@ __global__ void __launch_bounds__(256, 2) row_update_wide_kernel(const __grid_co
     key_grad<G, VPL, GP, GU>(g, p, k.s0, k.s1, k.first, nullptr, 0, acc);
     apply_update<G, VPL, ADAM>(g, p, k.row, r, acc);
   }
+  pdl_trigger();
 }
 
 // ------------------------------------------------------------------ host
@@ -449,8 +462,7 @@ static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t uca
     if (p.long_chunks && blocks > 3 * kSMs) blocks = 3 * kSMs;
     if (blocks < 1) blocks = 1;
     LaunchScope ls("seg_reduce", s);
-    seg_reduce_kernel<G, VPL, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_pdl(seg_reduce_kernel<G, VPL, GP, GU>, (unsigned)blocks, 256, 0, s, p);
     if (e != cudaSuccess) return e;
   }
   // persistent: as many CTAs as fit at once (U is known only on the device)
@@ -460,25 +472,27 @@ static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t uca
   if (blocks < 1) blocks = 1;
   LaunchScope ls("row_update", s);
   if constexpr (VPL == 1) {
+    // keys per group decide the depth (U <= ucap)
+    const bool deep = ucap / (blocks * (256 / G)) >= 64;
+    const int S = deep ? 4 : 2;
     const int ns = ((adam ? 3 : 2) * VPL + VPL);
-    const size_t smem = (size_t)2 * ns * 256 * sizeof(float4);
+    const size_t smem = (size_t)S * ns * 256 * sizeof(float4) + (size_t)S * (256 / G) * sizeof(KeyIdx);
     cudaError_t e;
-    if (adam) {
-      if ((e = cudaFuncSetAttribute(row_update_kernel<G, VPL, true, GP, GU>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-        return e;
-      row_update_kernel<G, VPL, true, GP, GU><<<(unsigned)blocks, 256, smem, s>>>(p);
-    } else {
-      if ((e = cudaFuncSetAttribute(row_update_kernel<G, VPL, false, GP, GU>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-        return e;
-      row_update_kernel<G, VPL, false, GP, GU><<<(unsigned)blocks, 256, smem, s>>>(p);
-    }
+    auto go = [&](auto kernel) -> cudaError_t {
+      cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (err != cudaSuccess) return err;
+      return launch_pdl(kernel, (unsigned)blocks, 256, smem, s, p);
+    };
+    if (adam)
+      e = deep ? go(row_update_kernel<G, VPL, true, GP, GU, 4>) : go(row_update_kernel<G, VPL, true, GP, GU, 2>);
+    else
+      e = deep ? go(row_update_kernel<G, VPL, false, GP, GU, 4>) : go(row_update_kernel<G, VPL, false, GP, GU, 2>);
+    if (e != cudaSuccess) return e;
   } else {
     if (adam)
-      row_update_wide_kernel<G, VPL, true, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
+      return launch_pdl(row_update_wide_kernel<G, VPL, true, GP, GU>, (unsigned)blocks, 256, 0, s, p);
     else
-      row_update_wide_kernel<G, VPL, false, GP, GU><<<(unsigned)blocks, 256, 0, s>>>(p);
+      return launch_pdl(row_update_wide_kernel<G, VPL, false, GP, GU>, (unsigned)blocks, 256, 0, s, p);
   }
   return cudaGetLastError();
 }
