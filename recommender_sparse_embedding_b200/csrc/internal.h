@@ -39,8 +39,8 @@ constexpr size_t kCtlZeroBytes = offsetof(SortCtl, active);
 // Control block of the sample-sort dedup (samplesort.cu).  Every field is
 // written by the kernels of each call before it is read; nothing is cleared
 // on the host.
-constexpr int kMaxSplitters = 1024;       // distinct splitters <= 1023
-constexpr int kMaxBucketSlots = 2048;     // buckets 0 .. 2 * nsplit (<= 2046)
+constexpr int kMaxSplitters = 2048;       // distinct splitters <= 2047
+constexpr int kMaxBucketSlots = 4096;     // buckets 0 .. 2 * nsplit (<= 4094)
 constexpr int kMaxSample = 8192;          // sample size of the largest batches
 // Segments (occurrences of one unique key) longer than this are summed by a
 // separate chunked reduction in the backward; the dedup marks their positions.
@@ -54,8 +54,10 @@ struct SsCtl {
   unsigned base[kMaxBucketSlots];         // first sorted position of each bucket
   unsigned hcnt[kMaxBucketSlots];         // distinct keys (heads) per bucket
   unsigned ncnt[kMaxBucketSlots];         // new keys per bucket
-  unsigned hpre[kMaxBucketSlots];         // heads in earlier buckets
-  unsigned npre[kMaxBucketSlots];         // new keys in earlier buckets
+  unsigned hpre[kMaxBucketSlots];         // heads in earlier buckets of the same local CTA
+  unsigned npre[kMaxBucketSlots];         // new keys in earlier buckets of the same local CTA
+  unsigned long long cta_tot[kMaxBucketSlots / 2];  // per local CTA: new keys << 32 | heads
+  unsigned long long cta_pre[kMaxBucketSlots / 2];  // the same, summed over earlier local CTAs
 };
 constexpr int64_t kSampleSortMaxN = (int64_t)1600 * 1000;  // larger batches use the radix sort
 
@@ -139,6 +141,7 @@ struct recis_batch {
   cudaEvent_t ev_pfork = nullptr, ev_probe = nullptr;  // IDMap probes beside the sort
   int cand_parity = 0;          // which candidate array the next call reads
   int64_t cand_n = 0;           // batch size that wrote it (0: none yet)
+  int cand_splits = 0;          // its splitter slots (quantiles written: cand_splits - 1)
   int32_t* seg_counter = nullptr;  // [capN] last-arrival counters (self-resetting)
   int32_t* bag_counter = nullptr;  // [capBags]
   double* partials = nullptr;

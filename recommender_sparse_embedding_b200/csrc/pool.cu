@@ -5,12 +5,12 @@
 //
 // Bags are contiguous ranges of occurrences, so the forward is a segmented
 // reduction over occurrence order (segreduce.cuh): a group of G lanes owns a
-// chunk of C occurrences, each lane one 16-byte column of the row.  Per batch
-// of K occurrences the group issues the index loads (inverse index, then row
-// offset) and then all K row loads before it accumulates, so every lane keeps
-// K independent 16-byte loads in flight.  The bag of the chunk's first
-// occurrence is found by a G-ary search over the bag offsets; later bag
-// boundaries come from a window of G bag ends held one per lane.
+// chunk of C occurrences, each lane one 16-byte column of the row.  Rows
+// stream through a ring of R slots per lane in shared memory (cp.async), so R
+// row loads per lane are in flight while the group adds.  The bag of the
+// chunk's first occurrence comes from the bag preparation; later bag
+// boundaries come from a window of G bag ends held one per lane.  A chunk
+// whose bags all hold one occurrence (one-hot features) is a plain gather.
 // Outputs: pooled rows [B][F][D] (sum, or mean = sum / length), optional
 // unpooled rows [N][D], and the gradient source of every occurrence for the
 // backward.
@@ -105,6 +105,26 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
   const int p0 = (int)chunk * C;
   const int p1 = p0 + C < N ? p0 + C : N;
 
+  // Row, sorted position and unique index of the G positions of one
+  // sub-block, one position per lane.  The row of an occurrence whose key
+  // was already present comes straight from the IDMap result of the dedup.
+  struct Ids {
+    int row, spos, seg;
+  };
+  auto resolve = [&](int sub) {
+    Ids r{-1, 0, 0};
+    const int q = sub + g.lane;
+    if (q < p1) {
+      r.seg = __ldg(p.inv + q);
+      r.spos = (int)__ldg(p.spos + q);
+      const int64_t pr = p.pocc ? __ldcg(p.pocc + q) : -2;
+      r.row = pr >= 0 ? (int)pr : (int)__ldg(p.rows + r.seg);
+    }
+    return r;
+  };
+  // the ids of the first sub-block are in flight while the bag walk starts
+  const Ids ids0 = resolve(p0);
+
   // bag containing p0 (precomputed), its start, and a window of G bag ends
   int j0 = p.chunk_bag[chunk];
   if (j0 < 0 || j0 >= nbags) {  // only with malformed offsets
@@ -157,23 +177,6 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     has = false;
   };
 
-  // Row, sorted position and unique index of the G positions of one
-  // sub-block, one position per lane.  The row of an occurrence whose key
-  // was already present comes straight from the IDMap result of the dedup.
-  struct Ids {
-    int row, spos, seg;
-  };
-  auto resolve = [&](int sub) {
-    Ids r{-1, 0, 0};
-    const int q = sub + g.lane;
-    if (q < p1) {
-      r.seg = __ldg(p.inv + q);
-      r.spos = (int)__ldg(p.spos + q);
-      const int64_t pr = p.pocc ? __ldcg(p.pocc + q) : -2;
-      r.row = pr >= 0 ? (int)pr : (int)__ldg(p.rows + r.seg);
-    }
-    return r;
-  };
   // rows stream through a ring of R slots per lane in shared memory: row t+R
   // is in flight (cp.async) while row t is added
   extern __shared__ float4 s_ring[];  // [R][VPL][blockDim]
@@ -192,7 +195,73 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     cp_async_commit();
   };
   const int m = p1 - p0;
-  Ids cur_ids = resolve(p0), nxt_ids = resolve(p0 + G);
+
+  // A chunk whose bags each hold exactly one occurrence (one-hot features, or
+  // a one-hot stretch of a multi-hot one) is a plain gather: position p0 + t
+  // is bag j0 + t, and the pooled row (sum, or mean over one row) is the row
+  // itself.  K row loads per lane are in flight at once.
+  bool onehot = cur_start == p0;
+  for (int s = 0; onehot && s < m; s += G) {
+    const int e = s == 0 ? wend
+                         : ((j0 + s + g.lane < nbags) ? (int)p.offs[j0 + s + g.lane + 1] : INT_MAX);
+    onehot = g.ballot(s + g.lane < m && e != p0 + s + g.lane + 1) == 0u;
+  }
+  if (onehot) {
+    constexpr int K = (VPL >= 8 ? 1 : 8 / VPL) < G ? (VPL >= 8 ? 1 : 8 / VPL) : G;
+    for (int s = 0; s < m; s += G) {
+      const Ids ids = s == 0 ? ids0 : resolve(p0 + s);
+      int out = 0;  // pooled row b*F+f of this lane's bag
+      if (s + g.lane < m) {
+        const int j = j0 + s + g.lane;
+        const int f = j / B;
+        out = (j - f * B) * F + f;
+        const int4 src = make_int4(out, 1, p0 + s + g.lane, 0);
+        p.gsrc[ids.spos] = src;
+        p.gfirst[ids.seg] = src;
+      }
+      const int cnt = m - s < G ? m - s : G;
+      for (int t0 = 0; t0 < cnt; t0 += K) {
+        float4 val[K][VPL];
+#pragma unroll
+        for (int u = 0; u < K; ++u) {
+          const int row = g.bcast(ids.row, (t0 + u) % G);
+          const bool ok = t0 + u < cnt && row >= 0;
+          const float4* src =
+              reinterpret_cast<const float4*>(p.row_data + (int64_t)(ok ? row : 0) * p.row_floats);
+#pragma unroll
+          for (int v = 0; v < VPL; ++v) {
+            const int col = g.lane + v * G;
+            val[u][v] = (ok && col < ncol) ? __ldcg(src + col) : f4_zero();
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < K; ++u) {
+          if (t0 + u >= cnt) break;
+          const int ob = g.bcast(out, (t0 + u) % G);
+          if (p.pooled) {
+            float4* o = reinterpret_cast<float4*>(p.pooled + (int64_t)ob * D);
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+              const int col = g.lane + v * G;
+              if (col < ncol) __stcs(o + col, val[u][v]);
+            }
+          }
+          if (p.unpooled) {
+            float4* o = reinterpret_cast<float4*>(p.unpooled + (int64_t)(p0 + s + t0 + u) * D);
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+              const int col = g.lane + v * G;
+              if (col < ncol) __stcs(o + col, val[u][v]);
+            }
+          }
+        }
+      }
+    }
+    pdl_trigger();
+    return;
+  }
+
+  Ids cur_ids = ids0, nxt_ids = resolve(p0 + G);
 #pragma unroll
   for (int t = 0; t < R; ++t) issue(t, t < m ? g.bcast(cur_ids.row, t) : -1);
   for (int t = 0; t < m; ++t) {

@@ -8,10 +8,11 @@
 // key order), segment starts, the segment and the occurrence of each sorted
 // position, and initialised new rows.  The digit passes are replaced by six
 // short launches, none of which waits on another CTA:
-//   ss_rank      a strided sample of the keys (2048 to 8192 by batch size) is
+//   ss_rank      a strided sample of the keys (4096 or 8192 by batch size) is
 //                sorted by ranking: every sample's rank is its count of
 //                smaller samples (ties by position), spread over many CTAs.
-//   ss_count     per tile of 2048 keys: up to 1023 distinct splitters from the
+//   ss_count     per tile of 2048 keys: up to 2047 (batches of at most
+//                327680 keys) or 1023 distinct splitters from the
 //                sorted sample, the bucket of every key (key u goes to bucket
 //                2r + [u == split[r]], r = #splitters < u, so buckets are
 //                ordered by key and a key equal to a splitter -- a hot key --
@@ -22,12 +23,14 @@
 //                the scatter is stable); the last CTA scans the bucket totals
 //                into bucket starts.
 //   ss_scatter   moves (key, occurrence) into bucket order, stably.
-//   ss_local     sorts every key-range bucket by (key, occurrence): one warp
-//                per bucket of up to 512 keys, in registers; the whole CTA in
-//                shared memory for larger ones.  An equality bucket holds one
-//                key, already in occurrence order.  Heads (first position of
-//                each distinct key) and new keys are numbered within the
-//                bucket; the last CTA scans the per-bucket counts.
+//   ss_local     one CTA per key-range bucket and the equality bucket after
+//                it.  A key-range bucket is sorted by (key, occurrence): up
+//                to 4 keys per thread in registers (lanes of a warp exchange
+//                by shuffles, warps through shared memory), larger buckets in
+//                shared memory.  An equality bucket holds one key, already in
+//                occurrence order.  Heads (first position of each distinct
+//                key) and new keys are numbered within the bucket; the last
+//                CTA scans the per-bucket counts.
 //   ss_finish    a flat pass over the sorted positions writes every output and
 //                initialises the new rows.
 // A key-range bucket larger than shared memory (only for adversarial key
@@ -109,6 +112,93 @@ __device__ void staged_sort(KeyPtr key, IdxPtr idx, int n) {
       if (local) __syncwarp(); else __syncthreads();
       prev_local = local;
     }
+  }
+  __syncthreads();
+}
+
+// (key, idx) of the lower position of a comparator keeps the smaller pair
+__device__ __forceinline__ bool pair_less(uint64_t ka, uint32_t xa, uint64_t kb, uint32_t xb) {
+  return ka < kb || (ka == kb && xa < xb);
+}
+
+// The same network on NT*E elements held in registers, element i = E*t + e
+// in element e of thread t.  A comparator whose block (k for the first stage
+// of a merge, 2d otherwise) fits in one thread is a register swap; one that
+// fits in E*32 elements pairs lanes of a warp by shuffles (first stage: lane
+// t ^ (k/E - 1), element E-1-e; otherwise lane t ^ (d/E), element e); the rest
+// exchange through shared memory sk/sx (NT*E entries).  Ends with the sorted
+// elements in sk/sx and a __syncthreads.
+template <int NT, int E>
+__device__ void reg_sort(uint64_t (&k)[E], uint32_t (&x)[E], uint64_t* sk, uint32_t* sx) {
+  const int t = threadIdx.x, lane = t & 31;
+#pragma unroll
+  for (int kk = 2; kk <= NT * E; kk <<= 1) {
+#pragma unroll
+    for (int d = kk >> 1; d > 0; d >>= 1) {
+      const bool mirror = d == (kk >> 1);
+      const int span = mirror ? kk : 2 * d;
+      if (span <= E) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int f = mirror ? (e ^ (kk - 1)) : (e ^ d);
+          if (f > e && pair_less(k[f], x[f], k[e], x[e])) {
+            const uint64_t tk = k[e];
+            const uint32_t tx = x[e];
+            k[e] = k[f];
+            x[e] = x[f];
+            k[f] = tk;
+            x[f] = tx;
+          }
+        }
+      } else if (span <= 32 * E) {
+        const int lm = mirror ? (kk / E - 1) : (d / E);
+        // this lane holds the lower positions of its pairs
+        const bool low = (lane & (mirror ? kk / (2 * E) : d / E)) == 0;
+        uint64_t nk[E];
+        uint32_t nx[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int send = mirror ? (E - 1 - e) : e;
+          const uint64_t pk = __shfl_xor_sync(0xffffffffu, k[send], lm);
+          const uint32_t px = __shfl_xor_sync(0xffffffffu, x[send], lm);
+          const bool pl = pair_less(pk, px, k[e], x[e]);
+          const bool take = low ? pl : !pl;
+          nk[e] = take ? pk : k[e];
+          nx[e] = take ? px : x[e];
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          k[e] = nk[e];
+          x[e] = nx[e];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          sk[E * t + e] = k[e];
+          sx[E * t + e] = x[e];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = E * t + e;
+          const int j = mirror ? (i ^ (kk - 1)) : (i ^ d);
+          const uint64_t pk = sk[j];
+          const uint32_t px = sx[j];
+          const bool pl = pair_less(pk, px, k[e], x[e]);
+          const bool take = i < j ? pl : !pl;
+          if (take) {
+            k[e] = pk;
+            x[e] = px;
+          }
+        }
+        __syncthreads();
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    sk[E * t + e] = k[e];
+    sx[E * t + e] = x[e];
   }
   __syncthreads();
 }
@@ -204,6 +294,7 @@ struct SsParams {
   SsCtl* ctl;
   const uint64_t* cand;     // candidate splitters: cand[(i+1)*cand_step - 1], i < S, ascending
   int cand_step;
+  int local_bpc_shift;      // log2 of the buckets per CTA of the local kernel
   uint64_t* cand_next;      // [S] quantiles of this call's sorted keys, for the next call
   uint32_t* th;             // [tiles][nbp] tile histograms, then their column prefix
   uint16_t* bkt;            // [N] bucket of each key
@@ -295,9 +386,9 @@ __global__ void __launch_bounds__(kCountThreads) ss_count_kernel(const __grid_co
     const int64_t pos = pos0 + j * 32;
     k[j] = pos < p.N ? __ldcs(p.keys + pos) : 0;
   }
-  // splitters: 4 candidates per thread, in order
+  // splitters: up to 8 candidates per thread, in order
   const int S = p.splits - 1, step = p.cand_step;
-  constexpr int kCand = kMaxSplitters / kCountThreads;  // 4
+  constexpr int kCand = kMaxSplitters / kCountThreads;  // 8
   uint64_t c[kCand];
   unsigned keepm = 0, nkeep = 0;
 #pragma unroll
@@ -423,18 +514,24 @@ __global__ void __launch_bounds__(1024) ss_tilescan_kernel(const __grid_constant
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // bucket starts: two consecutive buckets per thread
+  // bucket starts: consecutive buckets per thread
+  constexpr int PER = kMaxBucketSlots / 1024;
   const int nb = (int)p.ctl->nb;
-  unsigned c[2];
+  unsigned c[PER], own = 0;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int b = 2 * tid + h;
+  for (int h = 0; h < PER; ++h) {
+    const int b = PER * tid + h;
     c[h] = b < nb ? __ldcg(&p.ctl->tot[b]) : 0u;
+    own += c[h];
   }
   unsigned total;
-  const unsigned ex = block_excl_scan<1024>(c[0] + c[1], s_warp, &total);
-  if (2 * tid < nb) p.ctl->base[2 * tid] = ex;
-  if (2 * tid + 1 < nb) p.ctl->base[2 * tid + 1] = ex + c[0];
+  unsigned ex = block_excl_scan<1024>(own, s_warp, &total);
+#pragma unroll
+  for (int h = 0; h < PER; ++h) {
+    const int b = PER * tid + h;
+    if (b < nb) p.ctl->base[b] = ex;
+    ex += c[h];
+  }
   pdl_trigger();
 }
 
@@ -508,6 +605,21 @@ struct LocalShared {
   bool last;
 };
 
+// Sort a bucket of up to NT*E keys in registers (positions past m are
+// padded with the largest pair); leaves it in sk/sx.
+template <int NT, int E>
+__device__ void reg_load_sort(const SsParams& p, uint64_t* sk, uint32_t* sx, int64_t m, int64_t off) {
+  uint64_t k[E];
+  uint32_t x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = E * (int)threadIdx.x + e;
+    k[e] = i < m ? __ldcg(p.kb + off + i) : ~0ULL;
+    x[e] = i < m ? __ldcg(p.vb + off + i) : ~0u;
+  }
+  reg_sort<NT, E>(k, x, sk, sx);
+}
+
 // Number heads and new keys of a sorted bucket (in shared memory, or in
 // global memory for an oversized one) in rounds of NT positions, write the
 // sorted keys and occurrences (from shared memory) and every position's meta.
@@ -576,79 +688,97 @@ __device__ void block_number(const SsParams& p, LocalShared<NT, CAP>& sh, unsign
   }
 }
 
-// One CTA per key-range bucket and the equality bucket after it.  A
-// key-range bucket is sorted by (key, occurrence) in
-// shared memory (oversized ones in global memory), then numbered; an
-// equality bucket holds one key, already in occurrence order (stable
-// scatter).  The last CTA scans the bucket counts into the call's segment and
-// new-row prefixes.
+// Equality bucket b (one key, m > 0 positions, already in occurrence order
+// from the stable scatter; isnew: the key was claimed by this call): one
+// segment, numbered by threads first, first + stride, ...; `first == 0` also
+// writes the bucket's counts.
+__device__ __forceinline__ void local_equal(const SsParams& p, unsigned b, int64_t m, int64_t off,
+                                            bool isnew, int first, int stride) {
+  const uint64_t lng = m > kShortSeg ? kMetaLong : 0ULL;
+  for (int64_t i = first; i < m; i += stride)
+    p.meta[off + i] = pack_meta(b, 1u, isnew ? 1u : 0u, i == 0, i == 0 && isnew) | lng;
+  if (first == 0) {
+    p.ctl->hcnt[b] = 1;
+    p.ctl->ncnt[b] = isnew ? 1u : 0u;
+  }
+}
+
+// Key-range bucket b (m > 0) by the whole CTA: sorted by (key, occurrence) in
+// registers (up to 4 keys per thread), in shared memory, or in global memory
+// for an oversized one (adversarial key orders), then numbered.
 template <int NT, int CAP>
-__global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ SsParams p) {
-  pdl_wait();
-  extern __shared__ __align__(16) unsigned char s_raw[];
-  LocalShared<NT, CAP>& sh = *reinterpret_cast<LocalShared<NT, CAP>*>(s_raw);
+__device__ void local_range_block(const SsParams& p, LocalShared<NT, CAP>& sh, unsigned b, int64_t m,
+                                  int64_t off) {
   const int tid = threadIdx.x;
-  const unsigned nb = p.ctl->nb;
-  // CTA c: key-range bucket 2c, then equality bucket 2c+1
-  for (unsigned b = 2 * blockIdx.x; b < 2 * blockIdx.x + 2 && b < nb; ++b) {
-    const int64_t m = (int64_t)p.ctl->tot[b];
-    const int64_t off = (int64_t)p.ctl->base[b];
-    if (m == 0) {
-      if (tid == 0) {
-        p.ctl->hcnt[b] = 0;
-        p.ctl->ncnt[b] = 0;
-      }
-    } else if (b & 1u) {
-      const bool isnew = __ldcg(p.pocc + __ldcg(p.vb + off)) <= -2;
-      const uint64_t lng = m > kShortSeg ? kMetaLong : 0ULL;
-      for (int64_t i = tid; i < m; i += NT)
-        p.meta[off + i] = pack_meta(b, 1u, isnew ? 1u : 0u, i == 0, i == 0 && isnew) | lng;
-      if (tid == 0) {
-        p.ctl->hcnt[b] = 1;
-        p.ctl->ncnt[b] = isnew ? 1u : 0u;
-      }
-    } else if (m <= CAP) {
-      for (int i = tid; i < m; i += NT) {
-        sh.key[i] = __ldcg(p.kb + off + i);
-        sh.idx[i] = __ldcg(p.vb + off + i);
-      }
-      __syncthreads();
-      staged_sort<NT, true>(sh.key, sh.idx, (int)m);
-      block_number<NT, CAP>(p, sh, b, m, off, true);
-    } else {
-      staged_sort<NT, true>(p.kb + off, p.vb + off, (int)m);
-      __threadfence_block();
-      block_number<NT, CAP>(p, sh, b, m, off, false);
+  if (m <= NT * 4) {
+    if (m <= NT * 2) reg_load_sort<NT, 2>(p, sh.key, sh.idx, m, off);
+    else reg_load_sort<NT, 4>(p, sh.key, sh.idx, m, off);
+    block_number<NT, CAP>(p, sh, b, m, off, true);
+  } else if (m <= CAP) {
+    for (int i = tid; i < m; i += NT) {
+      sh.key[i] = __ldcg(p.kb + off + i);
+      sh.idx[i] = __ldcg(p.vb + off + i);
     }
     __syncthreads();
+    staged_sort<NT, true>(sh.key, sh.idx, (int)m);
+    block_number<NT, CAP>(p, sh, b, m, off, true);
+  } else {
+    staged_sort<NT, true>(p.kb + off, p.vb + off, (int)m);
+    __threadfence_block();
+    block_number<NT, CAP>(p, sh, b, m, off, false);
   }
-  // the last CTA scans the bucket counts and publishes the call's totals
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) sh.last = atomicAdd(&p.ctl->ticket_local, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!sh.last) return;
-  __threadfence();
-  // thread t owns buckets PER*t .. PER*t+PER-1: all loads at once, a serial
-  // scan of its own, one block scan
-  constexpr int PER = (kMaxBucketSlots + NT - 1) / NT;
-  unsigned long long v[PER], own = 0;
+}
+
+// Bucket prefixes in two levels.  Every CTA turns the counts of its BPC
+// buckets into prefixes within the CTA and publishes its total; the last CTA
+// to finish scans the CTA totals and publishes the call's totals.  A bucket's
+// place is then cta_pre[b / BPC] + hpre[b] (heads) and the same for new keys.
+// Called by every thread after its CTA's buckets are written.
+template <int NT, int BPC>
+__device__ void local_final_scan(const SsParams& p, unsigned long long* s_warp, bool* s_last) {
+  const int tid = threadIdx.x;
+  const unsigned nb = p.ctl->nb;
+  if (tid == 0) {
+    const unsigned b0 = blockIdx.x * BPC;
+    unsigned long long v[BPC], run = 0;
 #pragma unroll
-  for (int q = 0; q < PER; ++q) {
-    const unsigned i = (unsigned)(tid * PER + q);
-    v[q] = i < nb ? ((unsigned long long)__ldcg(&p.ctl->ncnt[i]) << 32) | __ldcg(&p.ctl->hcnt[i]) : 0ULL;
-  }
-#pragma unroll
-  for (int q = 0; q < PER; ++q) own += v[q];
-  unsigned long long carry;
-  unsigned long long ex = block_excl_scan2<NT>(own, sh.warp, &carry);
-#pragma unroll
-  for (int q = 0; q < PER; ++q) {
-    const unsigned i = (unsigned)(tid * PER + q);
-    if (i < nb) {
-      p.ctl->hpre[i] = (unsigned)(ex & 0xffffffffULL);
-      p.ctl->npre[i] = (unsigned)(ex >> 32);
+    for (int j = 0; j < BPC; ++j) {
+      const unsigned b = b0 + j;
+      v[j] = b < nb ? ((unsigned long long)__ldcg(&p.ctl->ncnt[b]) << 32) | __ldcg(&p.ctl->hcnt[b]) : 0ULL;
     }
+#pragma unroll
+    for (int j = 0; j < BPC; ++j) {
+      if (b0 + j < nb) {
+        p.ctl->hpre[b0 + j] = (unsigned)(run & 0xffffffffULL);
+        p.ctl->npre[b0 + j] = (unsigned)(run >> 32);
+      }
+      run += v[j];
+    }
+    p.ctl->cta_tot[blockIdx.x] = run;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) *s_last = atomicAdd(&p.ctl->ticket_local, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!*s_last) return;
+  __threadfence();
+  // thread t owns CTA totals per*t .. per*t+per-1 (per <= kMaxPer)
+  constexpr int kMaxPer = (kMaxBucketSlots / 2 + NT - 1) / NT;
+  const int G = (int)gridDim.x;
+  const int per = (G + NT - 1) / NT;
+  unsigned long long v[kMaxPer], own = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxPer; ++q) {
+    const int i = tid * per + q;
+    v[q] = (q < per && i < G) ? __ldcg(&p.ctl->cta_tot[i]) : 0ULL;
+    own += v[q];
+  }
+  unsigned long long carry;
+  unsigned long long ex = block_excl_scan2<NT>(own, s_warp, &carry);
+#pragma unroll
+  for (int q = 0; q < kMaxPer; ++q) {
+    const int i = tid * per + q;
+    if (q < per && i < G) p.ctl->cta_pre[i] = ex;
     ex += v[q];
   }
   if (tid == 0) {
@@ -665,6 +795,329 @@ __global__ void __launch_bounds__(NT) ss_local_kernel(const __grid_constant__ Ss
     }
     p.seg_start[U] = (int32_t)p.N;
   }
+}
+
+// One CTA per key-range bucket and the equality bucket after it (larger
+// batches, whose buckets hold hundreds to thousands of keys).
+template <int NT, int CAP>
+__global__ void __launch_bounds__(NT, NT >= 512 ? 2 : 4) ss_local_kernel(const __grid_constant__ SsParams p) {
+  pdl_wait();
+  extern __shared__ __align__(16) unsigned char s_raw[];
+  LocalShared<NT, CAP>& sh = *reinterpret_cast<LocalShared<NT, CAP>*>(s_raw);
+  const int tid = threadIdx.x;
+  const unsigned nb = p.ctl->nb;
+  // CTA c: key-range bucket 2c, then equality bucket 2c+1
+  for (unsigned b = 2 * blockIdx.x; b < 2 * blockIdx.x + 2 && b < nb; ++b) {
+    const int64_t m = (int64_t)p.ctl->tot[b];
+    const int64_t off = (int64_t)p.ctl->base[b];
+    if (m == 0) {
+      if (tid == 0) {
+        p.ctl->hcnt[b] = 0;
+        p.ctl->ncnt[b] = 0;
+      }
+    } else if (b & 1u) {
+      local_equal(p, b, m, off, __ldcg(p.pocc + __ldcg(p.vb + off)) <= -2, tid, NT);
+    } else {
+      local_range_block<NT, CAP>(p, sh, b, m, off);
+    }
+    __syncthreads();
+  }
+  local_final_scan<NT, 2>(p, sh.warp, &sh.last);
+  pdl_trigger();
+}
+
+// ------------------------------------------------------------------ local, one warp per bucket
+// For batches of up to kLocalWarpMaxN keys (2047 splitters: key-range
+// buckets of about 100 keys), one warp sorts and numbers one bucket.  A bucket of m <= 32E keys (E = 4, 8 or 16 per lane)
+// whose keys span less than 2^55 is sorted as single 64-bit words
+// (u - min) << log2(32E) | position: the positions are distinct and in
+// occurrence order (stable scatter), so the word order is the (key,
+// occurrence) order.  Lane l holds positions E*l .. E*l+E-1; the network is
+// the one of reg_sort on one warp.
+constexpr int64_t kLocalWarpMaxN = 327680;  // batches whose buckets go one per warp
+constexpr int kLocalWarps = 4;
+constexpr int kLocalWarpThreads = 32 * kLocalWarps;
+constexpr int kWarpSortMax = 512;
+
+template <int CAP>
+struct LocalWarpShared {
+  LocalShared<kLocalWarpThreads, CAP> blk;        // buckets left to the whole CTA
+  uint32_t idx[kLocalWarps][kWarpSortMax];        // occurrence of every bucket position
+  uint8_t hl[kLocalWarps][kWarpSortMax];          // per bucket-local segment: long
+  unsigned fallback;                              // bit w: warp w left its bucket to the CTA
+};
+
+__device__ __forceinline__ uint64_t u64_min(uint64_t a, uint64_t b) { return a < b ? a : b; }
+__device__ __forceinline__ uint64_t u64_max(uint64_t a, uint64_t b) { return a < b ? b : a; }
+
+template <int E>
+__device__ __forceinline__ void warp_sort_unrolled(uint64_t (&c)[E]) {
+  constexpr unsigned kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int kk = 2; kk <= 32 * E; kk <<= 1) {
+#pragma unroll
+    for (int d = kk >> 1; d > 0; d >>= 1) {
+      const bool mirror = d == (kk >> 1);
+      if ((mirror ? kk : 2 * d) <= E) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int f = mirror ? (e ^ (kk - 1)) : (e ^ d);
+          if (f > e) {
+            const uint64_t lo = u64_min(c[e], c[f]), hi = u64_max(c[e], c[f]);
+            c[e] = lo;
+            c[f] = hi;
+          }
+        }
+      } else if (mirror) {
+        // lane ^ (kk/E - 1): my element e meets its element E-1-e
+        const int lm = kk / E - 1;
+        const bool low = (lane & (kk / (2 * E))) == 0;
+#pragma unroll
+        for (int e = 0; e < E / 2; ++e) {
+          const uint64_t a = __shfl_xor_sync(kFull, c[E - 1 - e], lm);
+          const uint64_t b = __shfl_xor_sync(kFull, c[e], lm);
+          c[e] = low ? u64_min(c[e], a) : u64_max(c[e], a);
+          c[E - 1 - e] = low ? u64_min(c[E - 1 - e], b) : u64_max(c[E - 1 - e], b);
+        }
+      } else {
+        const int lm = d / E;
+        const bool low = (lane & lm) == 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const uint64_t a = __shfl_xor_sync(kFull, c[e], lm);
+          c[e] = low ? u64_min(c[e], a) : u64_max(c[e], a);
+        }
+      }
+    }
+  }
+}
+
+// one stage whose comparators lie inside a thread: partner e ^ (V-1) (first
+// stage of a merge of V) or e ^ V
+template <int E, bool MIRROR, int V>
+__device__ __forceinline__ void thread_stage(uint64_t (&c)[E]) {
+  if constexpr ((MIRROR ? V : 2 * V) <= E) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int f = MIRROR ? (e ^ (V - 1)) : (e ^ V);
+      if (f > e) {
+        const uint64_t lo = u64_min(c[e], c[f]), hi = u64_max(c[e], c[f]);
+        c[e] = lo;
+        c[f] = hi;
+      }
+    }
+  }
+}
+
+// The same network with its stages in a loop (compact code for the rare
+// buckets of up to 512 keys)
+template <int E>
+__device__ void warp_sort_loop(uint64_t (&c)[E]) {
+  constexpr unsigned kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  for (int kk = 2; kk <= 32 * E; kk <<= 1) {
+    for (int d = kk >> 1; d > 0; d >>= 1) {
+      const bool mirror = d == (kk >> 1);
+      if ((mirror ? kk : 2 * d) <= E) {
+        if (mirror) {
+          switch (kk) {
+            case 2: thread_stage<E, true, 2>(c); break;
+            case 4: thread_stage<E, true, 4>(c); break;
+            case 8: thread_stage<E, true, 8>(c); break;
+            default: thread_stage<E, true, 16>(c); break;
+          }
+        } else {
+          switch (d) {
+            case 1: thread_stage<E, false, 1>(c); break;
+            case 2: thread_stage<E, false, 2>(c); break;
+            case 4: thread_stage<E, false, 4>(c); break;
+            default: thread_stage<E, false, 8>(c); break;
+          }
+        }
+      } else if (mirror) {
+        const int lm = kk / E - 1;
+        const bool low = (lane & (kk / (2 * E))) == 0;
+#pragma unroll
+        for (int e = 0; e < E / 2; ++e) {
+          const uint64_t a = __shfl_xor_sync(kFull, c[E - 1 - e], lm);
+          const uint64_t b = __shfl_xor_sync(kFull, c[e], lm);
+          c[e] = low ? u64_min(c[e], a) : u64_max(c[e], a);
+          c[E - 1 - e] = low ? u64_min(c[E - 1 - e], b) : u64_max(c[E - 1 - e], b);
+        }
+      } else {
+        const int lm = d / E;
+        const bool low = (lane & lm) == 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const uint64_t a = __shfl_xor_sync(kFull, c[e], lm);
+          c[e] = low ? u64_min(c[e], a) : u64_max(c[e], a);
+        }
+      }
+    }
+  }
+}
+
+template <int E>
+__device__ __forceinline__ void warp_sort(uint64_t (&c)[E]) {
+  if constexpr (E <= 8) warp_sort_unrolled<E>(c);
+  else warp_sort_loop<E>(c);
+}
+
+// Key-range bucket b (0 < m <= 32E) by one warp: sort, number heads and new
+// keys, write the sorted keys, occurrences and meta.  Returns false, having
+// written nothing, when the bucket's keys span 2^55 or more.  *extra (when
+// not null) is loaded into extra_val together with the heads' IDMap results.
+template <int E>
+__device__ bool local_range_warp(const SsParams& p, unsigned b, int m, int64_t off, uint32_t* widx,
+                                 uint8_t* whl, const int64_t* extra, int64_t& extra_val) {
+  constexpr unsigned kFull = 0xffffffffu;
+  constexpr int PB = E == 4 ? 7 : (E == 8 ? 8 : 9);  // position bits
+  static_assert((32 * E) == (1 << PB), "one position per low bit pattern");
+  const int lane = threadIdx.x & 31;
+  uint64_t c[E];
+  uint64_t lo = ~0ULL, hi = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = E * lane + e;
+    c[e] = 0;
+    if (i < m) {
+      c[e] = __ldcg(p.kb + off + i);
+      widx[i] = __ldcg(p.vb + off + i);
+      lo = u64_min(lo, c[e]);
+      hi = u64_max(hi, c[e]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = u64_min(lo, __shfl_xor_sync(kFull, lo, o));
+    hi = u64_max(hi, __shfl_xor_sync(kFull, hi, o));
+  }
+  if (hi - lo >= (1ULL << 55)) return false;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = E * lane + e;
+    c[e] = i < m ? ((c[e] - lo) << PB) | (uint64_t)i : ~0ULL;
+  }
+  warp_sort<E>(c);
+  __syncwarp();
+  // heads (first position of a key), new keys, and long segments (the key 16
+  // positions after the head is the same)
+  const uint64_t before = __shfl_up_sync(kFull, c[E - 1] >> PB, 1);
+  uint32_t occ[E];
+  unsigned hmask = 0, nmask = 0, lmask = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = E * lane + e;
+    const uint64_t rel = c[e] >> PB;
+    const uint64_t after16 = __shfl_down_sync(kFull, rel, kShortSeg / E);
+    occ[e] = i < m ? widx[c[e] & ((1u << PB) - 1u)] : 0u;
+    const uint64_t prev = e == 0 ? before : (c[e - 1] >> PB);
+    if (i < m && (i == 0 || rel != prev)) {
+      hmask |= 1u << e;
+      if (i + kShortSeg < m && after16 == rel) lmask |= 1u << e;
+    }
+  }
+  // the IDMap results of the heads (and the caller's extra one), all in
+  // flight at once
+  int64_t pv[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) pv[e] = ((hmask >> e) & 1u) ? __ldcg(p.pocc + occ[e]) : 0;
+  if (extra) extra_val = __ldcg(extra);
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (pv[e] <= -2) nmask |= 1u << e;
+  const unsigned long long own = ((unsigned long long)__popc(nmask) << 32) | (unsigned)__popc(hmask);
+  unsigned long long y = own;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long z = __shfl_up_sync(kFull, y, o);
+    if (lane >= o) y += z;
+  }
+  const unsigned long long total = __shfl_sync(kFull, y, 31);
+  const unsigned lh0 = (unsigned)((y - own) & 0xffffffffULL), ln0 = (unsigned)((y - own) >> 32);
+  unsigned lh = lh0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    lh += (hmask >> e) & 1u;
+    if ((hmask >> e) & 1u) whl[lh - 1] = (uint8_t)((lmask >> e) & 1u);
+  }
+  __syncwarp();
+  lh = lh0;
+  unsigned ln = ln0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = E * lane + e;
+    lh += (hmask >> e) & 1u;
+    ln += (nmask >> e) & 1u;
+    if (i < m) {
+      p.kb[off + i] = lo + (c[e] >> PB);
+      p.vb[off + i] = occ[e];
+      p.meta[off + i] = pack_meta(b, lh, ln, (hmask >> e) & 1u, (nmask >> e) & 1u) |
+                        (whl[lh - 1] ? kMetaLong : 0ULL);
+    }
+  }
+  if (lane == 0) {
+    p.ctl->hcnt[b] = (unsigned)(total & 0xffffffffULL);
+    p.ctl->ncnt[b] = (unsigned)(total >> 32);
+  }
+  return true;
+}
+
+// Warp w of CTA c: key-range bucket 2q and equality bucket 2q+1 of pair
+// q = 4c + w.  Key-range buckets too large (over 512 keys) or too wide for
+// one warp are then done by the whole CTA, one after another.
+template <int CAP>
+__global__ void __launch_bounds__(kLocalWarpThreads) ss_local_warp_kernel(const __grid_constant__ SsParams p) {
+  pdl_wait();
+  extern __shared__ __align__(16) unsigned char s_raw[];
+  LocalWarpShared<CAP>& sh = *reinterpret_cast<LocalWarpShared<CAP>*>(s_raw);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const unsigned nb = p.ctl->nb;
+  if (tid == 0) sh.fallback = 0;
+  __syncthreads();
+  const unsigned q = kLocalWarps * blockIdx.x + w;
+  // both buckets' sizes and starts, and the equality bucket's first
+  // occurrence, are loaded at once (the control arrays hold every slot)
+  const unsigned br = 2 * q, be = 2 * q + 1;
+  const bool has_r = br < nb, has_e = be < nb;
+  const int64_t mr = (int64_t)__ldcg(&p.ctl->tot[br]), offr = (int64_t)__ldcg(&p.ctl->base[br]);
+  const int64_t me = (int64_t)__ldcg(&p.ctl->tot[be]), offe = (int64_t)__ldcg(&p.ctl->base[be]);
+  const bool eq = has_e && me > 0;
+  const int64_t* eq_pocc = eq ? p.pocc + __ldcg(p.vb + offe) : nullptr;
+  int64_t eq_val = 0;
+  bool eq_loaded = false;
+  if (has_r && mr == 0) {
+    if (lane == 0) {
+      p.ctl->hcnt[br] = 0;
+      p.ctl->ncnt[br] = 0;
+    }
+  } else if (has_r) {
+    bool done = false;
+    if (mr <= 128)
+      done = local_range_warp<4>(p, br, (int)mr, offr, sh.idx[w], sh.hl[w], eq_pocc, eq_val);
+    else if (mr <= 256)
+      done = local_range_warp<8>(p, br, (int)mr, offr, sh.idx[w], sh.hl[w], eq_pocc, eq_val);
+    else if (mr <= 512)
+      done = local_range_warp<16>(p, br, (int)mr, offr, sh.idx[w], sh.hl[w], eq_pocc, eq_val);
+    eq_loaded = done;
+    if (!done && lane == 0) atomicOr(&sh.fallback, 1u << w);
+  }
+  if (eq) {
+    if (!eq_loaded) eq_val = __ldcg(eq_pocc);
+    local_equal(p, be, me, offe, eq_val <= -2, lane, 32);
+  } else if (has_e && lane == 0) {
+    p.ctl->hcnt[be] = 0;
+    p.ctl->ncnt[be] = 0;
+  }
+  __syncthreads();
+  for (unsigned fb = sh.fallback; fb; fb &= fb - 1) {
+    const unsigned b = 2 * (kLocalWarps * blockIdx.x + (unsigned)(__ffs(fb) - 1));
+    local_range_block<kLocalWarpThreads, CAP>(p, sh.blk, b, (int64_t)p.ctl->tot[b],
+                                              (int64_t)p.ctl->base[b]);
+    __syncthreads();
+  }
+  local_final_scan<kLocalWarpThreads, 2 * kLocalWarps>(p, sh.blk.warp, &sh.blk.last);
   pdl_trigger();
 }
 
@@ -709,7 +1162,8 @@ __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_con
     if (m >> 63) atomicOr(&sh.chunk_long, 1u << ((tid + j * kFinThreads) / kShortSeg));
     const unsigned b = (unsigned)(m >> 44) & 0xfffu;
     const unsigned lh = (unsigned)(m & 0x1fffffULL);
-    const unsigned seg = __ldg(&p.ctl->hpre[b]) + lh - 1u;
+    const unsigned long long cpre = __ldg(&p.ctl->cta_pre[b >> p.local_bpc_shift]);
+    const unsigned seg = (unsigned)(cpre & 0xffffffffULL) + __ldg(&p.ctl->hpre[b]) + lh - 1u;
     p.seg_of[q] = (int32_t)seg;
     p.svals[q] = occ[j];
     if (occ[j] < (uint32_t)p.N) {
@@ -722,7 +1176,7 @@ __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_con
       if ((m >> 42) & 1u) {
         const int64_t slot = -2 - row;
         const unsigned ln = (unsigned)((m >> 21) & 0x1fffffULL);
-        row = (int64_t)(row_base + __ldg(&p.ctl->npre[b]) + ln - 1u);
+        row = (int64_t)(row_base + (cpre >> 32) + __ldg(&p.ctl->npre[b]) + ln - 1u);
         if (row >= p.mapped_rows) {
           raise_error(p.st, p.mirror, kErrTableFull);
           row = -1;
@@ -784,12 +1238,14 @@ __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------------ host
-int samplesort_splits_for(int64_t) { return kMaxSplitters; }
+// splitter slots: key-range buckets of about 100 keys for batches the
+// one-warp local sort takes, else about N / 1023
+int samplesort_splits_for(int64_t N) { return N <= kLocalWarpMaxN ? 2048 : 1024; }
 
 int64_t samplesort_tiles_for(int64_t N) { return (N + kTile - 1) / kTile; }
 
+// sample of the first call: at least two keys per splitter slot
 static int sample_size_for(int64_t N) {
-  if (N <= 262144) return 2048;
   if (N <= 524288) return 4096;
   return 8192;
 }
@@ -812,6 +1268,17 @@ static cudaError_t launch_local(const SsParams& p, int dev, cudaStream_t s) {
                     sizeof(LocalShared<NT, CAP>), s, p);
 }
 
+template <int CAP>
+static cudaError_t launch_local_warp(const SsParams& p, int dev, cudaStream_t s) {
+  static bool attr[64] = {false};
+  cudaError_t e = set_smem(ss_local_warp_kernel<CAP>, (int)sizeof(LocalWarpShared<CAP>), attr, dev);
+  if (e != cudaSuccess) return e;
+  LaunchScope ls("ss_local", s);
+  const unsigned pairs = (unsigned)((p.max_buckets + 1) / 2);
+  return launch_pdl(ss_local_warp_kernel<CAP>, (pairs + kLocalWarps - 1) / kLocalWarps,
+                    kLocalWarpThreads, sizeof(LocalWarpShared<CAP>), s, p);
+}
+
 cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
                                 bool insert, cudaStream_t s) {
   SsParams p;
@@ -821,6 +1288,8 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   p.nsample = sample_size_for(N);
   p.tiles = (int)samplesort_tiles_for(N);
   p.max_buckets = 2 * (p.splits - 1) + 1;
+  static_assert(2 * kLocalWarps == 8, "buckets per CTA of the one-warp local kernel");
+  p.local_bpc_shift = N <= kLocalWarpMaxN ? 3 : 1;  // 8 or 2 buckets per local CTA
   p.ctl = b->ss;
   p.th = b->ss_th;
   p.bkt = reinterpret_cast<uint16_t*>(b->vbuf[1]);
@@ -862,12 +1331,15 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   // never reuses and leaves nothing to reuse: its key chunks may arrive
   // sorted, one key range after another, where old quantiles would put a
   // whole call into one bucket.
+  // The previous quantiles serve when they are at least as many as this
+  // call's splitters (every (prev / splits)-th of them).
   const int cur = b->cand_parity;
-  const bool reuse = !insert && b->cand_n > 0 && b->cand_n >= N / 2 && b->cand_n <= 2 * N;
+  const bool reuse = !insert && b->cand_n > 0 && b->cand_n >= N / 2 && b->cand_n <= 2 * N &&
+                     b->cand_splits >= p.splits;
   p.cand_next = b->ss->cand[cur ^ 1];
   if (reuse) {
     p.cand = b->ss->cand[cur];
-    p.cand_step = 1;
+    p.cand_step = b->cand_splits / p.splits;
   } else {
     p.cand = b->ss->samp;
     p.cand_step = p.nsample / p.splits;
@@ -879,6 +1351,7 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   }
   b->cand_parity = cur ^ 1;
   b->cand_n = insert ? 0 : N;
+  b->cand_splits = p.splits;
   // IDMap probes of every occurrence on the side stream, beside the sort
   if ((e = cudaEventRecord(b->ev_pfork, s)) != cudaSuccess ||
       (e = cudaStreamWaitEvent(b->side, b->ev_pfork, 0)) != cudaSuccess)
@@ -900,12 +1373,16 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   }
   {
     const int smem = (kCountThreads / 32) * nbp_max * (int)sizeof(unsigned);
-    if ((e = set_smem(ss_scatter_kernel, smem, scatter_attr, dev)) != cudaSuccess) return e;
+    if ((e = set_smem(ss_scatter_kernel, (kCountThreads / 32) * kMaxBucketSlots * (int)sizeof(unsigned),
+                      scatter_attr, dev)) != cudaSuccess)
+      return e;
     LaunchScope ls("ss_scatter", s);
     if ((e = launch_pdl(ss_scatter_kernel, (unsigned)p.tiles, kCountThreads, smem, s, p)) != cudaSuccess) return e;
   }
   if ((e = cudaStreamWaitEvent(s, b->ev_probe, 0)) != cudaSuccess) return e;
-  if (N <= 524288)
+  if (N <= kLocalWarpMaxN)
+    e = launch_local_warp<2048>(p, dev, s);
+  else if (N <= 524288)
     e = launch_local<128, 2048>(p, dev, s);
   else
     e = launch_local<512, 4096>(p, dev, s);

@@ -168,21 +168,72 @@ def test_one_huge_bag(R, comb):
     _single(R, keys, [60_000], D=16, comb=comb, unpooled=True)
 
 
+@pytest.mark.parametrize("D,comb", [(4, "sum"), (64, "mean"), (200, "sum"), (1024, "mean")])
+def test_one_hot_stretches_among_multi_hot(R, D, comb):
+    # runs of one-occurrence bags (gathered directly) cut by empty and
+    # multi-occurrence bags (the segmented walk), with the unpooled output
+    rng = np.random.default_rng(21 + D)
+    F, B = 3, 3000
+    lengths = np.ones(F * B, np.int64)
+    for s in rng.choice(F * B, size=60, replace=False):
+        lengths[s] = rng.choice([0, 2, 3])
+    keys = rng.integers(0, 4000, size=int(lengths.sum()))
+    _single(R, keys, lengths, D=D, comb=comb, F=F, unpooled=True, opt="adam")
+
+
 def test_all_occurrences_one_key(R):
     # one unique key: the sort has no active pass and one segment spans every chunk
     _single(R, np.full(70_000, 123456789), np.ones(70_000, np.int64), D=32, opt="adam")
 
 
 def test_adversarial_key_order_oversized_bucket(R):
-    # the dedup samples keys at fixed positions; put spread-out keys there and
-    # crowd every other key between two of them, so one bucket holds almost
-    # the whole batch and is sorted and streamed from global memory
+    # the first call's splitters come from keys at fixed positions; put
+    # spread-out keys there and crowd every other key between the two
+    # smallest, so one bucket holds almost the whole batch and is sorted and
+    # streamed from global memory
     N = 24_000
     rng = np.random.default_rng(12)
-    keys = 500_000 + rng.permutation(400_000)[: N].astype(np.int64)
-    sampled = (np.arange(2048, dtype=np.int64) * N) // 2048
-    keys[sampled] = np.arange(len(sampled), dtype=np.int64) * 1000
+    keys = 1 + rng.permutation(1_000_000)[: N].astype(np.int64)
+    for ns in (2048, 4096, 8192):
+        sampled = (np.arange(ns, dtype=np.int64) * N) // ns
+        keys[sampled] = np.arange(ns, dtype=np.int64) * 1_000_000_000
     _single(R, keys, np.ones(N, np.int64), D=8, steps=2)
+
+
+@pytest.mark.parametrize("B", [12_602, 12_603, 15_000])
+def test_batch_sizes_around_the_one_warp_local_sort(R, B):
+    # 26 x B keys: 327,652 and 327,678 (one warp per bucket, 2047
+    # splitters) and 390,000 (one CTA per bucket, 1023 splitters)
+    run_workload(R, W.WORKLOADS["criteo26"].scaled(B), steps=2)
+
+
+def test_splitter_reuse_across_batch_sizes(R):
+    # one batch object, calls of 200K, 390K, 200K and 100K keys: quantiles of
+    # 2047 splitters serve a 1023-splitter call (every second one); a call
+    # that needs more splitters than the last call left draws a sample
+    rng = np.random.default_rng(14)
+    D = 8
+    spec = W.TableSpec("t", [0], D, "adagrad", 0.05, "sum", pooled=True, init_seed=6)
+    p = Pair(R, spec)
+    for step, N in enumerate((200_000, 390_000, 200_000, 100_000)):
+        keys = np.minimum(rng.zipf(1.1, size=N), 10**9).astype(np.int64) * 7_919 + rng.integers(0, 3, size=N)
+        bo = np.arange(N + 1, dtype=np.int64)
+        pooled = torch.empty((N, 1, D), dtype=torch.float32, device=DEV)
+        p.gpu.lookup_pooled(p.batch, torch.from_numpy(keys).to(DEV), torch.from_numpy(bo).to(DEV),
+                            1, N, R.SUM, pooled)
+        r = p.ora.lookup(keys, bo, 1, N, O.SUM)
+        uq, inv, rows, n_new = p.batch.get_unique(N)
+        assert np.array_equal(uq.cpu().numpy(), r.uniq)
+        assert np.array_equal(inv.cpu().numpy(), r.inv)
+        assert np.array_equal(rows.cpu().numpy(), r.rows)
+        assert n_new == r.n_new
+        close(pooled.cpu().numpy(), r.pooled, f"pooled call {step}")
+        gp = W.make_grad((N, 1, D), 80 + step)
+        p.gpu.backward_update(p.batch, torch.from_numpy(gp).to(DEV))
+        p.ora.backward_update(gp)
+        p.gpu.status_sync()
+        compare_tables(p, f"call {step}")
+    p.close()
 
 
 def test_hot_key_among_others(R):
