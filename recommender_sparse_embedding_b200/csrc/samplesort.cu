@@ -29,8 +29,10 @@
 //                by shuffles, warps through shared memory), larger buckets in
 //                shared memory.  An equality bucket holds one key, already in
 //                occurrence order.  Heads (first position of each distinct
-//                key) and new keys are numbered within the bucket; the last
-//                CTA scans the per-bucket counts.
+//                key) and new keys are numbered within the bucket, and the
+//                bucket counts summed within the CTA; the CTA totals are
+//                scanned by the last CTA (one CTA per bucket) or by every
+//                finish CTA (one warp per bucket: a few hundred totals).
 //   ss_finish    a flat pass over the sorted positions writes every output and
 //                initialises the new rows.
 // A key-range bucket larger than shared memory (only for adversarial key
@@ -295,6 +297,8 @@ struct SsParams {
   const uint64_t* cand;     // candidate splitters: cand[(i+1)*cand_step - 1], i < S, ascending
   int cand_step;
   int local_bpc_shift;      // log2 of the buckets per CTA of the local kernel
+  int local_ctas;           // CTAs of the local kernel
+  int finish_scans;         // the finish kernel scans the local CTAs' totals
   uint64_t* cand_next;      // [S] quantiles of this call's sorted keys, for the next call
   uint32_t* th;             // [tiles][nbp] tile histograms, then their column prefix
   uint16_t* bkt;            // [N] bucket of each key
@@ -415,6 +419,7 @@ __global__ void __launch_bounds__(kCountThreads) ss_count_kernel(const __grid_co
     p.ctl->nbp = (unsigned)nbp;
     p.ctl->ticket_scan = 0;
     p.ctl->ticket_local = 0;
+    p.bdev->nlong = 0;
     p.bdev->row_base = *(volatile unsigned long long*)&p.st->next_free;
   }
   __syncthreads();
@@ -729,72 +734,75 @@ __device__ void local_range_block(const SsParams& p, LocalShared<NT, CAP>& sh, u
   }
 }
 
-// Bucket prefixes in two levels.  Every CTA turns the counts of its BPC
-// buckets into prefixes within the CTA and publishes its total; the last CTA
-// to finish scans the CTA totals and publishes the call's totals.  A bucket's
-// place is then cta_pre[b / BPC] + hpre[b] (heads) and the same for new keys.
-// Called by every thread after its CTA's buckets are written.
-template <int NT, int BPC>
-__device__ void local_final_scan(const SsParams& p, unsigned long long* s_warp, bool* s_last) {
-  const int tid = threadIdx.x;
+// Bucket prefixes, first level: every local CTA turns the counts of its BPC
+// buckets into prefixes within the CTA and publishes its total.  The finish
+// kernel scans the CTA totals; a bucket's place is then the CTA prefix plus
+// hpre[b] (heads), and the same for new keys.  Called by every thread after
+// its CTA's buckets are written.
+template <int BPC>
+__device__ __forceinline__ void local_publish(const SsParams& p) {
+  if (threadIdx.x != 0) return;
   const unsigned nb = p.ctl->nb;
-  if (tid == 0) {
-    const unsigned b0 = blockIdx.x * BPC;
-    unsigned long long v[BPC], run = 0;
+  const unsigned b0 = blockIdx.x * BPC;
+  unsigned long long v[BPC], run = 0;
 #pragma unroll
-    for (int j = 0; j < BPC; ++j) {
-      const unsigned b = b0 + j;
-      v[j] = b < nb ? ((unsigned long long)__ldcg(&p.ctl->ncnt[b]) << 32) | __ldcg(&p.ctl->hcnt[b]) : 0ULL;
-    }
-#pragma unroll
-    for (int j = 0; j < BPC; ++j) {
-      if (b0 + j < nb) {
-        p.ctl->hpre[b0 + j] = (unsigned)(run & 0xffffffffULL);
-        p.ctl->npre[b0 + j] = (unsigned)(run >> 32);
-      }
-      run += v[j];
-    }
-    p.ctl->cta_tot[blockIdx.x] = run;
+  for (int j = 0; j < BPC; ++j) {
+    const unsigned b = b0 + j;
+    v[j] = b < nb ? ((unsigned long long)__ldcg(&p.ctl->ncnt[b]) << 32) | __ldcg(&p.ctl->hcnt[b]) : 0ULL;
   }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) *s_last = atomicAdd(&p.ctl->ticket_local, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!*s_last) return;
-  __threadfence();
-  // thread t owns CTA totals per*t .. per*t+per-1 (per <= kMaxPer)
-  constexpr int kMaxPer = (kMaxBucketSlots / 2 + NT - 1) / NT;
-  const int G = (int)gridDim.x;
+#pragma unroll
+  for (int j = 0; j < BPC; ++j) {
+    if (b0 + j < nb) {
+      p.ctl->hpre[b0 + j] = (unsigned)(run & 0xffffffffULL);
+      p.ctl->npre[b0 + j] = (unsigned)(run >> 32);
+    }
+    run += v[j];
+  }
+  p.ctl->cta_tot[blockIdx.x] = run;
+}
+
+// The call's totals (tot = new keys << 32 | heads), published by one thread.
+__device__ __forceinline__ void publish_totals(const SsParams& p, unsigned long long tot,
+                                               unsigned long long row_base) {
+  const unsigned long long U = tot & 0xffffffffULL, nnew = tot >> 32;
+  p.bdev->U = (unsigned)U;
+  p.bdev->n_new = (unsigned)nnew;
+  unsigned long long nf = row_base + nnew;
+  if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
+  p.st->next_free = nf;
+  if (p.mirror) {
+    p.mirror->next_free = nf;
+    __threadfence_system();
+  }
+  p.seg_start[U] = (int32_t)p.N;
+}
+
+// Exclusive scan of the local CTAs' totals by one block of NT threads
+// (thread t owns per consecutive ones); dst(i, prefix) receives each prefix.
+// Returns the grand total.
+template <int NT, typename Dst>
+__device__ __forceinline__ unsigned long long scan_cta_totals(const SsParams& p, unsigned long long* s_warp,
+                                                              Dst dst) {
+  constexpr int kPer = (kMaxBucketSlots / 2 + NT - 1) / NT;
+  const int tid = threadIdx.x;
+  const int G = p.local_ctas;
   const int per = (G + NT - 1) / NT;
-  unsigned long long v[kMaxPer], own = 0;
+  unsigned long long v[kPer], own = 0;
 #pragma unroll
-  for (int q = 0; q < kMaxPer; ++q) {
-    const int i = tid * per + q;
-    v[q] = (q < per && i < G) ? __ldcg(&p.ctl->cta_tot[i]) : 0ULL;
-    own += v[q];
+  for (int r = 0; r < kPer; ++r) {
+    const int i = tid * per + r;
+    v[r] = (r < per && i < G) ? __ldcg(&p.ctl->cta_tot[i]) : 0ULL;
+    own += v[r];
   }
-  unsigned long long carry;
-  unsigned long long ex = block_excl_scan2<NT>(own, s_warp, &carry);
+  unsigned long long tot;
+  unsigned long long ex = block_excl_scan2<NT>(own, s_warp, &tot);
 #pragma unroll
-  for (int q = 0; q < kMaxPer; ++q) {
-    const int i = tid * per + q;
-    if (q < per && i < G) p.ctl->cta_pre[i] = ex;
-    ex += v[q];
+  for (int r = 0; r < kPer; ++r) {
+    const int i = tid * per + r;
+    if (r < per && i < G) dst(i, ex);
+    ex += v[r];
   }
-  if (tid == 0) {
-    const unsigned long long U = carry & 0xffffffffULL, nnew = carry >> 32;
-    p.bdev->U = (unsigned)U;
-    p.bdev->n_new = (unsigned)nnew;
-    p.bdev->nlong = 0;
-    unsigned long long nf = p.bdev->row_base + nnew;
-    if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
-    p.st->next_free = nf;
-    if (p.mirror) {
-      p.mirror->next_free = nf;
-      __threadfence_system();
-    }
-    p.seg_start[U] = (int32_t)p.N;
-  }
+  return tot;
 }
 
 // One CTA per key-range bucket and the equality bucket after it (larger
@@ -822,7 +830,19 @@ __global__ void __launch_bounds__(NT, NT >= 512 ? 2 : 4) ss_local_kernel(const _
     }
     __syncthreads();
   }
-  local_final_scan<NT, 2>(p, sh.warp, &sh.last);
+  local_publish<2>(p);
+  // the last CTA to finish scans the CTA totals (the finish kernel reads
+  // the prefixes per position)
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(&p.ctl->ticket_local, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (sh.last) {
+    __threadfence();
+    const unsigned long long tot =
+        scan_cta_totals<NT>(p, sh.warp, [&](int i, unsigned long long v) { p.ctl->cta_pre[i] = v; });
+    if (tid == 0) publish_totals(p, tot, p.bdev->row_base);
+  }
   pdl_trigger();
 }
 
@@ -1117,7 +1137,7 @@ __global__ void __launch_bounds__(kLocalWarpThreads) ss_local_warp_kernel(const 
                                               (int64_t)p.ctl->base[b]);
     __syncthreads();
   }
-  local_final_scan<kLocalWarpThreads, 2 * kLocalWarps>(p, sh.blk.warp, &sh.blk.last);
+  local_publish<2 * kLocalWarps>(p);
   pdl_trigger();
 }
 
@@ -1125,6 +1145,8 @@ __global__ void __launch_bounds__(kLocalWarpThreads) ss_local_warp_kernel(const 
 struct FinishShared {
   int64_t init_key[kFinThreads * kFinItems];
   int32_t init_row[kFinThreads * kFinItems];
+  unsigned long long cpre[kMaxBucketSlots / 2];  // per local CTA: new keys << 32 | heads before it
+  unsigned long long warp[kFinThreads / 32];
   unsigned chunk_long;  // bit c: chunk c (kShortSeg positions) of this CTA holds a long segment
   int ninit;
 };
@@ -1133,7 +1155,7 @@ static_assert(kSub / kShortSeg <= 32, "one bit per chunk of a finish CTA");
 // Flat pass over the sorted positions, kSub per CTA (position blk*kSub +
 // j*256 + t for item j of thread t): segment of every position from its
 // bucket's prefix, all outputs, and the initialisation of the new rows.
-__global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_constant__ SsParams p) {
+__global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_constant__ SsParams p) {
   pdl_wait();
   __shared__ FinishShared sh;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -1154,6 +1176,15 @@ __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_con
       occ[j] = __ldcs(p.vb + q);
     }
   }
+  // second level of the bucket prefixes, after the one-warp local kernel:
+  // every CTA scans the local CTAs' totals and CTA 0 publishes the call's
+  // totals (after the CTA local kernel its last CTA did both)
+  if (p.finish_scans) {
+    const unsigned long long tot = scan_cta_totals<kFinThreads>(
+        p, sh.warp, [&](int i, unsigned long long v) { sh.cpre[i] = v; });
+    if (blockIdx.x == 0 && tid == 0) publish_totals(p, tot, row_base);
+  }
+  __syncthreads();
 #pragma unroll
   for (int j = 0; j < kFinItems; ++j) {
     const int64_t q = q0 + j * kFinThreads;
@@ -1162,7 +1193,8 @@ __global__ void __launch_bounds__(kFinThreads) ss_finish_kernel(const __grid_con
     if (m >> 63) atomicOr(&sh.chunk_long, 1u << ((tid + j * kFinThreads) / kShortSeg));
     const unsigned b = (unsigned)(m >> 44) & 0xfffu;
     const unsigned lh = (unsigned)(m & 0x1fffffULL);
-    const unsigned long long cpre = __ldg(&p.ctl->cta_pre[b >> p.local_bpc_shift]);
+    const unsigned long long cpre = p.finish_scans ? sh.cpre[b >> p.local_bpc_shift]
+                                                   : __ldg(&p.ctl->cta_pre[b >> p.local_bpc_shift]);
     const unsigned seg = (unsigned)(cpre & 0xffffffffULL) + __ldg(&p.ctl->hpre[b]) + lh - 1u;
     p.seg_of[q] = (int32_t)seg;
     p.svals[q] = occ[j];
@@ -1264,8 +1296,8 @@ static cudaError_t launch_local(const SsParams& p, int dev, cudaStream_t s) {
   cudaError_t e = set_smem(ss_local_kernel<NT, CAP>, (int)sizeof(LocalShared<NT, CAP>), attr, dev);
   if (e != cudaSuccess) return e;
   LaunchScope ls("ss_local", s);
-  return launch_pdl(ss_local_kernel<NT, CAP>, (unsigned)((p.max_buckets + 1) / 2), NT,
-                    sizeof(LocalShared<NT, CAP>), s, p);
+  return launch_pdl(ss_local_kernel<NT, CAP>, (unsigned)p.local_ctas, NT, sizeof(LocalShared<NT, CAP>), s,
+                    p);
 }
 
 template <int CAP>
@@ -1274,9 +1306,8 @@ static cudaError_t launch_local_warp(const SsParams& p, int dev, cudaStream_t s)
   cudaError_t e = set_smem(ss_local_warp_kernel<CAP>, (int)sizeof(LocalWarpShared<CAP>), attr, dev);
   if (e != cudaSuccess) return e;
   LaunchScope ls("ss_local", s);
-  const unsigned pairs = (unsigned)((p.max_buckets + 1) / 2);
-  return launch_pdl(ss_local_warp_kernel<CAP>, (pairs + kLocalWarps - 1) / kLocalWarps,
-                    kLocalWarpThreads, sizeof(LocalWarpShared<CAP>), s, p);
+  return launch_pdl(ss_local_warp_kernel<CAP>, (unsigned)p.local_ctas, kLocalWarpThreads,
+                    sizeof(LocalWarpShared<CAP>), s, p);
 }
 
 cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
@@ -1290,6 +1321,9 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   p.max_buckets = 2 * (p.splits - 1) + 1;
   static_assert(2 * kLocalWarps == 8, "buckets per CTA of the one-warp local kernel");
   p.local_bpc_shift = N <= kLocalWarpMaxN ? 3 : 1;  // 8 or 2 buckets per local CTA
+  p.local_ctas = (p.max_buckets + 1) / 2;            // bucket pairs
+  if (N <= kLocalWarpMaxN) p.local_ctas = (p.local_ctas + kLocalWarps - 1) / kLocalWarps;
+  p.finish_scans = N <= kLocalWarpMaxN ? 1 : 0;
   p.ctl = b->ss;
   p.th = b->ss_th;
   p.bkt = reinterpret_cast<uint16_t*>(b->vbuf[1]);
