@@ -820,17 +820,17 @@ recis_status recis_backward_update(recis_table_t t, recis_batch_t b, const float
   cudaStream_t s = (cudaStream_t)stream;
   recis_status st = pending_error(t, s);
   if (st != RECIS_OK) return st;
-  float lr_t = (float)t->cfg.lr, sqrt_bc2 = 1.0f;
+  float lr_t = (float)t->cfg.lr, inv_sqrt_bc2 = 1.0f;
   if (t->cfg.optimizer == RECIS_ADAM) {
     t->step += 1;
     const double bc1 = 1.0 - std::pow(t->cfg.beta1, (double)t->step);
     const double bc2 = 1.0 - std::pow(t->cfg.beta2, (double)t->step);
     lr_t = (float)(t->cfg.lr / bc1);
-    sqrt_bc2 = (float)std::sqrt(bc2);
+    inv_sqrt_bc2 = (float)(1.0 / std::sqrt(bc2));
   }
   if (b->N > 0) {
     const cudaError_t e = launch_update(t, b, grad_pooled, grad_unpooled,
-                                       update_chunk_for(b->N, t->D), lr_t, sqrt_bc2, s);
+                                       update_chunk_for(b->N, t->D), lr_t, inv_sqrt_bc2, s);
     if (e != cudaSuccess) return cuda_fail(e, "update launch");
   }
   after_call(t, 0, s);

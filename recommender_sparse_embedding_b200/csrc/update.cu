@@ -58,7 +58,7 @@ struct UpdateParams {
   float eps;
   float beta1, beta2;
   float omb1, omb2;  // 1 - beta1, 1 - beta2 (formed in double, rounded once)
-  float sqrt_bc2;    // Adam: sqrt(1 - beta2^t)
+  float inv_sqrt_bc2;  // Adam: 1 / sqrt(1 - beta2^t) (formed in double, rounded once)
 };
 
 // gradient rows each lane loads before adding (fewer for wide rows: registers)
@@ -195,7 +195,8 @@ __device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateP
 // With the dedup's list of chunks holding a long segment, a persistent grid
 // of groups walks the list; without it, one group per chunk.
 template <int G, int VPL, bool GP, bool GU>
-__global__ void __launch_bounds__(256, 3) seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
+__global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
+    seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
   pdl_wait();
   const GroupCtx<G> g;
   const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
@@ -239,7 +240,7 @@ __device__ __forceinline__ void load_row(const GroupCtx<G>& g, const UpdateParam
 //            w -= (lr / (1-b1^t)) m / (sqrt(v) / sqrt(1-b2^t) + eps)
 template <int G, int VPL, bool ADAM>
 __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateParams& p, int64_t row,
-                                             const RowRegs<VPL, ADAM>& r, const Acc4 (&grad)[VPL]) {
+                                             const RowRegs<VPL, ADAM>& r, const float4 (&grad)[VPL]) {
   if (row < 0) return;
   float* base = p.row_data + row * p.row_floats;
   const int D = p.ncol * 4;
@@ -247,14 +248,16 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
   for (int v = 0; v < VPL; ++v) {
     const int col = g.lane + v * G;
     if (col >= p.ncol) continue;
-    const float gg[4] = {(float)grad[v].x, (float)grad[v].y, (float)grad[v].z, (float)grad[v].w};
+    const float gg[4] = {grad[v].x, grad[v].y, grad[v].z, grad[v].w};
     float ww[4] = {r.w[v].x, r.w[v].y, r.w[v].z, r.w[v].w};
     float a1[4] = {r.s1[v].x, r.s1[v].y, r.s1[v].z, r.s1[v].w};
+    // the step lr * x / denom: the quotient by __fdividef (within 2 ulp;
+    // denom >= eps is far from its overflow range)
     if (!ADAM) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float acc = a1[e] + gg[e] * gg[e];
-        ww[e] = ww[e] - p.lr * gg[e] / (sqrtf(acc) + p.eps);
+        ww[e] = ww[e] - __fdividef(p.lr * gg[e], sqrtf(acc) + p.eps);
         a1[e] = acc;
       }
     } else {
@@ -263,7 +266,7 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
       for (int e = 0; e < 4; ++e) {
         const float m = p.beta1 * a1[e] + p.omb1 * gg[e];
         const float vv = p.beta2 * a2[e] + p.omb2 * (gg[e] * gg[e]);
-        ww[e] = ww[e] - p.lr * m / (sqrtf(vv) / p.sqrt_bc2 + p.eps);
+        ww[e] = ww[e] - __fdividef(p.lr * m, fmaf(sqrtf(vv), p.inv_sqrt_bc2, p.eps));
         a1[e] = m;
         a2[e] = vv;
       }
@@ -286,15 +289,31 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
 template <int G, int VPL, bool GP, bool GU>
 __device__ __forceinline__ void key_grad(const GroupCtx<G>& g, const UpdateParams& p, int32_t s0,
                                          int32_t s1, int4 first, const float4* staged, int stride,
-                                         Acc4 (&acc)[VPL]) {
+                                         float4 (&out)[VPL]) {
   const int64_t D = (int64_t)p.ncol * 4;
-#pragma unroll
-  for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
   const int len = s1 - s0;
   constexpr int K = kRowsInFlight<VPL, GP && GU>;
+  if (len == 1 && staged && !p.mean) {
+    // a singleton's one pooled-gradient term, exactly
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) out[v] = staged[v * stride];
+    return;
+  }
+  if (len > kShortSeg) {
+    const float4* src = reinterpret_cast<const float4*>(p.gbuf + (int64_t)(s0 / kChunk) * D);
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const int col = g.lane + v * G;
+      out[v] = col < p.ncol ? __ldcg(src + col) : f4_zero();
+    }
+    return;
+  }
+  Acc4 acc[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
   if (len == 1) {
     if (staged) {
-      const double sc = p.mean ? 1.0 / (double)first.y : 1.0;
+      const double sc = 1.0 / (double)first.y;  // mean pooling
 #pragma unroll
       for (int v = 0; v < VPL; ++v) {
         const float4 t = staged[v * stride];
@@ -302,16 +321,6 @@ __device__ __forceinline__ void key_grad(const GroupCtx<G>& g, const UpdateParam
       }
     } else {
       add_terms<G, VPL, 1, GP, GU>(g, p, make_src(p, first), 0, 1, acc);
-    }
-  } else if (len > kShortSeg) {
-    const float4* src = reinterpret_cast<const float4*>(p.gbuf + (int64_t)(s0 / kChunk) * D);
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      const int col = g.lane + v * G;
-      if (col < p.ncol) {
-        const float4 t = __ldcg(src + col);
-        acc[v] = Acc4{(double)t.x, (double)t.y, (double)t.z, (double)t.w};
-      }
     }
   } else {
     for (int base = 0; base < len; base += G) {
@@ -322,6 +331,8 @@ __device__ __forceinline__ void key_grad(const GroupCtx<G>& g, const UpdateParam
         add_terms<G, VPL, K, GP, GU>(g, p, s, k0, m - k0 < K ? m - k0 : K, acc);
     }
   }
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) out[v] = acc_round(acc[v]);
 }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -412,10 +423,10 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
     const int stage = (int)(k % S);
     const KeyIdx cur = *key_slot(stage);
     const bool staged_grad = GP && !GU && cur.s1 - cur.s0 == 1;
-    Acc4 acc[VPL];
+    float4 grad[VPL];
     cp_async_wait<S - 1>();
     key_grad<G, VPL, GP, GU>(g, p, cur.s0, cur.s1, cur.first,
-                             staged_grad ? slot(stage, NR * VPL) : nullptr, nt, acc);
+                             staged_grad ? slot(stage, NR * VPL) : nullptr, nt, grad);
     if (cur.row >= 0) {
       RowRegs<VPL, ADAM> r;
 #pragma unroll
@@ -424,7 +435,7 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
         r.s1[v] = *slot(stage, 1 * VPL + v);
         if (ADAM) r.s2[v] = *slot(stage, 2 * VPL + v);
       }
-      apply_update<G, VPL, ADAM>(g, p, cur.row, r, acc);
+      apply_update<G, VPL, ADAM>(g, p, cur.row, r, grad);
     }
   }
   pdl_trigger();
@@ -443,9 +454,9 @@ __global__ void __launch_bounds__(256, 2) row_update_wide_kernel(const __grid_co
     const KeyIdx k = key_idx(p, u);
     RowRegs<VPL, ADAM> r;
     load_row<G, VPL, ADAM>(g, p, k.row, r);
-    Acc4 acc[VPL];
-    key_grad<G, VPL, GP, GU>(g, p, k.s0, k.s1, k.first, nullptr, 0, acc);
-    apply_update<G, VPL, ADAM>(g, p, k.row, r, acc);
+    float4 grad[VPL];
+    key_grad<G, VPL, GP, GU>(g, p, k.s0, k.s1, k.first, nullptr, 0, grad);
+    apply_update<G, VPL, ADAM>(g, p, k.row, r, grad);
   }
   pdl_trigger();
 }
@@ -506,7 +517,7 @@ static cudaError_t launch_update_t(const UpdateParams& p, bool adam, int64_t uca
 }
 
 cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pooled,
-                          const float* grad_unpooled, int64_t, float lr_t, float sqrt_bc2,
+                          const float* grad_unpooled, int64_t, float lr_t, float inv_sqrt_bc2,
                           cudaStream_t s) {
   UpdateParams p;
   p.N = b->N;
@@ -536,7 +547,7 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.beta2 = (float)t->cfg.beta2;
   p.omb1 = (float)(1.0 - t->cfg.beta1);
   p.omb2 = (float)(1.0 - t->cfg.beta2);
-  p.sqrt_bc2 = sqrt_bc2;
+  p.inv_sqrt_bc2 = inv_sqrt_bc2;
   if (p.N == 0) return cudaSuccess;
   const bool adam = t->cfg.optimizer == RECIS_ADAM;
   const int64_t ucap = b->N;  // U <= N; groups past U return at once
