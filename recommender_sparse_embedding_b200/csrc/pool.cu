@@ -350,9 +350,14 @@ int group_lanes_for(int D) {
 
 int64_t pool_chunk_for(int64_t N, int D) {
   const int G = group_lanes_for(D);
-  // enough groups for about one full wave of 148 SMs x 2048 threads
+  // enough groups for about one wave of the kernel's resident threads (3, 2
+  // or 1 CTAs of 256 per SM by row width, as its launch bounds say), so each
+  // group walks as long a chunk as that allows
+  const int ncol = D / 4;
+  const int vpl = ncol <= 32 ? 1 : (ncol <= 64 ? 2 : 4);
+  const int64_t resident = (int64_t)kSMs * 256 * (vpl == 1 ? 3 : (vpl == 2 ? 2 : 1));
   int64_t C = 8;
-  while (C < 256 && (N / (C * 2)) * G >= (int64_t)kSMs * 2048) C *= 2;
+  while (C < 256 && (N / (C * 2)) * G >= resident) C *= 2;
   return C;
 }
 
