@@ -67,7 +67,7 @@ struct BatchDev {
   unsigned int U;               // unique keys of the last lookup
   unsigned int n_new;           // new keys of the last lookup
   unsigned int nlong;           // chunks of kShortSeg positions holding a long segment
-  unsigned int pad;
+  unsigned int nmulti;          // keys seen 2 to kShortSeg times (sample-sort path)
 };
 
 // ---------------------------------------------------------------- table
@@ -147,6 +147,7 @@ struct recis_batch {
   double* partials = nullptr;
   float* gbuf = nullptr;          // [chunks][D] reduced gradients of long segments
   int32_t* long_chunks = nullptr; // [chunks] chunks holding a long segment (sample-sort path)
+  int32_t* multi_keys = nullptr;  // [N/2] unique keys seen 2 to kShortSeg times (sample-sort path)
   int32_t* chunk_counter = nullptr;  // [chunks][2] block-level tickets of the backward
   int64_t capGbuf = 0;            // floats
   recis::BatchDev* bdev = nullptr;

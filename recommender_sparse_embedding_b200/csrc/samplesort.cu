@@ -328,6 +328,7 @@ struct SsParams {
   int32_t* seg_start;
   BatchDev* bdev;
   int32_t* long_chunks;     // chunks (kShortSeg positions) holding a long segment
+  int32_t* multi_keys;      // keys seen 2 to kShortSeg times (appended by ss_finish)
   DevState* st;
   HostMirror* mirror;
 };
@@ -420,6 +421,7 @@ __global__ void __launch_bounds__(kCountThreads) ss_count_kernel(const __grid_co
     p.ctl->ticket_scan = 0;
     p.ctl->ticket_local = 0;
     p.bdev->nlong = 0;
+    p.bdev->nmulti = 0;
     p.bdev->row_base = *(volatile unsigned long long*)&p.st->next_free;
   }
   __syncthreads();
@@ -1149,6 +1151,10 @@ struct FinishShared {
   unsigned long long warp[kFinThreads / 32];
   unsigned chunk_long;  // bit c: chunk c (kShortSeg positions) of this CTA holds a long segment
   int ninit;
+  unsigned heads[kSub / 32];        // bit i: position i of this CTA is a head
+  int32_t multi[kSub / 2];          // keys of this CTA seen 2 to kShortSeg times
+  int nmulti;
+  unsigned multi_base;
 };
 static_assert(kSub / kShortSeg <= 32, "one bit per chunk of a finish CTA");
 
@@ -1162,6 +1168,7 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
   if (tid == 0) {
     sh.ninit = 0;
     sh.chunk_long = 0;
+    sh.nmulti = 0;
   }
   __syncthreads();
   const int64_t q0 = (int64_t)blockIdx.x * kSub + tid;
@@ -1183,6 +1190,13 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
     const unsigned long long tot = scan_cta_totals<kFinThreads>(
         p, sh.warp, [&](int i, unsigned long long v) { sh.cpre[i] = v; });
     if (blockIdx.x == 0 && tid == 0) publish_totals(p, tot, row_base);
+  }
+  // head bits of this CTA's positions (position j*kFinThreads + 32w + lane)
+#pragma unroll
+  for (int j = 0; j < kFinItems; ++j) {
+    const int64_t q = q0 + j * kFinThreads;
+    const unsigned hb = __ballot_sync(0xffffffffu, q < p.N && ((mt[j] >> 43) & 1u));
+    if (lane == 0) sh.heads[(j * kFinThreads) / 32 + w] = hb;
   }
   __syncthreads();
 #pragma unroll
@@ -1223,10 +1237,24 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
       p.uniq[seg] = key;
       p.rows[seg] = row;
       p.seg_start[seg] = (int32_t)q;
+      // a short segment (not long) whose next position is no head holds 2 to
+      // kShortSeg occurrences: listed for the row update
+      if (p.multi_keys && !(m >> 63)) {
+        const int i = tid + j * kFinThreads + 1;  // next position within this CTA
+        bool next_head;
+        if (q + 1 >= p.N) next_head = true;
+        else if (i < kSub) next_head = (sh.heads[i >> 5] >> (i & 31)) & 1u;
+        else next_head = (__ldcs(p.meta + q + 1) >> 43) & 1u;
+        if (!next_head) sh.multi[atomicAdd(&sh.nmulti, 1)] = (int32_t)seg;
+      }
     }
   }
-  // chunks of this CTA holding a long segment, for the backward's reduction
+  // chunks of this CTA holding a long segment, for the backward's reduction,
+  // and its keys seen 2 to kShortSeg times
   __syncthreads();
+  if (tid == 0 && sh.nmulti > 0) sh.multi_base = atomicAdd(&p.bdev->nmulti, (unsigned)sh.nmulti);
+  __syncthreads();
+  for (int i = tid; i < sh.nmulti; i += kFinThreads) p.multi_keys[sh.multi_base + i] = sh.multi[i];
   if (w == 0) {
     const bool has = (sh.chunk_long >> lane) & 1u;
     const unsigned bal = __ballot_sync(0xffffffffu, has);
@@ -1351,6 +1379,7 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   p.seg_start = b->seg_start;
   p.bdev = b->bdev;
   p.long_chunks = b->long_chunks;
+  p.multi_keys = b->multi_keys;
   p.st = t->dstate;
   p.mirror = t->mirror_dev;
 

@@ -373,7 +373,8 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
         (e = realloc_dev(b->spos, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->gsrc, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->gfirst, cap, true)) != cudaSuccess ||
-        (e = realloc_dev(b->seg_counter, cap, true)) != cudaSuccess)
+        (e = realloc_dev(b->seg_counter, cap, true)) != cudaSuccess ||
+        (e = realloc_dev(b->multi_keys, cap / 2 + 1, false)) != cudaSuccess)
       return cuda_fail(e, "batch alloc");
     const int64_t st = (cap + kSortTile - 1) / kSortTile;
     if ((e = realloc_dev(b->sort_lookback, (size_t)st * 256, true)) != cudaSuccess)
@@ -456,6 +457,7 @@ static void batch_free(recis_batch* b) {
   cudaFree(b->partials);
   cudaFree(b->gbuf);
   cudaFree(b->long_chunks);
+  cudaFree(b->multi_keys);
   cudaFree(b->chunk_counter);
   cudaFree(b->bdev);
   cudaFree(b->chunk_bag);

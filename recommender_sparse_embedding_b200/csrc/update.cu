@@ -53,6 +53,7 @@ struct UpdateParams {
   double* partials;         // [nchunks][2][D]
   int32_t* counters;        // [U] last-arrival tickets (self-resetting)
   int32_t* chunk_counters;  // [nchunks][2] block-level tickets (self-resetting)
+  const int32_t* multi_keys;  // keys seen 2 to kShortSeg times (bdev->nmulti of them), or null
   // optimiser
   float lr;        // Adagrad: lr; Adam: lr / (1 - beta1^t)
   float eps;
@@ -360,6 +361,22 @@ __device__ __forceinline__ KeyIdx key_idx(const UpdateParams& p, int64_t u) {
   return k;
 }
 
+// The listed keys (seen 2 to kShortSeg times) i = gid, gid + groups, ...:
+// indices, row and gradient rows loaded, then the update.  Kept out of line
+// so that the staged key walk of the row update is allocated on its own.
+template <int G, int VPL, bool ADAM, bool GP, bool GU>
+__device__ __noinline__ void update_listed(const UpdateParams& p, int64_t gid, int64_t groups, int64_t nm) {
+  const GroupCtx<G> g;
+  for (int64_t i = gid; i < nm; i += groups) {
+    const KeyIdx k = key_idx(p, __ldg(p.multi_keys + i));
+    RowRegs<VPL, ADAM> r;
+    load_row<G, VPL, ADAM>(g, p, k.row, r);
+    float4 grad[VPL];
+    key_grad<G, VPL, GP, GU>(g, p, k.s0, k.s1, k.first, nullptr, 0, grad);
+    apply_update<G, VPL, ADAM>(g, p, k.row, r, grad);
+  }
+}
+
 // A persistent grid of G-lane groups walks the unique keys u = gid, gid +
 // groups, ... (U from the lookup), S keys deep: while key u is
 // updated, the next S-1 keys' rows [emb | state] (and a singleton's
@@ -384,13 +401,22 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
   const int64_t U = (int64_t)p.bdev->U;
   const int D = p.ncol * 4;
   const int64_t u0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  // Keys seen 2 to kShortSeg times first, spread evenly over the groups,
+  // when there are a few per group: their gradient rows are gathered when
+  // the key is updated, so drawn by the stride below they would pile up in
+  // some groups.  The walk then skips them.  (With many per group the walk's
+  // staging is worth more than the balance; every group decides alike.)
+  const int64_t nm = p.multi_keys ? (int64_t)p.bdev->nmulti : 0;
+  const bool listed = p.multi_keys != nullptr && nm <= 4 * groups;
+  if (listed) update_listed<G, VPL, ADAM, GP, GU>(p, u0, groups, nm);
+  auto is_listed = [&](const KeyIdx& k) { return listed && k.s1 - k.s0 > 1 && k.s1 - k.s0 <= kShortSeg; };
   if (u0 >= U) return;
   KeyIdx* s_keys = reinterpret_cast<KeyIdx*>(s_stage + S * NS * nt);
   auto key_slot = [&](int st) -> KeyIdx* { return s_keys + st * ngrp + grp; };
   auto slot = [&](int stage, int sl) -> float4* { return s_stage + ((stage * NS + sl) * nt + tid); };
   auto issue = [&](int stage, const KeyIdx& k) {
     if (g.lane == 0) *key_slot(stage) = k;
-    if (k.row < 0) return;
+    if (k.row < 0 || is_listed(k)) return;
     const float* base = p.row_data + (int64_t)k.row * p.row_floats;
     const bool stage_grad = GP && !GU && k.s1 - k.s0 == 1;
     const float* gsrc_row = p.gp + (int64_t)k.first.x * D;
@@ -425,6 +451,7 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
     const bool staged_grad = GP && !GU && cur.s1 - cur.s0 == 1;
     float4 grad[VPL];
     cp_async_wait<S - 1>();
+    if (is_listed(cur)) continue;  // updated above
     key_grad<G, VPL, GP, GU>(g, p, cur.s0, cur.s1, cur.first,
                              staged_grad ? slot(stage, NR * VPL) : nullptr, nt, grad);
     if (cur.row >= 0) {
@@ -530,6 +557,7 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   // long-segment marks and the long-chunk list come from the sample-sort dedup
   p.meta = b->N <= kSampleSortMaxN ? b->ss_meta : nullptr;
   p.long_chunks = b->N <= kSampleSortMaxN ? b->long_chunks : nullptr;
+  p.multi_keys = b->N <= kSampleSortMaxN ? b->multi_keys : nullptr;
   p.seg_of = b->seg_of;
   p.seg_start = b->seg_start;
   p.rows = b->rows;
