@@ -9,7 +9,7 @@ one dim-64 fp32 table with Adam state, sum pooling); `--workload` selects the
 others (seq8, longseq, tiny) for profiling.
 
 Prints one JSON line: IDs/s (device time, inputs resident, L2 flushed between
-steps), the same through the API with host buffers (e2e), the roofline of the
+steps), the same through the API with host buffers and pipelined copies (e2e), the roofline of the
 dominant kernel, SM clocks sampled during the timed region, and the CPU
 oracle's rate on this host as a baseline.
 
@@ -327,14 +327,16 @@ def run_gpu(args):
     stream = torch.cuda.current_stream()
     combiner = [R.SUM if t.combiner == "sum" else R.MEAN for t in w.tables]
 
-    def run_step(vals, foffs, per_table, n, kbuf):
+    def run_step(vals, foffs, per_table, n, kbuf, pooled_bufs=None, unpooled_bufs=None):
+        pb = pooled if pooled_bufs is None else pooled_bufs
+        ub = unpooled if unpooled_bufs is None else unpooled_bufs
         k = kbuf[:n]
         R.feature_hash(feats, vals, foffs, keys_out=k)
         for i, t in enumerate(w.tables):
             lo, hi, bo, gp, gu = per_table[i]
-            up = unpooled[i][: hi - lo] if unpooled[i] is not None else None
+            up = ub[i][: hi - lo] if ub[i] is not None else None
             tables[i].lookup_pooled(batches[i], k[lo:hi], bo, len(t.features), w.B, combiner[i],
-                                    pooled_out=pooled[i], unpooled_out=up)
+                                    pooled_out=pb[i], unpooled_out=up)
             tables[i].backward_update(batches[i], gp, gu)
         return n
 
@@ -392,51 +394,86 @@ def run_gpu(args):
     for t in tables:
         t.status_sync()
 
-    # ---- e2e through the API with host buffers (pinned), copies inside the timing
+    # ---- e2e through the API with host buffers (pinned), copies inside the timing.
+    # Steps are pipelined the way a training loop feeds the engine: step j+1's
+    # inputs go up on a copy stream while step j computes, and step j's pooled
+    # rows come down on another, so the two PCIe directions and the kernels
+    # overlap.  Two sets of device buffers alternate.  The timed region runs
+    # from the first copy up to the last copy down and holds every step's
+    # copies, its L2 flush and its kernels.
     e2e_ids, h2d, d2h = 0, 0, 0
     pin = [dev_batch(b, g, pin=True) for b, g in host[: min(4, n_distinct)]]
-    dv = torch.empty(maxN, dtype=torch.int64, device=dev)
-    dbo = [torch.empty(w.F * w.B + 1, dtype=torch.int64, device=dev) for _ in w.tables]
-    dgp = [torch.empty_like(p) if p is not None else None for p in pooled]
-    dgu = [torch.empty_like(u) if u is not None else None for u in unpooled]
+    NBUF = 2
+    dv = [torch.empty(maxN, dtype=torch.int64, device=dev) for _ in range(NBUF)]
+    dbo = [[torch.empty(w.F * w.B + 1, dtype=torch.int64, device=dev) for _ in w.tables] for _ in range(NBUF)]
+    dgp = [[torch.empty_like(p) if p is not None else None for p in pooled] for _ in range(NBUF)]
+    dgu = [[torch.empty_like(u) if u is not None else None for u in unpooled] for _ in range(NBUF)]
+    dpool = [[torch.empty_like(p) if p is not None else None for p in pooled] for _ in range(NBUF)]
     pooled_h = [torch.empty(p.shape, dtype=p.dtype).pin_memory() if p is not None else None
                 for p in pooled]
     e2e_steps = max(3, min(args.steps, 50) // 2)
-    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(e2e_steps)]
-    torch.cuda.synchronize()
-    for j in range(e2e_steps):
+    up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_up = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_down = [torch.cuda.Event() for _ in range(e2e_steps)]
+    t_first, t_last = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def upload(j):
+        """Step j's inputs into buffer set j % NBUF (once step j - NBUF is done with it)."""
+        nonlocal h2d
         vals_h, foffs, per_h, n = pin[j % len(pin)]
-        flush.zero_()
-        eev[j][0].record(stream)
-        v = dv[:n]
-        v.copy_(vals_h, non_blocking=True)
-        h2d = vals_h.numel() * 8
-        per_d = []
-        for i, (lo, hi, bo_h, gp_h, gu_h) in enumerate(per_h):
-            bo = dbo[i][: bo_h.numel()]
-            bo.copy_(bo_h, non_blocking=True)
-            h2d += bo_h.numel() * 8
-            gp = gu = None
-            if gp_h is not None:
-                gp = dgp[i]
-                gp.copy_(gp_h, non_blocking=True)
-                h2d += gp_h.numel() * 4
-            if gu_h is not None:
-                gu = dgu[i][: gu_h.shape[0]]
-                gu.copy_(gu_h, non_blocking=True)
-                h2d += gu_h.numel() * 4
-            per_d.append((lo, hi, bo, gp, gu))
-        run_step(v, foffs, per_d, n, keys)
-        d2h = 0
-        for i, ph in enumerate(pooled_h):
-            if ph is not None:
-                ph.copy_(pooled[i], non_blocking=True)
-                d2h += ph.numel() * 4
-        eev[j][1].record(stream)
-        e2e_ids += n
+        sb = j % NBUF
+        with torch.cuda.stream(up_s):
+            if j >= NBUF:
+                up_s.wait_event(ev_done[j - NBUF])
+            v = dv[sb][:n]
+            v.copy_(vals_h, non_blocking=True)
+            nb = vals_h.numel() * 8
+            per_d = []
+            for i, (lo, hi, bo_h, gp_h, gu_h) in enumerate(per_h):
+                bo = dbo[sb][i][: bo_h.numel()]
+                bo.copy_(bo_h, non_blocking=True)
+                nb += bo_h.numel() * 8
+                gp = gu = None
+                if gp_h is not None:
+                    gp = dgp[sb][i]
+                    gp.copy_(gp_h, non_blocking=True)
+                    nb += gp_h.numel() * 4
+                if gu_h is not None:
+                    gu = dgu[sb][i][: gu_h.shape[0]]
+                    gu.copy_(gu_h, non_blocking=True)
+                    nb += gu_h.numel() * 4
+                per_d.append((lo, hi, bo, gp, gu))
+            ev_up[j].record(up_s)
+        h2d = nb
+        return v, foffs, per_d, n
+
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
+    t_first.record(up_s)
+    staged = upload(0)
+    for j in range(e2e_steps):
+        nxt = upload(j + 1) if j + 1 < e2e_steps else None
+        sb = j % NBUF
+        stream.wait_event(ev_up[j])
+        if j >= NBUF:
+            stream.wait_event(ev_down[j - NBUF])  # pooled buffers of set sb copied down
+        flush.zero_()
+        v, foffs, per_d, n = staged
+        run_step(v, foffs, per_d, n, keys, pooled_bufs=dpool[sb])
+        ev_done[j].record(stream)
+        with torch.cuda.stream(down_s):
+            down_s.wait_event(ev_done[j])
+            d2h = 0
+            for i, ph in enumerate(pooled_h):
+                if ph is not None:
+                    ph.copy_(dpool[sb][i], non_blocking=True)
+                    d2h += ph.numel() * 4
+            ev_down[j].record(down_s)
+        e2e_ids += n
+        staged = nxt
+    t_last.record(down_s)
+    torch.cuda.synchronize()
+    e2e_ms = t_first.elapsed_time(t_last)
     for t in tables:
         t.status_sync()
 
@@ -504,7 +541,9 @@ def run_gpu(args):
             "step_alg_gbs": step_alg / (dev_ms / args.steps / 1e3) / 1e9,
             "step_frac_of_peak": step_alg / (dev_ms / args.steps / 1e3) / 1e9 / peak,
             "e2e": {"value": e2e_value, "unit": "IDs/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h,
+                    "note": "steps pipelined: step j+1's inputs up and step j-1's pooled rows down "
+                            "overlap step j's kernels; timed from the first copy up to the last copy down"},
             "gpu_launches": launches,
             "kernels": kern,
             "kernels_note": f"CUDA events around every launch, {prof_steps} further steps after the "

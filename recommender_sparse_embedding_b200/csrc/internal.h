@@ -129,7 +129,6 @@ struct recis_batch {
   int64_t* rows = nullptr;
   int32_t* inv = nullptr;
   int32_t* seg_of = nullptr;    // segment (unique index) of each sorted position
-  uint32_t* svals = nullptr;    // occurrence index of each sorted position
   int32_t* seg_start = nullptr; // [U+1] first sorted position of each unique
   uint32_t* spos = nullptr;     // [capN] sorted position of each occurrence
   int4* gsrc = nullptr;         // [capN] per sorted position: {gradient row, bag length, occurrence, 0}

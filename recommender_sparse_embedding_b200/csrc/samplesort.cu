@@ -5,8 +5,8 @@
 //
 // It produces exactly what the radix-sort path (sort.cu + unique.cu) produces:
 // unique keys ascending, inverse index, rows (new keys get rows in ascending
-// key order), segment starts, the segment and the occurrence of each sorted
-// position, and initialised new rows.  The digit passes are replaced by six
+// key order), segment starts, the segment of each sorted position, the
+// sorted position of each occurrence, and initialised new rows.  The digit passes are replaced by six
 // short launches, none of which waits on another CTA:
 //   ss_rank      a strided sample of the keys (4096 or 8192 by batch size) is
 //                sorted by ranking: every sample's rank is its count of
@@ -324,7 +324,6 @@ struct SsParams {
   int32_t* inv;
   uint32_t* spos;
   int32_t* seg_of;
-  uint32_t* svals;
   int32_t* seg_start;
   BatchDev* bdev;
   int32_t* long_chunks;     // chunks (kShortSeg positions) holding a long segment
@@ -1211,7 +1210,6 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
                                                    : __ldg(&p.ctl->cta_pre[b >> p.local_bpc_shift]);
     const unsigned seg = (unsigned)(cpre & 0xffffffffULL) + __ldg(&p.ctl->hpre[b]) + lh - 1u;
     p.seg_of[q] = (int32_t)seg;
-    p.svals[q] = occ[j];
     if (occ[j] < (uint32_t)p.N) {
       p.inv[occ[j]] = (int32_t)seg;
       p.spos[occ[j]] = (uint32_t)q;
@@ -1375,7 +1373,6 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   p.inv = b->inv;
   p.spos = b->spos;
   p.seg_of = b->seg_of;
-  p.svals = b->svals;
   p.seg_start = b->seg_start;
   p.bdev = b->bdev;
   p.long_chunks = b->long_chunks;

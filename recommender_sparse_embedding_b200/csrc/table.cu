@@ -367,7 +367,6 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
         (e = realloc_dev(b->rows, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->inv, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_of, cap, true)) != cudaSuccess ||
-        (e = realloc_dev(b->svals, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->ss_meta, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_start, cap + 1, true)) != cudaSuccess ||
         (e = realloc_dev(b->spos, cap, true)) != cudaSuccess ||
@@ -447,7 +446,6 @@ static void batch_free(recis_batch* b) {
   cudaFree(b->rows);
   cudaFree(b->inv);
   cudaFree(b->seg_of);
-  cudaFree(b->svals);
   cudaFree(b->seg_start);
   cudaFree(b->spos);
   cudaFree(b->gsrc);

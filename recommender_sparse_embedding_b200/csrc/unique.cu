@@ -98,7 +98,6 @@ struct UniqueParams {
   int32_t* inv;
   uint32_t* spos;           // [N] sorted position of each occurrence
   int32_t* seg_of;
-  uint32_t* svals;
   int32_t* seg_start;
   BatchDev* bdev;
   DevState* st;
@@ -271,7 +270,6 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
     }
     const int32_t seg = (int32_t)(hrun - 1);
     p.seg_of[pos] = seg;
-    p.svals[pos] = v[j];
     if (v[j] < (uint64_t)N) {
       p.inv[v[j]] = seg;
       p.spos[v[j]] = (uint32_t)pos;
@@ -347,7 +345,6 @@ cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cuda
   p.inv = b->inv;
   p.spos = b->spos;
   p.seg_of = b->seg_of;
-  p.svals = b->svals;
   p.seg_start = b->seg_start;
   p.bdev = b->bdev;
   p.st = t->dstate;
