@@ -6,37 +6,41 @@
 // It produces exactly what the radix-sort path (sort.cu + unique.cu) produces:
 // unique keys ascending, inverse index, rows (new keys get rows in ascending
 // key order), segment starts, the segment of each sorted position, the
-// sorted position of each occurrence, and initialised new rows.  The digit passes are replaced by six
-// short launches, none of which waits on another CTA:
-//   ss_rank      a strided sample of the keys (4096 or 8192 by batch size) is
-//                sorted by ranking: every sample's rank is its count of
-//                smaller samples (ties by position), spread over many CTAs.
+// sorted position of each occurrence, and initialised new rows; besides,
+// the marks and lists the backward uses (positions in long segments, chunks
+// holding one, keys seen 2 to kShortSeg times).  The digit passes are
+// replaced by short launches, none of which waits on another CTA:
+//   ss_rank      (first call of a batch) a strided sample of 4096 or 8192
+//                keys is sorted by ranking: every sample's rank is its count
+//                of smaller samples (ties by position), over many CTAs.
+//   ss_probe     (second stream, beside the three below) the IDMap
+//                find-or-insert of every occurrence: a missing key claims a
+//                free slot by CAS; its row is assigned by ss_finish.
 //   ss_count     per tile of 2048 keys: up to 2047 (batches of at most
-//                327680 keys) or 1023 distinct splitters from the
-//                sorted sample, the bucket of every key (key u goes to bucket
-//                2r + [u == split[r]], r = #splitters < u, so buckets are
-//                ordered by key and a key equal to a splitter -- a hot key --
-//                has a bucket of its own), the tile's bucket histogram, and
-//                the IDMap find-or-insert of every occurrence (a missing key
-//                claims a free slot by CAS; its row is assigned later).
+//                327680 keys) or 1023 distinct splitters from the sorted
+//                sample or the previous call's quantiles, the bucket of every
+//                key (key u goes to bucket 2r + [u == split[r]],
+//                r = #splitters < u, so buckets are ordered by key and a key
+//                equal to a splitter -- a hot key -- has a bucket of its
+//                own), and the tile's bucket histogram.
 //   ss_tilescan  per bucket, the exclusive prefix of the tile histograms (so
 //                the scatter is stable); the last CTA scans the bucket totals
 //                into bucket starts.
 //   ss_scatter   moves (key, occurrence) into bucket order, stably.
-//   ss_local     one CTA per key-range bucket and the equality bucket after
-//                it.  A key-range bucket is sorted by (key, occurrence): up
-//                to 4 keys per thread in registers (lanes of a warp exchange
-//                by shuffles, warps through shared memory), larger buckets in
-//                shared memory.  An equality bucket holds one key, already in
-//                occurrence order.  Heads (first position of each distinct
-//                key) and new keys are numbered within the bucket, and the
+//   ss_local     sorts every key-range bucket by (key, occurrence): one warp
+//                per bucket (batches of at most 327680 keys: 64-bit words of
+//                key and position in registers, up to 16 per lane), else one
+//                CTA per bucket (up to 4 pairs per thread in registers, or
+//                shared memory); an equality bucket holds one key, already
+//                in occurrence order.  Heads (first position of each distinct
+//                key) and new keys are numbered within the bucket and the
 //                bucket counts summed within the CTA; the CTA totals are
 //                scanned by the last CTA (one CTA per bucket) or by every
 //                finish CTA (one warp per bucket: a few hundred totals).
 //   ss_finish    a flat pass over the sorted positions writes every output and
 //                initialises the new rows.
 // A key-range bucket larger than shared memory (only for adversarial key
-// orders) is sorted by the same network in global memory.
+// orders) is sorted by the CTA network in global memory.
 #include <climits>
 
 #include "internal.h"

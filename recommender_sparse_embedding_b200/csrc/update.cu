@@ -5,8 +5,9 @@
 // parameters in the EmbeddingBlocks).
 //
 // The dedup left the sorted positions grouped by unique key: segment u spans
-// sorted positions seg_start[u] .. seg_start[u+1]-1, position q holds
-// occurrence vals[q].  The gradient of u is
+// sorted positions seg_start[u] .. seg_start[u+1]-1, and the pooling
+// recorded each position's gradient source (pooled-gradient row, bag length,
+// occurrence).  The gradient of u is
 //   g(u) = sum over its positions of grad_pooled[bag] * (1 or 1/length)
 //          + grad_unpooled[occurrence],
 // summed in fp64 in position order and rounded once to fp32.  Two launches:
@@ -21,7 +22,9 @@
 //   row_update  one lane group per unique key loads the row [emb | state],
 //               sums the key's gradient terms itself when the segment is
 //               short (all loads issued before the sum) or reads gbuf, and
-//               applies Adagrad or Adam in place.
+//               applies Adagrad or Adam in place.  Keys seen 2 to kShortSeg
+//               times come from the dedup's list, spread evenly over the
+//               groups, when there are a few per group.
 // No float atomics anywhere; the result does not depend on scheduling.
 #include "segreduce.cuh"
 
@@ -387,7 +390,8 @@ __device__ __noinline__ void update_listed(const UpdateParams& p, int64_t gid, i
 // its lane 0, read after __syncwarp).  Other keys' gradients (repeated keys,
 // long segments, unpooled gradients) are gathered while the key is updated.
 // Pipeline depth: 4 when each group walks many keys (long-sequence batches),
-// 2 otherwise (filling and draining a deep pipeline costs more than it hides).
+// 2 otherwise (measured: 3 or 4 keys deep, or a fourth CTA per SM, only
+// lengthen every request on the 26-feature step).
 template <int G, int VPL, bool ADAM, bool GP, bool GU, int S>
 __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constant__ UpdateParams p) {
   pdl_wait();
