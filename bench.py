@@ -74,6 +74,23 @@ def _config(w: W.Workload, extra=None):
 
 
 # ------------------------------------------------------------------ CPU oracle
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, the nominal figure (the measured copy peak is the roofline)
+
+
+def _host_cpu() -> str:
+    """CPU model and hardware threads of this host, for the CPU baseline."""
+    model = "unknown CPU"
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for ln in fh:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return f"{model}, {os.cpu_count()} hardware threads"
+
+
 def _oracle_rate(w: W.Workload, budget_s: float, batches):
     """The CPU oracle (single thread) on full steps of the workload, ~budget_s."""
     import oracle as O
@@ -99,7 +116,7 @@ def _oracle_rate(w: W.Workload, budget_s: float, batches):
         if time.perf_counter() - t0 >= budget_s:
             break
     el = sum(times)
-    return {"value": n_ids / el, "unit": "IDs/s", "cores": 1, "kind": "oracle",
+    return {"value": n_ids / el, "unit": "IDs/s", "cores": 1, "kind": "oracle", "host": _host_cpu(),
             "sample": f"{steps} full {w.name} steps (feature hash + lookup + backward/"
                       f"optimiser) on the single-threaded CPU oracle, {el:.1f} s",
             "ms_per_step": 1e3 * el / steps, "steps": steps}
@@ -133,7 +150,7 @@ def run_reference(args):
             "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64-accumulate/f32-store", "data": "synthetic",
             "config": _config(w),
-            "cpu_baseline": {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "cpu_baseline": {k: res[k] for k in ("value", "unit", "cores", "kind", "sample", "host")},
             "e2e": {"value": res["value"], "unit": "IDs/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -521,6 +538,7 @@ def run_gpu(args):
                 roof = {"bound": "hbm", "kernel": top, "row": grp,
                         "row_kernels": members, "achieved": achieved, "peak": peak,
                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                        "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                         "traffic": traffic, "traffic_note": tnote,
                         "alg_bytes_per_launch": per_launch,
                         "note": ("algorithmic bytes of the row / its kernels' event time"
@@ -552,7 +570,7 @@ def run_gpu(args):
         }
         if world == 1 and not args.no_cpu_baseline:
             res = _oracle_rate(w, args.cpu_seconds, host[:2])
-            line["cpu_baseline"] = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")}
+            line["cpu_baseline"] = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample", "host")}
         print(json.dumps(line), flush=True)
 
     for t in tables:
