@@ -797,7 +797,7 @@ recis_status recis_lookup_pooled(recis_table_t t, recis_batch_t b, const int64_t
     set_error("lookup_pooled: pooled_out and unpooled_out are both null");
     return RECIS_ERR_INVALID_ARG;
   }
-  LookupArgs a{t, b, keys, N, bag_offsets, F, B, combiner, pooled_out, unpooled_out, nullptr};
+  LookupArgs a{t, b, keys, N, bag_offsets, F, B, combiner, pooled_out, unpooled_out, nullptr, false};
   return lookup_impl(a, (cudaStream_t)stream);
 }
 
