@@ -35,13 +35,15 @@ def _ofeat(f: W.FeatureSpec):
 class Pair:
     """One logical table on both sides."""
 
-    def __init__(self, R, spec: W.TableSpec, initial_capacity=0, block_rows=0):
+    def __init__(self, R, spec: W.TableSpec, initial_capacity=0, block_rows=0, init_acc=0.0):
         opt_r = R.ADAGRAD if spec.optimizer == "adagrad" else R.ADAM
         opt_o = O.ADAGRAD if spec.optimizer == "adagrad" else O.ADAM
         self.spec = spec
         self.gpu = R.Table(spec.dim, opt_r, spec.lr, init_seed=spec.init_seed,
-                           initial_capacity=initial_capacity, block_rows=block_rows)
-        self.ora = O.Table(spec.dim, opt_o, spec.lr, init_seed=spec.init_seed)
+                           initial_capacity=initial_capacity, block_rows=block_rows,
+                           adagrad_init_acc=init_acc)
+        self.ora = O.Table(spec.dim, opt_o, spec.lr, init_seed=spec.init_seed,
+                           adagrad_init_acc=init_acc)
         self.batch = R.Batch()
         self.combiner_r = R.SUM if spec.combiner == "sum" else R.MEAN
         self.combiner_o = O.SUM if spec.combiner == "sum" else O.MEAN

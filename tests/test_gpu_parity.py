@@ -111,7 +111,7 @@ def test_dims_optimisers_combiners(R, D, opt, comb):
 
 # ---------------------------------------------------------------- edge cases
 def _single(R, keys, lengths, D=16, opt="adagrad", comb="sum", F=1, steps=2, unpooled=False,
-            grad_signed=False):
+            grad_signed=False, init_acc=0.0):
     """Run explicit keys / bag lengths (F features x B bags) on both sides."""
     keys = np.asarray(keys, np.int64)
     lengths = np.asarray(lengths, np.int64)
@@ -121,7 +121,7 @@ def _single(R, keys, lengths, D=16, opt="adagrad", comb="sum", F=1, steps=2, unp
     assert bo[-1] == len(keys)
     spec = W.TableSpec("t", list(range(F)), D, opt, 0.05, comb, pooled=True, unpooled=unpooled,
                        init_seed=5)
-    p = Pair(R, spec)
+    p = Pair(R, spec, init_acc=init_acc)
     k_dev = torch.from_numpy(keys).to(DEV)
     bo_dev = torch.from_numpy(bo).to(DEV)
     N = len(keys)
@@ -146,6 +146,14 @@ def _single(R, keys, lengths, D=16, opt="adagrad", comb="sum", F=1, steps=2, unp
         p.gpu.status_sync()
         compare_tables(p, f"step {step}")
     p.close()
+
+
+def test_adagrad_initial_accumulator(R):
+    # new rows' Adagrad state starts at the table's initial accumulator
+    rng = np.random.default_rng(8)
+    lengths = rng.integers(0, 5, size=600)
+    keys = rng.integers(0, 2000, size=int(lengths.sum()))
+    _single(R, keys, lengths, D=24, opt="adagrad", comb="mean", F=3, init_acc=0.25)
 
 
 def test_empty_batch(R):

@@ -277,16 +277,17 @@ def test_adam_constant_gradient_closed_form():
     assert t.step == 5
 
 
-def _run_vs_torch(opt, steps=3, all_touched=True, eps=None):
+def _run_vs_torch(opt, steps=3, all_touched=True, eps=None, init_acc=0.0):
     D, F, B = 8, 2, 24
     rng = np.random.default_rng(11)
     keys0 = np.unique(rng.integers(0, 1000, size=60))
-    t = O.Table(D, opt, 0.05, eps=eps, init_seed=2)
+    t = O.Table(D, opt, 0.05, eps=eps, init_seed=2, adagrad_init_acc=init_acc)
     t.lookup(keys0, np.array([0, len(keys0)]), 1, 1)  # insert all keys, no update
     _, emb, st = t.export()
     Wt = torch.nn.Parameter(torch.from_numpy(emb.astype(np.float64)))
     if opt == O.ADAGRAD:
-        topt = torch.optim.Adagrad([Wt], lr=0.05, eps=1e-10 if eps is None else eps)
+        topt = torch.optim.Adagrad([Wt], lr=0.05, eps=1e-10 if eps is None else eps,
+                                   initial_accumulator_value=init_acc)
     elif all_touched:
         topt = torch.optim.Adam([Wt], lr=0.05, betas=(0.9, 0.999), eps=1e-8 if eps is None else eps)
     else:
@@ -319,6 +320,13 @@ def _run_vs_torch(opt, steps=3, all_touched=True, eps=None):
 
 def test_adagrad_matches_torch_adagrad():
     t, topt, Wt, st = _run_vs_torch(O.ADAGRAD)
+    np.testing.assert_allclose(st, topt.state[Wt]["sum"].numpy(), rtol=1e-5, atol=1e-6)
+
+
+def test_adagrad_initial_accumulator_matches_torch_adagrad():
+    # a table's Adagrad accumulator starts at adagrad_init_acc, like
+    # torch.optim.Adagrad's initial_accumulator_value
+    t, topt, Wt, st = _run_vs_torch(O.ADAGRAD, init_acc=0.25)
     np.testing.assert_allclose(st, topt.state[Wt]["sum"].numpy(), rtol=1e-5, atol=1e-6)
 
 
