@@ -395,6 +395,7 @@ def run_gpu(args):
         t.status_sync()
     new_rows = [(t.size()[0] - r0) / args.steps for t, r0 in zip(tables, rows0)]
     dev_ms = sum(a.elapsed_time(b) for a, b in ev)
+    step_ms = sorted(a.elapsed_time(b) for a, b in ev)  # this rank's steps, each between its events
 
     # ---- traced region: the same steps again with CUDA events around every
     # launch of the library (per-kernel durations for the roofline)
@@ -548,6 +549,8 @@ def run_gpu(args):
         line = {
             "metric": METRIC, "value": value, "unit": "IDs/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dev_ms / args.steps,
+            "ms_per_step_p50": statistics.median(step_ms),
+            "ms_per_step_p90": step_ms[min(len(step_ms) - 1, round(0.9 * (len(step_ms) - 1)))],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": _config(w, {"ids_per_step": Nm,
