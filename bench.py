@@ -2,20 +2,27 @@
 """Benchmark of the dynamic-hash embedding step (RecIS Embedding Engine hot path).
 
 One step = recis_feature_hash + recis_lookup_pooled + recis_backward_update
-over one batch of a synthetic workload.  The default workload is the
-26-feature one-hot one (26 categorical features, batch 8192, int64 IDs
-Zipf(1.05) over 10^7 per feature, hashed then mod 2^40, tagged and merged into
-one dim-64 fp32 table with Adam state, sum pooling); `--workload` selects the
-others (seq8, longseq, tiny) for profiling.
+over one batch of a synthetic workload.
 
-Prints one JSON line: IDs/s (device time, inputs resident, L2 flushed between
-steps), the same through the API with host buffers and pipelined copies (e2e), the roofline of the
-dominant kernel, SM clocks sampled during the timed region, and the CPU
-oracle's rate on this host as a baseline.
+The headline workload is the large table: about 50M live IDs pre-inserted
+(100 features, dim-64 fp32 rows with Adam m and v beside them, ~38 GB), batch
+65536 x 100 features with bag lengths geometric (mean 5), each occurrence a
+never-seen ID with probability 0.05 (fresh IDs for every step) and otherwise a
+Zipf(1.05) draw over its feature's share of the live set, sum pooling.  The
+same line carries sub-records for the 26-feature one-hot workload (criteo26),
+the long behaviour sequence (longseq) and the 8 multi-hot sequence features
+(seq8); `--workload` selects another headline and `--subs` the sub-records.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+Per workload: IDs/s (device time, inputs resident in HBM, L2 flushed between
+steps), the same through the API with host buffers (e2e: torch copies of
+pinned host buffers around the library's device-pointer calls, pipelined),
+the roofline of the dominant kernel group, SM clocks sampled during the timed
+region, and the CPU oracle's rate on this host as a baseline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--workload NAME] [--subs a,b,c|none]
 Multi-GPU runs (torchrun, one rank per GPU) are independent replicas: each rank
-owns its own table and batches; only the timing is reduced (max over ranks).
+owns its own tables and batches; only the timing is reduced (max over ranks).
 """
 from __future__ import annotations
 
@@ -37,10 +44,14 @@ import numpy as np  # noqa: E402
 import workloads as W  # noqa: E402
 
 METRIC = "lookups/sec (IDs/s) fwd+bwd+update per step; achieved HBM GB/s vs B200 peak"
-DEFAULT_WORKLOAD = "criteo26"
+DEFAULT_WORKLOAD = "large"
+DEFAULT_SUBS = "criteo26,longseq,seq8"
 FALLBACK_HBM_GBS = 6650.0
-CSRC = os.path.join(ROOT, "recommender_sparse_embedding_b200", "csrc")
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, the nominal figure (the measured copy peak is the roofline)
 TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+# the large-table workload's CPU baseline runs at this fraction of its batch
+# and of its live set (the full live set would need ~40 GB of host memory)
+LARGE_ORACLE_SCALE = 16
 
 
 def _peaks():
@@ -58,8 +69,14 @@ def _describe(w: W.Workload) -> str:
                      for t in w.tables)
     f0 = w.features[0]
     tf = "hash->mod 2^40->tag" if f0.flags & W.HASH else "tag"
-    return (f"{w.name}: F={w.F} features, B={w.B}, bag length {w.length}, IDs Zipf({w.zipf_a}) "
-            f"over {w.n_ids:.0e} per feature, {tf}, fp32 tables [{tabs}]")
+    if w.live_ids:
+        ids = (f"{w.live_ids:.0e} live IDs pre-inserted, each occurrence fresh with p={w.fresh_frac} "
+               f"(never-seen IDs every step) else Zipf({w.zipf_a}) over its feature's "
+               f"{w.live_ids // w.F} live IDs")
+    else:
+        ids = f"IDs Zipf({w.zipf_a}) over {w.n_ids:.0e} per feature"
+    return (f"{w.name}: F={w.F} features, B={w.B}, bag length {w.length}, {ids}, {tf}, "
+            f"fp32 tables [{tabs}]")
 
 
 def _config(w: W.Workload, extra=None):
@@ -74,9 +91,6 @@ def _config(w: W.Workload, extra=None):
 
 
 # ------------------------------------------------------------------ CPU oracle
-NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, the nominal figure (the measured copy peak is the roofline)
-
-
 def _host_cpu() -> str:
     """CPU model and hardware threads of this host, for the CPU baseline."""
     model = "unknown CPU"
@@ -91,37 +105,6 @@ def _host_cpu() -> str:
     return f"{model}, {os.cpu_count()} hardware threads"
 
 
-def _oracle_rate(w: W.Workload, budget_s: float, batches):
-    """The CPU oracle (single thread) on full steps of the workload, ~budget_s."""
-    import oracle as O
-    ops = [O.FeatureOp(flags=f.flags, hash_seed=f.hash_seed, mod=f.mod, tag=f.tag,
-                       tag_shift=f.tag_shift, boundaries=list(f.boundaries)) for f in w.features]
-    tabs = [O.Table(t.dim, O.ADAM if t.optimizer == "adam" else O.ADAGRAD, t.lr,
-                    init_seed=t.init_seed) for t in w.tables]
-    n_ids, steps, t0 = 0, 0, time.perf_counter()
-    times = []
-    while True:
-        b, grads = batches[steps % len(batches)]
-        s0 = time.perf_counter()
-        keys = O.feature_hash(ops, b.values, b.feat_offsets)
-        for t, tab, (gp, gu) in zip(w.tables, tabs, grads):
-            lo, hi, bo = b.table_slice(t, w.B)
-            tab.lookup(keys[lo:hi], bo, len(t.features), w.B,
-                       O.SUM if t.combiner == "sum" else O.MEAN, pooled=t.pooled,
-                       unpooled=t.unpooled)
-            tab.backward_update(gp, gu)
-        times.append(time.perf_counter() - s0)
-        n_ids += len(b.values)
-        steps += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    el = sum(times)
-    return {"value": n_ids / el, "unit": "IDs/s", "cores": 1, "kind": "oracle", "host": _host_cpu(),
-            "sample": f"{steps} full {w.name} steps (feature hash + lookup + backward/"
-                      f"optimiser) on the single-threaded CPU oracle, {el:.1f} s",
-            "ms_per_step": 1e3 * el / steps, "steps": steps}
-
-
 def _grads(w: W.Workload, b: W.Batch, seed: int):
     """Upstream gradients of one batch: (grad_pooled, grad_unpooled) per table."""
     out = []
@@ -133,18 +116,73 @@ def _grads(w: W.Workload, b: W.Batch, seed: int):
     return out
 
 
+def _oracle_sample(w: W.Workload):
+    """(workload the oracle runs, its pre-inserted live keys per table or None,
+    a description of the sample).  The large-table workload runs at
+    1/LARGE_ORACLE_SCALE of its batch and live set; the others in full."""
+    if not w.live_ids:
+        return w, None, "full steps"
+    s = LARGE_ORACLE_SCALE
+    ws = w.scaled(w.B // s)
+    ws.live_ids = w.live_ids // s
+    per = ws.live_ids // ws.F
+    live = np.concatenate([(np.int64(ws.features[f].tag) << np.int64(ws.features[f].tag_shift))
+                           | W.live_ids(ws, f, per) for f in range(ws.F)])
+    live.sort()
+    return ws, [live], (f"1/{s}-scale steps: batch {ws.B} x {ws.F} features against a table "
+                        f"pre-filled with {len(live)} live keys (1/{s} of the live set)")
+
+
+def _oracle_rate(w: W.Workload, budget_s: float, nbatch: int = 2):
+    """The CPU oracle (single thread) on steps of the workload for ~budget_s."""
+    import oracle as O
+    ws, live, what = _oracle_sample(w)
+    batches = []
+    for i in range(nbatch):
+        b = W.make_batch(ws, i)
+        batches.append((b, _grads(ws, b, 100 + i)))
+    ops = [O.FeatureOp(flags=f.flags, hash_seed=f.hash_seed, mod=f.mod, tag=f.tag,
+                       tag_shift=f.tag_shift, boundaries=list(f.boundaries)) for f in ws.features]
+    tabs = [O.Table(t.dim, O.ADAM if t.optimizer == "adam" else O.ADAGRAD, t.lr,
+                    init_seed=t.init_seed) for t in ws.tables]
+    if live is not None:  # pre-insert the live set (untimed)
+        for tab, keys in zip(tabs, live):
+            for c0 in range(0, len(keys), 1 << 20):
+                k = keys[c0:c0 + (1 << 20)]
+                tab.lookup(k, np.arange(len(k) + 1, dtype=np.int64), 1, len(k), pooled=False)
+    n_ids, steps, t0 = 0, 0, time.perf_counter()
+    times = []
+    while True:
+        b, grads = batches[steps % len(batches)]
+        vals = b.values if live is None else W.with_fresh_ids(ws, b, 200 + steps)
+        s0 = time.perf_counter()
+        keys = O.feature_hash(ops, vals, b.feat_offsets)
+        for t, tab, (gp, gu) in zip(ws.tables, tabs, grads):
+            lo, hi, bo = b.table_slice(t, ws.B)
+            tab.lookup(keys[lo:hi], bo, len(t.features), ws.B,
+                       O.SUM if t.combiner == "sum" else O.MEAN, pooled=t.pooled,
+                       unpooled=t.unpooled)
+            tab.backward_update(gp, gu)
+        times.append(time.perf_counter() - s0)
+        n_ids += len(vals)
+        steps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = sum(times)
+    return {"value": n_ids / el, "unit": "IDs/s", "cores": 1, "kind": "oracle", "host": _host_cpu(),
+            "sample": f"{steps} {what} of {w.name} (feature hash + lookup + backward/optimiser) "
+                      f"on the single-threaded CPU oracle, {el:.1f} s",
+            "ms_per_step": 1e3 * el / steps, "steps": steps}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     w = W.WORKLOADS[args.workload]
-    batches = []
-    for i in range(2):
-        b = W.make_batch(w, i)
-        batches.append((b, _grads(w, b, 100 + i)))
     if args.warmup > 0:
-        _oracle_rate(w, 0.0, batches)  # one untimed step
-    res = _oracle_rate(w, max(5.0, 2.0 * args.steps) if args.steps < 60 else 120.0, batches)
+        _oracle_rate(w, 0.0, nbatch=1)  # one untimed step
+    res = _oracle_rate(w, max(5.0, 2.0 * args.steps) if args.steps < 60 else 120.0)
     line = {"impl": "reference", "metric": METRIC, "value": res["value"], "unit": "IDs/s",
             "n_gpus": args.gpus, "steps": res["steps"], "warmup": args.warmup,
             "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
@@ -236,31 +274,35 @@ def _files_sha(files):
     return h.hexdigest()
 
 
-def _traffic(kernel: str, units: float):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, scaled
-    to `units` (occurrences) when it was captured on another size; None when the
-    kernel's sources changed since the capture."""
+def _traffic(workload: str, kernel: str, units: float):
+    """(DRAM bytes per launch, L2 hit rate %, note) of `kernel` on `workload` from
+    the committed ncu summary, scaled to `units` occurrences when it was
+    captured on another size; bytes None when the kernel's sources changed
+    since the capture."""
     if not os.path.exists(TRAFFIC):
-        return None, "no capture"
+        return None, None, "no capture"
     with open(TRAFFIC) as fh:
         d = json.load(fh)
-    e = d.get(kernel)
+    e = d.get(workload, {}).get(kernel)
     if not e:
-        return None, "no capture of this kernel"
+        return None, None, "no capture of this kernel on this workload"
     try:
         if _files_sha(e["files"]) != e["sha256"]:
-            return None, "kernel changed since the capture"
+            return None, None, "kernel changed since the capture"
     except OSError:
-        return None, "kernel sources missing"
+        return None, None, "kernel sources missing"
     scale = units / e["units"] if e.get("units") else 1.0
-    return e["dram_bytes_per_launch"] * scale, e.get("note", "")
+    note = e.get("note", "")
+    if abs(scale - 1.0) > 0.01:
+        note += f"; captured at {e['units']} occurrences, scaled by {scale:.3f}"
+    return e["dram_bytes_per_launch"] * scale, e.get("l2_hit_pct"), note
 
 
 # kernels of the step, grouped by the row of the method they implement
 GROUPS = {
     "feature_hash": ("feature_hash",),
-    "dedup": ("ss_rank", "ss_probe", "ss_count", "ss_tilescan", "ss_scatter", "ss_local", "ss_finish", "sort_hist",
-              "sort_pass", "unique_insert"),
+    "dedup": ("ss_rank", "ss_probe", "ss_count", "ss_tilescan", "ss_scatter", "ss_local", "ss_finish",
+              "sort_hist", "sort_pass", "unique_insert"),
     "gather_pool": ("bag_prep", "gather_pool"),
     "backward": ("seg_reduce", "row_update"),
 }
@@ -282,43 +324,47 @@ def _alg_bytes(w: W.Workload, stats):
     return out
 
 
-def run_gpu(args):
+def _live_keys(w: W.Workload, seed: int):
+    """Pre-inserted keys of the large-table workload, tagged, ascending."""
+    per = w.live_ids // w.F
+    live = np.concatenate([(np.int64(w.features[f].tag) << np.int64(w.features[f].tag_shift))
+                           | W.live_ids(w, f, per, seed=seed) for f in range(w.F)])
+    live.sort()
+    return live
+
+
+def measure(w: W.Workload, args, R, dist, world: int, rank: int, dev, headline: bool):
+    """One workload: setup, warm-up, timed steps, traced steps (per-kernel
+    event times), e2e steps with host buffers, the CPU baseline.  Returns the
+    record on rank 0 (None elsewhere)."""
     import torch
-    import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.device("cuda", torch.cuda.current_device())
-
-    from recommender_sparse_embedding_b200 import build as rbuild
-    if rank == 0:
-        rbuild.build()
-    if world > 1:
-        dist.barrier()
-    import recommender_sparse_embedding_b200 as R
-    R.load()
-
-    w = W.WORKLOADS[args.workload]
-    nb = args.warmup + args.steps
-    n_distinct = min(nb, args.batches)
+    large = bool(w.live_ids)
+    prof_steps = min(args.steps, 10 if large else 50)
+    e2e_steps = 4 if large else max(3, min(args.steps, 50) // 2)
     seed = 2025 + w.index + 1000 * rank
-    host = []
-    for i in range(n_distinct):
-        b = W.make_batch(w, i, seed=seed)
-        host.append((b, _grads(w, b, seed + i)))
     feats = [R.Feature(flags=f.flags, hash_seed=f.hash_seed, mod=f.mod, tag=f.tag,
                        tag_shift=f.tag_shift,
                        boundaries=(torch.tensor(list(f.boundaries), dtype=torch.int64, device=dev)
                                    if f.boundaries else None)) for f in w.features]
 
-    def dev_batch(b, grads, pin=False):
+    # ---- inputs: every step's batch resident on the device before timing
+    n_steps = args.warmup + args.steps + prof_steps
+    if large:
+        # two drawn batches; every step gives their fresh-ID positions IDs never
+        # seen before (stream index = step), so 5% of occurrences are new each step
+        base = [W.make_batch(w, i, seed=seed) for i in range(2)]
+        host = [(b, _grads(w, b, seed + i)) for i, b in enumerate(base)]
+        step_vals = [W.with_fresh_ids(w, base[j % 2], 10 + j, seed=seed) for j in range(n_steps)]
+    else:
+        n_distinct = min(n_steps, args.batches)
+        host = []
+        for i in range(n_distinct):
+            b = W.make_batch(w, i, seed=seed)
+            host.append((b, _grads(w, b, seed + i)))
+        step_vals = None
+
+    def dev_batch(b, grads, vals=None, pin=False):
         mv = (lambda a: torch.from_numpy(a).pin_memory()) if pin else \
             (lambda a: torch.from_numpy(a).to(dev))
         per_table = []
@@ -326,14 +372,40 @@ def run_gpu(args):
             lo, hi, bo = b.table_slice(t, w.B)
             per_table.append((lo, hi, mv(bo), None if gp is None else mv(gp),
                               None if gu is None else mv(gu)))
-        return mv(b.values), b.feat_offsets.tolist(), per_table, len(b.values)
+        v = b.values if vals is None else vals
+        return mv(v), b.feat_offsets.tolist(), per_table, len(v)
 
-    devb = [dev_batch(b, g) for b, g in host]
-    tables = [R.Table(t.dim, R.ADAM if t.optimizer == "adam" else R.ADAGRAD, t.lr,
-                      init_seed=t.init_seed,
-                      initial_capacity=1_000_000 if args.small else 8_000_000) for t in w.tables]
-    batches = [R.Batch() for _ in w.tables]
+    if large:
+        base_dev = [dev_batch(b, g) for b, g in host]
+        devb = []
+        for j, v in enumerate(step_vals):
+            _, foffs, per_table, n = base_dev[j % 2]
+            devb.append((torch.from_numpy(v).to(dev), foffs, per_table, n))
+        del step_vals
+    else:
+        devb = [dev_batch(b, g) for b, g in host]
+    nb = len(devb)
+
     maxN = max(x[3] for x in devb)
+    if large:
+        live = _live_keys(w, seed)
+        new_est = int(1.1 * w.fresh_frac * maxN) * (n_steps + e2e_steps + 2)
+        cap = len(live) + new_est + maxN
+    else:
+        live = None
+        cap = 1_000_000 if args.small else 8_000_000
+    tables = [R.Table(t.dim, R.ADAM if t.optimizer == "adam" else R.ADAGRAD, t.lr,
+                      init_seed=t.init_seed, initial_capacity=cap) for t in w.tables]
+    batches = [R.Batch() for _ in w.tables]
+    if large:  # pre-insert the live set, in chunks the dedup takes in one call
+        b_ins = R.Batch()
+        chunk = 1_500_000
+        for c0 in range(0, len(live), chunk):
+            tables[0].insert(b_ins, torch.from_numpy(live[c0:c0 + chunk]).to(dev))
+        torch.cuda.synchronize()
+        tables[0].status_sync()
+        b_ins.close()
+        assert tables[0].size()[0] == len(live)
     keys = torch.empty(maxN, dtype=torch.int64, device=dev)
     pooled = [torch.empty((w.B, len(t.features), t.dim), dtype=torch.float32, device=dev)
               if t.pooled else None for t in w.tables]
@@ -357,14 +429,15 @@ def run_gpu(args):
             tables[i].backward_update(batches[i], gp, gu)
         return n
 
-    # unique keys per table and batch (for the algorithmic bytes), outside any timing
+    # unique keys per table (for the algorithmic bytes) on a few batches, untimed
     uniq = []
-    for vals, foffs, per_table, n in devb:
+    for vals, foffs, per_table, n in devb[: min(nb, 4)]:
         k = R.feature_hash(feats, vals, foffs)
         uniq.append([int(torch.unique(k[lo:hi]).numel()) for (lo, hi, *_r) in per_table])
+        del k
 
     for i in range(args.warmup):
-        run_step(*devb[i % n_distinct], keys)
+        run_step(*devb[i % nb], keys)
     torch.cuda.synchronize()
     for t in tables:
         t.status_sync()
@@ -383,7 +456,7 @@ def run_gpu(args):
     for j in range(args.steps):
         flush.zero_()
         ev[j][0].record(stream)
-        ids += run_step(*devb[(args.warmup + j) % n_distinct], keys)
+        ids += run_step(*devb[(args.warmup + j) % nb], keys)
         ev[j][1].record(stream)
     torch.cuda.synchronize()
     h1 = time.perf_counter()
@@ -397,20 +470,25 @@ def run_gpu(args):
     dev_ms = sum(a.elapsed_time(b) for a, b in ev)
     step_ms = sorted(a.elapsed_time(b) for a, b in ev)  # this rank's steps, each between its events
 
-    # ---- traced region: the same steps again with CUDA events around every
-    # launch of the library (per-kernel durations for the roofline)
-    prof_steps = min(args.steps, 50)
+    # ---- traced region: further steps with CUDA events around every launch of
+    # the library (per-kernel durations for the roofline)
     R.profile_enable(True)
     R.profile_collect()
     torch.cuda.synchronize()
     for j in range(prof_steps):
         flush.zero_()
-        run_step(*devb[(args.warmup + j) % n_distinct], keys)
+        run_step(*devb[(args.warmup + args.steps + j) % nb], keys)
     torch.cuda.synchronize()
     prof = R.profile_collect()
     R.profile_enable(False)
     for t in tables:
         t.status_sync()
+    Nm = statistics.mean(x[3] for x in devb)
+    stats_N = [statistics.mean(x[2][i][1] - x[2][i][0] for x in devb) for i in range(len(w.tables))]
+    del devb
+    if large:
+        del base_dev
+    torch.cuda.empty_cache()
 
     # ---- e2e through the API with host buffers (pinned), copies inside the timing.
     # Steps are pipelined the way a training loop feeds the engine: step j+1's
@@ -418,18 +496,29 @@ def run_gpu(args):
     # rows come down on another, so the two PCIe directions and the kernels
     # overlap.  Two sets of device buffers alternate.  The timed region runs
     # from the first copy up to the last copy down and holds every step's
-    # copies, its L2 flush and its kernels.
+    # copies, its L2 flush and its kernels.  The copies are torch copies of
+    # pinned host tensors; the library calls take the device buffers.
     e2e_ids, h2d, d2h = 0, 0, 0
-    pin = [dev_batch(b, g, pin=True) for b, g in host[: min(4, n_distinct)]]
+    if large:
+        # every e2e step has never-seen fresh IDs too; the gradients and bag
+        # offsets of the two drawn batches are pinned once and shared
+        pin_base = [dev_batch(b, g, pin=True) for b, g in host]
+        pin = []
+        for j in range(e2e_steps):
+            _, foffs, per_h, n = pin_base[j % 2]
+            vals = W.with_fresh_ids(w, host[j % 2][0], 10 + n_steps + j, seed=seed)
+            pin.append((torch.from_numpy(vals).pin_memory(), foffs, per_h, n))
+    else:
+        pin = [dev_batch(b, g, pin=True) for b, g in host[: min(4, len(host))]]
     NBUF = 2
     dv = [torch.empty(maxN, dtype=torch.int64, device=dev) for _ in range(NBUF)]
-    dbo = [[torch.empty(w.F * w.B + 1, dtype=torch.int64, device=dev) for _ in w.tables] for _ in range(NBUF)]
+    dbo = [[torch.empty(w.F * w.B + 1, dtype=torch.int64, device=dev) for _ in w.tables]
+           for _ in range(NBUF)]
     dgp = [[torch.empty_like(p) if p is not None else None for p in pooled] for _ in range(NBUF)]
     dgu = [[torch.empty_like(u) if u is not None else None for u in unpooled] for _ in range(NBUF)]
     dpool = [[torch.empty_like(p) if p is not None else None for p in pooled] for _ in range(NBUF)]
     pooled_h = [torch.empty(p.shape, dtype=p.dtype).pin_memory() if p is not None else None
                 for p in pooled]
-    e2e_steps = max(3, min(args.steps, 50) // 2)
     up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()
     ev_up = [torch.cuda.Event() for _ in range(e2e_steps)]
     ev_done = [torch.cuda.Event() for _ in range(e2e_steps)]
@@ -446,24 +535,24 @@ def run_gpu(args):
                 up_s.wait_event(ev_done[j - NBUF])
             v = dv[sb][:n]
             v.copy_(vals_h, non_blocking=True)
-            nb = vals_h.numel() * 8
+            nbytes = vals_h.numel() * 8
             per_d = []
             for i, (lo, hi, bo_h, gp_h, gu_h) in enumerate(per_h):
                 bo = dbo[sb][i][: bo_h.numel()]
                 bo.copy_(bo_h, non_blocking=True)
-                nb += bo_h.numel() * 8
+                nbytes += bo_h.numel() * 8
                 gp = gu = None
                 if gp_h is not None:
                     gp = dgp[sb][i]
                     gp.copy_(gp_h, non_blocking=True)
-                    nb += gp_h.numel() * 4
+                    nbytes += gp_h.numel() * 4
                 if gu_h is not None:
                     gu = dgu[sb][i][: gu_h.shape[0]]
                     gu.copy_(gu_h, non_blocking=True)
-                    nb += gu_h.numel() * 4
+                    nbytes += gu_h.numel() * 4
                 per_d.append((lo, hi, bo, gp, gu))
             ev_up[j].record(up_s)
-        h2d = nb
+        h2d = nbytes
         return v, foffs, per_d, n
 
     torch.cuda.synchronize()
@@ -507,14 +596,13 @@ def run_gpu(args):
     value = ids / (dev_ms / 1e3)
     e2e_value = e2e_ids / (e2e_ms / 1e3)
 
+    rec = None
     if rank == 0:
         peak, peak_kind = _peaks()
-        Nm = statistics.mean(x[3] for x in devb)
         stats = []
         for i, t in enumerate(w.tables):
-            Ni = statistics.mean(x[2][i][1] - x[2][i][0] for x in devb)
             Ui = statistics.mean(u[i] for u in uniq)
-            stats.append((Ni, Ui, new_rows[i]))
+            stats.append((stats_N[i], Ui, new_rows[i]))
         alg = _alg_bytes(w, stats)
         kern = {k: {"launches": v[0], "total_ms": v[1], "avg_us": 1e3 * v[1] / max(v[0], 1)}
                 for k, v in prof.items()}
@@ -535,18 +623,25 @@ def run_gpu(args):
                 else:
                     per_launch = alg[grp]
                     achieved = alg[grp] / row_s / 1e9
-                traffic, tnote = _traffic(top, Nm)
+                traffic, l2hit, tnote = _traffic(w.name, top, Nm / top_launches_per_step)
                 roof = {"bound": "hbm", "kernel": top, "row": grp,
                         "row_kernels": members, "achieved": achieved, "peak": peak,
                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                         "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                         "traffic": traffic, "traffic_note": tnote,
+                        "l2_hit_rate_pct": l2hit,
                         "alg_bytes_per_launch": per_launch,
                         "note": ("algorithmic bytes of the row / its kernels' event time"
                                  if len(members) > 1 else
                                  "algorithmic bytes per launch / CUDA-event time per launch")}
+        l2 = {}
+        for k in kern:
+            _, hit, _n = _traffic(w.name, k, Nm)
+            if hit is not None:
+                l2[k] = hit
         step_alg = sum(alg.values()) - alg["feature_hash"] + 16 * Nm
-        line = {
+        step_s = dev_ms / args.steps / 1e3
+        rec = {
             "metric": METRIC, "value": value, "unit": "IDs/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dev_ms / args.steps,
             "ms_per_step_p50": statistics.median(step_ms),
@@ -556,30 +651,77 @@ def run_gpu(args):
             "config": _config(w, {"ids_per_step": Nm,
                                   "unique_per_step": [s[1] for s in stats],
                                   "new_rows_per_step": [s[2] for s in stats],
-                                  "distinct_batches": n_distinct}),
+                                  "distinct_batches": nb,
+                                  **({"live_rows_at_start": len(live)} if large else {})}),
             "roofline": roof,
             "step_alg_bytes": step_alg,
-            "step_alg_gbs": step_alg / (dev_ms / args.steps / 1e3) / 1e9,
-            "step_frac_of_peak": step_alg / (dev_ms / args.steps / 1e3) / 1e9 / peak,
+            "step_alg_gbs": step_alg / step_s / 1e9,
+            "step_frac_of_peak": step_alg / step_s / 1e9 / peak,
+            "l2_hit_rate_pct": l2 or None,
             "e2e": {"value": e2e_value, "unit": "IDs/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h,
-                    "note": "steps pipelined: step j+1's inputs up and step j-1's pooled rows down "
-                            "overlap step j's kernels; timed from the first copy up to the last copy down"},
+                    "note": "torch copies of pinned host buffers around the library's "
+                            "device-pointer calls, inside the timed region; steps pipelined: step "
+                            "j+1's inputs up and step j-1's pooled rows down overlap step j's "
+                            "kernels; timed from the first copy up to the last copy down"},
             "gpu_launches": launches,
             "kernels": kern,
-            "kernels_note": f"CUDA events around every launch, {prof_steps} further steps after the "
-                            "timed region (the timed region itself runs without them)",
+            "kernels_note": f"CUDA events around every launch, {prof_steps} further steps after "
+                            "the timed region (the timed region itself runs without them)",
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
-            res = _oracle_rate(w, args.cpu_seconds, host[:2])
-            line["cpu_baseline"] = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample", "host")}
-        print(json.dumps(line), flush=True)
+            res = _oracle_rate(w, args.cpu_seconds if headline else args.cpu_seconds / 2)
+            rec["cpu_baseline"] = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample",
+                                                       "host")}
 
     for t in tables:
         t.close()
     for b in batches:
         b.close()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    from recommender_sparse_embedding_b200 import build as rbuild
+    if rank == 0:
+        rbuild.build()
+    if world > 1:
+        dist.barrier()
+    import recommender_sparse_embedding_b200 as R
+    R.load()
+
+    subs = [] if args.subs in ("", "none") else [s for s in args.subs.split(",")
+                                                 if s != args.workload]
+    line = measure(W.WORKLOADS[args.workload], args, R, dist, world, rank, dev, headline=True)
+    sub_recs = {}
+    for name in subs:
+        r = measure(W.WORKLOADS[name], args, R, dist, world, rank, dev, headline=False)
+        if r is not None:
+            keep = ("value", "unit", "ms_per_step", "ms_per_step_p50", "ms_per_step_p90", "config",
+                    "roofline", "step_alg_bytes", "step_alg_gbs", "step_frac_of_peak",
+                    "l2_hit_rate_pct", "e2e", "gpu_launches", "kernels", "clocks", "cpu_baseline")
+            sub_recs[name] = {k: r[k] for k in keep if k in r}
+    if rank == 0:
+        if sub_recs:
+            line["configs"] = sub_recs
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -588,10 +730,12 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--subs", default=DEFAULT_SUBS,
+                    help="comma-separated workloads measured after the headline one, or none")
     ap.add_argument("--batches", type=int, default=32, help="distinct batches generated")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

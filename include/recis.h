@@ -117,6 +117,33 @@ typedef struct {
 typedef struct recis_table* recis_table_t;
 typedef struct recis_batch* recis_batch_t;
 
+/* Table merging at model-creation time (README, Key optimisations >
+ * Distributed optimisation > parameter aggregation: tables with the same
+ * attributes -- dimension, initialiser and so on -- are merged into one logical
+ * table, so one lookup serves them all).  Host only, synchronous, no GPU.
+ * feats[f].table holds feature f's own table attributes; features whose
+ * dim, optimizer, lr, beta1, beta2, eps, adagrad_init_acc, init_scale and
+ * init_seed are all equal share a logical table.  Tables are numbered in the
+ * order their first feature appears; a table's features keep their order.
+ * Outputs, per feature f: table_of_feature[f]; tag_of_feature[f] = its rank
+ * among its table's features (0, 1, ...); tag_shift_of_feature[f] = the
+ * largest value_bits of its table's features -- the RECIS_TAG op's tag and
+ * tag_shift that keep the features' IDs apart in the merged table.  Per table
+ * t < *n_tables_out: tables_out[t] = the shared attributes, with
+ * initial_capacity the sum over its features and max_rows their sum (0 if
+ * any feature's is 0).  All output arrays have room for F entries.  Returns
+ * RECIS_ERR_INVALID_ARG for value_bits outside 1..62 or when a table has more
+ * features than 2^(63 - tag_shift) tags. */
+typedef struct {
+  recis_table_config table;  /* the feature's own table attributes */
+  int32_t value_bits;        /* its transformed values are < 2^value_bits (1..62) */
+  int32_t reserved_;
+} recis_feature_spec;
+recis_status recis_plan_tables(const recis_feature_spec* feats, int32_t F,
+                               int32_t* table_of_feature, uint64_t* tag_of_feature,
+                               int32_t* tag_shift_of_feature, recis_table_config* tables_out,
+                               int32_t* n_tables_out);
+
 /* Create a table on the current device (README, Efficient dynamic embedding:
  * IDMap + EmbeddingBlocks).  Rows are [emb D][state s*D] fp32 (s = 1 Adagrad,
  * 2 Adam), kept side by side in EmbeddingBlocks that are physically separate
@@ -145,7 +172,15 @@ recis_status recis_batch_destroy(recis_batch_t b);
  * keys: device int64[N]; bag_offsets: device int64[F*B+1] (0 .. N, non-decreasing);
  * pooled_out: device fp32 [B][F][D] or NULL; unpooled_out: device fp32 [N][D]
  * or NULL.  keys and bag_offsets must stay unchanged until the matching
- * recis_backward_update has run.  N <= 2^31 - 1. */
+ * recis_backward_update has run.  0 <= N < 2^30 (larger N: RECIS_ERR_INVALID_ARG).
+ * A lookup whose keys include the reserved -1 is rejected as a whole: no key
+ * is inserted, no row is created, the table is left as it was, and
+ * RECIS_ERR_RESERVED_KEY is reported as a device-detected error.  Batches of
+ * up to 1,600,000 keys are rejected the same way (RECIS_ERR_TABLE_FULL) when
+ * their new keys would not fit in max_rows; for larger batches the host checks
+ * the bound live rows + N against max_rows before launching and returns
+ * RECIS_ERR_TABLE_FULL at once.  The outputs of a rejected lookup are
+ * undefined and its recis_backward_update updates no row. */
 recis_status recis_lookup_pooled(recis_table_t t, recis_batch_t b, const int64_t* keys,
                                  int64_t N, const int64_t* bag_offsets, int32_t F, int64_t B,
                                  int32_t combiner, float* pooled_out, float* unpooled_out,
@@ -165,6 +200,17 @@ recis_status recis_backward_update(recis_table_t t, recis_batch_t b, const float
  * int64[N].  rows_out: device int64[N] (row of each key) or NULL. */
 recis_status recis_table_insert(recis_table_t t, recis_batch_t b, const int64_t* keys, int64_t N,
                                 int64_t* rows_out, recis_stream_t stream);
+
+/* Row access by offset (README, Efficient dynamic embedding: parameters and
+ * optimiser state kept side by side).  For each of the n row offsets rows[i]
+ * (device int64[n]) writes its key to keys_out[i] (device int64[n] or NULL),
+ * its emb to emb_out[i][0..D) (device fp32 [n][D] or NULL) and its optimiser
+ * state to state_out[i][0..s*D) (device fp32 [n][s*D] or NULL; Adam: m then
+ * v).  A row offset outside [0, live rows) gives key -1 and zeros.  Waits for
+ * `stream` to learn the live row count, then gathers asynchronously on it. */
+recis_status recis_table_read_rows(recis_table_t t, const int64_t* rows, int64_t n,
+                                   int64_t* keys_out, float* emb_out, float* state_out,
+                                   recis_stream_t stream);
 
 /* Synchronous.  Number of live rows and the Adam step counter. */
 recis_status recis_table_size(recis_table_t t, int64_t* n_out, int64_t* step_out,
@@ -218,6 +264,24 @@ recis_status recis_batch_get_unique(recis_batch_t b, int64_t* uniq_out, int32_t*
  * the caller. */
 recis_status recis_unique_static(const int64_t* keys, int64_t N, int64_t* uniq_out,
                                  int32_t* inv_out, int64_t* U_out, recis_stream_t stream);
+
+/* ------------------------------------------------------------------ test hooks */
+/* Process-wide settings that let tests reach error paths without faulting the
+ * GPU.  The pages have no counterpart (they describe no failure handling).
+ *   RECIS_DEBUG_SPIN_LIMIT: polls a device-side wait on another CTA's progress
+ *     makes before it gives up and reports RECIS_ERR_TIMEOUT (value 0 restores
+ *     the default, about 4M polls).  Applies to launches made after the call:
+ *     the radix-sort dedup of batches over 1.6M keys and recis_unique_static.
+ *     A wait that gives up leaves the call's outputs undefined (every access
+ *     stays in bounds); on a table it also leaves the table's contents
+ *     undefined.
+ *   RECIS_DEBUG_MAP_LIMIT: EmbeddingBlock bytes one table may have mapped;
+ *     growth past it fails with RECIS_ERR_OOM as a failed allocation would
+ *     (0 = no cap, the default).
+ * Returns RECIS_ERR_INVALID_ARG for an unknown setting or a negative value. */
+#define RECIS_DEBUG_SPIN_LIMIT 1
+#define RECIS_DEBUG_MAP_LIMIT 2
+recis_status recis_debug_set(int32_t what, int64_t value);
 
 /* ------------------------------------------------------------------ tracing */
 /* Kernel timing: while enabled, every kernel launch is bracketed by CUDA

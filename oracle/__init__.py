@@ -241,3 +241,42 @@ class Table:
                                     _ptr(emb, ctypes.c_float), _ptr(st, ctypes.c_float), step)
         if rc != OK:
             raise OracleError(rc, "import")
+
+
+class _FeatureAttrs(ctypes.Structure):
+    _fields_ = [
+        ("dim", ctypes.c_int32),
+        ("optimizer", ctypes.c_int32),
+        ("lr", ctypes.c_double),
+        ("beta1", ctypes.c_double),
+        ("beta2", ctypes.c_double),
+        ("eps", ctypes.c_double),
+        ("adagrad_init_acc", ctypes.c_double),
+        ("init_scale", ctypes.c_double),
+        ("init_seed", ctypes.c_uint64),
+        ("capacity", ctypes.c_int64),
+        ("value_bits", ctypes.c_int32),
+        ("pad_", ctypes.c_int32),
+    ]
+
+
+def plan_tables(features):
+    """Table merging of the oracle.  features: sequence of dicts with keys dim,
+    optimizer, lr, beta1, beta2, eps, adagrad_init_acc, init_scale, init_seed,
+    capacity, value_bits.  Returns (table_of, tag_of, shift_of, capacities)."""
+    F = len(features)
+    arr = (_FeatureAttrs * max(F, 1))()
+    for f, a in enumerate(features):
+        for k, v in a.items():
+            setattr(arr[f], k, v)
+    table_of = np.empty(max(F, 1), np.int32)
+    tag_of = np.empty(max(F, 1), np.uint64)
+    shift_of = np.empty(max(F, 1), np.int32)
+    caps = np.empty(max(F, 1), np.int64)
+    n = ctypes.c_int32(0)
+    rc = lib().orc_plan_tables(arr, F, _ptr(table_of, ctypes.c_int32), _ptr(tag_of, ctypes.c_uint64),
+                               _ptr(shift_of, ctypes.c_int32), _ptr(caps, ctypes.c_int64),
+                               ctypes.byref(n))
+    if rc != OK:
+        raise OracleError(rc, "plan_tables")
+    return table_of[:F].copy(), tag_of[:F].copy(), shift_of[:F].copy(), caps[: n.value].copy()

@@ -13,6 +13,8 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <map>
+#include <tuple>
 #include <unordered_map>
 #include <vector>
 
@@ -356,5 +358,54 @@ extern "C" int orc_table_import(orc_table* t, int64_t n, const int64_t* keys, co
                   sizeof(float) * t->s * D);
   }
   t->step = step;
+  return ORC_OK;
+}
+
+// Table merging (README, Key optimisations > Distributed optimisation >
+// parameter aggregation and sharding: "tables of the same attributes --
+// dimension, initialiser and so on -- become one logical table when the model
+// is created").  Reading: the attributes are all of a table's settings except
+// its capacity (dimension, optimiser and its hyper-parameters, initialiser
+// scale and seed); a merged table keeps each feature's IDs apart with a tag,
+// the feature's rank among the table's features, written above the widest
+// value of the table's features.
+extern "C" int orc_plan_tables(const orc_feature_attrs* feats, int32_t F, int32_t* table_of,
+                               uint64_t* tag_of, int32_t* shift_of, int64_t* table_capacity,
+                               int32_t* n_tables) {
+  typedef std::tuple<int32_t, int32_t, double, double, double, double, double, double, uint64_t>
+      Attrs;
+  std::map<Attrs, int32_t> table_id;  // attributes -> logical table
+  std::vector<int64_t> members;       // features seen per table
+  std::vector<int32_t> widest;        // widest value per table
+  std::vector<int64_t> cap;
+  for (int32_t f = 0; f < F; ++f) {
+    const orc_feature_attrs& a = feats[f];
+    if (a.value_bits < 1 || a.value_bits > 62) return ORC_INVALID_ARG;
+    const Attrs key(a.dim, a.optimizer, a.lr, a.beta1, a.beta2, a.eps, a.adagrad_init_acc,
+                    a.init_scale, a.init_seed);
+    auto it = table_id.find(key);
+    if (it == table_id.end()) {
+      it = table_id.emplace(key, (int32_t)members.size()).first;
+      members.push_back(0);
+      widest.push_back(0);
+      cap.push_back(0);
+    }
+    const int32_t t = it->second;
+    table_of[f] = t;
+    tag_of[f] = (uint64_t)members[t];
+    members[t] += 1;
+    widest[t] = std::max(widest[t], a.value_bits);
+    cap[t] += a.capacity;
+  }
+  for (size_t t = 0; t < members.size(); ++t) {
+    // tags 0 .. members-1 need ceil(log2(members)) bits above the values,
+    // inside the 63 bits of a non-negative key
+    int bits = 0;
+    while (((int64_t)1 << bits) < members[t]) ++bits;
+    if (widest[t] + bits > 63) return ORC_INVALID_ARG;
+    if (table_capacity) table_capacity[t] = cap[t];
+  }
+  for (int32_t f = 0; f < F; ++f) shift_of[f] = widest[table_of[f]];
+  *n_tables = (int32_t)members.size();
   return ORC_OK;
 }

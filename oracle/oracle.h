@@ -88,6 +88,28 @@ int orc_table_export(const orc_table* t, int64_t* keys, float* emb, float* state
 int orc_table_import(orc_table* t, int64_t n, const int64_t* keys, const float* emb,
                      const float* state, int64_t step);
 
+/* Table merging (README, Key optimisations > Distributed optimisation >
+ * parameter aggregation: tables with the same attributes are merged into one
+ * logical table at model-creation time).  Per feature: its table attributes
+ * and the bit width of its transformed values.  Outputs per feature: the
+ * logical table (numbered by first appearance), the tag (rank among the
+ * table's features) and the tag shift (widest value of the table); per table:
+ * the summed initial capacity.  Returns ORC_INVALID_ARG when bits are outside
+ * 1..62 or a table's tags do not fit above its values. */
+typedef struct {
+  int32_t dim;
+  int32_t optimizer;
+  double lr, beta1, beta2, eps, adagrad_init_acc, init_scale;
+  uint64_t init_seed;
+  int64_t capacity;
+  int32_t value_bits;
+  int32_t pad_;
+} orc_feature_attrs;
+
+int orc_plan_tables(const orc_feature_attrs* feats, int32_t F, int32_t* table_of,
+                    uint64_t* tag_of, int32_t* shift_of, int64_t* table_capacity,
+                    int32_t* n_tables);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,9 @@ enum : int {
 };
 
 // Bound for every spin-wait on another CTA's progress: after this many polls
-// (with a short sleep each) the waiter records kErrTimeout and moves on.
+// (with a short sleep each) the waiter records kErrTimeout and moves on.  The
+// kernels take the bound as an argument (spin_limit()), which a test may lower
+// through recis_debug_set to make a wait give up.
 constexpr int kSpinLimit = 1 << 22;
 
 // H: SplitMix64 finaliser (Steele, Lea & Flood, "Fast splittable pseudorandom

@@ -64,10 +64,13 @@ constexpr int64_t kSampleSortMaxN = (int64_t)1600 * 1000;  // larger batches use
 // Per-batch device scalars.
 struct BatchDev {
   unsigned long long row_base;  // table's next_free when the lookup started
-  unsigned int U;               // unique keys of the last lookup
+  unsigned int U;               // unique keys of the last lookup (0 when it was rejected)
   unsigned int n_new;           // new keys of the last lookup
   unsigned int nlong;           // chunks of kShortSeg positions holding a long segment
   unsigned int nmulti;          // keys seen 2 to kShortSeg times (sample-sort path)
+  unsigned int reject_call;     // call number of a lookup rejected as a whole (reserved key,
+                                // or its new keys overflow the row space)
+  unsigned int pad;
 };
 
 // ---------------------------------------------------------------- table
@@ -151,6 +154,7 @@ struct recis_batch {
   int64_t capGbuf = 0;            // floats
   recis::BatchDev* bdev = nullptr;
   uint32_t epoch = 0;
+  uint32_t call_seq = 0;          // number of the current lookup on this batch (never 0)
   // the last lookup, for the backward
   recis_table* table = nullptr;
   int64_t N = 0;
@@ -166,6 +170,11 @@ struct recis_batch {
 namespace recis {
 
 void set_error(const std::string& msg);
+
+// Test hooks (recis_debug_set): the bound of the device-side spin-waits, and
+// a cap on the EmbeddingBlock bytes a table may map (0 = none).
+int spin_limit();
+int64_t map_limit_bytes();
 
 // Launches kernel<<<grid, block, smem, s>>>(args...) with programmatic
 // stream serialization (see pdl_wait in common.cuh).

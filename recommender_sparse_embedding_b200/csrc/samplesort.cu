@@ -334,7 +334,18 @@ struct SsParams {
   int32_t* multi_keys;      // keys seen 2 to kShortSeg times (appended by ss_finish)
   DevState* st;
   HostMirror* mirror;
+  uint32_t call_id;         // this lookup's number on the batch (BatchDev::reject_call)
 };
+
+// A lookup is rejected as a whole when one of its keys is the reserved -1
+// (marked by the probe kernel) or when its new keys would not fit the mapped
+// row space: then no key is inserted (the slots its probes claimed are given
+// back), no row is created, and U = 0, so the matching backward updates no row.
+__device__ __forceinline__ bool call_rejected(const SsParams& p, unsigned long long tot,
+                                              unsigned long long row_base) {
+  return __ldcg(&p.bdev->reject_call) == p.call_id ||
+         row_base + (tot >> 32) > (unsigned long long)p.mapped_rows;
+}
 
 // Per sorted position, written by ss_local: the bucket, the position's
 // segment within the bucket (1-based count of heads up to it), for a head
@@ -476,7 +487,10 @@ __global__ void __launch_bounds__(kProbeThreads) ss_probe_kernel(const __grid_co
     }
     p.pocc[pos] = r;
   }
-  if (reserved) raise_error(p.st, p.mirror, kErrReservedKey);
+  if (reserved) {
+    p.bdev->reject_call = p.call_id;
+    raise_error(p.st, p.mirror, kErrReservedKey);
+  }
 }
 
 // ------------------------------------------------------------------ tile scan
@@ -766,14 +780,21 @@ __device__ __forceinline__ void local_publish(const SsParams& p) {
   p.ctl->cta_tot[blockIdx.x] = run;
 }
 
-// The call's totals (tot = new keys << 32 | heads), published by one thread.
+// The call's totals (tot = new keys << 32 | heads), published by one thread;
+// a rejected call publishes U = 0 and no new rows, and marks the batch.
 __device__ __forceinline__ void publish_totals(const SsParams& p, unsigned long long tot,
                                                unsigned long long row_base) {
-  const unsigned long long U = tot & 0xffffffffULL, nnew = tot >> 32;
-  p.bdev->U = (unsigned)U;
+  const unsigned long long U = tot & 0xffffffffULL;
+  unsigned long long nnew = tot >> 32;
+  const bool rejected = call_rejected(p, tot, row_base);
+  if (rejected) {
+    if (__ldcg(&p.bdev->reject_call) != p.call_id) raise_error(p.st, p.mirror, kErrTableFull);
+    p.bdev->reject_call = p.call_id;
+    nnew = 0;
+  }
+  p.bdev->U = rejected ? 0u : (unsigned)U;
   p.bdev->n_new = (unsigned)nnew;
-  unsigned long long nf = row_base + nnew;
-  if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
+  const unsigned long long nf = row_base + nnew;
   p.st->next_free = nf;
   if (p.mirror) {
     p.mirror->next_free = nf;
@@ -1189,10 +1210,14 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
   // second level of the bucket prefixes, after the one-warp local kernel:
   // every CTA scans the local CTAs' totals and CTA 0 publishes the call's
   // totals (after the CTA local kernel its last CTA did both)
+  bool rejected;
   if (p.finish_scans) {
     const unsigned long long tot = scan_cta_totals<kFinThreads>(
         p, sh.warp, [&](int i, unsigned long long v) { sh.cpre[i] = v; });
+    rejected = call_rejected(p, tot, row_base);
     if (blockIdx.x == 0 && tid == 0) publish_totals(p, tot, row_base);
+  } else {
+    rejected = __ldcg(&p.bdev->reject_call) == p.call_id;  // published by the local kernel
   }
   // head bits of this CTA's positions (position j*kFinThreads + 32w + lane)
 #pragma unroll
@@ -1225,7 +1250,12 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
         const int64_t slot = -2 - row;
         const unsigned ln = (unsigned)((m >> 21) & 0x1fffffULL);
         row = (int64_t)(row_base + (cpre >> 32) + __ldg(&p.ctl->npre[b]) + ln - 1u);
-        if (row >= p.mapped_rows) {
+        if (rejected) {
+          // give the claimed slot back: every key claimed by this call is
+          // newer than every key that stays, so no probe chain is cut
+          p.slots[slot].key = kEmptyKey;
+          row = -1;
+        } else if (row >= p.mapped_rows) {
           raise_error(p.st, p.mirror, kErrTableFull);
           row = -1;
         } else {
@@ -1241,7 +1271,7 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
       p.seg_start[seg] = (int32_t)q;
       // a short segment (not long) whose next position is no head holds 2 to
       // kShortSeg occurrences: listed for the row update
-      if (p.multi_keys && !(m >> 63)) {
+      if (p.multi_keys && !rejected && !(m >> 63)) {
         const int i = tid + j * kFinThreads + 1;  // next position within this CTA
         bool next_head;
         if (q + 1 >= p.N) next_head = true;
@@ -1257,7 +1287,7 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
   if (tid == 0 && sh.nmulti > 0) sh.multi_base = atomicAdd(&p.bdev->nmulti, (unsigned)sh.nmulti);
   __syncthreads();
   for (int i = tid; i < sh.nmulti; i += kFinThreads) p.multi_keys[sh.multi_base + i] = sh.multi[i];
-  if (w == 0) {
+  if (w == 0 && !rejected) {
     const bool has = (sh.chunk_long >> lane) & 1u;
     const unsigned bal = __ballot_sync(0xffffffffu, has);
     unsigned at = 0;
@@ -1383,6 +1413,7 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   p.multi_keys = b->multi_keys;
   p.st = t->dstate;
   p.mirror = t->mirror_dev;
+  p.call_id = b->call_seq;
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

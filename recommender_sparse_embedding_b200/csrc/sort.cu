@@ -35,7 +35,8 @@ __device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long 
 
 __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restrict__ keys,
                                                         int64_t N, SortCtl* ctl, DevState* st,
-                                                        HostMirror* mirror, BatchDev* bdev) {
+                                                        HostMirror* mirror, BatchDev* bdev,
+                                                        uint32_t call_id) {
   constexpr int kPer = 4;  // keys per thread per round, loaded before they are counted
   __shared__ unsigned int sh[kSortPasses][256];
   __shared__ bool s_last;
@@ -67,7 +68,10 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restric
       }
     }
   }
-  if (__any_sync(0xffffffffu, reserved) && lane == 0) raise_error(st, mirror, kErrReservedKey);
+  if (__any_sync(0xffffffffu, reserved) && lane == 0) {
+    bdev->reject_call = call_id;  // the unique pass then inserts nothing
+    raise_error(st, mirror, kErrReservedKey);
+  }
   __syncthreads();
   for (int i = threadIdx.x; i < kSortPasses * 256; i += blockDim.x) {
     const unsigned c = (&sh[0][0])[i];
@@ -121,7 +125,7 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restric
 __global__ void __launch_bounds__(kSortBlock) sort_pass_kernel(
     int P, const int64_t* __restrict__ in_keys, uint64_t* kb0, uint64_t* kb1, uint32_t* vb0,
     uint32_t* vb1, int64_t N, SortCtl* ctl, unsigned long long* lookback, uint32_t epoch,
-    DevState* st, HostMirror* mirror) {
+    DevState* st, HostMirror* mirror, int spin_max) {
   if (!ctl->active[P]) return;
   const unsigned ord = ctl->ordinal[P];
   const uint64_t* ksrc = (ord & 1) ? kb0 : kb1;  // ord-1 parity
@@ -235,7 +239,7 @@ __global__ void __launch_bounds__(kSortBlock) sort_pass_kernel(
         }
         unsigned long long v = e[w];
         while ((uint32_t)(v >> 32) != epoch || ((v >> 30) & 3u) == 0) {
-          if (++spins > kSpinLimit) {
+          if (++spins > spin_max) {
             raise_error(st, mirror, kErrTimeout);
             done = true;
             break;
@@ -290,18 +294,26 @@ cudaError_t launch_sort(recis_batch* b, recis_table* t, const int64_t* keys, int
     if (blocks < 1) blocks = 1;
     LaunchScope ls("sort_hist", s);
     sort_hist_kernel<<<(unsigned)blocks, 256, 0, s>>>(keys, N, b->ctl, t->dstate, t->mirror_dev,
-                                                      b->bdev);
+                                                      b->bdev, b->call_seq);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   const int64_t tiles = (N + kSortTile - 1) / kSortTile;
   for (int p = 0; p < kSortPasses; ++p) {
     b->epoch += 1;
-    if (b->epoch == 0) b->epoch = 1;
+    if (b->epoch == 0) {
+      // the tag wrapped: entries left by passes 2^32 tags ago could carry the
+      // tag about to be used, so the look-back array starts over from zero
+      // (stream-ordered after every earlier pass)
+      b->epoch = 1;
+      e = cudaMemsetAsync(b->sort_lookback, 0,
+                          sizeof(unsigned long long) * 256 * (size_t)b->sort_lookback_tiles, s);
+      if (e != cudaSuccess) return e;
+    }
     LaunchScope ls("sort_pass", s);
     sort_pass_kernel<<<(unsigned)tiles, kSortBlock, 0, s>>>(
         p, keys, b->kbuf[0], b->kbuf[1], b->vbuf[0], b->vbuf[1], N, b->ctl, b->sort_lookback,
-        b->epoch, t->dstate, t->mirror_dev);
+        b->epoch, t->dstate, t->mirror_dev, spin_limit());
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

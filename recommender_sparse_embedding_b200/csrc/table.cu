@@ -42,6 +42,9 @@ std::vector<cudaEvent_t> g_event_pool;
 int* g_feat_status[128] = {nullptr};
 std::mutex g_feat_mu;
 
+std::atomic<int> g_spin_limit{kSpinLimit};
+std::atomic<int64_t> g_map_limit{0};
+
 constexpr double kMaxLoad = 0.5;
 
 cudaEvent_t pool_event() {
@@ -57,6 +60,9 @@ cudaEvent_t pool_event() {
 }  // namespace
 
 void set_error(const std::string& msg) { g_err = msg; }
+
+int spin_limit() { return g_spin_limit.load(std::memory_order_relaxed); }
+int64_t map_limit_bytes() { return g_map_limit.load(std::memory_order_relaxed); }
 
 recis_status cuda_fail(cudaError_t e, const char* what) {
   set_error(std::string(what) + ": " + cudaGetErrorString(e));
@@ -140,6 +146,11 @@ static recis_status vmm_map_to(VmmArray& a, size_t bytes, int dev) {
     return RECIS_ERR_TABLE_FULL;
   }
   const size_t sz = bytes - a.mapped;
+  const int64_t cap = map_limit_bytes();
+  if (cap > 0 && (int64_t)bytes > cap) {
+    set_error("EmbeddingBlocks: mapping refused by the test cap on mapped bytes");
+    return RECIS_ERR_OOM;
+  }
   CUmemAllocationProp prop = {};
   prop.type = CU_MEM_ALLOCATION_TYPE_PINNED;
   prop.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
@@ -201,7 +212,9 @@ static recis_status grow_rows(recis_table* t, int64_t rows) {
   const size_t kb = round_up((size_t)backed * sizeof(int64_t), t->gran);
   st = vmm_map_to(t->keys, std::min(kb, t->keys.reserved), t->dev);
   if (st != RECIS_OK) return st;
-  t->mapped_rows = std::min<int64_t>(backed, (int64_t)(t->keys.mapped / sizeof(int64_t)));
+  // rows past max_rows stay unused even where a block's rounding backs them
+  t->mapped_rows = std::min<int64_t>(std::min<int64_t>(backed, (int64_t)(t->keys.mapped / sizeof(int64_t))),
+                                     t->max_rows);
   return RECIS_OK;
 }
 
@@ -297,9 +310,14 @@ static recis_status pending_error(recis_table* t, cudaStream_t s) {
 }
 
 // Make room for up to `n_new` new keys without waiting in the common case.
-static recis_status reserve(recis_table* t, int64_t n_new, cudaStream_t s) {
+// device_checked: the call's kernels reject it as a whole when its actual new
+// keys do not fit the mapped rows, so a bound past max_rows maps up to
+// max_rows and lets the device decide; otherwise such a bound is an error.
+static recis_status reserve(recis_table* t, int64_t n_new, cudaStream_t s,
+                            bool device_checked = false) {
   refresh_mirror(t);
   int64_t need = t->rows_upper + n_new;
+  if (device_checked) need = std::min(need, std::max(t->max_rows, t->rows_upper));
   if (need > t->mapped_rows || (double)need > kMaxLoad * (double)t->capacity) {
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
@@ -309,6 +327,7 @@ static recis_status reserve(recis_table* t, int64_t n_new, cudaStream_t s) {
     t->rows_upper = (int64_t)h.next_free;
     t->ring_live = 0;
     need = t->rows_upper + n_new;
+    if (device_checked) need = std::min(need, std::max(t->max_rows, t->rows_upper));
     recis_status st = grow_rows(t, need);
     if (st != RECIS_OK) return st;
     st = grow_idmap(t, need, s);
@@ -486,7 +505,7 @@ static recis_status lookup_impl(const LookupArgs& a, cudaStream_t s) {
   recis_batch* b = a.b;
   recis_status st = pending_error(t, s);
   if (st != RECIS_OK) return st;
-  st = reserve(t, a.N, s);
+  st = reserve(t, a.N, s, a.N <= kSampleSortMaxN);
   if (st != RECIS_OK) return st;
   st = batch_ensure(b, a.N, (int64_t)a.F * a.B, t->D);
   if (st != RECIS_OK) return st;
@@ -498,6 +517,7 @@ static recis_status lookup_impl(const LookupArgs& a, cudaStream_t s) {
   b->keys = a.keys;
   b->bag_offsets = a.bag_offsets;
   b->have_lookup = true;
+  if (++b->call_seq == 0) b->call_seq = 1;
   cudaError_t e;
   const bool pool = a.pooled_out || a.unpooled_out;
   const int64_t cf = pool_chunk_for(a.N, t->D);
@@ -539,6 +559,22 @@ using namespace recis;
 extern "C" {
 
 const char* recis_last_error_string(void) { return g_err.c_str(); }
+
+recis_status recis_debug_set(int32_t what, int64_t value) {
+  switch (what) {
+    case RECIS_DEBUG_SPIN_LIMIT:
+      if (value < 0 || value > INT32_MAX) return RECIS_ERR_INVALID_ARG;
+      g_spin_limit.store(value == 0 ? kSpinLimit : (int)value);
+      return RECIS_OK;
+    case RECIS_DEBUG_MAP_LIMIT:
+      if (value < 0) return RECIS_ERR_INVALID_ARG;
+      g_map_limit.store(value);
+      return RECIS_OK;
+    default:
+      set_error("debug_set: unknown setting");
+      return RECIS_ERR_INVALID_ARG;
+  }
+}
 
 int64_t recis_launch_count(void) { return g_launches.load(); }
 

@@ -36,10 +36,12 @@ __device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long 
 }
 
 // IDMap find-or-insert.  Returns true when the key was inserted by this call
-// (slot index in *slot); otherwise *row holds the existing row.  *slot = -1
-// when the probe limit is reached.
+// (slot index in *slot); otherwise *row holds the existing row (-1 for a
+// missing key when insert is false).  *slot = -1 when the probe limit is
+// reached or the key is missing and insert is false.
 __device__ __forceinline__ bool idmap_find_or_insert(Slot* slots, uint64_t mask, int64_t key,
-                                                     int64_t* slot, int64_t* row) {
+                                                     int64_t* slot, int64_t* row,
+                                                     bool insert = true) {
   uint64_t h = mix64((uint64_t)key ^ kSlotSalt) & mask;
   const int64_t limit = (int64_t)mask + 1 < kMaxProbes ? (int64_t)mask + 1 : kMaxProbes;
   for (int64_t n = 0; n < limit; ++n) {
@@ -50,6 +52,7 @@ __device__ __forceinline__ bool idmap_find_or_insert(Slot* slots, uint64_t mask,
       return false;
     }
     if (sv.x == kEmptyKey) {
+      if (!insert) break;
       const unsigned long long old = atomicCAS(reinterpret_cast<unsigned long long*>(&slots[h].key),
                                                (unsigned long long)kEmptyKey,
                                                (unsigned long long)key);
@@ -102,6 +105,8 @@ struct UniqueParams {
   BatchDev* bdev;
   DevState* st;
   HostMirror* mirror;
+  uint32_t call_id;
+  int spin_max;             // polls before a look-back wait gives up
 };
 
 __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_constant__ UniqueParams p) {
@@ -155,6 +160,9 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
     have_prev = false;
   }
 
+  // a batch holding the reserved key (found by the histogram pass) is
+  // rejected as a whole: its keys are only looked up, nothing is inserted
+  const bool rejected = __ldcg(&p.bdev->reject_call) == p.call_id;
   bool head[kUqItems], isnew[kUqItems];
   int64_t slot[kUqItems], row[kUqItems];
   unsigned nh = 0, nn = 0;
@@ -167,8 +175,9 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
     slot[j] = -1;
     row[j] = -1;
     if (head[j] && from_ukey(k[j]) != kEmptyKey) {  // the reserved key is reported by the sort
-      isnew[j] = idmap_find_or_insert(p.slots, p.slot_mask, from_ukey(k[j]), &slot[j], &row[j]);
-      if (slot[j] < 0) raise_error(p.st, p.mirror, kErrTableFull);
+      isnew[j] = idmap_find_or_insert(p.slots, p.slot_mask, from_ukey(k[j]), &slot[j], &row[j],
+                                      !rejected);
+      if (slot[j] < 0 && !rejected) raise_error(p.st, p.mirror, kErrTableFull);
     }
     if (head[j]) {
       ++nh;
@@ -210,11 +219,11 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
         const int64_t idx = t - lane;
         unsigned long long e = idx >= 0 ? ld_relaxed(p.lookback + idx) : kUqIncl;
         while (!__all_sync(0xffffffffu, (e >> 62) != 0)) {
-          if (++spins > kSpinLimit) break;
+          if (++spins > p.spin_max) break;
           __nanosleep(32);
           if ((e >> 62) == 0) e = ld_relaxed(p.lookback + idx);
         }
-        if (spins > kSpinLimit) {
+        if (spins > p.spin_max) {
           if (lane == 0) raise_error(p.st, p.mirror, kErrTimeout);
           break;
         }
@@ -277,7 +286,7 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
   }
   if (tile == gridDim.x - 1 && tid == 0) {
     const unsigned long long U = Hx + tH, nnew = Nx + tN;
-    p.bdev->U = (unsigned)U;
+    p.bdev->U = rejected ? 0u : (unsigned)U;
     p.bdev->n_new = (unsigned)nnew;
     unsigned long long nf = row_base + nnew;
     if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
@@ -349,6 +358,8 @@ cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cuda
   p.bdev = b->bdev;
   p.st = t->dstate;
   p.mirror = t->mirror_dev;
+  p.call_id = b->call_seq;
+  p.spin_max = spin_limit();
   const int64_t tiles = (N + kUqTile - 1) / kUqTile;
   LaunchScope ls("unique_insert", s);
   unique_insert_kernel<<<(unsigned)tiles, kUqBlock, 0, s>>>(p);

@@ -58,7 +58,7 @@ __device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long 
 // bounded wait gave up here or in the sort.
 __global__ void __launch_bounds__(kUoBlock) unique_only_kernel(
     const int64_t* __restrict__ in_keys, StaticScratch* sc, int64_t N, int64_t* uniq,
-    int32_t* inv, int64_t* U_out) {
+    int32_t* inv, int64_t* U_out, int spin_max) {
   __shared__ uint64_t s_last[kUoBlock];
   __shared__ unsigned s_scan[kUoBlock / 32];
   __shared__ unsigned s_tile;
@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kUoBlock) unique_only_kernel(
         const unsigned long long e = ld_relaxed(sc->seg_lookback + t);
         const unsigned long long flag = e >> 62;
         if (flag == 0) {
-          if (++spins > kSpinLimit) {
+          if (++spins > spin_max) {
             atomicOr(&sc->st.status, kErrTimeout);
             break;
           }
@@ -195,9 +195,16 @@ extern "C" recis_status recis_unique_static(const int64_t* keys, int64_t N, int6
       g_scratch_addr[dev] = static_cast<StaticScratch*>(p);
     }
     sc = g_scratch_addr[dev];
+    // this call's sort tags its passes epoch+1, epoch+2, ... skipping 0 (see
+    // launch_sort, which also clears the look-back array when the tag wraps);
+    // the next call starts where this one ends
     epoch = g_epoch[dev];
-    g_epoch[dev] = epoch + kSortPasses;  // this call's sort uses epoch+1 .. epoch+8
-    if (g_epoch[dev] < epoch) g_epoch[dev] = 0;
+    uint32_t last = epoch;
+    for (int p = 0; p < kSortPasses; ++p) {
+      last += 1;
+      if (last == 0) last = 1;
+    }
+    g_epoch[dev] = last;
   }
   if (N == 0) {
     e = cudaMemsetAsync(U_out, 0, sizeof(int64_t), s);
@@ -224,7 +231,7 @@ extern "C" recis_status recis_unique_static(const int64_t* keys, int64_t N, int6
   e = launch_sort(&b, &t, keys, N, s);
   if (e != cudaSuccess) return cuda_fail(e, "sort launch");
   const unsigned tiles = (unsigned)((N + kUoTile - 1) / kUoTile);
-  unique_only_kernel<<<tiles, kUoBlock, 0, s>>>(keys, sc, N, uniq_out, inv_out, U_out);
+  unique_only_kernel<<<tiles, kUoBlock, 0, s>>>(keys, sc, N, uniq_out, inv_out, U_out, spin_limit());
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "unique launch");
   return RECIS_OK;

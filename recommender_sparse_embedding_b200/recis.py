@@ -31,8 +31,10 @@ EXPORTS = (
     "recis_backward_update", "recis_table_insert", "recis_table_size", "recis_table_export",
     "recis_table_import", "recis_table_status_sync", "recis_batch_get_unique",
     "recis_profile_enable", "recis_profile_collect", "recis_launch_count",
-    "recis_last_error_string", "recis_unique_static",
+    "recis_last_error_string", "recis_unique_static", "recis_table_read_rows",
+    "recis_debug_set", "recis_plan_tables",
 )
+DEBUG_SPIN_LIMIT, DEBUG_MAP_LIMIT = 1, 2
 
 
 class RecisError(RuntimeError):
@@ -71,6 +73,11 @@ class TableConfig(ctypes.Structure):
     ]
 
 
+class FeatureSpec(ctypes.Structure):
+    _fields_ = [("table", TableConfig), ("value_bits", ctypes.c_int32),
+                ("reserved_", ctypes.c_int32)]
+
+
 _lib = None
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -105,6 +112,9 @@ def load(path: str = LIB_PATH):
             "recis_launch_count": [],
             "recis_last_error_string": [],
             "recis_unique_static": [_vp, _i64, _vp, _vp, _vp, _vp],
+            "recis_table_read_rows": [_vp, _vp, _i64, _vp, _vp, _vp, _vp],
+            "recis_debug_set": [_i32, _i64],
+            "recis_plan_tables": [_vp, _i32, _vp, _vp, _vp, _vp, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -288,6 +298,19 @@ class Table:
                                          ctypes.byref(step), _stream(stream)), "recis_table_export")
         return keys[:n], emb[:n], st[:n], step.value
 
+    def read_rows(self, rows: torch.Tensor, stream=None):
+        """(keys int64[n], emb fp32[n, D], state fp32[n, s*D]) of the given row
+        offsets (device int64), gathered on the device."""
+        n = rows.numel()
+        dev = rows.device
+        keys = torch.empty(max(n, 1), dtype=torch.int64, device=dev)
+        emb = torch.empty((max(n, 1), self.dim), dtype=torch.float32, device=dev)
+        st = torch.empty((max(n, 1), self.s * self.dim), dtype=torch.float32, device=dev)
+        _check(load().recis_table_read_rows(self.handle, _dev(rows, torch.int64), n, keys.data_ptr(),
+                                            emb.data_ptr(), st.data_ptr(), _stream(stream)),
+               "recis_table_read_rows")
+        return keys[:n], emb[:n], st[:n]
+
     def import_rows(self, keys, emb, state=None, step: int = 0, stream=None):
         import numpy as np
         keys = np.ascontiguousarray(keys, np.int64)
@@ -311,6 +334,54 @@ def unique_static(keys: torch.Tensor, stream=None):
     _check(load().recis_unique_static(_dev(keys, torch.int64), n, uniq.data_ptr(), inv.data_ptr(),
                                       U.data_ptr(), _stream(stream)), "recis_unique_static")
     return uniq, inv, U
+
+
+@dataclass
+class TablePlan:
+    """Result of plan_tables: per feature its logical table, tag and tag shift;
+    per logical table its merged configuration (a TableConfig)."""
+    table_of: list
+    tag_of: list
+    tag_shift_of: list
+    tables: list
+
+
+def plan_tables(features) -> TablePlan:
+    """recis_plan_tables (host only): merge features whose table attributes
+    are equal into logical tables.  features: sequence of (TableConfig,
+    value_bits) pairs."""
+    F = len(features)
+    arr = (FeatureSpec * max(F, 1))()
+    for f, (cfg, bits) in enumerate(features):
+        arr[f].table = cfg
+        arr[f].value_bits = bits
+    table_of = (ctypes.c_int32 * max(F, 1))()
+    tag_of = (ctypes.c_uint64 * max(F, 1))()
+    shift_of = (ctypes.c_int32 * max(F, 1))()
+    tabs = (TableConfig * max(F, 1))()
+    n = ctypes.c_int32(0)
+    _check(load().recis_plan_tables(arr, F, table_of, tag_of, shift_of, tabs, ctypes.byref(n)),
+           "recis_plan_tables")
+    return TablePlan(list(table_of[:F]), list(tag_of[:F]), list(shift_of[:F]),
+                     [tabs[i] for i in range(n.value)])
+
+
+def table_config(dim: int, optimizer: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+                 eps: Optional[float] = None, adagrad_init_acc: float = 0.0,
+                 init_scale: float = 0.0, init_seed: int = 0, initial_capacity: int = 0,
+                 block_rows: int = 0, max_rows: int = 0) -> TableConfig:
+    """A recis_table_config with the library's usual defaults."""
+    if eps is None:
+        eps = 1e-10 if optimizer == ADAGRAD else 1e-8
+    return TableConfig(dim=dim, optimizer=optimizer, lr=lr, beta1=beta1, beta2=beta2, eps=eps,
+                       adagrad_init_acc=adagrad_init_acc, init_scale=init_scale,
+                       init_seed=init_seed & (2**64 - 1), initial_capacity=initial_capacity,
+                       block_rows=block_rows, max_rows=max_rows)
+
+
+def debug_set(what: int, value: int):
+    """recis_debug_set: test hooks (DEBUG_SPIN_LIMIT, DEBUG_MAP_LIMIT; 0 = default)."""
+    _check(load().recis_debug_set(what, value), "recis_debug_set")
 
 
 def profile_enable(on: bool = True):

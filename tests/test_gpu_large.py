@@ -4,13 +4,17 @@ full large-table workload.
 - A 2.5M-occurrence batch (above the 1.6M sample-sort limit) runs through the
   LSD radix dedup and is compared with the oracle element by element.
 - The large-table workload at full size (50M pre-inserted keys, 65536 x 100
-  bags of geometric length, 32.8M occurrences) is too large for the oracle,
-  so integers are checked by properties that hold at any size (unique keys
-  strictly ascending, keys == uniq[inv], pre-inserted keys keep their rows,
-  new keys take the next rows in ascending key order) and floating point on
-  sampled bags and keys, each recomputed by the oracle from the pages'
-  definitions (pooled sum of the sampled bags; one Adam step of sampled keys
-  with their gradient summed over all their occurrences in float64).
+  bags of geometric length, 32.8M occurrences, two steps) is too large for the
+  oracle, so integers are checked by properties that hold at any size (unique
+  keys strictly ascending, keys == uniq[inv], every unique key has an
+  occurrence, U equals the number of distinct keys, pre-inserted keys keep
+  their rows, new keys take the next rows in ascending key order) and floating
+  point on sampled bags and keys, each recomputed by the oracle from the
+  pages' definitions: the pooled sums of sampled bags, and emb, Adam m and
+  Adam v of sampled keys after two steps with signed gradients, the oracle fed
+  each key's gradient summed over all its occurrences in float64 (m after the
+  first step is (1 - beta1) g, so the gradient's magnitude is pinned, not only
+  its sign).
 """
 import numpy as np
 import pytest
@@ -65,7 +69,43 @@ def test_radix_path_parity(R):
     p.close()
 
 
+def _host_grad(inv_dev, u, bag_offsets, gp, B):
+    """fp32 gradient of unique index u: its occurrences' pooled-gradient rows
+    summed in float64, rounded once (the oracle's definition of g(u))."""
+    occ = torch.nonzero(inv_dev == int(u)).flatten().cpu().numpy()
+    bag = np.searchsorted(bag_offsets, occ, side="right") - 1
+    return gp[bag % B, bag // B].astype(np.float64).sum(axis=0).astype(np.float32), len(occ)
+
+
+def _check_dedup(R, t, b, keys, N, live_dev, live_before, n_before):
+    """Integer checks of one full-size lookup that hold at any size."""
+    uq, inv, rows, n_new = b.get_unique(N)
+    torch.cuda.synchronize()
+    U = uq.numel()
+    assert bool((uq[1:] > uq[:-1]).all())                       # strictly ascending
+    assert torch.equal(uq[inv.long()], keys)                     # keys == uniq[inv]
+    cnt = torch.bincount(inv.long(), minlength=U)
+    assert cnt.numel() == U and int((cnt == 0).sum()) == 0       # every unique key occurs
+    assert U == int(torch.unique(keys).numel())                  # U = distinct keys
+    n_live = live_dev.numel()
+    at = torch.searchsorted(live_dev, uq)
+    found = (at < n_live) & (live_dev[at.clamp(max=n_live - 1)] == uq)
+    assert torch.equal(rows[found], at[found])                   # pre-inserted keys keep their rows
+    # keys already added by an earlier step keep their rows too; the rest are new
+    old = rows[~found] < n_before
+    assert int((rows[~found][old] >= live_before).sum()) == int(old.sum())
+    assert n_new == int((~found).sum()) - int(old.sum())
+    fresh_rows = rows[~found][~old]
+    assert torch.equal(fresh_rows, n_before + torch.arange(n_new, device=DEV))  # ascending key order
+    assert t.size()[0] == n_before + n_new
+    return uq, inv, rows, n_new, cnt
+
+
 def test_large_workload_full_size_sampled(R):
+    """Two steps of the large-table workload at full size with signed
+    gradients: integers by properties, pooled rows of sampled bags, and the
+    emb, Adam m and Adam v of sampled keys after both steps against the oracle
+    fed each key's gradient summed in float64 over all its occurrences."""
     w = W.WORKLOADS["large"]
     spec = w.tables[0]
     D, F, B = spec.dim, w.F, w.B
@@ -82,69 +122,88 @@ def test_large_workload_full_size_sampled(R):
         t.insert(b_ins, torch.from_numpy(live[c0:c0 + 1_500_000]).to(DEV))
     t.status_sync()
     assert t.size()[0] == n_live  # rows 0 .. n_live-1 in ascending key order
-
-    # one step of the workload at full size
-    bt = W.make_batch(w, 0)
-    N = len(bt.values)
-    ops = [O.FeatureOp(flags=f.flags, tag=f.tag, tag_shift=f.tag_shift) for f in w.features]
-    okeys = O.feature_hash(ops, bt.values, bt.feat_offsets)
-    keys = R.feature_hash([R.Feature(flags=f.flags, tag=f.tag, tag_shift=f.tag_shift)
-                           for f in w.features],
-                          torch.from_numpy(bt.values).to(DEV), bt.feat_offsets.tolist())
-    assert np.array_equal(keys.cpu().numpy(), okeys)
-    bo_dev = torch.from_numpy(bt.bag_offsets).to(DEV)
-    pooled = torch.empty((B, F, D), dtype=torch.float32, device=DEV)
-    b = R.Batch()
-    t.lookup_pooled(b, keys, bo_dev, F, B, R.SUM, pooled)
-    uq, inv, rows, n_new = b.get_unique(N)
-    torch.cuda.synchronize()
-
-    # integers, at full size: ascending unique keys, inverse, row assignment
-    assert bool((uq[1:] > uq[:-1]).all())
-    assert torch.equal(uq[inv.long()], keys)
     live_dev = torch.from_numpy(live).to(DEV)
-    at = torch.searchsorted(live_dev, uq)
-    found = (at < n_live) & (live_dev[at.clamp(max=n_live - 1)] == uq)
-    assert torch.equal(rows[found], at[found])  # pre-inserted keys keep their rows
-    assert n_new == int((~found).sum())
-    assert torch.equal(rows[~found], n_live + torch.arange(n_new, device=DEV))  # ascending key order
-    assert t.size()[0] == n_live + n_new
 
-    # pooled sums of sampled bags against the oracle on those bags alone
-    # (every row is still at its initial value)
-    bags = rng.choice(F * B, size=300, replace=False)
-    lo, hi = bt.bag_offsets[bags], bt.bag_offsets[bags + 1]
-    mkeys = np.concatenate([okeys[a:c] for a, c in zip(lo, hi)])
-    mbo = np.concatenate([[0], np.cumsum(hi - lo)]).astype(np.int64)
+    ops = [O.FeatureOp(flags=f.flags, tag=f.tag, tag_shift=f.tag_shift) for f in w.features]
+    rfeats = [R.Feature(flags=f.flags, tag=f.tag, tag_shift=f.tag_shift) for f in w.features]
+    b = R.Batch()
+    pooled = torch.empty((B, F, D), dtype=torch.float32, device=DEV)
+    steps = []
+    n_before = n_live
+    for step in range(2):
+        bt = W.make_batch(w, step)
+        N = len(bt.values)
+        okeys = O.feature_hash(ops, bt.values, bt.feat_offsets)
+        keys = R.feature_hash(rfeats, torch.from_numpy(bt.values).to(DEV), bt.feat_offsets.tolist())
+        assert np.array_equal(keys.cpu().numpy(), okeys)
+        bo_dev = torch.from_numpy(bt.bag_offsets).to(DEV)
+        t.lookup_pooled(b, keys, bo_dev, F, B, R.SUM, pooled)
+        uq, inv, rows, n_new, cnt = _check_dedup(R, t, b, keys, N, live_dev, n_live, n_before)
+        assert n_new > 0.04 * N  # the workload's 5% fresh IDs are new rows
+        if step == 0:
+            # pooled sums of sampled bags against the oracle on those bags alone
+            # (every row is still at its initial value)
+            bags = rng.choice(F * B, size=300, replace=False)
+            lo, hi = bt.bag_offsets[bags], bt.bag_offsets[bags + 1]
+            mkeys = np.concatenate([okeys[a:c] for a, c in zip(lo, hi)])
+            mbo = np.concatenate([[0], np.cumsum(hi - lo)]).astype(np.int64)
+            ot = O.Table(D, O.ADAM, spec.lr, init_seed=spec.init_seed)
+            ref = ot.lookup(mkeys, mbo, 1, len(bags), O.SUM).pooled[:, 0, :]
+            pc = pooled.cpu().numpy()
+            got = np.stack([pc[j % B, j // B] for j in bags])
+            close(got, ref, "pooled, sampled bags")
+        gp = W.make_grad((B, F, D), 4242 + step, signed=True)
+        t.backward_update(b, torch.from_numpy(gp).to(DEV))
+        t.status_sync()
+        steps.append((bt, uq, inv, rows, cnt, gp))
+        n_before += n_new
+
+    # sampled keys: random and hottest keys of step 0, fresh keys of step 0,
+    # random keys of step 1 (some present in both steps)
+    uq0, inv0, rows0, cnt0 = steps[0][1], steps[0][2], steps[0][3], steps[0][4]
+    uq1, inv1, rows1, cnt1 = steps[1][1], steps[1][2], steps[1][3], steps[1][4]
+    U0, U1 = uq0.numel(), uq1.numel()
+    fresh0 = torch.nonzero(rows0 >= n_live).flatten().cpu().numpy()
+    pick0 = np.unique(np.concatenate([rng.choice(U0, 40, replace=False),
+                                      torch.argsort(cnt0, descending=True)[:8].cpu().numpy(),
+                                      rng.choice(fresh0, 8, replace=False)]))
+    skeys = set(uq0[torch.from_numpy(pick0).to(DEV)].cpu().tolist())
+    skeys |= set(uq1[torch.from_numpy(rng.choice(U1, 24, replace=False)).to(DEV)].cpu().tolist())
+    skeys = np.array(sorted(skeys), np.int64)
+    # each sampled key's gradient per step (zero when absent), its row, and
+    # the oracle table stepped the same way (a dummy key keeps its Adam step
+    # counter in line with the GPU table's when no sampled key is present)
     ot = O.Table(D, O.ADAM, spec.lr, init_seed=spec.init_seed)
-    ref = ot.lookup(mkeys, mbo, 1, len(bags), O.SUM).pooled[:, 0, :]
-    pc = pooled.cpu().numpy()
-    got = np.stack([pc[j % B, j // B] for j in bags])
-    close(got, ref, "pooled, sampled bags")
-
-    # one Adam step: updated rows of sampled keys against the oracle fed the
-    # key's gradient summed in float64 over all its occurrences
-    gp = W.make_grad((B, F, D), 4242)
-    t.backward_update(b, torch.from_numpy(gp).to(DEV))
-    t.status_sync()
-    U = len(uq)
-    pick = np.unique(np.concatenate([rng.choice(U, size=48, replace=False),
-                                     np.argsort(-torch.bincount(inv.long()).cpu().numpy())[:8]]))
-    skeys = uq[torch.from_numpy(pick).to(DEV)]
-    cur = torch.empty((len(pick), D), dtype=torch.float32, device=DEV)
-    b3 = R.Batch()
-    sbo = torch.arange(len(pick) + 1, dtype=torch.int64, device=DEV)
-    t.lookup_pooled(b3, skeys, sbo, 1, len(pick), R.SUM, None, cur)
-    cur = cur.cpu().numpy()
-    for n, u in enumerate(pick):
-        occ = torch.nonzero(inv == int(u)).flatten().cpu().numpy()
-        bag = np.searchsorted(bt.bag_offsets, occ, side="right") - 1
-        g = gp[bag % B, bag // B].astype(np.float64).sum(axis=0).astype(np.float32)
-        o1 = O.Table(D, O.ADAM, spec.lr, init_seed=spec.init_seed)
-        o1.lookup(np.array([int(skeys[n])], np.int64), np.array([0, 1], np.int64), 1, 1, O.SUM)
-        o1.backward_update(g.reshape(1, 1, D))
-        _, emb, _ = o1.export()
-        close(cur[n], emb[0], f"updated row of unique key {int(u)} ({len(occ)} occurrences)")
-    for x in (b3, b, b_ins):
+    dummy = np.int64(-7)
+    row_of = {}
+    for s_i, (bt, uq, inv, rows, cnt, gp) in enumerate(steps):
+        uqh = uq.cpu().numpy()
+        pos = np.searchsorted(uqh, skeys)
+        present = (pos < len(uqh)) & (uqh[np.minimum(pos, len(uqh) - 1)] == skeys)
+        ks, gs = [dummy], [np.zeros(D, np.float32)]
+        for k, pz, pr in zip(skeys, pos, present):
+            if not pr:
+                continue
+            g, nocc = _host_grad(inv, pz, bt.bag_offsets, gp, B)
+            assert nocc == int(cnt[pz])
+            ks.append(k)
+            gs.append(g)
+            row_of[int(k)] = int(rows[pz])
+        order = np.argsort(np.array(ks))
+        kk = np.array(ks, np.int64)[order]
+        gg = np.stack(gs)[order]
+        ot.lookup(kk, np.arange(len(kk) + 1, dtype=np.int64), 1, len(kk), O.SUM)
+        ot.backward_update(gg.reshape(len(kk), 1, D))
+    rsel = torch.tensor([row_of[int(k)] for k in skeys], dtype=torch.int64, device=DEV)
+    gk, ge, gs_ = t.read_rows(rsel)
+    assert np.array_equal(gk.cpu().numpy(), skeys)
+    okeys_, oemb, ostate = ot.export()
+    idx = np.searchsorted(okeys_, skeys)
+    assert np.array_equal(okeys_[idx], skeys)
+    close(ge.cpu().numpy(), oemb[idx], "emb of sampled keys after two Adam steps")
+    close(gs_.cpu().numpy()[:, :D], ostate[idx][:, :D], "Adam m of sampled keys")
+    close(gs_.cpu().numpy()[:, D:], ostate[idx][:, D:], "Adam v of sampled keys")
+    assert t.size()[1] == 2
+    for x in (b, b_ins):
         x.close()
     t.close()

@@ -197,6 +197,7 @@ class Batch:
     feat_offsets: np.ndarray  # int64 [F+1]
     bag_offsets: np.ndarray   # int64 [F*B+1]
     lengths: np.ndarray       # int64 [F*B]
+    fresh_pos: Optional[List[np.ndarray]] = None  # per feature: positions holding fresh IDs
 
     def table_slice(self, t: TableSpec, B: int):
         """(value range, bag offsets rebased to 0) for the features of table t."""
@@ -228,25 +229,46 @@ def make_batch(w: Workload, batch_index: int = 0, seed: Optional[int] = None) ->
     N = int(bag_offsets[-1])
     feat_offsets = bag_offsets[:: w.B].copy()
     values = np.empty(N, np.int64)
-    zipf = Zipf(w.live_ids if w.live_ids else w.n_ids, w.zipf_a)
-    fresh_counter = 0
+    # large-table workload: Zipf over each feature's share of the live set (the
+    # pre-inserted IDs of live_ids()), so every non-fresh occurrence is live
+    zipf = Zipf(w.live_ids // w.F if w.live_ids else w.n_ids, w.zipf_a)
+    fresh_pos = [] if w.fresh_frac > 0 else None
     for f in range(w.F):
         lo, hi = int(feat_offsets[f]), int(feat_offsets[f + 1])
         n = hi - lo
         ranks0 = zipf.sample(rng, n) - 1
         if w.fresh_frac > 0:
-            fresh = rng.random(n) < w.fresh_frac
-            nf = int(fresh.sum())
-            # never-seen IDs: ranks beyond the live set, from a per-batch counter
-            ranks0[fresh] = (w.live_ids + ((batch_index + 1) << 32) + fresh_counter
-                             + np.arange(nf, dtype=np.int64))
-            fresh_counter += nf
+            fresh = np.nonzero(rng.random(n) < w.fresh_frac)[0]
+            ranks0[fresh] = _fresh_ranks(w, f, batch_index, len(fresh))
+            fresh_pos.append(lo + fresh)
         values[lo:hi] = scramble(ranks0, w.n_ids, key=(base << 8) + f)
-    return Batch(values, feat_offsets, bag_offsets, lengths)
+    return Batch(values, feat_offsets, bag_offsets, lengths, fresh_pos)
+
+
+def _fresh_ranks(w: Workload, f: int, stream_index: int, count: int) -> np.ndarray:
+    """Ranks of never-seen IDs: past the live set, from a counter range of
+    feature f and stream index (disjoint for different (f, index) pairs)."""
+    assert 0 <= stream_index < 4095 and f < 256 and count < (1 << 28)
+    return (w.live_ids + ((stream_index + 1) << 36) + (f << 28)
+            + np.arange(count, dtype=np.int64))
+
+
+def with_fresh_ids(w: Workload, b: Batch, stream_index: int,
+                   seed: Optional[int] = None) -> np.ndarray:
+    """Values of batch b with every fresh-ID position given a never-seen ID of
+    counter range `stream_index` (the rest unchanged): one more step of the
+    large-table workload without drawing its Zipf part again."""
+    base = 2025 + w.index if seed is None else seed
+    vals = b.values.copy()
+    for f, pos in enumerate(b.fresh_pos or []):
+        ranks0 = _fresh_ranks(w, f, stream_index, len(pos))
+        vals[pos] = scramble(ranks0, w.n_ids, key=(base << 8) + f)
+    return vals
 
 
 def live_ids(w: Workload, f: int, count: int, seed: Optional[int] = None) -> np.ndarray:
-    """The IDs of ranks 1..count of feature f (the pre-inserted live set)."""
+    """The IDs of ranks 1..count of feature f (the pre-inserted live set:
+    count = live_ids // F per feature)."""
     base = 2025 + w.index if seed is None else seed
     return scramble(np.arange(count, dtype=np.int64), w.n_ids, key=(base << 8) + f)
 
