@@ -137,6 +137,7 @@ struct recis_batch {
   int4* gsrc = nullptr;         // [capN] per sorted position: {gradient row, bag length, occurrence, 0}
   int4* gfirst = nullptr;       // [capN] per unique key: the same, of one of its occurrences
   int32_t* chunk_bag = nullptr; // bag of each pool chunk's first occurrence
+  int32_t* bag_of = nullptr;    // [capN] bag of every occurrence (written beside the dedup)
   int64_t capChunks = 0;
   cudaStream_t side = nullptr;  // bag preparation runs here, beside the dedup
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;

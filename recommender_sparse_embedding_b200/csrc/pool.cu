@@ -7,10 +7,14 @@
 // reduction over occurrence order (segreduce.cuh): a group of G lanes owns a
 // chunk of C occurrences, each lane one 16-byte column of the row.  Rows
 // stream through a ring of R slots per lane in shared memory (cp.async), so R
-// row loads per lane are in flight while the group adds.  The bag of the
-// chunk's first occurrence comes from the bag preparation; later bag
-// boundaries come from a window of G bag ends held one per lane.  A chunk
-// whose bags all hold one occurrence (one-hot features) is a plain gather.
+// row loads per lane are in flight while the group adds.  The bag
+// preparation (beside the dedup) writes the bag of every occurrence; the
+// group resolves G positions at a time, one per lane (row, sorted position,
+// unique key, bag and its bounds, one sub-block ahead), writes their
+// gradient-source records lane-parallel, and marks the positions that end a
+// bag in one ballot, so the walk itself only adds rows and flushes at the
+// marks.  A chunk whose bags all hold one occurrence (one-hot features) is a
+// plain gather.
 // Outputs: pooled rows [B][F][D] (sum, or mean = sum / length), optional
 // unpooled rows [N][D], and the gradient source of every occurrence for the
 // backward.
@@ -42,6 +46,7 @@ struct PoolParams {
   int4* gsrc;            // [N] per sorted position: {gradient row b*F+f, bag length, occurrence, 0}
   int4* gfirst;          // [U] per unique key: the same, of one of its occurrences
   int32_t* chunk_bag;    // [nchunks] bag of each chunk's first occurrence
+  int32_t* bag_of;       // [N] bag of every occurrence
   double* partials;
   int32_t* counters;     // [nbags]
   DevState* st;
@@ -49,29 +54,46 @@ struct PoolParams {
 };
 
 // Bag preparation, one thread per bag (runs beside the dedup on a side
-// stream): checks the offsets, writes the bag of every chunk's first
-// occurrence, and zeroes the pooled output of empty bags.
+// stream): checks the offsets, writes the bag of every occurrence and of every
+// chunk's first occurrence, and zeroes the pooled output of empty bags.  A bag
+// of more than 32 occurrences has its bag ids written by the whole warp.
 __global__ void __launch_bounds__(256) bag_prep_kernel(const __grid_constant__ PoolParams p) {
   const int64_t D = (int64_t)p.ncol * 4;
+  const int lane = threadIdx.x & 31;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   if (blockIdx.x == 0 && threadIdx.x == 0 &&
       (p.offs[0] != 0 || p.offs[p.nbags] != p.N))
     raise_error(p.st, p.mirror, kErrBadOffsets);
-  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < p.nbags; j += stride) {
-    const int64_t lo = p.offs[j], hi = p.offs[j + 1];
-    if (lo < 0 || hi < lo || hi > p.N) {
-      raise_error(p.st, p.mirror, kErrBadOffsets);
-      continue;
-    }
-    if (hi == lo) {
-      if (p.pooled) {
-        const int64_t f = j / p.B, b = j - f * p.B;
-        float4* o = reinterpret_cast<float4*>(p.pooled + (b * p.F + f) * D);
-        for (int c = 0; c < p.ncol; ++c) o[c] = f4_zero();
+  // warp-uniform trip count, so the warp can share out its long bags
+  for (int64_t j0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); j0 < p.nbags; j0 += stride) {
+    const int64_t j = j0 + lane;
+    int64_t lo = 0, hi = 0;
+    if (j < p.nbags) {
+      lo = p.offs[j];
+      hi = p.offs[j + 1];
+      if (lo < 0 || hi < lo || hi > p.N) {
+        raise_error(p.st, p.mirror, kErrBadOffsets);
+        lo = hi = 0;
+      } else if (hi == lo) {
+        if (p.pooled) {
+          const int64_t f = j / p.B, b = j - f * p.B;
+          float4* o = reinterpret_cast<float4*>(p.pooled + (b * p.F + f) * D);
+          for (int c = 0; c < p.ncol; ++c) o[c] = f4_zero();
+        }
+      } else {
+        for (int64_t c = (lo + p.C - 1) / p.C; c * p.C < hi; ++c) p.chunk_bag[c] = (int32_t)j;
+        if (hi - lo <= 32)
+          for (int64_t q = lo; q < hi; ++q) p.bag_of[q] = (int32_t)j;
       }
-      continue;
     }
-    for (int64_t c = (lo + p.C - 1) / p.C; c * p.C < hi; ++c) p.chunk_bag[c] = (int32_t)j;
+    unsigned lng = __ballot_sync(0xffffffffu, hi - lo > 32);
+    while (lng) {
+      const int l = __ffs(lng) - 1;
+      const int64_t a = __shfl_sync(0xffffffffu, lo, l), e = __shfl_sync(0xffffffffu, hi, l);
+      const int32_t jl = (int32_t)(j0 + l);
+      for (int64_t q = a + lane; q < e; q += 32) p.bag_of[q] = jl;
+      lng &= lng - 1;
+    }
   }
 }
 
@@ -122,31 +144,45 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     }
     return r;
   };
+  // bag of a position and its bounds (bag_of is written beside the dedup)
+  struct Bag {
+    int j, lo, hi;
+  };
+  auto bag_at = [&](int sub) {
+    Bag r{0, 0, 0};
+    const int q = sub + g.lane;
+    if (q < p1) {
+      int j = __ldg(p.bag_of + q);
+      if (j < 0 || j >= nbags) j = 0;  // only with malformed bag offsets (reported by the preparation)
+      r.j = j;
+      r.lo = (int)__ldg(p.offs + j);
+      r.hi = (int)__ldg(p.offs + j + 1);
+    }
+    return r;
+  };
   // the ids of the first sub-block are in flight while the bag walk starts
   const Ids ids0 = resolve(p0);
 
-  // bag containing p0 (precomputed), its start, and a window of G bag ends
+  // bag containing p0 (precomputed), its start, and the ends of the G bags
+  // from it on (for the one-hot test)
   int j0 = p.chunk_bag[chunk];
   if (j0 < 0 || j0 >= nbags) {  // only with malformed offsets
     if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
     j0 = 0;
   }
-  int cur = j0;
-  int cf = cur / B, cb = cur - cf * B;  // feature and sample of the current bag
-  int cur_start = (int)p.offs[j0];
-  int wbase = j0;
-  int wend = (wbase + g.lane < nbags) ? (int)p.offs[wbase + g.lane + 1] : INT_MAX;
-  int cur_end = g.bcast(wend, 0);
+  const int cur_start = (int)p.offs[j0];
+  const int wend = (j0 + g.lane < nbags) ? (int)p.offs[j0 + g.lane + 1] : INT_MAX;
 
   Acc4 acc[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
-  bool has = false;
 
-  auto epilogue = [&]() {
+  // the pooled row of bag j (sum, or mean over its len occurrences)
+  auto store_bag = [&](int j, int len) {
     if (!p.pooled) return;
-    float4* o = reinterpret_cast<float4*>(p.pooled + (int64_t)(cb * F + cf) * D);
-    const double dlen = (double)(cur_end - cur_start);
+    const int f = j / B;
+    float4* o = reinterpret_cast<float4*>(p.pooled + (int64_t)((j - f * B) * F + f) * D);
+    const double dlen = (double)len;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       const int col = g.lane + v * G;
@@ -161,20 +197,6 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
         __stcs(o + col, acc_round(r));
       }
     }
-  };
-  auto flush = [&]() {
-    if (!has) return;
-    if (!(cur_start >= 0 && cur_start < cur_end && cur_end <= N)) {  // malformed bag offsets
-      if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
-    } else if (cur_start >= p0 && cur_end <= p1) {
-      epilogue();
-    } else if (combine_split<G, VPL>(g, acc, p.partials, p.counters, cur, chunk, cur == j0,
-                                     cur_start, cur_end, C, ncol)) {
-      epilogue();
-    }
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
-    has = false;
   };
 
   // rows stream through a ring of R slots per lane in shared memory: row t+R
@@ -261,70 +283,64 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     return;
   }
 
+  // The bag walk.  Per sub-block of G positions (one per lane, resolved one
+  // sub-block ahead): the positions' gradient sources are written by their
+  // own lanes, and `ends` marks the positions after which the running sum is
+  // flushed -- the last position of a bag, or of the chunk.
+  auto flush_bag = [&](int j, int lo, int hi) {
+    if (!(lo >= 0 && lo < hi && hi <= N)) {  // malformed bag offsets
+      if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
+    } else if (lo >= p0 && hi <= p1) {
+      store_bag(j, hi - lo);
+    } else if (combine_split<G, VPL>(g, acc, p.partials, p.counters, j, chunk, lo <= p0, lo, hi, C,
+                                     ncol)) {
+      store_bag(j, hi - lo);
+    }
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
+  };
+  auto emit = [&](int sub, const Ids& ids, const Bag& bg) {
+    const int q = sub + g.lane;
+    if (q < p1) {
+      const int f = bg.j / B;
+      const int4 src = make_int4((bg.j - f * B) * F + f, bg.hi - bg.lo, q, 0);
+      p.gsrc[ids.spos] = src;
+      p.gfirst[ids.seg] = src;
+    }
+    return g.ballot(q < p1 && (q + 1 == bg.hi || q + 1 == p1));
+  };
   Ids cur_ids = ids0, nxt_ids = resolve(p0 + G);
+  Bag cur_bag = bag_at(p0), nxt_bag = bag_at(p0 + G);
+  unsigned ends = emit(p0, cur_ids, cur_bag);
 #pragma unroll
   for (int t = 0; t < R; ++t) issue(t, t < m ? g.bcast(cur_ids.row, t) : -1);
   for (int t = 0; t < m; ++t) {
-    const int pos = p0 + t;
     const int ln = t % G;
     const int row = g.bcast(cur_ids.row, ln);
-    const int spos = g.bcast(cur_ids.spos, ln);
-    const int seg = g.bcast(cur_ids.seg, ln);
     cp_async_wait<R - 1>();
-    float4 val[VPL];
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       const int col = g.lane + v * G;
-      val[v] = (row >= 0 && col < ncol) ? *slot(t % R, v) : f4_zero();
+      const float4 val = (row >= 0 && col < ncol) ? *slot(t % R, v) : f4_zero();
+      acc_add(acc[v], val);
+      if (p.unpooled && col < ncol)
+        __stcs(reinterpret_cast<float4*>(p.unpooled + (int64_t)(p0 + t) * D) + col, val);
     }
     // the row R positions ahead (in this sub-block or the next) into the slot just read
     const int ta = t + R;
     int arow = -1;
     if (ta < m) arow = (ta / G == t / G) ? g.bcast(cur_ids.row, ta % G) : g.bcast(nxt_ids.row, ta % G);
     issue(ta, arow);
-    while (pos >= cur_end) {  // leave the current bag (and any empty ones)
-      flush();
-      if (cur + 1 >= nbags) {  // only reachable with malformed bag offsets
-        if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
-        cur_end = INT_MAX;
-        break;
-      }
-      ++cur;
-      if (++cb == B) {
-        cb = 0;
-        ++cf;
-      }
-      cur_start = cur_end;
-      if (cur - wbase >= G) {
-        wbase = cur;
-        wend = (wbase + g.lane < nbags) ? (int)p.offs[wbase + g.lane + 1] : INT_MAX;
-      }
-      cur_end = g.bcast(wend, cur - wbase);
-    }
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) acc_add(acc[v], val[v]);
-    has = true;
-    if (p.unpooled) {
-      float4* dst = reinterpret_cast<float4*>(p.unpooled + (int64_t)pos * D);
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) {
-        const int col = g.lane + v * G;
-        if (col < ncol) __stcs(dst + col, val[v]);
-      }
-    }
-    // for the backward: this occurrence's gradient source, by sorted
-    // position and by unique key
-    if (g.lane == 0) {
-      const int4 src = make_int4(cb * F + cf, cur_end - cur_start, pos, 0);
-      p.gsrc[spos] = src;
-      p.gfirst[seg] = src;
-    }
-    if (ln == G - 1) {  // next sub-block
+    if ((ends >> ln) & 1u)
+      flush_bag(g.bcast(cur_bag.j, ln), g.bcast(cur_bag.lo, ln), g.bcast(cur_bag.hi, ln));
+    if (ln == G - 1 && t + 1 < m) {  // next sub-block
       cur_ids = nxt_ids;
+      cur_bag = nxt_bag;
+      ends = emit(p0 + t + 1, cur_ids, cur_bag);
       nxt_ids = resolve(p0 + t + 1 + G);
+      nxt_bag = bag_at(p0 + t + 1 + G);
     }
   }
-  flush();
   pdl_trigger();
 }
 
@@ -385,6 +401,7 @@ static PoolParams pool_params(const LookupArgs& a, int64_t chunk) {
   p.gsrc = b->gsrc;
   p.gfirst = b->gfirst;
   p.chunk_bag = b->chunk_bag;
+  p.bag_of = b->bag_of;
   p.partials = b->partials;
   p.counters = b->bag_counter;
   p.st = t->dstate;

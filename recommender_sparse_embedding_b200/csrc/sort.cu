@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restric
                                                         int64_t N, SortCtl* ctl, DevState* st,
                                                         HostMirror* mirror, BatchDev* bdev,
                                                         uint32_t call_id) {
-  constexpr int kPer = 4;  // keys per thread per round, loaded before they are counted
+  constexpr int kPer = 8;  // keys per thread per round, all loaded before they are counted
   __shared__ unsigned int sh[kSortPasses][256];
   __shared__ bool s_last;
   for (int i = threadIdx.x; i < kSortPasses * 256; i += blockDim.x) (&sh[0][0])[i] = 0;
@@ -45,26 +45,31 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restric
   const int lane = threadIdx.x & 31;
   bool reserved = false;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x * kPer;
-  // warp-uniform trip count so that match/ballot see the whole warp
+  // warp-uniform trip count so that the votes see the whole warp
   const int64_t base0 = ((int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31)) * kPer;
   for (int64_t wb = base0; wb < N; wb += stride) {
     int64_t k[kPer];
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int64_t i = wb + j * 32 + lane;
-      k[j] = i < N ? keys[i] : 0;
+      k[j] = i < N ? __ldcs(keys + i) : 0;
     }
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const bool valid = wb + j * 32 + lane < N;
       reserved |= valid && (k[j] == kEmptyKey);
       const uint64_t u = to_ukey(k[j]);
-      const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+      const bool full = __all_sync(0xffffffffu, valid);
 #pragma unroll
       for (int p = 0; p < kSortPasses; ++p) {
         const unsigned d = (unsigned)(u >> (p * kSortBits)) & 255u;
-        const unsigned peers = __match_any_sync(0xffffffffu, valid ? d : 256u) & vmask;
-        if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh[p][d], (unsigned)__popc(peers));
+        // a digit the whole warp shares (the constant high digits of tagged
+        // keys) is one add of 32; the others one shared atomic per key
+        if (full && __all_sync(0xffffffffu, d == __shfl_sync(0xffffffffu, d, 0))) {
+          if (lane == 0) atomicAdd(&sh[p][d], 32u);
+        } else if (valid) {
+          atomicAdd(&sh[p][d], 1u);
+        }
       }
     }
   }
@@ -289,7 +294,7 @@ cudaError_t launch_sort(recis_batch* b, recis_table* t, const int64_t* keys, int
     if (e != cudaSuccess) return e;
   }
   {
-    int64_t blocks = (N + 1023) / 1024;  // 4 keys per thread
+    int64_t blocks = (N + 2047) / 2048;  // 8 keys per thread
     if (blocks > 8 * kSMs) blocks = 8 * kSMs;
     if (blocks < 1) blocks = 1;
     LaunchScope ls("sort_hist", s);

@@ -392,6 +392,7 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
         (e = realloc_dev(b->gsrc, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->gfirst, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_counter, cap, true)) != cudaSuccess ||
+        (e = realloc_dev(b->bag_of, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->multi_keys, cap / 2 + 1, false)) != cudaSuccess)
       return cuda_fail(e, "batch alloc");
     const int64_t st = (cap + kSortTile - 1) / kSortTile;
@@ -478,6 +479,7 @@ static void batch_free(recis_batch* b) {
   cudaFree(b->chunk_counter);
   cudaFree(b->bdev);
   cudaFree(b->chunk_bag);
+  cudaFree(b->bag_of);
   if (b->side) cudaStreamDestroy(b->side);
   if (b->ev_fork) cudaEventDestroy(b->ev_fork);
   if (b->ev_join) cudaEventDestroy(b->ev_join);

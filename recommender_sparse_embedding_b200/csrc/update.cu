@@ -137,6 +137,17 @@ __device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateP
   const int64_t D = (int64_t)p.ncol * 4;
   const int64_t p0 = chunk * kChunk;
   const int64_t p1 = p0 + kChunk < p.N ? p0 + kChunk : p.N;
+  if (!p.meta && !p.long_chunks) {
+    // no marks from the dedup: a segment lying wholly inside the chunk is
+    // short (kChunk <= kShortSeg), so only the segments of the chunk's first
+    // and last positions can be long; a chunk where neither is ends here
+    bool lng = false;
+    for (int e = g.lane; e < 2; e += G) {
+      const int32_t sg = __ldg(p.seg_of + (e == 0 ? p0 : p1 - 1));
+      lng |= __ldg(p.seg_start + sg + 1) - __ldg(p.seg_start + sg) > kShortSeg;
+    }
+    if (!g.ballot(lng)) return;
+  }
   Acc4 acc[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
@@ -198,8 +209,12 @@ __device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateP
 
 // With the dedup's list of chunks holding a long segment, a persistent grid
 // of groups walks the list; without it, one group per chunk.
+// resident CTAs of 256 threads per SM of the long-segment reduction
+template <int VPL>
+constexpr int kSegReduceCtas = VPL == 1 ? 3 : (VPL == 2 ? 2 : 1);
+
 template <int G, int VPL, bool GP, bool GU>
-__global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
+__global__ void __launch_bounds__(256, kSegReduceCtas<VPL>)
     seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
   pdl_wait();
   const GroupCtx<G> g;
@@ -501,7 +516,7 @@ template <int G, int VPL, bool GP, bool GU>
 static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t ucap, cudaStream_t s) {
   {
     int64_t blocks = (p.nchunks * G + 255) / 256;
-    if (p.long_chunks && blocks > 3 * kSMs) blocks = 3 * kSMs;
+    if (p.long_chunks && blocks > kSegReduceCtas<VPL> * kSMs) blocks = kSegReduceCtas<VPL> * kSMs;
     if (blocks < 1) blocks = 1;
     LaunchScope ls("seg_reduce", s);
     const cudaError_t e = launch_pdl(seg_reduce_kernel<G, VPL, GP, GU>, (unsigned)blocks, 256, 0, s, p);
