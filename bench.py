@@ -436,12 +436,19 @@ def measure(w: W.Workload, args, R, dist, world: int, rank: int, dev, headline: 
         uniq.append([int(torch.unique(k[lo:hi]).numel()) for (lo, hi, *_r) in per_table])
         del k
 
+    rows_pre = [t.size()[0] for t in tables]
     for i in range(args.warmup):
         run_step(*devb[i % nb], keys)
     torch.cuda.synchronize()
     for t in tables:
         t.status_sync()
     rows0 = [t.size()[0] for t in tables]
+    # make room now for every row the remaining steps may add (from the
+    # warm-up's growth), so that no block is mapped and no IDMap rehashed
+    # inside the timed region
+    for t, r_pre, r0, (lo, hi, *_r) in zip(tables, rows_pre, rows0, devb[0][2]):
+        per_step = (r0 - r_pre) / max(args.warmup, 1)
+        t.reserve(int(r0 + 1.1 * per_step * (args.steps + prof_steps + e2e_steps + 2)) + (hi - lo))
 
     # ---- timed region: K steps, no tracing events between the kernels
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

@@ -212,6 +212,15 @@ recis_status recis_table_read_rows(recis_table_t t, const int64_t* rows, int64_t
                                    int64_t* keys_out, float* emb_out, float* state_out,
                                    recis_stream_t stream);
 
+/* Synchronous.  Makes room for `rows` live rows in total (README, Efficient
+ * dynamic embedding: EmbeddingBlocks grow on demand): maps EmbeddingBlocks and
+ * sizes the IDMap for them now, so that lookups that keep the table at or
+ * below that many rows map nothing and rehash nothing while they run (a
+ * lookup may still wait for earlier work when its host-side bound on new rows
+ * says it could pass the mapped rows).  Waits for `stream` first and returns
+ * any pending device-detected error.  rows > max_rows: RECIS_ERR_TABLE_FULL. */
+recis_status recis_table_reserve(recis_table_t t, int64_t rows, recis_stream_t stream);
+
 /* Synchronous.  Number of live rows and the Adam step counter. */
 recis_status recis_table_size(recis_table_t t, int64_t* n_out, int64_t* step_out,
                               recis_stream_t stream);

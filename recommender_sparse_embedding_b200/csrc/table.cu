@@ -875,6 +875,20 @@ recis_status recis_backward_update(recis_table_t t, recis_batch_t b, const float
   return RECIS_OK;
 }
 
+recis_status recis_table_reserve(recis_table_t t, int64_t rows, recis_stream_t stream) {
+  if (!t || rows < 0) {
+    set_error("table_reserve: bad arguments");
+    return RECIS_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  recis_status st = take_status(t, s);  // waits for the stream; exact live rows
+  if (st != RECIS_OK) return st;
+  const int64_t target = std::max(rows, t->rows_upper);
+  st = grow_rows(t, target);
+  if (st != RECIS_OK) return st;
+  return grow_idmap(t, target, s);
+}
+
 recis_status recis_table_status_sync(recis_table_t t, recis_stream_t stream) {
   if (!t) return RECIS_ERR_INVALID_ARG;
   return take_status(t, (cudaStream_t)stream);

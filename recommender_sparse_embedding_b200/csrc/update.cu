@@ -229,6 +229,157 @@ __global__ void __launch_bounds__(256, kSegReduceCtas<VPL>)
   pdl_trigger();
 }
 
+// ------------------------------------------------------------------ seg_reduce, staged
+// The same reduction for one 16-byte column per lane (D = 4G) and one kind of
+// gradient (pooled or unpooled), G >= 8: groups walk the listed chunks (one
+// each when the grid covers the list); a chunk's positions are resolved by
+// the group (each lane kChunk / G of them), and the gradient rows of all its
+// long positions are copied into shared memory by cp.async at once, one slot
+// per position and lane, so a chunk costs one round trip for its rows instead
+// of one per few rows.  Each lane copies and reads back only its own columns.
+__device__ __forceinline__ void cp_async16_(void* smem, const void* gmem) {
+  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+
+template <int G>
+struct ChunkPos {
+  static constexpr int E = G >= kChunk ? 1 : kChunk / G;  // positions per lane
+  int32_t seg[E], st[E], en[E], src[E];
+  double scale[E];
+  unsigned mask;  // bit t: position t of the chunk is in a long segment
+};
+
+template <int G, bool GP>
+__device__ __forceinline__ void chunk_indices(const GroupCtx<G>& g, const UpdateParams& p, int64_t chunk,
+                                              ChunkPos<G>& c) {
+  constexpr int E = ChunkPos<G>::E;
+  const int64_t p0 = chunk * kChunk;
+  bool lng[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int t = g.lane + e * G;
+    const int64_t q = p0 + t;
+    lng[e] = false;
+    c.seg[e] = 0;
+    c.st[e] = c.en[e] = c.src[e] = 0;
+    c.scale[e] = 1.0;
+    if (chunk >= 0 && t < kChunk && q < p.N) {
+      const bool marked = p.meta ? (__ldg(p.meta + q) >> 63) != 0 : true;
+      const int32_t sg = __ldg(p.seg_of + q);
+      const int4 gs = __ldg(p.gsrc + q);
+      const int32_t a = __ldg(p.seg_start + sg), b = __ldg(p.seg_start + sg + 1);
+      lng[e] = marked && b - a > kShortSeg;
+      c.seg[e] = sg;
+      c.st[e] = a;
+      c.en[e] = b;
+      c.src[e] = GP ? gs.x : gs.z;
+      c.scale[e] = (GP && p.mean) ? 1.0 / (double)gs.y : 1.0;
+    }
+  }
+  c.mask = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) c.mask |= g.ballot(lng[e]) << (e * G);
+}
+
+template <int G, bool GP>
+__global__ void __launch_bounds__(256, 3) seg_reduce_staged_kernel(const __grid_constant__ UpdateParams p) {
+  pdl_wait();
+  constexpr int E = ChunkPos<G>::E;
+  extern __shared__ float4 s_rows[];  // [groups of the CTA][kChunk][G]
+  const GroupCtx<G> g;
+  float4* rows = s_rows + (size_t)(threadIdx.x / G) * kChunk * G;
+  const int64_t groups = (int64_t)gridDim.x * blockDim.x / G;
+  const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  const int64_t n = (int64_t)p.bdev->nlong;
+  const int64_t D = (int64_t)p.ncol * 4;
+  const float* grad = GP ? p.gp : p.gu;
+  auto chunk_of = [&](int64_t i) -> int64_t { return i < n ? (int64_t)__ldg(p.long_chunks + i) : -1; };
+  ChunkPos<G> cur;
+  int64_t i = gid;
+  int64_t chunk = chunk_of(i);
+  chunk_indices<G, GP>(g, p, chunk, cur);
+  while (chunk >= 0) {
+    // this chunk's gradient rows into shared memory
+    for (unsigned m = cur.mask; m; m &= m - 1) {
+      const int t = __ffs(m) - 1;
+      const int32_t src = g.bcast(t / G == 0 ? cur.src[0] : cur.src[E - 1], t % G);
+      if (g.lane < p.ncol) cp_async16_(rows + t * G + g.lane, grad + (int64_t)src * D + 4 * g.lane);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    // the next chunk's positions meanwhile
+    const int64_t next = chunk_of(i + groups);
+    ChunkPos<G> nxt;
+    chunk_indices<G, GP>(g, p, next, nxt);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    // the long positions in order, one segment run at a time
+    const int64_t p0 = chunk * kChunk;
+    Acc4 acc = acc_zero();
+    int32_t sg = -1, cst = 0, cen = 0;
+    auto flush = [&]() {
+      Acc4 a1[1] = {acc};
+      const bool two_level = (cen - 1) / kChunk - cst / kChunk >= 2 * kCombineBlock;
+      if (two_level ? combine_split2<G, 1, 2, kCombineBlock>(g, a1, p.partials, p.chunk_counters, p.counters,
+                                                            sg, chunk, cst <= p0, cst, cen, kChunk, p.ncol)
+                    : combine_split<G, 1, 2>(g, a1, p.partials, p.counters, sg, chunk, cst <= p0, cst, cen,
+                                             kChunk, p.ncol)) {
+        if (g.lane < p.ncol) __stcg(reinterpret_cast<float4*>(p.gbuf + (cst / kChunk) * D) + g.lane,
+                                    acc_round(a1[0]));
+      }
+      acc = acc_zero();
+    };
+    for (unsigned m = cur.mask; m; m &= m - 1) {
+      const int t = __ffs(m) - 1;
+      const int e = t / G, l = t % G;
+      const int32_t s = g.bcast(e == 0 ? cur.seg[0] : cur.seg[E - 1], l);
+      if (s != sg) {
+        if (sg >= 0) flush();
+        sg = s;
+        cst = g.bcast(e == 0 ? cur.st[0] : cur.st[E - 1], l);
+        cen = g.bcast(e == 0 ? cur.en[0] : cur.en[E - 1], l);
+      }
+      const double sc = g.bcast(e == 0 ? cur.scale[0] : cur.scale[E - 1], l);
+      if (g.lane < p.ncol) {
+        const float4 v = rows[t * G + g.lane];
+        acc.x += (double)v.x * sc;
+        acc.y += (double)v.y * sc;
+        acc.z += (double)v.z * sc;
+        acc.w += (double)v.w * sc;
+      }
+    }
+    if (sg >= 0) flush();
+    i += groups;
+    chunk = next;
+    cur = nxt;
+  }
+  pdl_trigger();
+}
+
+// Chunks of kChunk positions holding a position of a long segment, listed
+// for the staged reduction when the dedup listed none (the radix path): only
+// the segments of a chunk's first and last positions can be long (a segment
+// lying wholly inside a chunk is short).  The list's order depends on
+// scheduling; every chunk's partial and every combine do not.
+__global__ void __launch_bounds__(256) list_long_chunks_kernel(const __grid_constant__ UpdateParams p,
+                                                               int32_t* out, BatchDev* bdev) {
+  pdl_wait();
+  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  bool lng = false;
+  if (c < p.nchunks) {
+    const int64_t p0 = c * kChunk, p1 = p0 + kChunk < p.N ? p0 + kChunk : p.N;
+    const int32_t a = __ldg(p.seg_of + p0), b = __ldg(p.seg_of + p1 - 1);
+    lng = __ldg(p.seg_start + a + 1) - __ldg(p.seg_start + a) > kShortSeg ||
+          __ldg(p.seg_start + b + 1) - __ldg(p.seg_start + b) > kShortSeg;
+  }
+  const unsigned bal = __ballot_sync(0xffffffffu, lng);
+  const int lane = threadIdx.x & 31;
+  unsigned at = 0;
+  if (lane == 0 && bal) at = atomicAdd(&bdev->nlong, (unsigned)__popc(bal));
+  at = __shfl_sync(0xffffffffu, at, 0);
+  if (lng) out[at + __popc(bal & ((1u << lane) - 1u))] = (int32_t)c;
+  pdl_trigger();
+}
+
 // ------------------------------------------------------------------ row_update
 // Row data of one unique key: emb and the optimiser state, VPL 16-byte
 // columns per lane.
@@ -514,7 +665,28 @@ int64_t update_chunk_for(int64_t, int) { return kChunk; }
 
 template <int G, int VPL, bool GP, bool GU>
 static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t ucap, cudaStream_t s) {
-  {
+  if constexpr (VPL == 1 && G >= 8 && GP != GU) {
+    if (p.long_chunks) {
+      constexpr size_t smem = (size_t)256 * kChunk * sizeof(float4);  // one slot per position and lane
+      static bool attr[64] = {false};
+      int dev = 0;
+      cudaGetDevice(&dev);
+      if (dev < 0 || dev >= 64 || !attr[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(seg_reduce_staged_kernel<G, GP>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr[dev] = true;
+      }
+      // one group per chunk (the list holds at most nchunks; groups past its
+      // length return at once): many groups in flight hide the combines'
+      // fences and ticket round trips
+      LaunchScope ls("seg_reduce", s);
+      const int64_t blocks = (p.nchunks * G + 255) / 256;
+      const cudaError_t e = launch_pdl(seg_reduce_staged_kernel<G, GP>, (unsigned)(blocks < 1 ? 1 : blocks), 256,
+                                       smem, s, p);
+      if (e != cudaSuccess) return e;
+    }
+  } else {
     int64_t blocks = (p.nchunks * G + 255) / 256;
     if (p.long_chunks && blocks > kSegReduceCtas<VPL> * kSMs) blocks = kSegReduceCtas<VPL> * kSMs;
     if (blocks < 1) blocks = 1;
@@ -596,6 +768,15 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.omb2 = (float)(1.0 - t->cfg.beta2);
   p.inv_sqrt_bc2 = inv_sqrt_bc2;
   if (p.N == 0) return cudaSuccess;
+  if (!p.long_chunks) {
+    // the radix-path dedup lists no chunks: list those holding a long segment
+    cudaError_t e = cudaMemsetAsync(&b->bdev->nlong, 0, sizeof(unsigned), s);
+    if (e != cudaSuccess) return e;
+    LaunchScope ls("list_long", s);
+    list_long_chunks_kernel<<<(unsigned)((p.nchunks + 255) / 256), 256, 0, s>>>(p, b->long_chunks, b->bdev);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    p.long_chunks = b->long_chunks;
+  }
   const bool adam = t->cfg.optimizer == RECIS_ADAM;
   const int64_t ucap = b->N;  // U <= N; groups past U return at once
   const int ncol = p.ncol;

@@ -32,7 +32,7 @@ EXPORTS = (
     "recis_table_import", "recis_table_status_sync", "recis_batch_get_unique",
     "recis_profile_enable", "recis_profile_collect", "recis_launch_count",
     "recis_last_error_string", "recis_unique_static", "recis_table_read_rows",
-    "recis_debug_set", "recis_plan_tables",
+    "recis_debug_set", "recis_plan_tables", "recis_table_reserve",
 )
 DEBUG_SPIN_LIMIT, DEBUG_MAP_LIMIT = 1, 2
 
@@ -115,6 +115,7 @@ def load(path: str = LIB_PATH):
             "recis_table_read_rows": [_vp, _vp, _i64, _vp, _vp, _vp, _vp],
             "recis_debug_set": [_i32, _i64],
             "recis_plan_tables": [_vp, _i32, _vp, _vp, _vp, _vp, _vp],
+            "recis_table_reserve": [_vp, _i64, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -275,6 +276,10 @@ class Table:
                                          keys.numel(), _dev(rows_out, torch.int64),
                                          _stream(stream)), "recis_table_insert")
         return rows_out
+
+    def reserve(self, rows: int, stream=None):
+        """recis_table_reserve: room for `rows` live rows in total, mapped now."""
+        _check(load().recis_table_reserve(self.handle, rows, _stream(stream)), "recis_table_reserve")
 
     def size(self, stream=None):
         n, st = ctypes.c_int64(), ctypes.c_int64()
