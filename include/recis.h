@@ -112,7 +112,26 @@ typedef struct {
   int64_t initial_capacity;  /* expected live keys; the IDMap starts at >= 2x this */
   int64_t block_rows;        /* rows per EmbeddingBlock (growth unit); 0 = 65536 */
   int64_t max_rows;          /* upper bound on live rows (address space reserved); 0 = 2^28 */
+  int32_t admit_threshold;   /* admission: lookups a new key must appear in before it gets a
+                                row (0 or 1: at once; at most 65535) */
+  int32_t evictable;         /* 1: keep each row's last-lookup clock for recis_table_evict */
+  int32_t placement;         /* RECIS_PLACE_* flags: where the table's memory lives (0: all in HBM) */
+  int32_t reserved_;
 } recis_table_config;
+
+/* Placement (README, Key optimisations > Efficient dynamic embedding: the
+ * IDMap and the EmbeddingBlocks can be kept in GPU or in CPU memory).
+ *   RECIS_PLACE_BLOCKS_HOST: EmbeddingBlocks (rows, row keys, last-lookup
+ *     clocks) are allocated in host memory of the GPU's NUMA node and mapped
+ *     into the same contiguous virtual range, so kernels reach them over the
+ *     host link with no change; tables beyond HBM fit, at host-link speed.
+ *     Needs the driver's host-NUMA support for virtual-memory mappings.
+ *   RECIS_PLACE_IDMAP_HOST: the IDMap slot array is mapped pinned host
+ *     memory.  Needs native GPU atomics on host memory (the insert is a CAS).
+ * A placement the system cannot provide gives RECIS_ERR_INVALID_ARG at
+ * create, with the reason in recis_last_error_string(). */
+#define RECIS_PLACE_BLOCKS_HOST 1
+#define RECIS_PLACE_IDMAP_HOST 2
 
 typedef struct recis_table* recis_table_t;
 typedef struct recis_batch* recis_batch_t;
@@ -143,6 +162,27 @@ recis_status recis_plan_tables(const recis_feature_spec* feats, int32_t F,
                                int32_t* table_of_feature, uint64_t* tag_of_feature,
                                int32_t* tag_shift_of_feature, recis_table_config* tables_out,
                                int32_t* n_tables_out);
+
+/* Admission and eviction (README, Core architecture > Embedding Engine: the
+ * table supports feature eviction and admission policies; the README names no
+ * policy, so these are the readings):
+ *   - Admission: a key not in the table is a candidate.  Each lookup it appears
+ *     in (however often) raises its count by one; the lookup that brings the
+ *     count to admit_threshold gives it a row (new rows in ascending key order,
+ *     as always).  Until then its occurrences pool as zero vectors (MEAN still
+ *     divides by the whole bag length), its unpooled rows are zeros, its
+ *     gradient is dropped, and recis_batch_get_unique reports row -1 for it.
+ *     Candidates live in IDMap slots only; they use no EmbeddingBlock row.
+ *   - Clock: every lookup or insert that launches work advances the table's
+ *     clock by one; an evictable table records in each row (and each
+ *     candidate) the clock of the last lookup that touched it.
+ *   - Eviction: recis_table_evict removes every row and candidate last touched
+ *     before a given clock.  An evicted key keeps its IDMap slot as a
+ *     tombstone (so no probe chain is cut) until an IDMap growth drops it; if
+ *     it comes back it starts over as a new candidate with an initial row.
+ *     Freed rows (key -1) join a queue in ascending row order; later new keys
+ *     take them, oldest first, before rows past the end.  Exports, saves and
+ *     recis_table_size count live rows only. */
 
 /* Create a table on the current device (README, Efficient dynamic embedding:
  * IDMap + EmbeddingBlocks).  Rows are [emb D][state s*D] fp32 (s = 1 Adagrad,
@@ -196,8 +236,9 @@ recis_status recis_lookup_pooled(recis_table_t t, recis_batch_t b, const int64_t
 recis_status recis_backward_update(recis_table_t t, recis_batch_t b, const float* grad_pooled,
                                    const float* grad_unpooled, recis_stream_t stream);
 
-/* Find-or-insert only (no pooling): used to pre-load a table.  keys: device
- * int64[N].  rows_out: device int64[N] (row of each key) or NULL. */
+/* Find-or-insert only (no pooling): used to pre-load a table; its keys are
+ * admitted at once whatever the admission threshold.  keys: device int64[N].
+ * rows_out: device int64[N] (row of each key) or NULL. */
 recis_status recis_table_insert(recis_table_t t, recis_batch_t b, const int64_t* keys, int64_t N,
                                 int64_t* rows_out, recis_stream_t stream);
 
@@ -206,7 +247,9 @@ recis_status recis_table_insert(recis_table_t t, recis_batch_t b, const int64_t*
  * (device int64[n]) writes its key to keys_out[i] (device int64[n] or NULL),
  * its emb to emb_out[i][0..D) (device fp32 [n][D] or NULL) and its optimiser
  * state to state_out[i][0..s*D) (device fp32 [n][s*D] or NULL; Adam: m then
- * v).  A row offset outside [0, live rows) gives key -1 and zeros.  Waits for
+ * v).  A row offset outside [0, rows in use) gives key -1 and zeros; a row
+ * freed by eviction and not yet reused gives key -1 (its values are left
+ * over from its last key).  Waits for
  * `stream` to learn the live row count, then gathers asynchronously on it. */
 recis_status recis_table_read_rows(recis_table_t t, const int64_t* rows, int64_t n,
                                    int64_t* keys_out, float* emb_out, float* state_out,
@@ -221,6 +264,16 @@ recis_status recis_table_read_rows(recis_table_t t, const int64_t* rows, int64_t
  * any pending device-detected error.  rows > max_rows: RECIS_ERR_TABLE_FULL. */
 recis_status recis_table_reserve(recis_table_t t, int64_t rows, recis_stream_t stream);
 
+/* Synchronous (README, Core architecture > Embedding Engine: feature eviction).
+ * Evicts every row and candidate whose last lookup clock is below min_clock
+ * (rows touched by the lookups numbered min_clock and later stay); *n_evicted
+ * (may be NULL) receives the number of rows freed.  The table must have been
+ * created with evictable = 1 (else RECIS_ERR_INVALID_ARG).  *clock_out of
+ * recis_table_clock is the number of lookups so far. */
+recis_status recis_table_evict(recis_table_t t, int64_t min_clock, int64_t* n_evicted,
+                               recis_stream_t stream);
+recis_status recis_table_clock(recis_table_t t, int64_t* clock_out);
+
 /* Synchronous.  Number of live rows and the Adam step counter. */
 recis_status recis_table_size(recis_table_t t, int64_t* n_out, int64_t* step_out,
                               recis_stream_t stream);
@@ -233,6 +286,24 @@ recis_status recis_table_size(recis_table_t t, int64_t* n_out, int64_t* step_out
 recis_status recis_table_export(recis_table_t t, int64_t* keys, float* emb, float* state,
                                 int64_t capacity, int64_t* n_out, int64_t* step_out,
                                 recis_stream_t stream);
+
+/* Synchronous (README, Core architecture > Saver: sparse parameters stored and
+ * delivered in the SafeTensors standard format).  Writes the table to the file
+ * `path` in the SafeTensors format: tensors "keys" (I64 [n]), "emb" (F32 [n, D])
+ * and the optimiser state, "accum" (Adagrad) or "adam_m" and "adam_v" (Adam),
+ * each F32 [n, D], rows in ascending row order; metadata "format" =
+ * "recis-embedding-table", "dim", "optimizer", "step", "rows", "lr", "beta1",
+ * "beta2", "eps", "adagrad_init_acc", "init_scale", "init_seed" (strings).  The
+ * rows stream through host memory in chunks of about 64 MB.  An unwritable path
+ * gives RECIS_ERR_INVALID_ARG. */
+recis_status recis_table_save(recis_table_t t, const char* path, recis_stream_t stream);
+/* Synchronous.  Reads a SafeTensors file holding "keys", "emb" and this table's
+ * optimiser-state tensors (as recis_table_save writes them) with dim D and
+ * appends its rows after the live rows, as recis_table_import does (keys must
+ * be new); the metadata "step", when present, becomes the table's step
+ * counter.  A file without those tensors, or with another dim, gives
+ * RECIS_ERR_INVALID_ARG and leaves the table unchanged. */
+recis_status recis_table_load(recis_table_t t, const char* path, recis_stream_t stream);
 
 /* Synchronous.  Appends n rows from HOST buffers after the live rows (keys must
  * not be present; state NULL = initial state) and sets the step counter. */

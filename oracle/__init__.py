@@ -74,6 +74,10 @@ def lib():
                                     ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                     ctypes.c_double, ctypes.c_uint64, ctypes.c_double]
         L.orc_table_free.argtypes = [ctypes.c_void_p]
+        L.orc_table_clock.restype = ctypes.c_int64
+        L.orc_table_clock.argtypes = [ctypes.c_void_p]
+        L.orc_table_set_admission.argtypes = [ctypes.c_void_p, ctypes.c_int32]
+        L.orc_table_evict.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
         L.orc_lookup.restype = ctypes.c_int
         L.orc_lookup.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64,
                                  ctypes.POINTER(ctypes.c_int64), ctypes.c_int32, ctypes.c_int64,
@@ -163,7 +167,7 @@ class Table:
     def __init__(self, dim: int, optimizer: int, lr: float, beta1: float = 0.9,
                  beta2: float = 0.999, eps: Optional[float] = None,
                  adagrad_init_acc: float = 0.0, init_seed: int = 0,
-                 init_scale: Optional[float] = None):
+                 init_scale: Optional[float] = None, admit_threshold: int = 0):
         if eps is None:
             eps = 1e-10 if optimizer == ADAGRAD else 1e-8
         if init_scale is None:
@@ -174,6 +178,8 @@ class Table:
                                       ctypes.c_uint64(init_seed & (2**64 - 1)), init_scale)
         if not self._h:
             raise OracleError(INVALID_ARG, "table_new")
+        if admit_threshold:
+            lib().orc_table_set_admission(self._h, admit_threshold)
 
     def __del__(self):
         h = getattr(self, "_h", None)
@@ -222,6 +228,18 @@ class Table:
     @property
     def step(self) -> int:
         return int(lib().orc_table_step(self._h))
+
+    @property
+    def clock(self) -> int:
+        return int(lib().orc_table_clock(self._h))
+
+    def evict(self, min_clock: int) -> int:
+        """Remove rows and candidates last touched before lookup `min_clock`."""
+        n = ctypes.c_int64(0)
+        rc = lib().orc_table_evict(self._h, ctypes.c_int64(min_clock), ctypes.byref(n))
+        if rc != OK:
+            raise OracleError(rc, "evict")
+        return n.value
 
     def export(self):
         n, D = self.size, self.dim

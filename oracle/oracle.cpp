@@ -45,6 +45,20 @@ struct orc_table {
   // First level: IDMap, feature ID -> row offset (README, Key optimisations,
   // "Efficient dynamic embedding", IDMap bullet).
   std::unordered_map<int64_t, int64_t> idmap;
+  // Admission and eviction (README, Core architecture > Embedding Engine: the
+  // table supports feature eviction and admission policies).  Reading: a key
+  // not in the IDMap is a candidate whose count rises by one per lookup it
+  // appears in; it gets a row on the lookup where the count reaches
+  // admit_threshold (<= 1: at once).  Every lookup advances the clock; a row
+  // (or a candidate) remembers the clock of the last lookup that touched it,
+  // and eviction removes those last touched before a given clock.  Freed rows
+  // queue in ascending row order and are handed to new keys first.
+  int32_t admit_threshold = 1;
+  int64_t clock = 0;
+  std::unordered_map<int64_t, std::pair<int64_t, int64_t>> cand;  // key -> (count, last clock)
+  std::vector<int64_t> last_seen;                                  // per row
+  std::vector<int64_t> free_rows;                                  // queue of freed rows
+  size_t free_head = 0;
   // Second level: rows of [emb D][state s*D] fp32 in row order
   // (same section, EmbeddingBlocks bullet: parameters and optimiser state kept
   // together).  One flat vector stands for the chunked blocks.
@@ -151,13 +165,28 @@ static void init_row(orc_table* t, int64_t key, int64_t row) {
   }
 }
 
+// A new row at the end of the table.
 static int64_t add_row(orc_table* t, int64_t key) {
   const int64_t row = (int64_t)t->row_key.size();
   t->row_key.push_back(key);
   t->emb.resize((size_t)(row + 1) * t->D);
   t->state.resize((size_t)(row + 1) * t->s * t->D);
+  t->last_seen.push_back(t->clock);
   t->idmap.emplace(key, row);
   return row;
+}
+
+// The row of a key admitted by a lookup: the oldest freed row if any, else a
+// new one at the end.
+static int64_t take_row(orc_table* t, int64_t key) {
+  if (t->free_head < t->free_rows.size()) {
+    const int64_t row = t->free_rows[t->free_head++];
+    t->row_key[row] = key;
+    t->last_seen[row] = t->clock;
+    t->idmap.emplace(key, row);
+    return row;
+  }
+  return add_row(t, key);
 }
 
 // Forward.  Steps, in order:
@@ -184,6 +213,7 @@ extern "C" int orc_lookup(orc_table* t, const int64_t* keys, int64_t N, const in
   } else if (N != 0) {
     return ORC_INVALID_ARG;
   }
+  t->clock += 1;  // every accepted call advances the clock, even one rejected below
   for (int64_t i = 0; i < N; ++i)
     if (keys[i] == kReserved) return ORC_RESERVED_KEY;
 
@@ -203,10 +233,20 @@ extern "C" int orc_lookup(orc_table* t, const int64_t* keys, int64_t N, const in
     auto it = t->idmap.find(uniq[j]);
     if (it != t->idmap.end()) {
       rows[j] = it->second;
-    } else {
-      rows[j] = add_row(t, uniq[j]);
+      t->last_seen[rows[j]] = t->clock;
+      continue;
+    }
+    // a candidate: admitted when this lookup brings its count to the threshold
+    auto c = t->cand.find(uniq[j]);
+    const int64_t count = (c == t->cand.end() ? 0 : c->second.first) + 1;
+    if (count >= t->admit_threshold) {
+      if (c != t->cand.end()) t->cand.erase(c);
+      rows[j] = take_row(t, uniq[j]);
       init_row(t, uniq[j], rows[j]);
       ++n_new;
+    } else {
+      t->cand[uniq[j]] = std::make_pair(count, t->clock);
+      rows[j] = -1;  // no row yet: pooled as zeros, gradient dropped
     }
   }
 
@@ -220,6 +260,7 @@ extern "C" int orc_lookup(orc_table* t, const int64_t* keys, int64_t N, const in
         std::fill(acc.begin(), acc.end(), 0.0);
         const int64_t lo = bag_offsets[bag], hi = bag_offsets[bag + 1];
         for (int64_t i = lo; i < hi; ++i) {
+          if (rows[inv[i]] < 0) continue;  // a candidate's occurrence adds zeros
           const float* e = &t->emb[(size_t)rows[inv[i]] * D];
           for (int j = 0; j < D; ++j) acc[j] += (double)e[j];
         }
@@ -235,6 +276,10 @@ extern "C" int orc_lookup(orc_table* t, const int64_t* keys, int64_t N, const in
   }
   if (unpooled_out) {
     for (int64_t i = 0; i < N; ++i) {
+      if (rows[inv[i]] < 0) {
+        std::memset(unpooled_out + (size_t)i * D, 0, sizeof(float) * D);
+        continue;
+      }
       const float* e = &t->emb[(size_t)rows[inv[i]] * D];
       std::memcpy(unpooled_out + (size_t)i * D, e, sizeof(float) * D);
     }
@@ -308,6 +353,7 @@ extern "C" int orc_backward_update(orc_table* t, const float* grad_pooled,
   const double bc2 = 1.0 - std::pow(t->beta2, (double)t->step);
   for (int64_t u = 0; u < U; ++u) {
     const int64_t row = t->rows[u];
+    if (row < 0) continue;  // a candidate without a row: its gradient is dropped
     float* w = &t->emb[(size_t)row * D];
     float* st = &t->state[(size_t)row * t->s * D];
     const double* gu = &g[(size_t)u * D];
@@ -332,15 +378,50 @@ extern "C" int orc_backward_update(orc_table* t, const float* grad_pooled,
   return ORC_OK;
 }
 
-extern "C" int64_t orc_table_size(const orc_table* t) { return (int64_t)t->row_key.size(); }
+// live rows: every row that holds a key (freed rows hold -1)
+extern "C" int64_t orc_table_size(const orc_table* t) {
+  return (int64_t)t->row_key.size() - (int64_t)(t->free_rows.size() - t->free_head);
+}
 extern "C" int64_t orc_table_step(const orc_table* t) { return t->step; }
+extern "C" int64_t orc_table_clock(const orc_table* t) { return t->clock; }
 
+// the live rows in ascending row order (freed rows left out)
 extern "C" int orc_table_export(const orc_table* t, int64_t* keys, float* emb, float* state) {
-  const int64_t n = (int64_t)t->row_key.size();
-  if (keys) std::copy(t->row_key.begin(), t->row_key.end(), keys);
-  if (emb) std::copy(t->emb.begin(), t->emb.end(), emb);
-  if (state) std::copy(t->state.begin(), t->state.end(), state);
-  (void)n;
+  const int D = t->D, SD = t->s * t->D;
+  int64_t k = 0;
+  for (size_t row = 0; row < t->row_key.size(); ++row) {
+    if (t->row_key[row] == kReserved) continue;
+    if (keys) keys[k] = t->row_key[row];
+    if (emb) std::copy(&t->emb[row * D], &t->emb[row * D] + D, emb + (size_t)k * D);
+    if (state) std::copy(&t->state[row * SD], &t->state[row * SD] + SD, state + (size_t)k * SD);
+    ++k;
+  }
+  return ORC_OK;
+}
+
+extern "C" int orc_table_set_admission(orc_table* t, int32_t threshold) {
+  if (!t || threshold < 0) return ORC_INVALID_ARG;
+  t->admit_threshold = threshold < 1 ? 1 : threshold;
+  return ORC_OK;
+}
+
+// Eviction: every row, and every candidate, whose last lookup came before
+// min_clock is removed; the freed rows join the queue in ascending row order.
+extern "C" int orc_table_evict(orc_table* t, int64_t min_clock, int64_t* n_evicted) {
+  if (!t) return ORC_INVALID_ARG;
+  int64_t n = 0;
+  for (size_t row = 0; row < t->row_key.size(); ++row) {
+    if (t->row_key[row] == kReserved || t->last_seen[row] >= min_clock) continue;
+    t->idmap.erase(t->row_key[row]);
+    t->row_key[row] = kReserved;
+    t->free_rows.push_back((int64_t)row);
+    ++n;
+  }
+  for (auto it = t->cand.begin(); it != t->cand.end();) {
+    if (it->second.second < min_clock) it = t->cand.erase(it);
+    else ++it;
+  }
+  if (n_evicted) *n_evicted = n;
   return ORC_OK;
 }
 
@@ -350,6 +431,7 @@ extern "C" int orc_table_import(orc_table* t, int64_t n, const int64_t* keys, co
     if (keys[i] == kReserved || t->idmap.count(keys[i])) return ORC_INVALID_ARG;
   const int D = t->D;
   for (int64_t i = 0; i < n; ++i) {
+    t->cand.erase(keys[i]);  // an imported key is admitted
     const int64_t row = add_row(t, keys[i]);
     init_row(t, keys[i], row);  // default state when none is given
     std::memcpy(&t->emb[(size_t)row * D], emb + (size_t)i * D, sizeof(float) * D);

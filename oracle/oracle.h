@@ -80,9 +80,18 @@ int orc_lookup(orc_table* t, const int64_t* keys, int64_t N, const int64_t* bag_
 int orc_backward_update(orc_table* t, const float* grad_pooled, const float* grad_unpooled,
                         double* grad_u_out);
 
+/* live rows (rows freed by eviction excluded) */
 int64_t orc_table_size(const orc_table* t);
 int64_t orc_table_step(const orc_table* t);
-/* rows in ascending row order; state is [n][s*D] (s = 1 Adagrad, 2 Adam: m then v) */
+/* lookups so far (the clock eviction compares against) */
+int64_t orc_table_clock(const orc_table* t);
+/* admission: a key gets a row on the lookup that brings its count of lookups
+ * seen in to `threshold` (0 or 1: at once) */
+int orc_table_set_admission(orc_table* t, int32_t threshold);
+/* eviction: rows and candidates last touched by a lookup before min_clock are
+ * removed; freed rows are reused by later keys, oldest first */
+int orc_table_evict(orc_table* t, int64_t min_clock, int64_t* n_evicted);
+/* live rows in ascending row order; state is [n][s*D] (s = 1 Adagrad, 2 Adam: m then v) */
 int orc_table_export(const orc_table* t, int64_t* keys, float* emb, float* state);
 /* append rows (key, emb, state) after the live rows; keys must be new */
 int orc_table_import(orc_table* t, int64_t n, const int64_t* keys, const float* emb,

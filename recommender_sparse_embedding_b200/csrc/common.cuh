@@ -1,5 +1,6 @@
 // common.cuh -- device-side helpers shared by the kernels of the embedding engine.
 #pragma once
+#include <climits>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -39,14 +40,43 @@ constexpr uint64_t kSlotSalt = 0x2545F4914F6CDD1DULL;
 
 struct __align__(16) Slot {
   int64_t key;  // kEmptyKey when free
-  int64_t row;
+  int64_t row;  // see the row states below
 };
+
+// Row field of a slot whose key is set (admission and eviction: RecIS README,
+// Core architecture > Embedding Engine, feature eviction and admission):
+//   >= 0          the key's row;
+//   -1            claimed by the running call, no row yet;
+//   kTombRow      the key was evicted: it keeps its slot (so no other key's
+//                 probe chain is cut) and has no row; if it comes back it
+//                 takes this slot again;
+//   kReclaimRow   an evicted key's slot taken again by the running call;
+//   candidate     a key seen by earlier lookups but not admitted yet:
+//                 -2 - (clock << 16 | count), count = lookups it appeared in
+//                 (1 .. 65535), clock = the last of them (< 2^40).
+constexpr int64_t kTombRow = INT64_MIN;
+constexpr int64_t kReclaimRow = INT64_MIN + 1;
+constexpr int kMaxAdmitThreshold = 65535;
+__host__ __device__ __forceinline__ bool is_cand_row(int64_t r) { return r <= -2 && r > kReclaimRow; }
+__host__ __device__ __forceinline__ int cand_count(int64_t r) { return (int)((-2 - r) & 0xffff); }
+__host__ __device__ __forceinline__ uint64_t cand_clock(int64_t r) { return (uint64_t)(-2 - r) >> 16; }
+__host__ __device__ __forceinline__ int64_t cand_row(uint64_t clock, int count) {
+  return -2 - (int64_t)((clock << 16) | (uint64_t)(count < 0xffff ? count : 0xffff));
+}
+// lookups the key had appeared in before the running call, from its row field
+__host__ __device__ __forceinline__ int prior_count(int64_t r) { return is_cand_row(r) ? cand_count(r) : 0; }
+// last-lookup clock of a row freed by an eviction that has not yet joined
+// the free-row queue
+constexpr uint32_t kFreedMark = 0xffffffffu;
 
 // Table-wide device state.
 struct DevState {
-  unsigned long long next_free;  // number of live rows
-  int status;                    // OR of error bits
+  unsigned long long next_free;   // rows in use: live rows and freed rows below it
+  int status;                     // OR of error bits
   int pad;
+  unsigned long long slots_used;  // IDMap slots holding a key (tombstones included)
+  unsigned long long free_head;   // freed rows not yet reused: queue [free_head, free_tail)
+  unsigned long long free_tail;
 };
 
 // Host-mapped mirror: written by kernels so the host can read progress and
@@ -55,7 +85,73 @@ struct HostMirror {
   volatile unsigned long long next_free;
   volatile int error_seen;
   volatile int pad;
+  volatile unsigned long long slots_used;
 };
+
+// Result of an IDMap probe for one key.
+struct Probe {
+  int64_t row;   // the key's row (>= 0), or -1 when it has none
+  int64_t slot;  // its slot when it has no row (claimed, candidate or reclaimed); -1 otherwise
+  int prior;     // lookups it appeared in before this call (candidates; 0 otherwise)
+  bool limit;    // the probe limit was reached (the IDMap is too full)
+};
+
+constexpr int kProbeLimit = 1 << 16;
+
+// IDMap find-or-insert with admission: linear probing from slot h (sv = the
+// slot already loaded there).  A key found with a row returns it; a key
+// without one (claimed by this call, a candidate, or evicted -- an evicted
+// key's slot is reclaimed for it) returns its slot and its prior count; a
+// missing key claims the first free slot by a 64-bit CAS on its key (each
+// claim adds one to *claims).  With insert false nothing is claimed and a
+// missing or evicted key returns row -1 and slot -1.
+__device__ __forceinline__ Probe idmap_probe(Slot* slots, uint64_t mask, int64_t key, uint64_t h,
+                                             longlong2 sv, bool insert, unsigned* claims) {
+  const int64_t limit = (int64_t)mask + 1 < kProbeLimit ? (int64_t)mask + 1 : kProbeLimit;
+  for (int64_t n = 0; n < limit; ++n) {
+    if (n > 0) sv = __ldcg(reinterpret_cast<const longlong2*>(slots + h));
+    bool mine = sv.x == key;
+    if (!mine && sv.x == kEmptyKey) {
+      if (!insert) return Probe{-1, -1, 0, false};
+      const unsigned long long old = atomicCAS(reinterpret_cast<unsigned long long*>(&slots[h].key),
+                                               (unsigned long long)kEmptyKey, (unsigned long long)key);
+      if ((int64_t)old == kEmptyKey) {
+        atomicAdd(claims, 1u);
+        return Probe{-1, (int64_t)h, 0, false};
+      }
+      mine = (int64_t)old == key;
+    }
+    if (mine) {
+      const int64_t r = sv.x == key && sv.y >= 0 ? sv.y : __ldcg(&slots[h].row);
+      if (r >= 0) return Probe{r, -1, 0, false};
+      if (r == kTombRow || r == kReclaimRow) {
+        if (!insert) return Probe{-1, -1, 0, false};
+        if (r == kTombRow)
+          atomicCAS(reinterpret_cast<unsigned long long*>(&slots[h].row), (unsigned long long)kTombRow,
+                    (unsigned long long)kReclaimRow);
+        return Probe{-1, (int64_t)h, 0, false};
+      }
+      return Probe{-1, (int64_t)h, prior_count(r), false};  // claimed by this call (-1) or a candidate
+    }
+    h = (h + 1) & mask;
+  }
+  return Probe{-1, -1, 0, true};
+}
+
+// Gives back a slot the running call took for a key it then did not keep (a
+// rejected call): a fresh claim empties it again (returns 1, one slot less in
+// use), a reclaimed evicted key's slot becomes a tombstone again; a
+// candidate's slot keeps its state.  Every key claimed by the call is newer
+// than every key that stays, so emptying its slot cuts no probe chain.
+__device__ __forceinline__ unsigned idmap_give_back(Slot* slots, int64_t slot) {
+  const int64_t r = __ldcg(&slots[slot].row);
+  if (r == -1) {
+    slots[slot].key = kEmptyKey;
+    return 1u;
+  }
+  if (r == kReclaimRow) slots[slot].row = kTombRow;
+  return 0u;
+}
 
 __device__ __forceinline__ void raise_error(DevState* st, HostMirror* mirror, int bit) {
   atomicOr(&st->status, bit);

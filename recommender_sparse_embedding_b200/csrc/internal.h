@@ -64,6 +64,8 @@ constexpr int64_t kSampleSortMaxN = (int64_t)1600 * 1000;  // larger batches use
 // Per-batch device scalars.
 struct BatchDev {
   unsigned long long row_base;  // table's next_free when the lookup started
+  unsigned long long free_base; // table's free_head when the lookup started
+  unsigned long long free_avail;// freed rows queued then (free_tail - free_head)
   unsigned int U;               // unique keys of the last lookup (0 when it was rejected)
   unsigned int n_new;           // new keys of the last lookup
   unsigned int nlong;           // chunks of kShortSeg positions holding a long segment
@@ -78,6 +80,7 @@ struct VmmArray {
   CUdeviceptr va = 0;
   size_t reserved = 0;   // bytes of address space
   size_t mapped = 0;     // bytes backed by physical blocks
+  int host_numa = -1;    // >= 0: blocks are host memory of this NUMA node
   std::vector<CUmemGenericAllocationHandle> handles;
   std::vector<size_t> sizes;
 };
@@ -95,8 +98,14 @@ struct recis_table {
   int64_t max_rows = 0;
   int64_t mapped_rows = 0;
   recis::VmmArray rows;         // [row][emb D | state s*D] fp32
-  recis::VmmArray keys;         // [row] int64, key of each row
-  recis::Slot* slots = nullptr; // IDMap
+  recis::VmmArray keys;         // [row] int64, key of each row (-1: freed)
+  recis::VmmArray seen;         // [row] uint32, clock of the last lookup that touched it (evictable tables)
+  int32_t* free_rows = nullptr; // queue of freed rows (DevState free_head .. free_tail)
+  int64_t free_cap = 0;         // entries of free_rows
+  int64_t clock = 0;            // lookups so far
+  int64_t slots_upper = 0;      // upper bound on IDMap slots holding a key
+  recis::Slot* slots = nullptr; // IDMap (device address; mapped pinned host memory with PLACE_IDMAP_HOST)
+  recis::Slot* slots_host = nullptr;  // host address of a host-placed IDMap
   int64_t capacity = 0;         // slots, power of two
   recis::DevState* dstate = nullptr;
   recis::HostMirror* mirror = nullptr;  // host-mapped
@@ -227,7 +236,7 @@ struct LookupArgs {
 
 cudaError_t launch_sort(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
                         cudaStream_t s);
-cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cudaStream_t s);
+cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, bool insert, cudaStream_t s);
 cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* keys, int64_t N,
                                 bool insert, cudaStream_t s);
 int samplesort_splits_for(int64_t N);
@@ -239,7 +248,8 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
                           const float* grad_unpooled, int64_t chunk, float lr_t, float inv_sqrt_bc2,
                           cudaStream_t s);
 cudaError_t launch_import(recis_table* t, const int64_t* keys, int64_t n, int64_t row0,
-                          cudaStream_t s);
+                          int64_t clock, cudaStream_t s);
+recis_status table_counts(recis_table* t, cudaStream_t s, int64_t* in_use, int64_t* live);
 cudaError_t launch_rehash(recis_table* t, const Slot* old_slots, int64_t old_cap, cudaStream_t s);
 
 int64_t pool_chunk_for(int64_t N, int D);

@@ -56,8 +56,8 @@ extern "C" recis_status recis_table_read_rows(recis_table_t t, const int64_t* ro
   cudaStream_t s = (cudaStream_t)stream;
   // rows at or past the live count read as key -1 and zeros; the live count
   // is exact once the table's earlier work has finished
-  int64_t live = 0;
-  recis_status st = recis_table_size(t, &live, nullptr, stream);
+  int64_t live = 0;  // rows in use (a freed row reads as key -1)
+  recis_status st = table_counts(t, s, &live, nullptr);
   if (st != RECIS_OK) return st;
   const int64_t total = n * (t->row_floats / 4);
   int64_t blocks = (total + 255) / 256;

@@ -58,10 +58,13 @@ constexpr int kFinItems = 2;
 constexpr int kSub = kFinThreads * kFinItems;       // sorted positions per finish CTA
 constexpr int kMaxProbes = 1 << 16;
 
-// IDMap probe result of a head: row >= 0 for a key already present; -2 - slot
-// for a new key whose slot this call claimed; -1 when there is no row
-// (reserved key, or the IDMap was exhausted).
-__device__ __forceinline__ int64_t encode_new(int64_t slot) { return -2 - slot; }
+// IDMap result of an occurrence (from the probe kernel): the key's row
+// (>= 0); -2 - slot for a key without a row that this call admits (new: it
+// gets a row); kCandPocc - slot for one that stays a candidate; -1 when there
+// is no row and no slot (reserved key, or the IDMap was exhausted).
+constexpr int64_t kCandPocc = -((int64_t)1 << 40) - 2;
+__device__ __forceinline__ bool pocc_new(int64_t v) { return v <= -2 && v > kCandPocc; }
+__device__ __forceinline__ bool pocc_cand(int64_t v) { return v <= kCandPocc; }
 
 // bucket of ukey u: 2r + [u == split[r]], r = number of splitters < u
 __device__ __forceinline__ unsigned bucket_of(const uint64_t* split, int nsplit, uint64_t u) {
@@ -209,35 +212,6 @@ __device__ void reg_sort(uint64_t (&k)[E], uint32_t (&x)[E], uint64_t* sk, uint3
   __syncthreads();
 }
 
-// IDMap find-or-insert: linear probing from slot h = H(key ^ salt); a free
-// slot is claimed by a 64-bit CAS on its key.  Returns the row of a key
-// already present, -2 - slot for a key claimed in this call (its row is -1
-// until the call assigns it, whichever occurrence claimed it), or -1 when
-// the probe limit was reached.
-__device__ __forceinline__ int64_t idmap_resolve(Slot* slots, uint64_t mask, int64_t key, uint64_t h,
-                                                 longlong2 sv) {
-  const int64_t limit = (int64_t)mask + 1 < kMaxProbes ? (int64_t)mask + 1 : kMaxProbes;
-  for (int64_t n = 0; n < limit; ++n) {
-    if (n > 0) sv = __ldcg(reinterpret_cast<const longlong2*>(slots + h));
-    if (sv.x == key) {
-      const int64_t row = sv.y >= 0 ? sv.y : __ldcg(&slots[h].row);
-      return row >= 0 ? row : encode_new((int64_t)h);
-    }
-    if (sv.x == kEmptyKey) {
-      const unsigned long long old = atomicCAS(reinterpret_cast<unsigned long long*>(&slots[h].key),
-                                               (unsigned long long)kEmptyKey,
-                                               (unsigned long long)key);
-      if ((int64_t)old == kEmptyKey) return encode_new((int64_t)h);
-      if ((int64_t)old == key) {
-        const int64_t row = __ldcg(&slots[h].row);
-        return row >= 0 ? row : encode_new((int64_t)h);
-      }
-    }
-    h = (h + 1) & mask;
-  }
-  return -1;
-}
-
 // exclusive block scan of one value per thread; *total gets the block sum
 template <int NT>
 __device__ __forceinline__ unsigned block_excl_scan(unsigned x, unsigned* s_warp, unsigned* total) {
@@ -335,7 +309,17 @@ struct SsParams {
   DevState* st;
   HostMirror* mirror;
   uint32_t call_id;         // this lookup's number on the batch (BatchDev::reject_call)
+  int admit;                // admission threshold (>= 1)
+  uint64_t clock;           // this lookup's clock
+  uint32_t* seen;           // [row] clock of the last lookup that touched the row, or null
+  const int32_t* free_rows; // queue of freed rows (bdev->free_base .. + free_avail)
 };
+
+// New rows a call takes past the table's end: its new keys beyond the freed
+// rows it reuses.
+__device__ __forceinline__ unsigned long long fresh_rows(unsigned long long nnew, unsigned long long avail) {
+  return nnew > avail ? nnew - avail : 0ULL;
+}
 
 // A lookup is rejected as a whole when one of its keys is the reserved -1
 // (marked by the probe kernel) or when its new keys would not fit the mapped
@@ -344,7 +328,7 @@ struct SsParams {
 __device__ __forceinline__ bool call_rejected(const SsParams& p, unsigned long long tot,
                                               unsigned long long row_base) {
   return __ldcg(&p.bdev->reject_call) == p.call_id ||
-         row_base + (tot >> 32) > (unsigned long long)p.mapped_rows;
+         row_base + fresh_rows(tot >> 32, p.bdev->free_avail) > (unsigned long long)p.mapped_rows;
 }
 
 // Per sorted position, written by ss_local: the bucket, the position's
@@ -437,6 +421,9 @@ __global__ void __launch_bounds__(kCountThreads) ss_count_kernel(const __grid_co
     p.bdev->nlong = 0;
     p.bdev->nmulti = 0;
     p.bdev->row_base = *(volatile unsigned long long*)&p.st->next_free;
+    const unsigned long long fh = *(volatile unsigned long long*)&p.st->free_head;
+    p.bdev->free_base = fh;
+    p.bdev->free_avail = *(volatile unsigned long long*)&p.st->free_tail - fh;
   }
   __syncthreads();
 #pragma unroll
@@ -458,10 +445,16 @@ __global__ void __launch_bounds__(kCountThreads) ss_count_kernel(const __grid_co
 // IDMap find-or-insert of every occurrence (runs on a second stream beside
 // count, tile scan and scatter): two keys per thread, both first slots loaded
 // before either is resolved.  A missing key claims a free slot by CAS; every
-// occurrence of it then sees the slot with row -1 and records -2 - slot.
+// occurrence of a key without a row records its slot and whether this call
+// admits it (the count of lookups it appeared in reaches the threshold).  All
+// occurrences of a key see the same slot state, so they agree.  Claims are
+// counted per CTA and added to the table's slot count once.
 constexpr int kProbeThreads = 256;
 constexpr int kProbeItems = 2;
 __global__ void __launch_bounds__(kProbeThreads) ss_probe_kernel(const __grid_constant__ SsParams p) {
+  __shared__ unsigned s_claims;
+  if (threadIdx.x == 0) s_claims = 0;
+  __syncthreads();
   const int64_t pos0 = (int64_t)blockIdx.x * (kProbeThreads * kProbeItems) + threadIdx.x;
   int64_t k[kProbeItems];
   uint64_t h[kProbeItems];
@@ -482,8 +475,10 @@ __global__ void __launch_bounds__(kProbeThreads) ss_probe_kernel(const __grid_co
     if (k[j] == kEmptyKey) {
       reserved = true;
     } else {
-      r = idmap_resolve(p.slots, p.slot_mask, k[j], h[j], sv[j]);
-      if (r == -1) raise_error(p.st, p.mirror, kErrTableFull);
+      const Probe pr = idmap_probe(p.slots, p.slot_mask, k[j], h[j], sv[j], true, &s_claims);
+      if (pr.limit) raise_error(p.st, p.mirror, kErrTableFull);
+      else if (pr.row >= 0) r = pr.row;
+      else r = pr.prior + 1 >= p.admit ? -2 - pr.slot : kCandPocc - pr.slot;
     }
     p.pocc[pos] = r;
   }
@@ -491,6 +486,8 @@ __global__ void __launch_bounds__(kProbeThreads) ss_probe_kernel(const __grid_co
     p.bdev->reject_call = p.call_id;
     raise_error(p.st, p.mirror, kErrReservedKey);
   }
+  __syncthreads();
+  if (threadIdx.x == 0 && s_claims) atomicAdd(&p.st->slots_used, (unsigned long long)s_claims);
 }
 
 // ------------------------------------------------------------------ tile scan
@@ -664,7 +661,7 @@ __device__ void block_number(const SsParams& p, LocalShared<NT, CAP>& sh, unsign
       occ = in_smem ? sh.idx[i] : __ldcg(p.vb + off + i);
       const uint64_t before = i == 0 ? 0 : (in_smem ? sh.key[i - 1] : __ldcg(p.kb + off + i - 1));
       if (i == 0 || u != before) {
-        f = 1u | (__ldcg(p.pocc + occ) <= -2 ? 2u : 0u);
+        f = 1u | (pocc_new(__ldcg(p.pocc + occ)) ? 2u : 0u);
         const int64_t j = i + kShortSeg;
         lng = j < m && (in_smem ? sh.key[j] : __ldcg(p.kb + off + j)) == u;
       }
@@ -794,10 +791,14 @@ __device__ __forceinline__ void publish_totals(const SsParams& p, unsigned long 
   }
   p.bdev->U = rejected ? 0u : (unsigned)U;
   p.bdev->n_new = (unsigned)nnew;
-  const unsigned long long nf = row_base + nnew;
+  // new keys take the queued freed rows first, then rows past the end
+  const unsigned long long avail = p.bdev->free_avail;
+  const unsigned long long nf = row_base + fresh_rows(nnew, avail);
   p.st->next_free = nf;
+  p.st->free_head = p.bdev->free_base + (nnew < avail ? nnew : avail);
   if (p.mirror) {
     p.mirror->next_free = nf;
+    p.mirror->slots_used = *(volatile unsigned long long*)&p.st->slots_used;
     __threadfence_system();
   }
   p.seg_start[U] = (int32_t)p.N;
@@ -850,7 +851,7 @@ __global__ void __launch_bounds__(NT, NT >= 512 ? 2 : 4) ss_local_kernel(const _
         p.ctl->ncnt[b] = 0;
       }
     } else if (b & 1u) {
-      local_equal(p, b, m, off, __ldcg(p.pocc + __ldcg(p.vb + off)) <= -2, tid, NT);
+      local_equal(p, b, m, off, pocc_new(__ldcg(p.pocc + __ldcg(p.vb + off))), tid, NT);
     } else {
       local_range_block<NT, CAP>(p, sh, b, m, off);
     }
@@ -1072,7 +1073,7 @@ __device__ bool local_range_warp(const SsParams& p, unsigned b, int m, int64_t o
   if (extra) extra_val = __ldcg(extra);
 #pragma unroll
   for (int e = 0; e < E; ++e)
-    if (pv[e] <= -2) nmask |= 1u << e;
+    if (pocc_new(pv[e])) nmask |= 1u << e;
   const unsigned long long own = ((unsigned long long)__popc(nmask) << 32) | (unsigned)__popc(hmask);
   unsigned long long y = own;
 #pragma unroll
@@ -1151,7 +1152,7 @@ __global__ void __launch_bounds__(kLocalWarpThreads) ss_local_warp_kernel(const 
   }
   if (eq) {
     if (!eq_loaded) eq_val = __ldcg(eq_pocc);
-    local_equal(p, be, me, offe, eq_val <= -2, lane, 32);
+    local_equal(p, be, me, offe, pocc_new(eq_val), lane, 32);
   } else if (has_e && lane == 0) {
     p.ctl->hcnt[be] = 0;
     p.ctl->ncnt[be] = 0;
@@ -1197,6 +1198,7 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
   __syncthreads();
   const int64_t q0 = (int64_t)blockIdx.x * kSub + tid;
   const uint64_t row_base = p.bdev->row_base;
+  unsigned sh_unclaim = 0;  // slots this thread gave back (a rejected call)
   uint64_t mt[kFinItems];
   uint32_t occ[kFinItems];
 #pragma unroll
@@ -1247,13 +1249,16 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
       const int64_t key = from_ukey(__ldcs(p.kb + q));
       int64_t row = __ldcg(p.pocc + occ[j]);
       if ((m >> 42) & 1u) {
+        // admitted by this call: the k-th new key (ascending key order) takes
+        // the k-th queued freed row, or a row past the end
         const int64_t slot = -2 - row;
         const unsigned ln = (unsigned)((m >> 21) & 0x1fffffULL);
-        row = (int64_t)(row_base + (cpre >> 32) + __ldg(&p.ctl->npre[b]) + ln - 1u);
+        const unsigned long long k = (cpre >> 32) + __ldg(&p.ctl->npre[b]) + ln - 1u;
+        const unsigned long long avail = p.bdev->free_avail;
+        row = k < avail ? (int64_t)__ldg(p.free_rows + p.bdev->free_base + k)
+                        : (int64_t)(row_base + (k - avail));
         if (rejected) {
-          // give the claimed slot back: every key claimed by this call is
-          // newer than every key that stays, so no probe chain is cut
-          p.slots[slot].key = kEmptyKey;
+          sh_unclaim += idmap_give_back(p.slots, slot);
           row = -1;
         } else if (row >= p.mapped_rows) {
           raise_error(p.st, p.mirror, kErrTableFull);
@@ -1261,10 +1266,19 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
         } else {
           p.slots[slot].row = row;
           p.row_keys[row] = key;
+          if (p.seen) p.seen[row] = (uint32_t)p.clock;
           const int at = atomicAdd(&sh.ninit, 1);
           sh.init_key[at] = key;
           sh.init_row[at] = (int32_t)row;
         }
+      } else if (pocc_cand(row)) {
+        // stays a candidate: one more lookup counted, at this clock
+        const int64_t slot = kCandPocc - row;
+        if (rejected) sh_unclaim += idmap_give_back(p.slots, slot);
+        else p.slots[slot].row = cand_row(p.clock, prior_count(__ldcg(&p.slots[slot].row)) + 1);
+        row = -1;
+      } else if (row >= 0 && p.seen && !rejected) {
+        p.seen[row] = (uint32_t)p.clock;
       }
       p.uniq[seg] = key;
       p.rows[seg] = row;
@@ -1281,6 +1295,7 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
       }
     }
   }
+  if (sh_unclaim) atomicAdd(&p.st->slots_used, (unsigned long long)(0ULL - sh_unclaim));
   // chunks of this CTA holding a long segment, for the backward's reduction,
   // and its keys seen 2 to kShortSeg times
   __syncthreads();
@@ -1414,6 +1429,11 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   p.st = t->dstate;
   p.mirror = t->mirror_dev;
   p.call_id = b->call_seq;
+  // a bulk insert pre-loads: its keys are admitted at once
+  p.admit = (!insert && t->cfg.admit_threshold > 1) ? t->cfg.admit_threshold : 1;
+  p.clock = (uint64_t)t->clock;
+  p.seen = t->cfg.evictable ? reinterpret_cast<uint32_t*>(t->seen.va) : nullptr;
+  p.free_rows = t->free_rows;
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

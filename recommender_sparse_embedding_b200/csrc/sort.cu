@@ -117,6 +117,9 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restric
   __syncthreads();
   if (threadIdx.x == 0) {
     bdev->row_base = *(volatile unsigned long long*)&st->next_free;
+    const unsigned long long fh = *(volatile unsigned long long*)&st->free_head;
+    bdev->free_base = fh;
+    bdev->free_avail = *(volatile unsigned long long*)&st->free_tail - fh;
     unsigned n = 0;
     for (int p = 0; p < kSortPasses; ++p) {
       ctl->active[p] = s_active[p];

@@ -81,6 +81,8 @@ struct Drv {
   decltype(&::cuMemSetAccess) MemSetAccess = nullptr;
   decltype(&::cuMemGetAllocationGranularity) MemGetAllocationGranularity = nullptr;
   decltype(&::cuGetErrorString) GetErrorString = nullptr;
+  decltype(&::cuDeviceGet) DeviceGet = nullptr;
+  decltype(&::cuDeviceGetAttribute) DeviceGetAttribute = nullptr;
   bool ok = false;
 };
 
@@ -99,7 +101,8 @@ static const Drv& drv() {
            get("cuMemMap", (void**)&x.MemMap) && get("cuMemUnmap", (void**)&x.MemUnmap) &&
            get("cuMemSetAccess", (void**)&x.MemSetAccess) &&
            get("cuMemGetAllocationGranularity", (void**)&x.MemGetAllocationGranularity) &&
-           get("cuGetErrorString", (void**)&x.GetErrorString);
+           get("cuGetErrorString", (void**)&x.GetErrorString) && get("cuDeviceGet", (void**)&x.DeviceGet) &&
+           get("cuDeviceGetAttribute", (void**)&x.DeviceGetAttribute);
     return x;
   }();
   return d;
@@ -153,8 +156,13 @@ static recis_status vmm_map_to(VmmArray& a, size_t bytes, int dev) {
   }
   CUmemAllocationProp prop = {};
   prop.type = CU_MEM_ALLOCATION_TYPE_PINNED;
-  prop.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
-  prop.location.id = dev;
+  if (a.host_numa >= 0) {  // host memory, reached by the GPU through the mapping
+    prop.location.type = CU_MEM_LOCATION_TYPE_HOST_NUMA;
+    prop.location.id = a.host_numa;
+  } else {
+    prop.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
+    prop.location.id = dev;
+  }
   CUmemGenericAllocationHandle h;
   CUresult r = drv().MemCreate(&h, sz, &prop, 0);
   if (r != CUDA_SUCCESS) return cu_fail(r, "cuMemCreate (EmbeddingBlock)");
@@ -164,7 +172,8 @@ static recis_status vmm_map_to(VmmArray& a, size_t bytes, int dev) {
     return cu_fail(r, "cuMemMap");
   }
   CUmemAccessDesc acc = {};
-  acc.location = prop.location;
+  acc.location.type = CU_MEM_LOCATION_TYPE_DEVICE;  // the GPU reads and writes every block
+  acc.location.id = dev;
   acc.flags = CU_MEM_ACCESS_FLAGS_PROT_READWRITE;
   r = drv().MemSetAccess(a.va + a.mapped, sz, &acc, 1);
   if (r != CUDA_SUCCESS) {
@@ -212,10 +221,36 @@ static recis_status grow_rows(recis_table* t, int64_t rows) {
   const size_t kb = round_up((size_t)backed * sizeof(int64_t), t->gran);
   st = vmm_map_to(t->keys, std::min(kb, t->keys.reserved), t->dev);
   if (st != RECIS_OK) return st;
+  int64_t m = std::min<int64_t>(backed, (int64_t)(t->keys.mapped / sizeof(int64_t)));
+  if (t->cfg.evictable) {
+    const size_t sb = round_up((size_t)m * sizeof(uint32_t), t->gran);
+    st = vmm_map_to(t->seen, std::min(sb, t->seen.reserved), t->dev);
+    if (st != RECIS_OK) return st;
+    m = std::min<int64_t>(m, (int64_t)(t->seen.mapped / sizeof(uint32_t)));
+  }
   // rows past max_rows stay unused even where a block's rounding backs them
-  t->mapped_rows = std::min<int64_t>(std::min<int64_t>(backed, (int64_t)(t->keys.mapped / sizeof(int64_t))),
-                                     t->max_rows);
+  t->mapped_rows = std::min<int64_t>(m, t->max_rows);
   return RECIS_OK;
+}
+
+// A slot array of cap slots: device memory, or mapped pinned host memory for
+// a host-placed IDMap (*host receives its host address, else null).
+static cudaError_t alloc_slots(recis_table* t, int64_t cap, Slot** dev_ptr, Slot** host) {
+  *host = nullptr;
+  if (!(t->cfg.placement & RECIS_PLACE_IDMAP_HOST)) return cudaMalloc(dev_ptr, sizeof(Slot) * cap);
+  cudaError_t e = cudaHostAlloc(host, sizeof(Slot) * cap, cudaHostAllocMapped);
+  if (e != cudaSuccess) return e;
+  e = cudaHostGetDevicePointer((void**)dev_ptr, *host, 0);
+  if (e != cudaSuccess) {
+    cudaFreeHost(*host);
+    *host = nullptr;
+  }
+  return e;
+}
+
+static void free_slots(Slot* dev_ptr, Slot* host) {
+  if (host) cudaFreeHost(host);
+  else cudaFree(dev_ptr);
 }
 
 // IDMap growth: a new slot array, every live (key, row) re-inserted.
@@ -224,22 +259,32 @@ static recis_status grow_idmap(recis_table* t, int64_t keys_needed, cudaStream_t
   while ((double)keys_needed > kMaxLoad * (double)cap) cap *= 2;
   if (cap == t->capacity) return RECIS_OK;
   Slot* ns = nullptr;
-  cudaError_t e = cudaMalloc(&ns, sizeof(Slot) * cap);
+  Slot* ns_host = nullptr;
+  cudaError_t e = alloc_slots(t, cap, &ns, &ns_host);
   if (e != cudaSuccess) {
-    set_error("IDMap growth: cudaMalloc failed");
+    set_error("IDMap growth: allocation failed");
     return RECIS_ERR_OOM;
   }
   e = cudaMemsetAsync(ns, 0xff, sizeof(Slot) * cap, s);
   if (e != cudaSuccess) return cuda_fail(e, "IDMap growth memset");
   Slot* old = t->slots;
+  Slot* old_host = t->slots_host;
   const int64_t old_cap = t->capacity;
   t->slots = ns;
+  t->slots_host = ns_host;
   t->capacity = cap;
+  // the rehash drops tombstones and counts the slots it fills
+  e = cudaMemsetAsync(&t->dstate->slots_used, 0, sizeof(unsigned long long), s);
+  if (e != cudaSuccess) return cuda_fail(e, "IDMap growth memset");
   e = launch_rehash(t, old, old_cap, s);
   if (e != cudaSuccess) return cuda_fail(e, "IDMap rehash");
   e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "IDMap rehash");
-  cudaFree(old);
+  free_slots(old, old_host);
+  unsigned long long used = 0;
+  e = cudaMemcpy(&used, &t->dstate->slots_used, sizeof(used), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "IDMap rehash count");
+  t->slots_upper = (int64_t)used;
   return RECIS_OK;
 }
 
@@ -251,6 +296,8 @@ static void refresh_mirror(recis_table* t) {
     if (cudaEventQuery(t->ring[k]) == cudaSuccess) {
       const int64_t bound = (int64_t)t->mirror->next_free + (t->cum_issued - t->ring_cum[k]);
       if (bound < t->rows_upper) t->rows_upper = bound;
+      const int64_t sbound = (int64_t)t->mirror->slots_used + (t->cum_issued - t->ring_cum[k]);
+      if (sbound < t->slots_upper) t->slots_upper = sbound;
       t->ring_live = i;  // this event and older ones are consumed
       return;
     }
@@ -293,6 +340,7 @@ static recis_status take_status(recis_table* t, cudaStream_t s) {
   e = cudaMemcpy(&h, t->dstate, sizeof(DevState), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   t->rows_upper = (int64_t)h.next_free;
+  t->slots_upper = (int64_t)h.slots_used;
   t->ring_live = 0;
   t->mirror->error_seen = 0;
   if (h.status) {
@@ -318,19 +366,22 @@ static recis_status reserve(recis_table* t, int64_t n_new, cudaStream_t s,
   refresh_mirror(t);
   int64_t need = t->rows_upper + n_new;
   if (device_checked) need = std::min(need, std::max(t->max_rows, t->rows_upper));
-  if (need > t->mapped_rows || (double)need > kMaxLoad * (double)t->capacity) {
+  // IDMap slots: keys with rows, candidates and tombstones all hold one
+  const int64_t slots_need = std::max(need, t->slots_upper + n_new);
+  if (need > t->mapped_rows || (double)slots_need > kMaxLoad * (double)t->capacity) {
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
     DevState h;
     e = cudaMemcpy(&h, t->dstate, sizeof(DevState), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "row count read");
     t->rows_upper = (int64_t)h.next_free;
+    t->slots_upper = (int64_t)h.slots_used;
     t->ring_live = 0;
     need = t->rows_upper + n_new;
     if (device_checked) need = std::min(need, std::max(t->max_rows, t->rows_upper));
     recis_status st = grow_rows(t, need);
     if (st != RECIS_OK) return st;
-    st = grow_idmap(t, need, s);
+    st = grow_idmap(t, std::max(need, t->slots_upper + n_new), s);
     if (st != RECIS_OK) return st;
   }
   return RECIS_OK;
@@ -338,6 +389,7 @@ static recis_status reserve(recis_table* t, int64_t n_new, cudaStream_t s,
 
 static void after_call(recis_table* t, int64_t n_new_bound, cudaStream_t s) {
   t->rows_upper += n_new_bound;
+  t->slots_upper += n_new_bound;
   t->cum_issued += n_new_bound;
   const int k = t->ring_next;
   if (cudaEventRecord(t->ring[k], s) == cudaSuccess) {
@@ -520,6 +572,7 @@ static recis_status lookup_impl(const LookupArgs& a, cudaStream_t s) {
   b->bag_offsets = a.bag_offsets;
   b->have_lookup = true;
   if (++b->call_seq == 0) b->call_seq = 1;
+  t->clock += 1;  // this call's lookups touch rows at this clock
   cudaError_t e;
   const bool pool = a.pooled_out || a.unpooled_out;
   const int64_t cf = pool_chunk_for(a.N, t->D);
@@ -537,7 +590,7 @@ static recis_status lookup_impl(const LookupArgs& a, cudaStream_t s) {
         return cuda_fail(e, "dedup launch");
     } else {
       if ((e = launch_sort(b, t, a.keys, a.N, s)) != cudaSuccess) return cuda_fail(e, "sort launch");
-      if ((e = launch_unique_insert(b, t, a.N, s)) != cudaSuccess)
+      if ((e = launch_unique_insert(b, t, a.N, a.insert, s)) != cudaSuccess)
         return cuda_fail(e, "unique launch");
     }
     if (a.rows_out && (e = launch_rows_per_key(b, a.N, a.rows_out, s)) != cudaSuccess)
@@ -551,6 +604,19 @@ static recis_status lookup_impl(const LookupArgs& a, cudaStream_t s) {
     if ((e = launch_pool(a, cf, s)) != cudaSuccess) return cuda_fail(e, "pool launch");
   }
   after_call(t, a.N, s);
+  return RECIS_OK;
+}
+
+// Synchronous: rows in use (live rows and the freed rows below them) and live
+// rows of a table.
+recis_status table_counts(recis_table* t, cudaStream_t s, int64_t* in_use, int64_t* live) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  DevState h;
+  e = cudaMemcpy(&h, t->dstate, sizeof(DevState), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "size read");
+  if (in_use) *in_use = (int64_t)h.next_free;
+  if (live) *live = (int64_t)h.next_free - (int64_t)(h.free_tail - h.free_head);
   return RECIS_OK;
 }
 
@@ -691,7 +757,8 @@ recis_status recis_table_create(const recis_table_config* cfg, recis_stream_t st
   if (cfg->dim < 4 || cfg->dim > 1024 || cfg->dim % 4 != 0 ||
       (cfg->optimizer != RECIS_ADAGRAD && cfg->optimizer != RECIS_ADAM) ||
       cfg->initial_capacity < 0 || cfg->block_rows < 0 || cfg->max_rows < 0 ||
-      !(cfg->eps >= 0.0) || !std::isfinite(cfg->lr)) {
+      !(cfg->eps >= 0.0) || !std::isfinite(cfg->lr) || cfg->admit_threshold < 0 ||
+      cfg->admit_threshold > kMaxAdmitThreshold || (cfg->evictable != 0 && cfg->evictable != 1)) {
     set_error("table_create: invalid config (dim must be a multiple of 4 in [4, 1024])");
     return RECIS_ERR_INVALID_ARG;
   }
@@ -717,10 +784,42 @@ recis_status recis_table_create(const recis_table_config* cfg, recis_stream_t st
   t->max_rows = cfg->max_rows > 0 ? cfg->max_rows : (int64_t)1 << 28;
   if (t->max_rows > INT32_MAX) t->max_rows = INT32_MAX;  // row offsets are 31-bit in the kernels
 
+  if (cfg->placement & ~(RECIS_PLACE_BLOCKS_HOST | RECIS_PLACE_IDMAP_HOST)) {
+    delete t;
+    set_error("table_create: unknown placement flags");
+    return RECIS_ERR_INVALID_ARG;
+  }
+  if (cfg->placement & RECIS_PLACE_IDMAP_HOST) {
+    int native = 0;
+    cudaDeviceGetAttribute(&native, cudaDevAttrHostNativeAtomicSupported, t->dev);
+    if (!native) {
+      delete t;
+      set_error("table_create: an IDMap in host memory needs native GPU atomics on host memory, "
+                "which this system does not provide");
+      return RECIS_ERR_INVALID_ARG;
+    }
+  }
+  int host_numa = -1;
+  if (cfg->placement & RECIS_PLACE_BLOCKS_HOST) {
+    CUdevice cd = 0;
+    int vmm_host = 0, numa = -1;
+    if (drv().DeviceGet(&cd, t->dev) == CUDA_SUCCESS) {
+      drv().DeviceGetAttribute(&vmm_host, CU_DEVICE_ATTRIBUTE_HOST_NUMA_VIRTUAL_MEMORY_MANAGEMENT_SUPPORTED, cd);
+      drv().DeviceGetAttribute(&numa, CU_DEVICE_ATTRIBUTE_HOST_NUMA_ID, cd);
+    }
+    if (!vmm_host) {
+      delete t;
+      set_error("table_create: EmbeddingBlocks in host memory need host-NUMA virtual-memory mappings, "
+                "which this driver and device do not provide");
+      return RECIS_ERR_INVALID_ARG;
+    }
+    host_numa = numa < 0 ? 0 : numa;
+    t->rows.host_numa = t->keys.host_numa = t->seen.host_numa = host_numa;
+  }
   CUmemAllocationProp prop = {};
   prop.type = CU_MEM_ALLOCATION_TYPE_PINNED;
-  prop.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
-  prop.location.id = t->dev;
+  prop.location.type = host_numa >= 0 ? CU_MEM_LOCATION_TYPE_HOST_NUMA : CU_MEM_LOCATION_TYPE_DEVICE;
+  prop.location.id = host_numa >= 0 ? host_numa : t->dev;
   r = drv().MemGetAllocationGranularity(&t->gran, &prop, CU_MEM_ALLOC_GRANULARITY_RECOMMENDED);
   if (r != CUDA_SUCCESS) {
     delete t;
@@ -729,14 +828,16 @@ recis_status recis_table_create(const recis_table_config* cfg, recis_stream_t st
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
   if ((st = vmm_reserve(t->rows, round_up((size_t)t->max_rows * t->row_bytes, t->gran))) != RECIS_OK ||
-      (st = vmm_reserve(t->keys, round_up((size_t)t->max_rows * sizeof(int64_t), t->gran))) != RECIS_OK)
+      (st = vmm_reserve(t->keys, round_up((size_t)t->max_rows * sizeof(int64_t), t->gran))) != RECIS_OK ||
+      (cfg->evictable &&
+       (st = vmm_reserve(t->seen, round_up((size_t)t->max_rows * sizeof(uint32_t), t->gran))) != RECIS_OK))
     goto fail;
   if ((st = grow_rows(t, std::max<int64_t>(cfg->initial_capacity, 1))) != RECIS_OK) goto fail;
   {
     int64_t cap = 1024;
     while ((double)cfg->initial_capacity > kMaxLoad * (double)cap) cap *= 2;
     t->capacity = cap;
-    if ((e = cudaMalloc(&t->slots, sizeof(Slot) * cap)) != cudaSuccess) {
+    if ((e = alloc_slots(t, cap, &t->slots, &t->slots_host)) != cudaSuccess) {
       st = RECIS_ERR_OOM;
       set_error("IDMap allocation failed");
       goto fail;
@@ -776,7 +877,9 @@ recis_status recis_table_destroy(recis_table_t t) {
   cudaDeviceSynchronize();
   vmm_release(t->rows);
   vmm_release(t->keys);
-  cudaFree(t->slots);
+  vmm_release(t->seen);
+  cudaFree(t->free_rows);
+  free_slots(t->slots, t->slots_host);
   cudaFree(t->dstate);
   if (t->mirror) cudaFreeHost((void*)t->mirror);
   for (int k = 0; k < recis_table::kRing; ++k)
@@ -894,16 +997,19 @@ recis_status recis_table_status_sync(recis_table_t t, recis_stream_t stream) {
   return take_status(t, (cudaStream_t)stream);
 }
 
+
 recis_status recis_table_size(recis_table_t t, int64_t* n_out, int64_t* step_out,
                               recis_stream_t stream) {
   if (!t) return RECIS_ERR_INVALID_ARG;
-  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-  DevState h;
-  e = cudaMemcpy(&h, t->dstate, sizeof(DevState), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return cuda_fail(e, "size read");
-  if (n_out) *n_out = (int64_t)h.next_free;
+  recis_status st = table_counts(t, (cudaStream_t)stream, nullptr, n_out);
+  if (st != RECIS_OK) return st;
   if (step_out) *step_out = t->step;
+  return RECIS_OK;
+}
+
+recis_status recis_table_clock(recis_table_t t, int64_t* clock_out) {
+  if (!t || !clock_out) return RECIS_ERR_INVALID_ARG;
+  *clock_out = t->clock;
   return RECIS_OK;
 }
 
@@ -911,31 +1017,35 @@ recis_status recis_table_export(recis_table_t t, int64_t* keys, float* emb, floa
                                 int64_t capacity, int64_t* n_out, int64_t* step_out,
                                 recis_stream_t stream) {
   if (!t || capacity < 0) return RECIS_ERR_INVALID_ARG;
-  int64_t n = 0;
-  recis_status st = recis_table_size(t, &n, step_out, stream);
+  int64_t in_use = 0, n = 0;
+  recis_status st = table_counts(t, (cudaStream_t)stream, &in_use, &n);
   if (st != RECIS_OK) return st;
   if (n_out) *n_out = n;
+  if (step_out) *step_out = t->step;
   const int64_t m = std::min(n, capacity);
-  cudaError_t e;
-  if (keys && m > 0) {
-    e = cudaMemcpy(keys, (const void*)t->keys.va, sizeof(int64_t) * m, cudaMemcpyDeviceToHost);
+  if (m == 0) return RECIS_OK;
+  // the live rows (freed rows hold key -1) in ascending row order, in chunks
+  const int64_t chunk = std::max<int64_t>(1, ((int64_t)64 << 20) / (int64_t)t->row_bytes);
+  std::vector<int64_t> kb((size_t)std::min(chunk, in_use));
+  std::vector<float> buf((emb || state) ? (size_t)std::min(chunk, in_use) * t->row_floats : 0);
+  int64_t k = 0;
+  for (int64_t r0 = 0; r0 < in_use && k < m; r0 += chunk) {
+    const int64_t nr = std::min(chunk, in_use - r0);
+    cudaError_t e = cudaMemcpy(kb.data(), (const int64_t*)t->keys.va + r0, sizeof(int64_t) * nr,
+                               cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "export keys");
-  }
-  if ((emb || state) && m > 0) {
-    const int64_t chunk = std::max<int64_t>(1, ((int64_t)64 << 20) / (int64_t)t->row_bytes);
-    std::vector<float> buf((size_t)std::min(chunk, m) * t->row_floats);
-    for (int64_t r0 = 0; r0 < m; r0 += chunk) {
-      const int64_t nr = std::min(chunk, m - r0);
+    if (emb || state) {
       e = cudaMemcpy(buf.data(), (const char*)t->rows.va + (size_t)r0 * t->row_bytes,
                      (size_t)nr * t->row_bytes, cudaMemcpyDeviceToHost);
       if (e != cudaSuccess) return cuda_fail(e, "export rows");
-      for (int64_t i = 0; i < nr; ++i) {
-        const float* src = buf.data() + (size_t)i * t->row_floats;
-        if (emb) std::memcpy(emb + (size_t)(r0 + i) * t->D, src, sizeof(float) * t->D);
-        if (state)
-          std::memcpy(state + (size_t)(r0 + i) * t->s * t->D, src + t->D,
-                      sizeof(float) * t->s * t->D);
-      }
+    }
+    for (int64_t i = 0; i < nr && k < m; ++i) {
+      if (kb[i] == kEmptyKey) continue;
+      if (keys) keys[k] = kb[i];
+      const float* src = buf.data() + (size_t)i * t->row_floats;
+      if (emb) std::memcpy(emb + (size_t)k * t->D, src, sizeof(float) * t->D);
+      if (state) std::memcpy(state + (size_t)k * t->s * t->D, src + t->D, sizeof(float) * t->s * t->D);
+      ++k;
     }
   }
   return RECIS_OK;
@@ -958,8 +1068,8 @@ recis_status recis_table_import(recis_table_t t, const int64_t* keys, const floa
   if (st != RECIS_OK) return st;
   st = reserve(t, n, s);
   if (st != RECIS_OK) return st;
-  int64_t row0 = 0;
-  st = recis_table_size(t, &row0, nullptr, stream);
+  int64_t row0 = 0;  // imported rows go after every row in use
+  st = table_counts(t, s, &row0, nullptr);
   if (st != RECIS_OK) return st;
   if (row0 + n > t->mapped_rows) {
     st = grow_rows(t, row0 + n);
@@ -989,7 +1099,7 @@ recis_status recis_table_import(recis_table_t t, const int64_t* keys, const floa
     int64_t* dkeys = nullptr;
     if ((e = cudaMalloc(&dkeys, sizeof(int64_t) * n)) != cudaSuccess) return cuda_fail(e, "import");
     e = cudaMemcpy(dkeys, keys, sizeof(int64_t) * n, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = launch_import(t, dkeys, n, row0, s);
+    if (e == cudaSuccess) e = launch_import(t, dkeys, n, row0, t->clock, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     cudaFree(dkeys);
     if (e != cudaSuccess) return cuda_fail(e, "import");

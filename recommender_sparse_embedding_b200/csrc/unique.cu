@@ -23,7 +23,6 @@ namespace recis {
 namespace {
 
 constexpr int kUqBlock = 256, kUqItems = 4, kUqTile = kUqBlock * kUqItems;
-constexpr int kMaxProbes = 1 << 16;
 constexpr unsigned long long kUqAgg = 1ULL << 62, kUqIncl = 2ULL << 62;
 
 __device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
@@ -33,45 +32,6 @@ __device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long lon
 }
 __device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v) {
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-// IDMap find-or-insert.  Returns true when the key was inserted by this call
-// (slot index in *slot); otherwise *row holds the existing row (-1 for a
-// missing key when insert is false).  *slot = -1 when the probe limit is
-// reached or the key is missing and insert is false.
-__device__ __forceinline__ bool idmap_find_or_insert(Slot* slots, uint64_t mask, int64_t key,
-                                                     int64_t* slot, int64_t* row,
-                                                     bool insert = true) {
-  uint64_t h = mix64((uint64_t)key ^ kSlotSalt) & mask;
-  const int64_t limit = (int64_t)mask + 1 < kMaxProbes ? (int64_t)mask + 1 : kMaxProbes;
-  for (int64_t n = 0; n < limit; ++n) {
-    const longlong2 sv = __ldcg(reinterpret_cast<const longlong2*>(slots + h));
-    if (sv.x == key) {
-      *slot = (int64_t)h;
-      *row = sv.y;
-      return false;
-    }
-    if (sv.x == kEmptyKey) {
-      if (!insert) break;
-      const unsigned long long old = atomicCAS(reinterpret_cast<unsigned long long*>(&slots[h].key),
-                                               (unsigned long long)kEmptyKey,
-                                               (unsigned long long)key);
-      if ((int64_t)old == kEmptyKey) {
-        *slot = (int64_t)h;
-        *row = -1;
-        return true;
-      }
-      if ((int64_t)old == key) {
-        *slot = (int64_t)h;
-        *row = __ldcg(&slots[h].row);
-        return false;
-      }
-    }
-    h = (h + 1) & mask;
-  }
-  *slot = -1;
-  *row = -1;
-  return false;
 }
 
 }  // namespace
@@ -107,6 +67,10 @@ struct UniqueParams {
   HostMirror* mirror;
   uint32_t call_id;
   int spin_max;             // polls before a look-back wait gives up
+  int admit;                // admission threshold (>= 1)
+  uint64_t clock;           // this lookup's clock
+  uint32_t* seen;           // [row] last-lookup clock of each row, or null
+  const int32_t* free_rows; // queue of freed rows (bdev->free_base .. + free_avail)
 };
 
 __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_constant__ UniqueParams p) {
@@ -115,6 +79,7 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
   __shared__ unsigned s_tile;
   __shared__ unsigned long long s_prefix;
   __shared__ int s_ninit;
+  __shared__ unsigned s_claims;
   __shared__ int64_t s_init_key[kUqTile];
   __shared__ int64_t s_init_row[kUqTile];
 
@@ -122,6 +87,7 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
   if (tid == 0) {
     s_tile = atomicAdd(&p.ctl->seg_tile_counter, 1u);
     s_ninit = 0;
+    s_claims = 0;
   }
   __syncthreads();
   const unsigned tile = s_tile;
@@ -165,6 +131,7 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
   const bool rejected = __ldcg(&p.bdev->reject_call) == p.call_id;
   bool head[kUqItems], isnew[kUqItems];
   int64_t slot[kUqItems], row[kUqItems];
+  int prior[kUqItems];
   unsigned nh = 0, nn = 0;
 #pragma unroll
   for (int j = 0; j < kUqItems; ++j) {
@@ -174,10 +141,20 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
     isnew[j] = false;
     slot[j] = -1;
     row[j] = -1;
+    prior[j] = 0;
     if (head[j] && from_ukey(k[j]) != kEmptyKey) {  // the reserved key is reported by the sort
-      isnew[j] = idmap_find_or_insert(p.slots, p.slot_mask, from_ukey(k[j]), &slot[j], &row[j],
-                                      !rejected);
-      if (slot[j] < 0 && !rejected) raise_error(p.st, p.mirror, kErrTableFull);
+      const int64_t key = from_ukey(k[j]);
+      const uint64_t h = mix64((uint64_t)key ^ kSlotSalt) & p.slot_mask;
+      const Probe pr = idmap_probe(p.slots, p.slot_mask, key, h,
+                                   __ldcg(reinterpret_cast<const longlong2*>(p.slots + h)), !rejected,
+                                   &s_claims);
+      if (pr.limit && !rejected) raise_error(p.st, p.mirror, kErrTableFull);
+      row[j] = pr.row;
+      slot[j] = pr.slot;
+      prior[j] = pr.prior;
+      // a key without a row is admitted when this lookup brings its count to
+      // the threshold; otherwise it stays a candidate (slot kept, no row)
+      isnew[j] = !rejected && pr.row < 0 && pr.slot >= 0 && pr.prior + 1 >= p.admit;
     }
     if (head[j]) {
       ++nh;
@@ -259,7 +236,10 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
       const unsigned seg = hrun;
       int64_t r = row[j];
       if (isnew[j]) {
-        r = (int64_t)(row_base + nrun);
+        // the k-th new key takes the k-th queued freed row, or a row past the end
+        const unsigned long long kk = nrun, avail = p.bdev->free_avail;
+        r = kk < avail ? (int64_t)__ldg(p.free_rows + p.bdev->free_base + kk)
+                       : (int64_t)(row_base + (kk - avail));
         ++nrun;
         if (r >= p.mapped_rows) {
           raise_error(p.st, p.mirror, kErrTableFull);
@@ -267,10 +247,16 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
         } else {
           p.slots[slot[j]].row = r;
           p.row_keys[r] = from_ukey(k[j]);
+          if (p.seen) p.seen[r] = (uint32_t)p.clock;
           const int q = atomicAdd(&s_ninit, 1);
           s_init_key[q] = from_ukey(k[j]);
           s_init_row[q] = r;
         }
+      } else if (r < 0 && slot[j] >= 0 && !rejected) {
+        // stays a candidate: one more lookup counted, at this clock
+        p.slots[slot[j]].row = cand_row(p.clock, prior[j] + 1);
+      } else if (r >= 0 && p.seen && !rejected) {
+        p.seen[r] = (uint32_t)p.clock;
       }
       p.uniq[seg] = from_ukey(k[j]);
       p.rows[seg] = r;
@@ -284,15 +270,19 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
       p.spos[v[j]] = (uint32_t)pos;
     }
   }
+  if (tid == 0 && s_claims) atomicAdd(&p.st->slots_used, (unsigned long long)s_claims);
   if (tile == gridDim.x - 1 && tid == 0) {
     const unsigned long long U = Hx + tH, nnew = Nx + tN;
     p.bdev->U = rejected ? 0u : (unsigned)U;
     p.bdev->n_new = (unsigned)nnew;
-    unsigned long long nf = row_base + nnew;
+    const unsigned long long avail = p.bdev->free_avail;
+    unsigned long long nf = row_base + (nnew > avail ? nnew - avail : 0ULL);
     if (nf > (unsigned long long)p.mapped_rows) nf = (unsigned long long)p.mapped_rows;
     p.st->next_free = nf;
+    p.st->free_head = p.bdev->free_base + (nnew < avail ? nnew : avail);
     if (p.mirror) {
       p.mirror->next_free = nf;
+      p.mirror->slots_used = *(volatile unsigned long long*)&p.st->slots_used;
       __threadfence_system();
     }
     p.seg_start[U] = (int32_t)N;
@@ -328,7 +318,7 @@ __global__ void rows_per_key_kernel(const int32_t* __restrict__ inv, const int64
     out[i] = rows[inv[i]];
 }
 
-cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cudaStream_t s) {
+cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, bool insert, cudaStream_t s) {
   UniqueParams p;
   p.in_keys = b->keys;
   p.kb0 = b->kbuf[0];
@@ -360,6 +350,11 @@ cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, cuda
   p.mirror = t->mirror_dev;
   p.call_id = b->call_seq;
   p.spin_max = spin_limit();
+  // a bulk insert pre-loads: its keys are admitted at once
+  p.admit = (!insert && t->cfg.admit_threshold > 1) ? t->cfg.admit_threshold : 1;
+  p.clock = (uint64_t)t->clock;
+  p.seen = t->cfg.evictable ? reinterpret_cast<uint32_t*>(t->seen.va) : nullptr;
+  p.free_rows = t->free_rows;
   const int64_t tiles = (N + kUqTile - 1) / kUqTile;
   LaunchScope ls("unique_insert", s);
   unique_insert_kernel<<<(unsigned)tiles, kUqBlock, 0, s>>>(p);
@@ -374,33 +369,50 @@ cudaError_t launch_rows_per_key(recis_batch* b, int64_t N, int64_t* rows_out, cu
   return cudaGetLastError();
 }
 
+// Every key of the old slot array into the new one with its row state (a row
+// or a candidate count); tombstones are dropped.  Counts the slots filled.
 __global__ void rehash_kernel(const Slot* __restrict__ old_slots, int64_t old_cap, Slot* slots,
                               uint64_t mask, DevState* st, HostMirror* mirror) {
+  __shared__ unsigned s_claims;
+  if (threadIdx.x == 0) s_claims = 0;
+  __syncthreads();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < old_cap; i += stride) {
     const Slot sl = old_slots[i];
-    if (sl.key == kEmptyKey) continue;
-    int64_t slot, row;
-    if (idmap_find_or_insert(slots, mask, sl.key, &slot, &row))
-      slots[slot].row = sl.row;
-    else
-      raise_error(st, mirror, slot < 0 ? kErrTableFull : kErrDuplicateImport);
+    if (sl.key == kEmptyKey || sl.row == kTombRow) continue;
+    const uint64_t h = mix64((uint64_t)sl.key ^ kSlotSalt) & mask;
+    const Probe pr = idmap_probe(slots, mask, sl.key, h, __ldcg(reinterpret_cast<const longlong2*>(slots + h)),
+                                 true, &s_claims);
+    if (pr.slot >= 0 && pr.row < 0 && pr.prior == 0) slots[pr.slot].row = sl.row;
+    else raise_error(st, mirror, pr.limit ? kErrTableFull : kErrDuplicateImport);
   }
+  __syncthreads();
+  if (threadIdx.x == 0 && s_claims) atomicAdd(&st->slots_used, (unsigned long long)s_claims);
 }
 
+// Imported keys get rows row0 + i; a key already holding a row is an error, a
+// candidate or an evicted key is admitted with its imported row.
 __global__ void import_kernel(const int64_t* __restrict__ keys, int64_t n, int64_t row0,
-                              Slot* slots, uint64_t mask, int64_t* row_keys, DevState* st,
-                              HostMirror* mirror) {
+                              Slot* slots, uint64_t mask, int64_t* row_keys, uint32_t* seen,
+                              uint32_t clock, DevState* st, HostMirror* mirror) {
+  __shared__ unsigned s_claims;
+  if (threadIdx.x == 0) s_claims = 0;
+  __syncthreads();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
-    int64_t slot, row;
-    if (idmap_find_or_insert(slots, mask, keys[i], &slot, &row)) {
-      slots[slot].row = row0 + i;
+    const uint64_t h = mix64((uint64_t)keys[i] ^ kSlotSalt) & mask;
+    const Probe pr = idmap_probe(slots, mask, keys[i], h, __ldcg(reinterpret_cast<const longlong2*>(slots + h)),
+                                 true, &s_claims);
+    if (pr.slot >= 0 && pr.row < 0) {
+      slots[pr.slot].row = row0 + i;
       row_keys[row0 + i] = keys[i];
+      if (seen) seen[row0 + i] = clock;
     } else {
-      raise_error(st, mirror, slot < 0 ? kErrTableFull : kErrDuplicateImport);
+      raise_error(st, mirror, pr.limit ? kErrTableFull : kErrDuplicateImport);
     }
   }
+  __syncthreads();
+  if (threadIdx.x == 0 && s_claims) atomicAdd(&st->slots_used, (unsigned long long)s_claims);
 }
 
 cudaError_t launch_rehash(recis_table* t, const Slot* old_slots, int64_t old_cap, cudaStream_t s) {
@@ -414,14 +426,15 @@ cudaError_t launch_rehash(recis_table* t, const Slot* old_slots, int64_t old_cap
 }
 
 cudaError_t launch_import(recis_table* t, const int64_t* keys, int64_t n, int64_t row0,
-                          cudaStream_t s) {
+                          int64_t clock, cudaStream_t s) {
   int64_t blocks = (n + 255) / 256;
   if (blocks > 16 * kSMs) blocks = 16 * kSMs;
   if (blocks < 1) return cudaSuccess;
   LaunchScope ls("idmap_import", s);
-  import_kernel<<<(unsigned)blocks, 256, 0, s>>>(keys, n, row0, t->slots, (uint64_t)t->capacity - 1,
-                                                 reinterpret_cast<int64_t*>(t->keys.va), t->dstate,
-                                                 t->mirror_dev);
+  import_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+      keys, n, row0, t->slots, (uint64_t)t->capacity - 1, reinterpret_cast<int64_t*>(t->keys.va),
+      t->cfg.evictable ? reinterpret_cast<uint32_t*>(t->seen.va) : nullptr, (uint32_t)clock, t->dstate,
+      t->mirror_dev);
   return cudaGetLastError();
 }
 

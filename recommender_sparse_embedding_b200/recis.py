@@ -23,6 +23,7 @@ ERR_INVALID_ARG, ERR_OOM, ERR_TABLE_FULL, ERR_RESERVED_KEY, ERR_CUDA, ERR_TIMEOU
 BUCKETIZE, HASH, MOD, TAG = 1, 2, 4, 8
 ADAGRAD, ADAM = 0, 1
 SUM, MEAN = 0, 1
+PLACE_BLOCKS_HOST, PLACE_IDMAP_HOST = 1, 2
 
 # every entry point declared in include/recis.h
 EXPORTS = (
@@ -32,7 +33,8 @@ EXPORTS = (
     "recis_table_import", "recis_table_status_sync", "recis_batch_get_unique",
     "recis_profile_enable", "recis_profile_collect", "recis_launch_count",
     "recis_last_error_string", "recis_unique_static", "recis_table_read_rows",
-    "recis_debug_set", "recis_plan_tables", "recis_table_reserve",
+    "recis_debug_set", "recis_plan_tables", "recis_table_reserve", "recis_table_save",
+    "recis_table_load", "recis_table_evict", "recis_table_clock",
 )
 DEBUG_SPIN_LIMIT, DEBUG_MAP_LIMIT = 1, 2
 
@@ -70,6 +72,10 @@ class TableConfig(ctypes.Structure):
         ("initial_capacity", ctypes.c_int64),
         ("block_rows", ctypes.c_int64),
         ("max_rows", ctypes.c_int64),
+        ("admit_threshold", ctypes.c_int32),
+        ("evictable", ctypes.c_int32),
+        ("placement", ctypes.c_int32),
+        ("reserved_", ctypes.c_int32),
     ]
 
 
@@ -116,6 +122,10 @@ def load(path: str = LIB_PATH):
             "recis_debug_set": [_i32, _i64],
             "recis_plan_tables": [_vp, _i32, _vp, _vp, _vp, _vp, _vp],
             "recis_table_reserve": [_vp, _i64, _vp],
+            "recis_table_save": [_vp, ctypes.c_char_p, _vp],
+            "recis_table_load": [_vp, ctypes.c_char_p, _vp],
+            "recis_table_evict": [_vp, _i64, _vp, _vp],
+            "recis_table_clock": [_vp, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -228,13 +238,16 @@ class Table:
     def __init__(self, dim: int, optimizer: int, lr: float, beta1: float = 0.9,
                  beta2: float = 0.999, eps: Optional[float] = None, adagrad_init_acc: float = 0.0,
                  init_scale: float = 0.0, init_seed: int = 0, initial_capacity: int = 0,
-                 block_rows: int = 0, max_rows: int = 0, stream=None):
+                 block_rows: int = 0, max_rows: int = 0, admit_threshold: int = 0,
+                 evictable: bool = False, placement: int = 0, stream=None):
         if eps is None:
             eps = 1e-10 if optimizer == ADAGRAD else 1e-8
         cfg = TableConfig(dim=dim, optimizer=optimizer, lr=lr, beta1=beta1, beta2=beta2, eps=eps,
                           adagrad_init_acc=adagrad_init_acc, init_scale=init_scale,
                           init_seed=init_seed & (2**64 - 1), initial_capacity=initial_capacity,
-                          block_rows=block_rows, max_rows=max_rows)
+                          block_rows=block_rows, max_rows=max_rows,
+                          admit_threshold=admit_threshold, evictable=1 if evictable else 0,
+                          placement=placement)
         h = ctypes.c_void_p()
         _check(load().recis_table_create(ctypes.byref(cfg), _stream(stream), ctypes.byref(h)),
                "recis_table_create")
@@ -277,6 +290,20 @@ class Table:
                                          _stream(stream)), "recis_table_insert")
         return rows_out
 
+    def evict(self, min_clock: int, stream=None) -> int:
+        """recis_table_evict: remove keys last touched before lookup `min_clock`;
+        returns the rows freed."""
+        n = ctypes.c_int64()
+        _check(load().recis_table_evict(self.handle, min_clock, ctypes.byref(n), _stream(stream)),
+               "recis_table_evict")
+        return n.value
+
+    @property
+    def clock(self) -> int:
+        c = ctypes.c_int64()
+        _check(load().recis_table_clock(self.handle, ctypes.byref(c)), "recis_table_clock")
+        return c.value
+
     def reserve(self, rows: int, stream=None):
         """recis_table_reserve: room for `rows` live rows in total, mapped now."""
         _check(load().recis_table_reserve(self.handle, rows, _stream(stream)), "recis_table_reserve")
@@ -315,6 +342,16 @@ class Table:
                                             emb.data_ptr(), st.data_ptr(), _stream(stream)),
                "recis_table_read_rows")
         return keys[:n], emb[:n], st[:n]
+
+    def save(self, path: str, stream=None):
+        """recis_table_save: the table as a SafeTensors file."""
+        _check(load().recis_table_save(self.handle, os.fsencode(path), _stream(stream)),
+               "recis_table_save")
+
+    def load_file(self, path: str, stream=None):
+        """recis_table_load: append the rows of a SafeTensors file."""
+        _check(load().recis_table_load(self.handle, os.fsencode(path), _stream(stream)),
+               "recis_table_load")
 
     def import_rows(self, keys, emb, state=None, step: int = 0, stream=None):
         import numpy as np

@@ -35,15 +35,17 @@ def _ofeat(f: W.FeatureSpec):
 class Pair:
     """One logical table on both sides."""
 
-    def __init__(self, R, spec: W.TableSpec, initial_capacity=0, block_rows=0, init_acc=0.0):
+    def __init__(self, R, spec: W.TableSpec, initial_capacity=0, block_rows=0, init_acc=0.0,
+                 admit_threshold=0, evictable=False, placement=0):
         opt_r = R.ADAGRAD if spec.optimizer == "adagrad" else R.ADAM
         opt_o = O.ADAGRAD if spec.optimizer == "adagrad" else O.ADAM
         self.spec = spec
         self.gpu = R.Table(spec.dim, opt_r, spec.lr, init_seed=spec.init_seed,
                            initial_capacity=initial_capacity, block_rows=block_rows,
-                           adagrad_init_acc=init_acc)
+                           adagrad_init_acc=init_acc, admit_threshold=admit_threshold,
+                           evictable=evictable, placement=placement)
         self.ora = O.Table(spec.dim, opt_o, spec.lr, init_seed=spec.init_seed,
-                           adagrad_init_acc=init_acc)
+                           adagrad_init_acc=init_acc, admit_threshold=admit_threshold)
         self.batch = R.Batch()
         self.combiner_r = R.SUM if spec.combiner == "sum" else R.MEAN
         self.combiner_o = O.SUM if spec.combiner == "sum" else O.MEAN
@@ -54,10 +56,15 @@ class Pair:
 
 
 def run_workload(R, w: W.Workload, steps=2, batch_seed=None, check_unique=True, pairs=None,
-                 initial_capacity=0, block_rows=0, grad_signed=False, return_pairs=False):
+                 initial_capacity=0, block_rows=0, grad_signed=False, return_pairs=False,
+                 admit_threshold=0, evict_every=0, evict_age=1):
+    """Steps of workload w on both sides, compared after every step.  With
+    evict_every > 0 both sides evict, after every evict_every-th step, the keys
+    last touched more than evict_age lookups before the current clock."""
     dev = torch.device("cuda", torch.cuda.current_device())
     if pairs is None:
-        pairs = [Pair(R, t, initial_capacity, block_rows) for t in w.tables]
+        pairs = [Pair(R, t, initial_capacity, block_rows, admit_threshold=admit_threshold,
+                      evictable=evict_every > 0) for t in w.tables]
     rfeats = [_rfeat(R, f, dev) for f in w.features]
     ofeats = [_ofeat(f) for f in w.features]
     for step in range(steps):
@@ -98,6 +105,11 @@ def run_workload(R, w: W.Workload, steps=2, batch_seed=None, check_unique=True, 
             p.ora.backward_update(gp, gu)
             p.gpu.status_sync()
             compare_tables(p, f"{t.name} step {step}")
+            if evict_every and (step + 1) % evict_every == 0:
+                assert p.gpu.clock == p.ora.clock
+                cut = p.ora.clock - evict_age + 1
+                assert p.gpu.evict(cut) == p.ora.evict(cut)
+                compare_tables(p, f"{t.name} after eviction at step {step}")
     if return_pairs:
         return pairs
     for p in pairs:
