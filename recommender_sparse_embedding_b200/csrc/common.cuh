@@ -98,6 +98,14 @@ struct Probe {
 
 constexpr int kProbeLimit = 1 << 16;
 
+// IDMap result of one occurrence, as the probe kernel records it: the key's
+// row (>= 0); -2 - slot for a key without a row that this call admits (it
+// gets a row); kCandPocc - slot for one that stays a candidate; -1 when there
+// is no row and no slot (reserved key, or the IDMap was exhausted).
+constexpr int64_t kCandPocc = -((int64_t)1 << 40) - 2;
+__device__ __forceinline__ bool pocc_new(int64_t v) { return v <= -2 && v > kCandPocc; }
+__device__ __forceinline__ bool pocc_cand(int64_t v) { return v <= kCandPocc; }
+
 // IDMap find-or-insert with admission: linear probing from slot h (sv = the
 // slot already loaded there).  A key found with a row returns it; a key
 // without one (claimed by this call, a candidate, or evicted -- an evicted

@@ -16,8 +16,8 @@ namespace recis {
 constexpr int kSortBits = 8;
 constexpr int kSortPasses = 64 / kSortBits;
 constexpr int kSortBlock = 256;
-constexpr int kSortItems = 8;
-constexpr int kSortTile = kSortBlock * kSortItems;  // 2048 keys per tile
+constexpr int kSortItems = 12;
+constexpr int kSortTile = kSortBlock * kSortItems;  // 3072 keys per tile
 
 // Per-call control block of the sort and of the unique pass.  The first
 // kCtlZeroBytes bytes are cleared before every lookup.
@@ -147,6 +147,8 @@ struct recis_batch {
   int4* gfirst = nullptr;       // [capN] per unique key: the same, of one of its occurrences
   int32_t* chunk_bag = nullptr; // bag of each pool chunk's first occurrence
   int32_t* bag_of = nullptr;    // [capN] bag of every occurrence (written beside the dedup)
+  int64_t* pocc = nullptr;      // [capN] IDMap result of each head, by sorted position (radix-sort path)
+  int64_t capPocc = 0;
   int64_t capChunks = 0;
   cudaStream_t side = nullptr;  // bag preparation runs here, beside the dedup
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;

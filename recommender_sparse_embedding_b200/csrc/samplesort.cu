@@ -58,14 +58,6 @@ constexpr int kFinItems = 2;
 constexpr int kSub = kFinThreads * kFinItems;       // sorted positions per finish CTA
 constexpr int kMaxProbes = 1 << 16;
 
-// IDMap result of an occurrence (from the probe kernel): the key's row
-// (>= 0); -2 - slot for a key without a row that this call admits (new: it
-// gets a row); kCandPocc - slot for one that stays a candidate; -1 when there
-// is no row and no slot (reserved key, or the IDMap was exhausted).
-constexpr int64_t kCandPocc = -((int64_t)1 << 40) - 2;
-__device__ __forceinline__ bool pocc_new(int64_t v) { return v <= -2 && v > kCandPocc; }
-__device__ __forceinline__ bool pocc_cand(int64_t v) { return v <= kCandPocc; }
-
 // bucket of ukey u: 2r + [u == split[r]], r = number of splitters < u
 __device__ __forceinline__ unsigned bucket_of(const uint64_t* split, int nsplit, uint64_t u) {
   int lo = 0, hi = nsplit;

@@ -226,10 +226,11 @@ __global__ void __launch_bounds__(kSortBlock) sort_pass_kernel(
     s_doff[d] = pre + x - total;
   }
   // decoupled look-back for digit d: kWin predecessor entries are loaded at
-  // once, then consumed nearest first until an inclusive one is met
+  // once, then consumed nearest first until an inclusive one is met (a window
+  // of 4 measured faster than 1 or 16 on 32.8M keys)
   unsigned excl = 0;
   if (tile > 0) {
-    constexpr int kWin = 16;
+    constexpr int kWin = 4;
     int64_t t = (int64_t)tile - 1;
     int spins = 0;
     bool done = false;

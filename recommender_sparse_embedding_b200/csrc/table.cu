@@ -470,6 +470,11 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
         (e = cudaEventCreateWithFlags(&b->ev_probe, cudaEventDisableTiming)) != cudaSuccess)
       return cuda_fail(e, "batch stream");
   }
+  if (N > kSampleSortMaxN && N > b->capPocc) {
+    const int64_t cap = N + N / 8;
+    if ((e = realloc_dev(b->pocc, cap, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
+    b->capPocc = cap;
+  }
   if (N <= kSampleSortMaxN) {
     const int64_t th = samplesort_tiles_for(N) * kMaxBucketSlots;
     if (th > b->ss_th_cap) {
@@ -532,6 +537,7 @@ static void batch_free(recis_batch* b) {
   cudaFree(b->bdev);
   cudaFree(b->chunk_bag);
   cudaFree(b->bag_of);
+  cudaFree(b->pocc);
   if (b->side) cudaStreamDestroy(b->side);
   if (b->ev_fork) cudaEventDestroy(b->ev_fork);
   if (b->ev_join) cudaEventDestroy(b->ev_join);

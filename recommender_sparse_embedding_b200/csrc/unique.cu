@@ -71,7 +71,56 @@ struct UniqueParams {
   uint64_t clock;           // this lookup's clock
   uint32_t* seen;           // [row] last-lookup clock of each row, or null
   const int32_t* free_rows; // queue of freed rows (bdev->free_base .. + free_avail)
+  int64_t* pocc;            // [N] IDMap result of each head, at its sorted position
 };
+
+// IDMap find-or-insert of every head (first position of a key) of the
+// sorted keys, with admission, before the unique pass: the result lands at
+// the head's sorted position (pocc[pos], as the probe kernel of the sample
+// sort encodes it), so the unique pass reads it coalesced and its look-back
+// never waits on a probe.  A call rejected for a reserved key (found by the
+// histogram pass) only looks keys up.
+__global__ void __launch_bounds__(kUqBlock) head_probe_kernel(const __grid_constant__ UniqueParams p) {
+  __shared__ unsigned s_claims;
+  if (threadIdx.x == 0) s_claims = 0;
+  __syncthreads();
+  const int64_t N = p.N;
+  const unsigned na = p.ctl->n_active;
+  const uint64_t* ks = na == 0 ? nullptr : (((na - 1) & 1) ? p.kb1 : p.kb0);
+  const bool rejected = __ldcg(&p.bdev->reject_call) == p.call_id;
+  const int64_t pos0 = ((int64_t)blockIdx.x * kUqBlock + threadIdx.x) * kUqItems;
+  uint64_t k[kUqItems + 1];
+#pragma unroll
+  for (int j = 0; j <= kUqItems; ++j) {
+    const int64_t pos = pos0 + j - 1;
+    k[j] = (pos >= 0 && pos < N) ? (ks ? ks[pos] : to_ukey(p.in_keys[pos])) : 0;
+  }
+  bool head[kUqItems];
+  uint64_t h[kUqItems];
+  longlong2 sv[kUqItems];
+#pragma unroll
+  for (int j = 0; j < kUqItems; ++j) {
+    const int64_t pos = pos0 + j;
+    head[j] = pos < N && (pos == 0 || k[j] != k[j + 1]);
+    h[j] = mix64((uint64_t)from_ukey(k[j + 1]) ^ kSlotSalt) & p.slot_mask;
+    if (head[j] && from_ukey(k[j + 1]) != kEmptyKey)
+      sv[j] = __ldcg(reinterpret_cast<const longlong2*>(p.slots + h[j]));
+  }
+#pragma unroll
+  for (int j = 0; j < kUqItems; ++j) {
+    if (!head[j]) continue;
+    int64_t r = -1;  // the reserved key (reported by the histogram pass) has no row
+    if (from_ukey(k[j + 1]) != kEmptyKey) {
+      const Probe pr = idmap_probe(p.slots, p.slot_mask, from_ukey(k[j + 1]), h[j], sv[j], !rejected, &s_claims);
+      if (pr.limit) raise_error(p.st, p.mirror, kErrTableFull);
+      else if (pr.row >= 0) r = pr.row;
+      else if (pr.slot >= 0) r = pr.prior + 1 >= p.admit ? -2 - pr.slot : kCandPocc - pr.slot;
+    }
+    p.pocc[pos0 + j] = r;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && s_claims) atomicAdd(&p.st->slots_used, (unsigned long long)s_claims);
+}
 
 __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_constant__ UniqueParams p) {
   __shared__ uint64_t s_last[kUqBlock];
@@ -79,7 +128,7 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
   __shared__ unsigned s_tile;
   __shared__ unsigned long long s_prefix;
   __shared__ int s_ninit;
-  __shared__ unsigned s_claims;
+  __shared__ unsigned s_unclaim;
   __shared__ int64_t s_init_key[kUqTile];
   __shared__ int64_t s_init_row[kUqTile];
 
@@ -87,7 +136,7 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
   if (tid == 0) {
     s_tile = atomicAdd(&p.ctl->seg_tile_counter, 1u);
     s_ninit = 0;
-    s_claims = 0;
+    s_unclaim = 0;
   }
   __syncthreads();
   const unsigned tile = s_tile;
@@ -126,36 +175,23 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
     have_prev = false;
   }
 
-  // a batch holding the reserved key (found by the histogram pass) is
-  // rejected as a whole: its keys are only looked up, nothing is inserted
+  // a batch holding the reserved key (found by the histogram pass and the
+  // probe) is rejected as a whole: the probe's claims are given back
   const bool rejected = __ldcg(&p.bdev->reject_call) == p.call_id;
+  // the heads' IDMap results, recorded at their sorted positions by head_probe
   bool head[kUqItems], isnew[kUqItems];
-  int64_t slot[kUqItems], row[kUqItems];
-  int prior[kUqItems];
+  int64_t pv[kUqItems];
   unsigned nh = 0, nn = 0;
 #pragma unroll
   for (int j = 0; j < kUqItems; ++j) {
     const int64_t pos = pos0 + j;
     const uint64_t pk = j == 0 ? prev : k[j - 1];
     head[j] = pos < N && (!(j == 0 ? have_prev : true) || pk != k[j]);
-    isnew[j] = false;
-    slot[j] = -1;
-    row[j] = -1;
-    prior[j] = 0;
-    if (head[j] && from_ukey(k[j]) != kEmptyKey) {  // the reserved key is reported by the sort
-      const int64_t key = from_ukey(k[j]);
-      const uint64_t h = mix64((uint64_t)key ^ kSlotSalt) & p.slot_mask;
-      const Probe pr = idmap_probe(p.slots, p.slot_mask, key, h,
-                                   __ldcg(reinterpret_cast<const longlong2*>(p.slots + h)), !rejected,
-                                   &s_claims);
-      if (pr.limit && !rejected) raise_error(p.st, p.mirror, kErrTableFull);
-      row[j] = pr.row;
-      slot[j] = pr.slot;
-      prior[j] = pr.prior;
-      // a key without a row is admitted when this lookup brings its count to
-      // the threshold; otherwise it stays a candidate (slot kept, no row)
-      isnew[j] = !rejected && pr.row < 0 && pr.slot >= 0 && pr.prior + 1 >= p.admit;
-    }
+    pv[j] = head[j] ? __ldcg(p.pocc + pos) : -1;
+  }
+#pragma unroll
+  for (int j = 0; j < kUqItems; ++j) {
+    isnew[j] = !rejected && pocc_new(pv[j]);  // admitted by this call: gets a row
     if (head[j]) {
       ++nh;
       nn += isnew[j];
@@ -234,9 +270,10 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
     if (pos >= N) break;
     if (head[j]) {
       const unsigned seg = hrun;
-      int64_t r = row[j];
+      int64_t r = pv[j] >= 0 ? pv[j] : -1;
       if (isnew[j]) {
         // the k-th new key takes the k-th queued freed row, or a row past the end
+        const int64_t slot = -2 - pv[j];
         const unsigned long long kk = nrun, avail = p.bdev->free_avail;
         r = kk < avail ? (int64_t)__ldg(p.free_rows + p.bdev->free_base + kk)
                        : (int64_t)(row_base + (kk - avail));
@@ -245,16 +282,19 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
           raise_error(p.st, p.mirror, kErrTableFull);
           r = -1;
         } else {
-          p.slots[slot[j]].row = r;
+          p.slots[slot].row = r;
           p.row_keys[r] = from_ukey(k[j]);
           if (p.seen) p.seen[r] = (uint32_t)p.clock;
           const int q = atomicAdd(&s_ninit, 1);
           s_init_key[q] = from_ukey(k[j]);
           s_init_row[q] = r;
         }
-      } else if (r < 0 && slot[j] >= 0 && !rejected) {
-        // stays a candidate: one more lookup counted, at this clock
-        p.slots[slot[j]].row = cand_row(p.clock, prior[j] + 1);
+      } else if (pv[j] <= -2) {
+        // no row: a rejected call gives its claims back; otherwise the key
+        // stays a candidate with one more lookup counted, at this clock
+        const int64_t slot = pocc_new(pv[j]) ? -2 - pv[j] : kCandPocc - pv[j];
+        if (rejected) atomicAdd(&s_unclaim, idmap_give_back(p.slots, slot));
+        else p.slots[slot].row = cand_row(p.clock, prior_count(__ldcg(&p.slots[slot].row)) + 1);
       } else if (r >= 0 && p.seen && !rejected) {
         p.seen[r] = (uint32_t)p.clock;
       }
@@ -270,7 +310,8 @@ __global__ void __launch_bounds__(kUqBlock) unique_insert_kernel(const __grid_co
       p.spos[v[j]] = (uint32_t)pos;
     }
   }
-  if (tid == 0 && s_claims) atomicAdd(&p.st->slots_used, (unsigned long long)s_claims);
+  __syncthreads();
+  if (tid == 0 && s_unclaim) atomicAdd(&p.st->slots_used, 0ULL - (unsigned long long)s_unclaim);
   if (tile == gridDim.x - 1 && tid == 0) {
     const unsigned long long U = Hx + tH, nnew = Nx + tN;
     p.bdev->U = rejected ? 0u : (unsigned)U;
@@ -355,7 +396,14 @@ cudaError_t launch_unique_insert(recis_batch* b, recis_table* t, int64_t N, bool
   p.clock = (uint64_t)t->clock;
   p.seen = t->cfg.evictable ? reinterpret_cast<uint32_t*>(t->seen.va) : nullptr;
   p.free_rows = t->free_rows;
+  p.pocc = b->pocc;
   const int64_t tiles = (N + kUqTile - 1) / kUqTile;
+  {
+    LaunchScope ls("head_probe", s);
+    head_probe_kernel<<<(unsigned)tiles, kUqBlock, 0, s>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   LaunchScope ls("unique_insert", s);
   unique_insert_kernel<<<(unsigned)tiles, kUqBlock, 0, s>>>(p);
   return cudaGetLastError();

@@ -23,8 +23,8 @@ namespace {
 
 constexpr int64_t kStaticMaxKeys = (int64_t)1 << 18;  // 262,144 keys per call
 constexpr int kUoBlock = 256, kUoItems = 4, kUoTile = kUoBlock * kUoItems;
-constexpr int64_t kStaticSortTiles = kStaticMaxKeys / kSortTile;
-constexpr int64_t kStaticUniqueTiles = kStaticMaxKeys / kUoTile;
+constexpr int64_t kStaticSortTiles = (kStaticMaxKeys + kSortTile - 1) / kSortTile;
+constexpr int64_t kStaticUniqueTiles = (kStaticMaxKeys + kUoTile - 1) / kUoTile;
 
 struct StaticScratch {
   SortCtl ctl;
