@@ -345,6 +345,49 @@ recis_status recis_batch_get_unique(recis_batch_t b, int64_t* uniq_out, int32_t*
 recis_status recis_unique_static(const int64_t* keys, int64_t N, int64_t* uniq_out,
                                  int32_t* inv_out, int64_t* U_out, recis_stream_t stream);
 
+/* ------------------------------------------------------------------ sharded tables */
+/* Building blocks of tables sharded over GPUs (README, Key optimisations >
+ * Distributed optimisation: parameters split evenly over the nodes; each node
+ * merges and deduplicates its requests and fetches the embeddings from their
+ * owners with an All-to-All).  A requesting GPU dedups its batch, groups the
+ * unique keys by owner, exchanges them (an NCCL all-to-all issued by the
+ * caller), pools the rows that come back, and in the backward sends each
+ * unique key's summed gradient to its owner, which applies it with
+ * recis_backward_update as an unpooled gradient of a lookup that had one bag
+ * per received key.  All asynchronous on `stream` unless marked synchronous.
+ *
+ * recis_batch_dedup: uniq_out (device int64[N]) = distinct keys ascending,
+ *   inv_out (device int32[N]) = index of keys[i] in uniq_out, *U_out (device
+ *   int64) = their number (-1 if a bounded wait gave up).  The batch keeps
+ *   the grouping of occurrences by unique key for recis_reduce_grad; any int64
+ *   key is allowed.  0 <= N < 2^30.
+ * recis_partition_keys (synchronous): a stable partition of keys[0..n) by
+ *   owner = H(key ^ salt) mod G (H: the SplitMix64 finaliser): out_keys
+ *   (device int64[n]) holds the keys of owner 0, then owner 1, ..., each in
+ *   input order; out_pos[i] (device int32[n]) = where keys[i] went;
+ *   counts_out (device int64[G]) = keys per owner.  1 <= G <= 256.
+ * recis_pool_rows: pooled_out[b][f] = sum (MEAN: / bag length; empty bag: 0)
+ *   over the occurrences i of bag f*B+b of rows[r(inv[i])], r(u) =
+ *   row_of_unique[u] (device int32, or NULL for u); rows: device fp32
+ *   [*][D]; fp64 sums rounded once.
+ * recis_reduce_grad: for every unique key u of the batch's last
+ *   recis_batch_dedup, g(u) = the sum over its occurrences i of
+ *   grad_pooled[bag(i)] (x 1/length for MEAN) + grad_unpooled[i] (either may
+ *   be NULL), in occurrence order in fp64, rounded once, written to
+ *   grad_out[o(u)][0..D), o(u) = out_index[u] (device int32, or NULL for u). */
+recis_status recis_batch_dedup(recis_batch_t b, const int64_t* keys, int64_t N, int64_t* uniq_out,
+                               int32_t* inv_out, int64_t* U_out, recis_stream_t stream);
+recis_status recis_partition_keys(recis_batch_t b, const int64_t* keys, int64_t n, int32_t G,
+                                  uint64_t salt, int64_t* out_keys, int32_t* out_pos,
+                                  int64_t* counts_out, recis_stream_t stream);
+recis_status recis_pool_rows(const float* rows, const int32_t* row_of_unique, const int32_t* inv,
+                             const int64_t* bag_offsets, int32_t F, int64_t B, int32_t D,
+                             int32_t combiner, float* pooled_out, recis_stream_t stream);
+recis_status recis_reduce_grad(recis_batch_t b, const int64_t* bag_offsets, int32_t F, int64_t B,
+                               int32_t D, int32_t combiner, const float* grad_pooled,
+                               const float* grad_unpooled, const int32_t* out_index,
+                               float* grad_out, recis_stream_t stream);
+
 /* ------------------------------------------------------------------ test hooks */
 /* Process-wide settings that let tests reach error paths without faulting the
  * GPU.  The pages have no counterpart (they describe no failure handling).

@@ -149,6 +149,12 @@ struct recis_batch {
   int32_t* bag_of = nullptr;    // [capN] bag of every occurrence (written beside the dedup)
   int64_t* pocc = nullptr;      // [capN] IDMap result of each head, by sorted position (radix-sort path)
   int64_t capPocc = 0;
+  // table-less dedup of the sharded path (recis_batch_dedup, recis_reduce_grad)
+  int32_t* socc = nullptr;      // [capN] occurrence at each sorted position
+  recis::DevState* dstate_local = nullptr;  // status word of the batch's own calls
+  int64_t dedup_N = -1;         // occurrences of the last batch dedup (-1: none)
+  unsigned* part_hist = nullptr;  // recis_partition_keys: per-tile owner counts, then offsets
+  int64_t capPart = 0;
   int64_t capChunks = 0;
   cudaStream_t side = nullptr;  // bag preparation runs here, beside the dedup
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
@@ -252,6 +258,7 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
 cudaError_t launch_import(recis_table* t, const int64_t* keys, int64_t n, int64_t row0,
                           int64_t clock, cudaStream_t s);
 recis_status table_counts(recis_table* t, cudaStream_t s, int64_t* in_use, int64_t* live);
+recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D);
 cudaError_t launch_rehash(recis_table* t, const Slot* old_slots, int64_t old_cap, cudaStream_t s);
 
 int64_t pool_chunk_for(int64_t N, int D);

@@ -412,7 +412,7 @@ static cudaError_t realloc_dev(T*& p, size_t count, bool zero) {
 
 int64_t unique_tiles_for(int64_t N);
 
-static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D) {
+recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (b->dev >= 0 && b->dev != dev) {
@@ -445,6 +445,7 @@ static recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D
         (e = realloc_dev(b->gfirst, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->seg_counter, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->bag_of, cap, true)) != cudaSuccess ||
+        (e = realloc_dev(b->socc, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->multi_keys, cap / 2 + 1, false)) != cudaSuccess)
       return cuda_fail(e, "batch alloc");
     const int64_t st = (cap + kSortTile - 1) / kSortTile;
@@ -538,6 +539,9 @@ static void batch_free(recis_batch* b) {
   cudaFree(b->chunk_bag);
   cudaFree(b->bag_of);
   cudaFree(b->pocc);
+  cudaFree(b->socc);
+  cudaFree(b->part_hist);
+  cudaFree(b->dstate_local);
   if (b->side) cudaStreamDestroy(b->side);
   if (b->ev_fork) cudaEventDestroy(b->ev_fork);
   if (b->ev_join) cudaEventDestroy(b->ev_join);

@@ -34,7 +34,8 @@ EXPORTS = (
     "recis_profile_enable", "recis_profile_collect", "recis_launch_count",
     "recis_last_error_string", "recis_unique_static", "recis_table_read_rows",
     "recis_debug_set", "recis_plan_tables", "recis_table_reserve", "recis_table_save",
-    "recis_table_load", "recis_table_evict", "recis_table_clock",
+    "recis_table_load", "recis_table_evict", "recis_table_clock", "recis_batch_dedup",
+    "recis_partition_keys", "recis_pool_rows", "recis_reduce_grad",
 )
 DEBUG_SPIN_LIMIT, DEBUG_MAP_LIMIT = 1, 2
 
@@ -126,6 +127,10 @@ def load(path: str = LIB_PATH):
             "recis_table_load": [_vp, ctypes.c_char_p, _vp],
             "recis_table_evict": [_vp, _i64, _vp, _vp],
             "recis_table_clock": [_vp, _vp],
+            "recis_batch_dedup": [_vp, _vp, _i64, _vp, _vp, _vp, _vp],
+            "recis_partition_keys": [_vp, _vp, _i64, _i32, ctypes.c_uint64, _vp, _vp, _vp, _vp],
+            "recis_pool_rows": [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp],
+            "recis_reduce_grad": [_vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
