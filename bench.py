@@ -79,12 +79,27 @@ def _describe(w: W.Workload) -> str:
             f"fp32 tables [{tabs}]")
 
 
+def _workload(name: str, scale: int) -> W.Workload:
+    """The named workload, or for profiler captures the same recipe with a
+    batch 1/scale as large (and, for the large table, 1/(2 scale) of its live
+    rows)."""
+    w = W.WORKLOADS[name]
+    if scale <= 1:
+        return w
+    s = w.scaled(max(1, w.B // scale))
+    s.live_ids = w.live_ids // (2 * scale)
+    s.scale = scale
+    return s
+
+
 def _config(w: W.Workload, extra=None):
     c = {"workload": _describe(w), "F": w.F, "B": w.B,
          "tables": [{"dim": t.dim, "features": len(t.features), "optimizer": t.optimizer,
                      "combiner": t.combiner, "pooled": t.pooled, "unpooled": t.unpooled}
                     for t in w.tables],
          "l2": "flushed (256 MiB write) between timed steps", "parallelism": "replicas"}
+    if getattr(w, "scale", 1) > 1:
+        c["scale"] = f"batch 1/{w.scale} of the workload's (profiler capture case)"
     if extra:
         c.update(extra)
     return c
@@ -304,7 +319,7 @@ GROUPS = {
     "dedup": ("ss_rank", "ss_probe", "ss_count", "ss_tilescan", "ss_scatter", "ss_local", "ss_finish",
               "sort_hist", "sort_pass", "unique_insert"),
     "gather_pool": ("bag_prep", "gather_pool"),
-    "backward": ("seg_reduce", "row_update"),
+    "backward": ("seg_partial", "seg_combine", "row_update"),
 }
 
 
@@ -716,10 +731,10 @@ def run_gpu(args):
 
     subs = [] if args.subs in ("", "none") else [s for s in args.subs.split(",")
                                                  if s != args.workload]
-    line = measure(W.WORKLOADS[args.workload], args, R, dist, world, rank, dev, headline=True)
+    line = measure(_workload(args.workload, args.scale), args, R, dist, world, rank, dev, headline=True)
     sub_recs = {}
     for name in subs:
-        r = measure(W.WORKLOADS[name], args, R, dist, world, rank, dev, headline=False)
+        r = measure(_workload(name, args.scale), args, R, dist, world, rank, dev, headline=False)
         if r is not None:
             keep = ("value", "unit", "ms_per_step", "ms_per_step_p50", "ms_per_step_p90", "config",
                     "roofline", "step_alg_bytes", "step_alg_gbs", "step_frac_of_peak",
@@ -748,6 +763,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--small", action="store_true",
                     help="smaller table reservation (for profiler captures)")
+    ap.add_argument("--scale", type=int, default=1,
+                    help="run each workload with a batch 1/scale as large (profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "own":
         args.warmup = 3

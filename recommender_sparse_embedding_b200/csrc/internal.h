@@ -68,11 +68,12 @@ struct BatchDev {
   unsigned long long free_avail;// freed rows queued then (free_tail - free_head)
   unsigned int U;               // unique keys of the last lookup (0 when it was rejected)
   unsigned int n_new;           // new keys of the last lookup
-  unsigned int nlong;           // chunks of kShortSeg positions holding a long segment
+  unsigned int nseg_med;        // long segments cut by seg_reduce span ends, combined by one lane group
+  unsigned int nseg_huge;       // ... over many spans, combined by a whole CTA
+  unsigned int seg_work;        // work counter of the combine
   unsigned int nmulti;          // keys seen 2 to kShortSeg times (sample-sort path)
   unsigned int reject_call;     // call number of a lookup rejected as a whole (reserved key,
                                 // or its new keys overflow the row space)
-  unsigned int pad;
 };
 
 // ---------------------------------------------------------------- table
@@ -162,13 +163,12 @@ struct recis_batch {
   int cand_parity = 0;          // which candidate array the next call reads
   int64_t cand_n = 0;           // batch size that wrote it (0: none yet)
   int cand_splits = 0;          // its splitter slots (quantiles written: cand_splits - 1)
-  int32_t* seg_counter = nullptr;  // [capN] last-arrival counters (self-resetting)
   int32_t* bag_counter = nullptr;  // [capBags]
   double* partials = nullptr;
   float* gbuf = nullptr;          // [chunks][D] reduced gradients of long segments
-  int32_t* long_chunks = nullptr; // [chunks] chunks holding a long segment (sample-sort path)
   int32_t* multi_keys = nullptr;  // [N/2] unique keys seen 2 to kShortSeg times (sample-sort path)
-  int32_t* chunk_counter = nullptr;  // [chunks][2] block-level tickets of the backward
+  int2* long_segs = nullptr;      // [capSegs] {start, end} of long segments cut by span ends
+  int64_t capSegs = 0;
   int64_t capGbuf = 0;            // floats
   recis::BatchDev* bdev = nullptr;
   uint32_t epoch = 0;

@@ -5,14 +5,14 @@
 //
 // Bags are contiguous ranges of occurrences, so the forward is a segmented
 // reduction over occurrence order (segreduce.cuh): a group of G lanes owns a
-// chunk of C occurrences, each lane one 16-byte column of the row.  Rows
-// stream through a ring of R slots per lane in shared memory (cp.async), so R
-// row loads per lane are in flight while the group adds.  The bag
+// chunk of C occurrences, each lane one 16-byte column of the row.  The bag
 // preparation (beside the dedup) writes the bag of every occurrence; the
 // group resolves G positions at a time, one per lane (row, sorted position,
-// unique key, bag and its bounds, one sub-block ahead), writes their
-// gradient-source records lane-parallel, and marks the positions that end a
-// bag in one ballot, so the walk itself only adds rows and flushes at the
+// unique key, bag and its bounds, two sub-blocks ahead), writes their
+// gradient-source records lane-parallel, marks the positions that end a bag
+// in one ballot, and copies the sub-block's rows into shared memory by
+// cp.async at once (one round trip per sub-block), so the walk itself only
+// adds rows and flushes at the
 // marks.  A chunk whose bags all hold one occurrence (one-hot features) is a
 // plain gather.
 // Outputs: pooled rows [B][F][D] (sum, or mean = sum / length), optional
@@ -51,7 +51,16 @@ struct PoolParams {
   int32_t* counters;     // [nbags]
   DevState* st;
   HostMirror* mirror;
+  uint64_t b_magic;      // ceil(2^64 / B) for B >= 2 (quotient by B as a high multiply), 0 for B = 1
 };
+
+// j / B for 0 <= j < 2^32: floor(j * ceil(2^64 / B) / 2^64) is exact, the
+// rounding of the magic number adding less than 2^-32 to a quotient whose
+// fraction is at most 1 - 1/B (division by invariant integers using
+// multiplication, Granlund and Montgomery 1994).
+__device__ __forceinline__ int div_b(const PoolParams& p, int j) {
+  return p.b_magic ? (int)__umul64hi((unsigned long long)(unsigned)j, p.b_magic) : j;
+}
 
 // Bag preparation, one thread per bag (runs beside the dedup on a side
 // stream): checks the offsets, writes the bag of every occurrence and of every
@@ -97,10 +106,11 @@ __global__ void __launch_bounds__(256) bag_prep_kernel(const __grid_constant__ P
   }
 }
 
-// depth of the row ring: up to 8 rows, at most one sub-block (G) ahead
+// rows per lane staged at once by the bag walk: a sub-block (G), at most
+// 16 16-byte slots per lane
 template <int G, int VPL>
-__host__ __device__ constexpr int pool_ring() {
-  return (VPL >= 4 ? 2 : (VPL == 2 ? 4 : 8)) < G ? (VPL >= 4 ? 2 : (VPL == 2 ? 4 : 8)) : G;
+__host__ __device__ constexpr int pool_piece() {
+  return 16 / VPL < G ? 16 / VPL : G;
 }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -115,7 +125,6 @@ template <int G, int VPL>
 __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     pool_kernel(const __grid_constant__ PoolParams p) {
   pdl_wait();
-  constexpr int R = pool_ring<G, VPL>();  // rows in flight per group
   // all positions, bags and rows fit in 32 bits (N < 2^30, F*B < 2^31,
   // rows < 2^31), so the walk runs on 32-bit integers
   const int ncol = p.ncol;
@@ -180,7 +189,7 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
   // the pooled row of bag j (sum, or mean over its len occurrences)
   auto store_bag = [&](int j, int len) {
     if (!p.pooled) return;
-    const int f = j / B;
+    const int f = div_b(p, j);
     float4* o = reinterpret_cast<float4*>(p.pooled + (int64_t)((j - f * B) * F + f) * D);
     const double dlen = (double)len;
 #pragma unroll
@@ -199,23 +208,7 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     }
   };
 
-  // rows stream through a ring of R slots per lane in shared memory: row t+R
-  // is in flight (cp.async) while row t is added
-  extern __shared__ float4 s_ring[];  // [R][VPL][blockDim]
-  auto slot = [&](int r, int v) -> float4* {
-    return s_ring + ((r * VPL + v) * (int)blockDim.x + (int)threadIdx.x);
-  };
-  auto issue = [&](int t, int row) {
-    if (row >= 0) {
-      const float4* src = reinterpret_cast<const float4*>(p.row_data + (int64_t)row * p.row_floats);
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) {
-        const int col = g.lane + v * G;
-        if (col < ncol) cp_async16(slot(t % R, v), src + col);
-      }
-    }
-    cp_async_commit();
-  };
+  extern __shared__ float4 s_ring[];  // [groups][PR][VPL][G] staged rows of the bag walk
   const int m = p1 - p0;
 
   // A chunk whose bags each hold exactly one occurrence (one-hot features, or
@@ -235,7 +228,7 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
       int out = 0;  // pooled row b*F+f of this lane's bag
       if (s + g.lane < m) {
         const int j = j0 + s + g.lane;
-        const int f = j / B;
+        const int f = div_b(p, j);
         out = (j - f * B) * F + f;
         const int4 src = make_int4(out, 1, p0 + s + g.lane, 0);
         p.gsrc[ids.spos] = src;
@@ -283,10 +276,13 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     return;
   }
 
-  // The bag walk.  Per sub-block of G positions (one per lane, resolved one
-  // sub-block ahead): the positions' gradient sources are written by their
-  // own lanes, and `ends` marks the positions after which the running sum is
-  // flushed -- the last position of a bag, or of the chunk.
+  // The bag walk, one sub-block of G positions at a time (one per lane,
+  // resolved one sub-block ahead): the positions' gradient sources are
+  // written by their own lanes, and `ends` marks the positions after which
+  // the running sum is flushed -- the last position of a bag, or of the
+  // chunk.  The sub-block's rows are copied into shared memory by cp.async,
+  // PR rows per lane at once (one round trip), while the sub-block after the
+  // next one is resolved; then they are added in position order.
   auto flush_bag = [&](int j, int lo, int hi) {
     if (!(lo >= 0 && lo < hi && hi <= N)) {  // malformed bag offsets
       if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
@@ -302,44 +298,61 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
   auto emit = [&](int sub, const Ids& ids, const Bag& bg) {
     const int q = sub + g.lane;
     if (q < p1) {
-      const int f = bg.j / B;
+      const int f = div_b(p, bg.j);
       const int4 src = make_int4((bg.j - f * B) * F + f, bg.hi - bg.lo, q, 0);
       p.gsrc[ids.spos] = src;
       p.gfirst[ids.seg] = src;
     }
     return g.ballot(q < p1 && (q + 1 == bg.hi || q + 1 == p1));
   };
+  constexpr int PR = pool_piece<G, VPL>();  // rows per lane staged at once
+  float4* stage = s_ring + (size_t)(threadIdx.x / G) * PR * VPL * G;
   Ids cur_ids = ids0, nxt_ids = resolve(p0 + G);
   Bag cur_bag = bag_at(p0), nxt_bag = bag_at(p0 + G);
-  unsigned ends = emit(p0, cur_ids, cur_bag);
+  for (int sub = p0; sub < p1; sub += G) {
+    const unsigned ends = emit(sub, cur_ids, cur_bag);
+    const unsigned has_row = g.ballot(cur_ids.row >= 0);
+    const int cnt = p1 - sub < G ? p1 - sub : G;
+    Ids nn_ids{-1, 0, 0};
+    Bag nn_bag{0, 0, 0};
+    for (int r0 = 0; r0 < cnt; r0 += PR) {
+      const int pc = cnt - r0 < PR ? cnt - r0 : PR;
+      for (int u = 0; u < pc; ++u) {
+        const int row = g.bcast(cur_ids.row, r0 + u);
+        if (row >= 0) {
+          const float4* src = reinterpret_cast<const float4*>(p.row_data + (int64_t)row * p.row_floats);
 #pragma unroll
-  for (int t = 0; t < R; ++t) issue(t, t < m ? g.bcast(cur_ids.row, t) : -1);
-  for (int t = 0; t < m; ++t) {
-    const int ln = t % G;
-    const int row = g.bcast(cur_ids.row, ln);
-    cp_async_wait<R - 1>();
+          for (int v = 0; v < VPL; ++v) {
+            const int col = g.lane + v * G;
+            if (col < ncol) cp_async16(stage + (u * VPL + v) * G + g.lane, src + col);
+          }
+        }
+      }
+      cp_async_commit();
+      if (r0 == 0) {  // the sub-block after the next one, while the rows are in flight
+        nn_ids = resolve(sub + 2 * G);
+        nn_bag = bag_at(sub + 2 * G);
+      }
+      cp_async_wait<0>();
+      for (int u = 0; u < pc; ++u) {
+        const int t = r0 + u;
+        const bool ok = (has_row >> t) & 1u;
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      const int col = g.lane + v * G;
-      const float4 val = (row >= 0 && col < ncol) ? *slot(t % R, v) : f4_zero();
-      acc_add(acc[v], val);
-      if (p.unpooled && col < ncol)
-        __stcs(reinterpret_cast<float4*>(p.unpooled + (int64_t)(p0 + t) * D) + col, val);
+        for (int v = 0; v < VPL; ++v) {
+          const int col = g.lane + v * G;
+          const float4 val = (ok && col < ncol) ? stage[(u * VPL + v) * G + g.lane] : f4_zero();
+          acc_add(acc[v], val);
+          if (p.unpooled && col < ncol)
+            __stcs(reinterpret_cast<float4*>(p.unpooled + (int64_t)(sub + t) * D) + col, val);
+        }
+        if ((ends >> t) & 1u)
+          flush_bag(g.bcast(cur_bag.j, t), g.bcast(cur_bag.lo, t), g.bcast(cur_bag.hi, t));
+      }
     }
-    // the row R positions ahead (in this sub-block or the next) into the slot just read
-    const int ta = t + R;
-    int arow = -1;
-    if (ta < m) arow = (ta / G == t / G) ? g.bcast(cur_ids.row, ta % G) : g.bcast(nxt_ids.row, ta % G);
-    issue(ta, arow);
-    if ((ends >> ln) & 1u)
-      flush_bag(g.bcast(cur_bag.j, ln), g.bcast(cur_bag.lo, ln), g.bcast(cur_bag.hi, ln));
-    if (ln == G - 1 && t + 1 < m) {  // next sub-block
-      cur_ids = nxt_ids;
-      cur_bag = nxt_bag;
-      ends = emit(p0 + t + 1, cur_ids, cur_bag);
-      nxt_ids = resolve(p0 + t + 1 + G);
-      nxt_bag = bag_at(p0 + t + 1 + G);
-    }
+    cur_ids = nxt_ids;
+    cur_bag = nxt_bag;
+    nxt_ids = nn_ids;
+    nxt_bag = nn_bag;
   }
   pdl_trigger();
 }
@@ -349,7 +362,7 @@ static cudaError_t launch_pool_t(const PoolParams& p, cudaStream_t s) {
   const int64_t threads = p.nchunks * G;
   int64_t blocks = (threads + 255) / 256;
   if (blocks < 1) blocks = 1;
-  const size_t smem = (size_t)pool_ring<G, VPL>() * VPL * 256 * sizeof(float4);
+  const size_t smem = (size_t)pool_piece<G, VPL>() * VPL * 256 * sizeof(float4);
   const cudaError_t e =
       cudaFuncSetAttribute(pool_kernel<G, VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -406,6 +419,8 @@ static PoolParams pool_params(const LookupArgs& a, int64_t chunk) {
   p.counters = b->bag_counter;
   p.st = t->dstate;
   p.mirror = t->mirror_dev;
+  // ceil(2^64 / B) = floor((2^64 - 1) / B) + 1 (B >= 2; 2^64 itself for B = 1)
+  p.b_magic = a.B >= 2 ? ~0ULL / (uint64_t)a.B + 1 : 0;
   return p;
 }
 

@@ -296,7 +296,6 @@ struct SsParams {
   int32_t* seg_of;
   int32_t* seg_start;
   BatchDev* bdev;
-  int32_t* long_chunks;     // chunks (kShortSeg positions) holding a long segment
   int32_t* multi_keys;      // keys seen 2 to kShortSeg times (appended by ss_finish)
   DevState* st;
   HostMirror* mirror;
@@ -410,7 +409,9 @@ __global__ void __launch_bounds__(kCountThreads) ss_count_kernel(const __grid_co
     p.ctl->nbp = (unsigned)nbp;
     p.ctl->ticket_scan = 0;
     p.ctl->ticket_local = 0;
-    p.bdev->nlong = 0;
+    p.bdev->nseg_med = 0;  // the backward's long-segment lists start empty
+    p.bdev->nseg_huge = 0;
+    p.bdev->seg_work = 0;
     p.bdev->nmulti = 0;
     p.bdev->row_base = *(volatile unsigned long long*)&p.st->next_free;
     const unsigned long long fh = *(volatile unsigned long long*)&p.st->free_head;
@@ -1166,7 +1167,6 @@ struct FinishShared {
   int32_t init_row[kFinThreads * kFinItems];
   unsigned long long cpre[kMaxBucketSlots / 2];  // per local CTA: new keys << 32 | heads before it
   unsigned long long warp[kFinThreads / 32];
-  unsigned chunk_long;  // bit c: chunk c (kShortSeg positions) of this CTA holds a long segment
   int ninit;
   unsigned heads[kSub / 32];        // bit i: position i of this CTA is a head
   int32_t multi[kSub / 2];          // keys of this CTA seen 2 to kShortSeg times
@@ -1184,7 +1184,6 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   if (tid == 0) {
     sh.ninit = 0;
-    sh.chunk_long = 0;
     sh.nmulti = 0;
   }
   __syncthreads();
@@ -1226,7 +1225,6 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
     const int64_t q = q0 + j * kFinThreads;
     if (q >= p.N) break;
     const uint64_t m = mt[j];
-    if (m >> 63) atomicOr(&sh.chunk_long, 1u << ((tid + j * kFinThreads) / kShortSeg));
     const unsigned b = (unsigned)(m >> 44) & 0xfffu;
     const unsigned lh = (unsigned)(m & 0x1fffffULL);
     const unsigned long long cpre = p.finish_scans ? sh.cpre[b >> p.local_bpc_shift]
@@ -1288,22 +1286,11 @@ __global__ void __launch_bounds__(kFinThreads, 3) ss_finish_kernel(const __grid_
     }
   }
   if (sh_unclaim) atomicAdd(&p.st->slots_used, (unsigned long long)(0ULL - sh_unclaim));
-  // chunks of this CTA holding a long segment, for the backward's reduction,
-  // and its keys seen 2 to kShortSeg times
+  // this CTA's keys seen 2 to kShortSeg times, for the backward's row update
   __syncthreads();
   if (tid == 0 && sh.nmulti > 0) sh.multi_base = atomicAdd(&p.bdev->nmulti, (unsigned)sh.nmulti);
   __syncthreads();
   for (int i = tid; i < sh.nmulti; i += kFinThreads) p.multi_keys[sh.multi_base + i] = sh.multi[i];
-  if (w == 0 && !rejected) {
-    const bool has = (sh.chunk_long >> lane) & 1u;
-    const unsigned bal = __ballot_sync(0xffffffffu, has);
-    unsigned at = 0;
-    if (lane == 0 && bal) at = atomicAdd(&p.bdev->nlong, (unsigned)__popc(bal));
-    at = __shfl_sync(0xffffffffu, at, 0);
-    if (has)
-      p.long_chunks[at + __popc(bal & ((1u << lane) - 1u))] =
-          (int32_t)(blockIdx.x * (kSub / kShortSeg) + lane);
-  }
   // the next call's candidate splitters: quantiles of this call's sorted keys
   if (blockIdx.x == 0) {
     const unsigned long long N = (unsigned long long)p.N;
@@ -1416,7 +1403,6 @@ cudaError_t launch_sample_dedup(recis_batch* b, recis_table* t, const int64_t* k
   p.seg_of = b->seg_of;
   p.seg_start = b->seg_start;
   p.bdev = b->bdev;
-  p.long_chunks = b->long_chunks;
   p.multi_keys = b->multi_keys;
   p.st = t->dstate;
   p.mirror = t->mirror_dev;

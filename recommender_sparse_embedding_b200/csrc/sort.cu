@@ -120,6 +120,9 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restric
     const unsigned long long fh = *(volatile unsigned long long*)&st->free_head;
     bdev->free_base = fh;
     bdev->free_avail = *(volatile unsigned long long*)&st->free_tail - fh;
+    bdev->nseg_med = 0;  // the backward's long-segment lists start empty
+    bdev->nseg_huge = 0;
+    bdev->seg_work = 0;
     unsigned n = 0;
     for (int p = 0; p < kSortPasses; ++p) {
       ctl->active[p] = s_active[p];

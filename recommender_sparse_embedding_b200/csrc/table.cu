@@ -443,7 +443,6 @@ recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D) {
         (e = realloc_dev(b->spos, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->gsrc, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->gfirst, cap, true)) != cudaSuccess ||
-        (e = realloc_dev(b->seg_counter, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->bag_of, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->socc, cap, true)) != cudaSuccess ||
         (e = realloc_dev(b->multi_keys, cap / 2 + 1, false)) != cudaSuccess)
@@ -497,14 +496,20 @@ recis_status batch_ensure(recis_batch* b, int64_t N, int64_t nbags, int D) {
     if ((e = realloc_dev(b->partials, cap, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
     b->capPartials = cap;
   }
-  const int64_t gneed = ((N + cu - 1) / cu + 1) * (int64_t)D;
+  // reduced gradients of long segments: one row per kShortSeg positions (a
+  // long segment is the only one starting in its row's positions); the list
+  // of long segments crossing a span end: at most one per span
+  const int64_t gneed = ((N + kShortSeg - 1) / kShortSeg + 1) * (int64_t)D;
   if (gneed > b->capGbuf) {
     const int64_t cap = gneed + gneed / 4;
     if ((e = realloc_dev(b->gbuf, cap, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
-    if ((e = realloc_dev(b->long_chunks, cap / D + 1, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
-    if ((e = realloc_dev(b->chunk_counter, 2 * (cap / D + 1), true)) != cudaSuccess)
-      return cuda_fail(e, "batch alloc");
     b->capGbuf = cap;
+  }
+  const int64_t sneed = (N + cu - 1) / cu + 1;
+  if (sneed > b->capSegs) {
+    const int64_t cap = sneed + sneed / 4;
+    if ((e = realloc_dev(b->long_segs, cap, false)) != cudaSuccess) return cuda_fail(e, "batch alloc");
+    b->capSegs = cap;
   }
   return RECIS_OK;
 }
@@ -528,13 +533,11 @@ static void batch_free(recis_batch* b) {
   cudaFree(b->spos);
   cudaFree(b->gsrc);
   cudaFree(b->gfirst);
-  cudaFree(b->seg_counter);
   cudaFree(b->bag_counter);
   cudaFree(b->partials);
   cudaFree(b->gbuf);
-  cudaFree(b->long_chunks);
   cudaFree(b->multi_keys);
-  cudaFree(b->chunk_counter);
+  cudaFree(b->long_segs);
   cudaFree(b->bdev);
   cudaFree(b->chunk_bag);
   cudaFree(b->bag_of);

@@ -10,15 +10,15 @@
 // occurrence).  The gradient of u is
 //   g(u) = sum over its positions of grad_pooled[bag] * (1 or 1/length)
 //          + grad_unpooled[occurrence],
-// summed in fp64 in position order and rounded once to fp32.  Two launches:
-//   seg_reduce  segments longer than kShortSeg (hot keys) are cut into
-//               chunks of kChunk positions; each lane group sums its chunk's
-//               part of a segment into an fp64 partial; the group that
-//               arrives last adds the partials in chunk order (for a segment
-//               of more than 64 chunks, in two levels: per block of 32
-//               chunks, then the block sums in block order) and stores g(u)
-//               in gbuf at row seg_start[u] / kChunk (a long segment is the
-//               only long one starting in its chunk).
+// summed in fp64 in position order and rounded once to fp32.  Three launches:
+//   seg_partial  segments longer than kShortSeg (hot keys): the positions
+//                are cut into spans; each lane group sums its span's part
+//                of every long segment in fp64, storing g(u) in gbuf at row
+//                seg_start[u] / kChunk when the segment lies inside the span
+//                (a long segment is the only long one starting in its
+//                kChunk positions), else a partial;
+//   seg_combine  adds the partials of each segment cut by span ends in a
+//                fixed order and stores g(u) in gbuf;
 //   row_update  one lane group per unique key loads the row [emb | state],
 //               sums the key's gradient terms itself when the segment is
 //               short (all loads issued before the sum) or reads gbuf, and
@@ -30,32 +30,30 @@
 
 namespace recis {
 
-constexpr int kChunk = 16;  // seg_reduce positions per group (<= kShortSeg + 1)
-static_assert(kChunk <= kShortSeg + 1, "a chunk must hold at most one long segment start");
-static_assert(kChunk == kShortSeg, "the dedup lists long chunks of kShortSeg positions");
-constexpr int kCombineBlock = 32;  // chunks per block of the two-level combine
+constexpr int kChunk = 16;  // positions per gbuf row; seg_reduce spans are multiples of it
+static_assert(kChunk <= kShortSeg + 1, "kChunk positions must hold at most one long segment start");
+static_assert(kChunk == kShortSeg, "gbuf holds one row per kShortSeg positions");
 
 struct UpdateParams {
   int64_t N;
   int32_t ncol;             // D / 4
   int32_t mean;
   int32_t row_floats;
-  int64_t nchunks;          // seg_reduce chunks
+  int64_t span;             // seg_reduce positions per lane group (a multiple of kChunk)
   const int4* gsrc;         // [N] per sorted position: {gradient row, bag length, occurrence, 0}
   const int4* gfirst;       // [U] per unique key: gsrc of one of its occurrences
-  const uint64_t* meta;     // [N] per sorted position, bit 63: long segment (null: use seg_start)
-  const int32_t* long_chunks;  // chunks holding a long segment, bdev->nlong of them (or null)
   const int32_t* seg_of;    // [N] sorted position -> unique index
   const int32_t* seg_start; // [U+1]
   const int64_t* rows;      // [U]
-  const BatchDev* bdev;     // U of the lookup
+  BatchDev* bdev;           // U of the lookup; the long-segment list counters
   const float* gp;          // grad_pooled [B][F][D] or null
   const float* gu;          // grad_unpooled [N][D] or null
-  float* gbuf;              // [nchunks][D] reduced gradients of long segments
+  float* gbuf;              // [N / kChunk + 1][D] reduced gradients of long segments
   float* row_data;
-  double* partials;         // [nchunks][2][D]
-  int32_t* counters;        // [U] last-arrival tickets (self-resetting)
-  int32_t* chunk_counters;  // [nchunks][2] block-level tickets (self-resetting)
+  double* partials;         // [spans][2][D]
+  int2* long_segs;          // [seg_cap] long segments crossing a span end: the CTA-combined ones
+                            // from the back, the others from the front
+  int64_t seg_cap;
   const int32_t* multi_keys;  // keys seen 2 to kShortSeg times (bdev->nmulti of them), or null
   // optimiser
   float lr;        // Adagrad: lr; Adam: lr / (1 - beta1^t)
@@ -125,258 +123,337 @@ __device__ __forceinline__ void add_terms(const GroupCtx<G>& g, const UpdatePara
 }
 
 // ------------------------------------------------------------------ seg_reduce
-// One group per chunk of kChunk sorted positions.  Lanes resolve G positions
-// at a time: the long-segment mark (or, without marks, the segment's bounds),
-// the segment and the gradient source; positions of short segments are
-// skipped, so a chunk without a long segment ends after one load.  A chunk
-// meets at most two long segments (one ending, one starting); each gets one
-// partial per chunk, in slot 0 if it starts at or before the chunk's first
-// position, else slot 1.
-template <int G, int VPL, bool GP, bool GU>
-__device__ __forceinline__ void reduce_chunk(const GroupCtx<G>& g, const UpdateParams& p, int64_t chunk) {
-  const int64_t D = (int64_t)p.ncol * 4;
-  const int64_t p0 = chunk * kChunk;
-  const int64_t p1 = p0 + kChunk < p.N ? p0 + kChunk : p.N;
-  if (!p.meta && !p.long_chunks) {
-    // no marks from the dedup: a segment lying wholly inside the chunk is
-    // short (kChunk <= kShortSeg), so only the segments of the chunk's first
-    // and last positions can be long; a chunk where neither is ends here
-    bool lng = false;
-    for (int e = g.lane; e < 2; e += G) {
-      const int32_t sg = __ldg(p.seg_of + (e == 0 ? p0 : p1 - 1));
-      lng |= __ldg(p.seg_start + sg + 1) - __ldg(p.seg_start + sg) > kShortSeg;
-    }
-    if (!g.ballot(lng)) return;
-  }
-  Acc4 acc[VPL];
+// Long segments (more than kShortSeg positions: hot keys).  The sorted
+// positions are cut into spans of p.span positions (a multiple of kChunk),
+// one lane group per span.  The group walks its span a step of Q positions
+// (one or a few per lane) at a time, with three steps in flight: the rows
+// of step k, the segment bounds of step k+1 and the segments and gradient
+// sources of step k+2.  A position is long when its segment is; the
+// gradient rows of a step's long positions are copied into shared memory by
+// cp.async, up to PR positions at once (one slot per position, row and
+// lane), then added in position order into one fp64 sum per segment run.
+// A run's sum is
+//   - the segment's gradient, rounded once and stored in gbuf at row
+//     start / kChunk, when the segment lies inside the span;
+//   - else a partial of the span: slot 0 for the segment that began before
+//     the span, slot 1 for the one that begins in it and runs past its end.
+// seg_partial lists the segment as {start, end} at its first span;
+// seg_combine adds its partials in a fixed order -- slot 1 of its first
+// span, then slot 0 of each following span -- with one lane group, or for a
+// segment of many spans with a whole CTA: lane group j takes terms j,
+// j + groups, ..., and the groups' sums are added in group order.  No
+// tickets, fences or float atomics; the result does not depend on
+// scheduling.
+constexpr int kHugeTerms = 16;  // partials above which a whole CTA combines a segment
+
+// Positions per step: one per lane (at least kChunk, at most 4 per lane).
+template <int G>
+struct SegStep {
+  static constexpr int Q = G >= kChunk ? G : (4 * G < kChunk ? 4 * G : kChunk);
+  static constexpr int E = Q / G;  // positions per lane
+};
+
+// A step's positions, loaded in two stages: the segment and the gradient
+// source of each position, then its segment's bounds.
+template <int E>
+struct StepA {
+  int32_t seg[E];
+  int4 src[E];
+};
+template <int E>
+struct StepB {
+  int32_t seg[E], st[E], en[E];
+  int4 src[E];
+};
+
+// a[e] for a run-time e without local-memory indexing
+template <int E, typename T>
+__device__ __forceinline__ T pick(const T (&a)[E], int e) {
+  T v = a[0];
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
-  int32_t cur = -1;
-  int64_t cst = 0, cen = 0;
-  auto flush = [&]() {
-    // segments of up to two blocks of chunks: one last-arrival combine;
-    // longer ones (hot keys of long sequences): two levels
-    const bool two_level = (cen - 1) / kChunk - cst / kChunk >= 2 * kCombineBlock;
-    if (two_level ? combine_split2<G, VPL, VPL >= 4 ? 1 : 4 / VPL, kCombineBlock>(
-                        g, acc, p.partials, p.chunk_counters, p.counters, cur, chunk, cst <= p0, cst, cen,
-                        kChunk, p.ncol)
-                  : combine_split<G, VPL, VPL >= 4 ? 1 : 4 / VPL>(g, acc, p.partials, p.counters, cur, chunk,
-                                                                 cst <= p0, cst, cen, kChunk, p.ncol)) {
-      float4* dst = reinterpret_cast<float4*>(p.gbuf + (cst / kChunk) * D);
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) {
-        const int col = g.lane + v * G;
-        if (col < p.ncol) __stcg(dst + col, acc_round(acc[v]));
-      }
-    }
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
-  };
-  for (int64_t sub = p0; sub < p1; sub += G) {
-    const int64_t q = sub + g.lane;
-    bool maybe = q < p1;
-    if (maybe && p.meta) maybe = (__ldg(p.meta + q) >> 63) != 0;
-    if (!g.ballot(maybe)) continue;
-    int32_t seg = -1, st = 0, en = 0;
-    Src s{0, 0, 1.0};
-    if (maybe) {
-      seg = __ldg(p.seg_of + q);
-      s = make_src(p, __ldg(p.gsrc + q));
-      st = __ldg(p.seg_start + seg);
-      en = __ldg(p.seg_start + seg + 1);
-    }
-    const bool is_long = maybe && en - st > kShortSeg;
-    unsigned rest = g.ballot(is_long);
-    while (rest) {
-      const int a = __ffs(rest) - 1;
-      const int32_t sg = g.bcast(seg, a);
-      const unsigned same = g.ballot(is_long && seg == sg);  // lanes a .. a+cnt-1
-      const int cnt = __popc(same);
-      if (sg != cur) {
-        if (cur >= 0) flush();
-        cur = sg;
-        cst = g.bcast(st, a);
-        cen = g.bcast(en, a);
-      }
-      constexpr int K = kRowsInFlight<VPL, GP && GU>;
-      for (int k0 = 0; k0 < cnt; k0 += K)
-        add_terms<G, VPL, K, GP, GU>(g, p, s, a + k0, cnt - k0 < K ? cnt - k0 : K, acc);
-      rest &= ~same;
-    }
-  }
-  if (cur >= 0) flush();
+  for (int i = 1; i < E; ++i)
+    if (i == e) v = a[i];
+  return v;
 }
 
-// With the dedup's list of chunks holding a long segment, a persistent grid
-// of groups walks the list; without it, one group per chunk.
-// resident CTAs of 256 threads per SM of the long-segment reduction
-template <int VPL>
-constexpr int kSegReduceCtas = VPL == 1 ? 3 : (VPL == 2 ? 2 : 1);
-
-template <int G, int VPL, bool GP, bool GU>
-__global__ void __launch_bounds__(256, kSegReduceCtas<VPL>)
-    seg_reduce_kernel(const __grid_constant__ UpdateParams p) {
-  pdl_wait();
-  const GroupCtx<G> g;
-  const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
-  if (p.long_chunks) {
-    const int64_t n = (int64_t)p.bdev->nlong;
-    const int64_t groups = (int64_t)gridDim.x * blockDim.x / G;
-    for (int64_t i = gid; i < n; i += groups) reduce_chunk<G, VPL, GP, GU>(g, p, __ldg(p.long_chunks + i));
-  } else if (gid < p.nchunks) {
-    reduce_chunk<G, VPL, GP, GU>(g, p, gid);
+template <int G, int E>
+__device__ __forceinline__ void load_step_a(const GroupCtx<G>& g, const UpdateParams& p, int64_t base,
+                                            int64_t end, StepA<E>& a) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int64_t q = base + g.lane + e * G;
+    a.seg[e] = -1;
+    a.src[e] = make_int4(0, 1, 0, 0);
+    if (q < end) {
+      a.seg[e] = __ldg(p.seg_of + q);
+      a.src[e] = __ldg(p.gsrc + q);
+    }
   }
-  pdl_trigger();
 }
 
-// ------------------------------------------------------------------ seg_reduce, staged
-// The same reduction for one 16-byte column per lane (D = 4G) and one kind of
-// gradient (pooled or unpooled), G >= 8: groups walk the listed chunks (one
-// each when the grid covers the list); a chunk's positions are resolved by
-// the group (each lane kChunk / G of them), and the gradient rows of all its
-// long positions are copied into shared memory by cp.async at once, one slot
-// per position and lane, so a chunk costs one round trip for its rows instead
-// of one per few rows.  Each lane copies and reads back only its own columns.
+template <int E>
+__device__ __forceinline__ void load_step_b(const UpdateParams& p, const StepA<E>& a, StepB<E>& b) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    b.seg[e] = a.seg[e];
+    b.src[e] = a.src[e];
+    b.st[e] = b.en[e] = 0;
+    if (a.seg[e] >= 0) {
+      b.st[e] = __ldg(p.seg_start + a.seg[e]);
+      b.en[e] = __ldg(p.seg_start + a.seg[e] + 1);
+    }
+  }
+}
+
+// bit t (t = lane + e * G): position t of the step lies in a long segment
+template <int G, int E>
+__device__ __forceinline__ unsigned long_mask(const GroupCtx<G>& g, const StepB<E>& b) {
+  unsigned m = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) m |= g.ballot(b.seg[e] >= 0 && b.en[e] - b.st[e] > kShortSeg) << (e * G);
+  return m;
+}
+
 __device__ __forceinline__ void cp_async16_(void* smem, const void* gmem) {
   const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
 }
 
-template <int G>
-struct ChunkPos {
-  static constexpr int E = G >= kChunk ? 1 : kChunk / G;  // positions per lane
-  int32_t seg[E], st[E], en[E], src[E];
-  double scale[E];
-  unsigned mask;  // bit t: position t of the chunk is in a long segment
-};
-
-template <int G, bool GP>
-__device__ __forceinline__ void chunk_indices(const GroupCtx<G>& g, const UpdateParams& p, int64_t chunk,
-                                              ChunkPos<G>& c) {
-  constexpr int E = ChunkPos<G>::E;
-  const int64_t p0 = chunk * kChunk;
-  bool lng[E];
+template <int G, int VPL>
+__device__ __forceinline__ void store_gbuf(const GroupCtx<G>& g, const UpdateParams& p, int64_t start,
+                                           const Acc4 (&acc)[VPL]) {
+  float4* dst = reinterpret_cast<float4*>(p.gbuf + (start / kChunk) * (int64_t)p.ncol * 4);
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int t = g.lane + e * G;
-    const int64_t q = p0 + t;
-    lng[e] = false;
-    c.seg[e] = 0;
-    c.st[e] = c.en[e] = c.src[e] = 0;
-    c.scale[e] = 1.0;
-    if (chunk >= 0 && t < kChunk && q < p.N) {
-      const bool marked = p.meta ? (__ldg(p.meta + q) >> 63) != 0 : true;
-      const int32_t sg = __ldg(p.seg_of + q);
-      const int4 gs = __ldg(p.gsrc + q);
-      const int32_t a = __ldg(p.seg_start + sg), b = __ldg(p.seg_start + sg + 1);
-      lng[e] = marked && b - a > kShortSeg;
-      c.seg[e] = sg;
-      c.st[e] = a;
-      c.en[e] = b;
-      c.src[e] = GP ? gs.x : gs.z;
-      c.scale[e] = (GP && p.mean) ? 1.0 / (double)gs.y : 1.0;
-    }
+  for (int v = 0; v < VPL; ++v) {
+    const int col = g.lane + v * G;
+    if (col < p.ncol) __stcg(dst + col, acc_round(acc[v]));
   }
-  c.mask = 0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) c.mask |= g.ballot(lng[e]) << (e * G);
 }
 
-template <int G, bool GP>
-__global__ void __launch_bounds__(256, 3) seg_reduce_staged_kernel(const __grid_constant__ UpdateParams p) {
+// resident CTAs per SM (registers: several positions per lane for narrow
+// rows, many accumulators for wide ones)
+template <int G, int VPL>
+constexpr int kPartialCtas = VPL >= 4 ? 1 : (G < 8 ? 2 : 3);
+
+// Staging: kChunk 16-byte slots per lane, PR long positions' rows at a time.
+template <int G, int VPL, bool GP, bool GU>
+__global__ void __launch_bounds__(256, kPartialCtas<G, VPL>) seg_partial_kernel(const __grid_constant__ UpdateParams p) {
   pdl_wait();
-  constexpr int E = ChunkPos<G>::E;
+  constexpr int NRW = (GP && GU) ? 2 : 1;  // gradient rows per position
+  constexpr int PR = kChunk / (VPL * NRW) > 0 ? kChunk / (VPL * NRW) : 1;  // positions staged at once
+  constexpr int Q = SegStep<G>::Q, E = SegStep<G>::E;
   extern __shared__ float4 s_rows[];  // [groups of the CTA][kChunk][G]
   const GroupCtx<G> g;
   float4* rows = s_rows + (size_t)(threadIdx.x / G) * kChunk * G;
-  const int64_t groups = (int64_t)gridDim.x * blockDim.x / G;
-  const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
-  const int64_t n = (int64_t)p.bdev->nlong;
+  const int64_t span = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  const int64_t p0 = span * p.span;
+  if (p0 >= p.N) return;
+  const int64_t p1 = p0 + p.span < p.N ? p0 + p.span : p.N;
   const int64_t D = (int64_t)p.ncol * 4;
-  const float* grad = GP ? p.gp : p.gu;
-  auto chunk_of = [&](int64_t i) -> int64_t { return i < n ? (int64_t)__ldg(p.long_chunks + i) : -1; };
-  ChunkPos<G> cur;
-  int64_t i = gid;
-  int64_t chunk = chunk_of(i);
-  chunk_indices<G, GP>(g, p, chunk, cur);
-  while (chunk >= 0) {
-    // this chunk's gradient rows into shared memory
-    for (unsigned m = cur.mask; m; m &= m - 1) {
-      const int t = __ffs(m) - 1;
-      const int32_t src = g.bcast(t / G == 0 ? cur.src[0] : cur.src[E - 1], t % G);
-      if (g.lane < p.ncol) cp_async16_(rows + t * G + g.lane, grad + (int64_t)src * D + 4 * g.lane);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    // the next chunk's positions meanwhile
-    const int64_t next = chunk_of(i + groups);
-    ChunkPos<G> nxt;
-    chunk_indices<G, GP>(g, p, next, nxt);
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    // the long positions in order, one segment run at a time
-    const int64_t p0 = chunk * kChunk;
-    Acc4 acc = acc_zero();
-    int32_t sg = -1, cst = 0, cen = 0;
-    auto flush = [&]() {
-      Acc4 a1[1] = {acc};
-      const bool two_level = (cen - 1) / kChunk - cst / kChunk >= 2 * kCombineBlock;
-      if (two_level ? combine_split2<G, 1, 2, kCombineBlock>(g, a1, p.partials, p.chunk_counters, p.counters,
-                                                            sg, chunk, cst <= p0, cst, cen, kChunk, p.ncol)
-                    : combine_split<G, 1, 2>(g, a1, p.partials, p.counters, sg, chunk, cst <= p0, cst, cen,
-                                             kChunk, p.ncol)) {
-        if (g.lane < p.ncol) __stcg(reinterpret_cast<float4*>(p.gbuf + (cst / kChunk) * D) + g.lane,
-                                    acc_round(a1[0]));
+  Acc4 acc[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
+  int32_t cur = -1, cst = 0, cen = 0;
+  auto flush = [&]() {
+    if (cst >= p0 && cen <= p1) {
+      store_gbuf<G, VPL>(g, p, cst, acc);
+    } else {
+      const int slot = cst < p0 ? 0 : 1;
+      double2* dst = reinterpret_cast<double2*>(p.partials + (span * 2 + slot) * D);
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int col = g.lane + v * G;
+        if (col < p.ncol) {
+          __stcg(dst + 2 * col, make_double2(acc[v].x, acc[v].y));
+          __stcg(dst + 2 * col + 1, make_double2(acc[v].z, acc[v].w));
+        }
       }
-      acc = acc_zero();
-    };
-    for (unsigned m = cur.mask; m; m &= m - 1) {
-      const int t = __ffs(m) - 1;
-      const int e = t / G, l = t % G;
-      const int32_t s = g.bcast(e == 0 ? cur.seg[0] : cur.seg[E - 1], l);
-      if (s != sg) {
-        if (sg >= 0) flush();
-        sg = s;
-        cst = g.bcast(e == 0 ? cur.st[0] : cur.st[E - 1], l);
-        cen = g.bcast(e == 0 ? cur.en[0] : cur.en[E - 1], l);
-      }
-      const double sc = g.bcast(e == 0 ? cur.scale[0] : cur.scale[E - 1], l);
-      if (g.lane < p.ncol) {
-        const float4 v = rows[t * G + g.lane];
-        acc.x += (double)v.x * sc;
-        acc.y += (double)v.y * sc;
-        acc.z += (double)v.z * sc;
-        acc.w += (double)v.w * sc;
+      // listed at its first span: segments of many spans from the back
+      if (slot == 1 && g.lane == 0) {
+        if ((cen - 1) / p.span - cst / p.span + 1 > kHugeTerms)
+          p.long_segs[p.seg_cap - 1 - atomicAdd(&p.bdev->nseg_huge, 1u)] = make_int2(cst, cen);
+        else
+          p.long_segs[atomicAdd(&p.bdev->nseg_med, 1u)] = make_int2(cst, cen);
       }
     }
-    if (sg >= 0) flush();
-    i += groups;
-    chunk = next;
-    cur = nxt;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
+  };
+  // three steps in flight: rows of step k, bounds of step k+1, segments of step k+2
+  StepA<E> a1, a2;
+  StepB<E> cur_b, nxt_b;
+  load_step_a<G, E>(g, p, p0, p1, a1);
+  load_step_b<E>(p, a1, cur_b);
+  load_step_a<G, E>(g, p, p0 + Q, p1, a1);
+  unsigned mask = long_mask<G, E>(g, cur_b);
+  for (int64_t base = p0; base < p1; base += Q) {
+    bool ahead = false;  // next steps' loads issued
+    unsigned rem = mask;
+    do {
+      // the next PR long positions of the step: rows into shared memory
+      unsigned piece = 0;
+      {
+        unsigned r = rem;
+        for (int u = 0; u < PR && r; ++u) {
+          piece |= r & (0u - r);
+          r &= r - 1;
+        }
+      }
+      rem &= ~piece;
+      int u = 0;
+      for (unsigned m = piece; m; m &= m - 1, ++u) {
+        const int t = __ffs(m) - 1;
+        const int e = t / G, l = t % G;
+        const int4 sv = pick(cur_b.src, e);
+        if (GP) {
+          const float* r = p.gp + (int64_t)g.bcast(sv.x, l) * D;
+#pragma unroll
+          for (int v = 0; v < VPL; ++v) {
+            const int col = g.lane + v * G;
+            if (col < p.ncol) cp_async16_(rows + ((u * NRW) * VPL + v) * G + g.lane, r + 4 * col);
+          }
+        }
+        if (GU) {
+          const float* r = p.gu + (int64_t)g.bcast(sv.z, l) * D;
+#pragma unroll
+          for (int v = 0; v < VPL; ++v) {
+            const int col = g.lane + v * G;
+            if (col < p.ncol)
+              cp_async16_(rows + ((u * NRW + (GP ? 1 : 0)) * VPL + v) * G + g.lane, r + 4 * col);
+          }
+        }
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      if (!ahead) {
+        load_step_b<E>(p, a1, nxt_b);
+        load_step_a<G, E>(g, p, base + 2 * Q, p1, a2);
+        ahead = true;
+      }
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      // the piece's positions in order, one segment run at a time
+      u = 0;
+      for (unsigned m = piece; m; m &= m - 1, ++u) {
+        const int t = __ffs(m) - 1;
+        const int e = t / G, l = t % G;
+        const int32_t sg = g.bcast(pick(cur_b.seg, e), l);
+        if (sg != cur) {
+          if (cur >= 0) flush();
+          cur = sg;
+          cst = g.bcast(pick(cur_b.st, e), l);
+          cen = g.bcast(pick(cur_b.en, e), l);
+        }
+        const double sc = (GP && p.mean) ? 1.0 / (double)g.bcast(pick(cur_b.src, e).y, l) : 1.0;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+          const int col = g.lane + v * G;
+          if (col < p.ncol) {
+            const float4 x = GP ? rows[((u * NRW) * VPL + v) * G + g.lane] : f4_zero();
+            const float4 y = GU ? rows[((u * NRW + (GP ? 1 : 0)) * VPL + v) * G + g.lane] : f4_zero();
+            // one term per position: pooled gradient * scale + unpooled gradient
+            acc[v].x += (GP ? (double)x.x * sc : 0.0) + (GU ? (double)y.x : 0.0);
+            acc[v].y += (GP ? (double)x.y * sc : 0.0) + (GU ? (double)y.y : 0.0);
+            acc[v].z += (GP ? (double)x.z * sc : 0.0) + (GU ? (double)y.z : 0.0);
+            acc[v].w += (GP ? (double)x.w * sc : 0.0) + (GU ? (double)y.w : 0.0);
+          }
+        }
+      }
+    } while (rem);
+    cur_b = nxt_b;
+    a1 = a2;
+    mask = long_mask<G, E>(g, cur_b);
   }
+  if (cur >= 0) flush();
   pdl_trigger();
 }
 
-// Chunks of kChunk positions holding a position of a long segment, listed
-// for the staged reduction when the dedup listed none (the radix path): only
-// the segments of a chunk's first and last positions can be long (a segment
-// lying wholly inside a chunk is short).  The list's order depends on
-// scheduling; every chunk's partial and every combine do not.
-__global__ void __launch_bounds__(256) list_long_chunks_kernel(const __grid_constant__ UpdateParams p,
-                                                               int32_t* out, BatchDev* bdev) {
-  pdl_wait();
-  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  bool lng = false;
-  if (c < p.nchunks) {
-    const int64_t p0 = c * kChunk, p1 = p0 + kChunk < p.N ? p0 + kChunk : p.N;
-    const int32_t a = __ldg(p.seg_of + p0), b = __ldg(p.seg_of + p1 - 1);
-    lng = __ldg(p.seg_start + a + 1) - __ldg(p.seg_start + a) > kShortSeg ||
-          __ldg(p.seg_start + b + 1) - __ldg(p.seg_start + b) > kShortSeg;
+__device__ __forceinline__ int64_t min_i64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// Terms i = i0, i0 + stride, ... (< n) of a listed segment whose first span
+// is c0, added in that order: term 0 is slot 1 of span c0, term i slot 0 of
+// span c0 + i; NB terms' loads in flight at a time.
+template <int G, int VPL, int NB>
+__device__ __forceinline__ void add_span_partials(const GroupCtx<G>& g, const UpdateParams& p, int64_t c0,
+                                                  int64_t n, int64_t i0, int64_t stride, Acc4 (&acc)[VPL]) {
+  const int64_t D = (int64_t)p.ncol * 4;
+  for (int64_t ib = i0; ib < n; ib += NB * stride) {
+    double2 pa[NB][VPL], pb[NB][VPL];
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      const int64_t i = ib + t * stride;
+      const double2* src = reinterpret_cast<const double2*>(p.partials + ((c0 + i) * 2 + (i == 0 ? 1 : 0)) * D);
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int col = g.lane + v * G;
+        if (i < n && col < p.ncol) {
+          pa[t][v] = __ldcg(src + 2 * col);
+          pb[t][v] = __ldcg(src + 2 * col + 1);
+        } else {
+          pa[t][v] = make_double2(0.0, 0.0);
+          pb[t][v] = make_double2(0.0, 0.0);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      if (ib + t * stride >= n) break;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) acc_add(acc[v], Acc4{pa[t][v].x, pa[t][v].y, pb[t][v].x, pb[t][v].y});
+    }
   }
-  const unsigned bal = __ballot_sync(0xffffffffu, lng);
-  const int lane = threadIdx.x & 31;
-  unsigned at = 0;
-  if (lane == 0 && bal) at = atomicAdd(&bdev->nlong, (unsigned)__popc(bal));
-  at = __shfl_sync(0xffffffffu, at, 0);
-  if (lng) out[at + __popc(bal & ((1u << lane) - 1u))] = (int32_t)c;
+}
+
+// A persistent grid takes work items from a counter: first the segments of
+// many spans (one CTA each), then the others (one lane group each, a CTA's
+// groups taking consecutive list entries).
+template <int G, int VPL>
+__global__ void __launch_bounds__(256) seg_combine_kernel(const __grid_constant__ UpdateParams p) {
+  pdl_wait();
+  constexpr int NB = VPL >= 4 ? 2 : 4;
+  const GroupCtx<G> g;
+  const int grp = threadIdx.x / G, ngrp = blockDim.x / G;
+  const int64_t cap = p.seg_cap;
+  const int64_t spans = (p.N + p.span - 1) / p.span;
+  int64_t nmed = p.bdev->nseg_med, nhuge = p.bdev->nseg_huge;
+  if (nmed > cap) nmed = cap;
+  if (nhuge > cap - nmed) nhuge = cap - nmed;
+  const int64_t items = nhuge + (nmed + ngrp - 1) / ngrp;
+  __shared__ unsigned s_item;
+  extern __shared__ Acc4 s_part[];  // [groups][VPL][G]
+  for (;;) {
+    __syncthreads();  // the previous item's s_part and s_item are read
+    if (threadIdx.x == 0) s_item = atomicAdd(&p.bdev->seg_work, 1u);
+    __syncthreads();
+    const int64_t item = s_item;
+    if (item >= items) break;
+    Acc4 acc[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
+    if (item < nhuge) {
+      const int2 sg = p.long_segs[cap - 1 - item];
+      const int64_t c0 = sg.x / p.span, n = min_i64((sg.y - 1) / p.span + 1, spans) - c0;
+      add_span_partials<G, VPL, NB>(g, p, c0, n, grp, ngrp, acc);
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) s_part[(grp * VPL + v) * G + g.lane] = acc[v];
+      __syncthreads();
+      if (grp == 0) {
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) acc[v] = acc_zero();
+        for (int j = 0; j < ngrp; ++j) {
+#pragma unroll
+          for (int v = 0; v < VPL; ++v) acc_add(acc[v], s_part[(j * VPL + v) * G + g.lane]);
+        }
+        store_gbuf<G, VPL>(g, p, sg.x, acc);
+      }
+    } else {
+      const int64_t j = (item - nhuge) * ngrp + grp;
+      if (j < nmed) {
+        const int2 sg = p.long_segs[j];
+        const int64_t c0 = sg.x / p.span, n = min_i64((sg.y - 1) / p.span + 1, spans) - c0;
+        add_span_partials<G, VPL, NB>(g, p, c0, n, 0, 1, acc);
+        store_gbuf<G, VPL>(g, p, sg.x, acc);
+      }
+    }
+  }
   pdl_trigger();
 }
 
@@ -661,37 +738,48 @@ __global__ void __launch_bounds__(256, 2) row_update_wide_kernel(const __grid_co
 // ------------------------------------------------------------------ host
 int group_lanes_for(int D);
 
-int64_t update_chunk_for(int64_t, int) { return kChunk; }
+// seg_reduce span: kChunk * 2^k positions (at most 8 steps), as long as 16K
+// lane groups remain to fill the GPU
+int64_t update_chunk_for(int64_t N, int) {
+  int64_t span = kChunk;
+  while (span < 8 * kChunk && (N + 2 * span - 1) / (2 * span) >= 16384) span *= 2;
+  return span;
+}
+
+// sets a kernel's dynamic shared memory limit once per device
+template <typename K>
+static cudaError_t smem_attr(K kernel, size_t smem, bool (&done)[64]) {
+  if (smem <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  return e;
+}
 
 template <int G, int VPL, bool GP, bool GU>
 static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t ucap, cudaStream_t s) {
-  if constexpr (VPL == 1 && G >= 8 && GP != GU) {
-    if (p.long_chunks) {
-      constexpr size_t smem = (size_t)256 * kChunk * sizeof(float4);  // one slot per position and lane
-      static bool attr[64] = {false};
-      int dev = 0;
-      cudaGetDevice(&dev);
-      if (dev < 0 || dev >= 64 || !attr[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(seg_reduce_staged_kernel<G, GP>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr[dev] = true;
-      }
-      // one group per chunk (the list holds at most nchunks; groups past its
-      // length return at once): many groups in flight hide the combines'
-      // fences and ticket round trips
-      LaunchScope ls("seg_reduce", s);
-      const int64_t blocks = (p.nchunks * G + 255) / 256;
-      const cudaError_t e = launch_pdl(seg_reduce_staged_kernel<G, GP>, (unsigned)(blocks < 1 ? 1 : blocks), 256,
-                                       smem, s, p);
+  {
+    // one lane group per span; one staging slot per position, row and lane
+    constexpr size_t smem = (size_t)256 * kChunk * sizeof(float4);
+    static bool attr[64] = {false};
+    cudaError_t e = smem_attr(seg_partial_kernel<G, VPL, GP, GU>, smem, attr);
+    if (e != cudaSuccess) return e;
+    const int64_t spans = (p.N + p.span - 1) / p.span;
+    const int64_t blocks = (spans * G + 255) / 256;
+    {
+      LaunchScope ls("seg_partial", s);
+      e = launch_pdl(seg_partial_kernel<G, VPL, GP, GU>, (unsigned)(blocks < 1 ? 1 : blocks), 256, smem, s, p);
       if (e != cudaSuccess) return e;
     }
-  } else {
-    int64_t blocks = (p.nchunks * G + 255) / 256;
-    if (p.long_chunks && blocks > kSegReduceCtas<VPL> * kSMs) blocks = kSegReduceCtas<VPL> * kSMs;
-    if (blocks < 1) blocks = 1;
-    LaunchScope ls("seg_reduce", s);
-    const cudaError_t e = launch_pdl(seg_reduce_kernel<G, VPL, GP, GU>, (unsigned)blocks, 256, 0, s, p);
+    constexpr size_t csmem = (size_t)256 * VPL * sizeof(Acc4);
+    static bool cattr[64] = {false};
+    if ((e = smem_attr(seg_combine_kernel<G, VPL>, csmem, cattr)) != cudaSuccess) return e;
+    int64_t cblocks = 4 * (int64_t)kSMs;
+    if (cblocks > spans) cblocks = spans;
+    LaunchScope ls("seg_combine", s);
+    e = launch_pdl(seg_combine_kernel<G, VPL>, (unsigned)(cblocks < 1 ? 1 : cblocks), 256, csmem, s, p);
     if (e != cudaSuccess) return e;
   }
   // persistent: as many CTAs as fit at once (U is known only on the device)
@@ -735,19 +823,17 @@ static cudaError_t launch_update_t(const UpdateParams& p, bool adam, int64_t uca
 }
 
 cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pooled,
-                          const float* grad_unpooled, int64_t, float lr_t, float inv_sqrt_bc2,
+                          const float* grad_unpooled, int64_t span, float lr_t, float inv_sqrt_bc2,
                           cudaStream_t s) {
   UpdateParams p;
   p.N = b->N;
   p.ncol = t->D / 4;
   p.mean = b->combiner == RECIS_MEAN;
   p.row_floats = t->row_floats;
-  p.nchunks = (b->N + kChunk - 1) / kChunk;
+  p.span = span;
   p.gsrc = b->gsrc;
   p.gfirst = b->gfirst;
-  // long-segment marks and the long-chunk list come from the sample-sort dedup
-  p.meta = b->N <= kSampleSortMaxN ? b->ss_meta : nullptr;
-  p.long_chunks = b->N <= kSampleSortMaxN ? b->long_chunks : nullptr;
+  // keys seen 2 to kShortSeg times are listed by the sample-sort dedup
   p.multi_keys = b->N <= kSampleSortMaxN ? b->multi_keys : nullptr;
   p.seg_of = b->seg_of;
   p.seg_start = b->seg_start;
@@ -758,8 +844,8 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.gbuf = b->gbuf;
   p.row_data = reinterpret_cast<float*>(t->rows.va);
   p.partials = b->partials;
-  p.counters = b->seg_counter;
-  p.chunk_counters = b->chunk_counter;
+  p.long_segs = b->long_segs;
+  p.seg_cap = b->capSegs;
   p.lr = lr_t;
   p.eps = (float)t->cfg.eps;
   p.beta1 = (float)t->cfg.beta1;
@@ -768,15 +854,6 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.omb2 = (float)(1.0 - t->cfg.beta2);
   p.inv_sqrt_bc2 = inv_sqrt_bc2;
   if (p.N == 0) return cudaSuccess;
-  if (!p.long_chunks) {
-    // the radix-path dedup lists no chunks: list those holding a long segment
-    cudaError_t e = cudaMemsetAsync(&b->bdev->nlong, 0, sizeof(unsigned), s);
-    if (e != cudaSuccess) return e;
-    LaunchScope ls("list_long", s);
-    list_long_chunks_kernel<<<(unsigned)((p.nchunks + 255) / 256), 256, 0, s>>>(p, b->long_chunks, b->bdev);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    p.long_chunks = b->long_chunks;
-  }
   const bool adam = t->cfg.optimizer == RECIS_ADAM;
   const int64_t ucap = b->N;  // U <= N; groups past U return at once
   const int ncol = p.ncol;

@@ -253,6 +253,29 @@ def test_hot_key_among_others(R):
     _single(R, keys, np.ones(N, np.int64), D=16, opt="adam", grad_signed=True)
 
 
+@pytest.mark.parametrize("D,opt,comb,unpooled", [(4, "adagrad", "sum", False), (8, "adam", "mean", True),
+                                                  (64, "adam", "sum", False), (256, "adam", "sum", True),
+                                                  (1024, "adagrad", "mean", False)])
+def test_long_segments_over_many_spans(R, D, opt, comb, unpooled):
+    # over 524K occurrences: the long-segment reduction walks spans of more
+    # than one 16-position chunk; keys of 20K occurrences span hundreds of
+    # spans (combined by a whole CTA), keys of 300 or 40 a few (one lane
+    # group), the rest are short; multi-hot bags, signed gradients
+    rng = np.random.default_rng(21)
+    keys = np.concatenate([np.repeat(np.arange(24, dtype=np.int64) * 1_000_003 + 11, 20_000),
+                           np.repeat(np.arange(100, dtype=np.int64) * 7_919 + 3, 300),
+                           np.repeat(np.arange(1000, dtype=np.int64) * 104_729 + 5, 40),
+                           rng.integers(1 << 20, 1 << 44, size=100_000 if D <= 256 else 20_000)])
+    keys = keys[rng.permutation(len(keys))]
+    lengths = rng.integers(1, 9, size=len(keys))
+    ends = np.cumsum(lengths)
+    last = int(np.searchsorted(ends, len(keys)))
+    lengths = lengths[: last + 1]
+    lengths[-1] -= ends[last] - len(keys)
+    assert lengths.min() > 0 and lengths.sum() == len(keys)
+    _single(R, keys, lengths, D=D, opt=opt, comb=comb, unpooled=unpooled, grad_signed=True)
+
+
 def test_all_new_then_all_old(R):
     keys = np.arange(50_000, dtype=np.int64) * 1_000_003
     _single(R, keys[::-1].copy(), np.ones(50_000, np.int64), D=8, steps=3)
