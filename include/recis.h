@@ -25,6 +25,11 @@
  *   - Device pointers are raw CUDA device addresses owned by the caller; they
  *     must stay valid until the work of the call has finished on the stream.
  *     Host pointers are plain host memory, read before the call returns.
+ *   - Device arrays are moved with vector loads and copies, so they must be
+ *     aligned: float row arrays (pooled and unpooled rows, gradients) to 16
+ *     bytes, int64 arrays (keys, offsets, rows) to 8, int32 arrays to 4.  A
+ *     misaligned pointer is rejected on the host with RECIS_ERR_INVALID_ARG
+ *     before any work is queued.
  *   - Device-detected errors (reserved key, table full, value too wide for its
  *     tag) are reported by recis_table_status_sync(), and by the first later
  *     call on the same table that finds the earlier work finished.

@@ -189,6 +189,11 @@ namespace recis {
 
 void set_error(const std::string& msg);
 
+// Device arrays are read and written with vector loads and copies: int64
+// arrays must be 8-byte aligned, float rows 16-byte aligned.  True when p
+// (non-null) is not a multiple of `bytes`, a power of two.
+inline bool misaligned(const void* p, uintptr_t bytes) { return ((uintptr_t)p & (bytes - 1)) != 0; }
+
 // Test hooks (recis_debug_set): the bound of the device-side spin-waits, and
 // a cap on the EmbeddingBlock bytes a table may map (0 = none).
 int spin_limit();

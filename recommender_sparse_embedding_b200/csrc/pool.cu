@@ -51,6 +51,7 @@ struct PoolParams {
   int32_t* counters;     // [nbags]
   DevState* st;
   HostMirror* mirror;
+  int spin_max;          // polls before a wait gives up
   uint64_t b_magic;      // ceil(2^64 / B) for B >= 2 (quotient by B as a high multiply), 0 for B = 1
 };
 
@@ -121,7 +122,9 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int G, int VPL>
+// TMA: the bag walk's rows are copied by the bulk-copy engine (EmbeddingBlocks
+// in device memory), else by cp.async.
+template <int G, int VPL, bool TMA>
 __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     pool_kernel(const __grid_constant__ PoolParams p) {
   pdl_wait();
@@ -307,6 +310,14 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
   };
   constexpr int PR = pool_piece<G, VPL>();  // rows per lane staged at once
   float4* stage = s_ring + (size_t)(threadIdx.x / G) * PR * VPL * G;
+  __shared__ uint64_t s_mbar[256];  // TMA: one transaction barrier per group
+  uint64_t* mbar = s_mbar + threadIdx.x / G;
+  unsigned phase = 0;
+  const unsigned row_bytes = (unsigned)ncol * 16u;
+  if (TMA) {
+    if (g.lane == 0) mbar_init(mbar, 1);
+    __syncwarp(g.mask);
+  }
   Ids cur_ids = ids0, nxt_ids = resolve(p0 + G);
   Bag cur_bag = bag_at(p0), nxt_bag = bag_at(p0 + G);
   for (int sub = p0; sub < p1; sub += G) {
@@ -317,23 +328,48 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     Bag nn_bag{0, 0, 0};
     for (int r0 = 0; r0 < cnt; r0 += PR) {
       const int pc = cnt - r0 < PR ? cnt - r0 : PR;
-      for (int u = 0; u < pc; ++u) {
-        const int row = g.bcast(cur_ids.row, r0 + u);
-        if (row >= 0) {
-          const float4* src = reinterpret_cast<const float4*>(p.row_data + (int64_t)row * p.row_floats);
+      unsigned nrows = 0;
+      if (TMA) {
+        // each lane copies its own position's row, one bulk copy
+        const bool mine = g.lane >= r0 && g.lane < r0 + pc && cur_ids.row >= 0;
+        nrows = (unsigned)__popc(g.ballot(mine));
+        if (nrows) {
+          __syncwarp(g.mask);  // the group has read the previous piece
+          fence_async_smem();
+          if (g.lane == 0) mbar_arrive_expect(mbar, nrows * row_bytes);
+          if (mine)
+            bulk_row(stage + (g.lane - r0) * VPL * G, p.row_data + (int64_t)cur_ids.row * p.row_floats, row_bytes,
+                     mbar);
+        }
+      } else {
+        for (int u = 0; u < pc; ++u) {
+          const int row = g.bcast(cur_ids.row, r0 + u);
+          if (row >= 0) {
+            const float4* src = reinterpret_cast<const float4*>(p.row_data + (int64_t)row * p.row_floats);
 #pragma unroll
-          for (int v = 0; v < VPL; ++v) {
-            const int col = g.lane + v * G;
-            if (col < ncol) cp_async16(stage + (u * VPL + v) * G + g.lane, src + col);
+            for (int v = 0; v < VPL; ++v) {
+              const int col = g.lane + v * G;
+              if (col < ncol) cp_async16(stage + (u * VPL + v) * G + g.lane, src + col);
+            }
           }
         }
+        cp_async_commit();
       }
-      cp_async_commit();
       if (r0 == 0) {  // the sub-block after the next one, while the rows are in flight
         nn_ids = resolve(sub + 2 * G);
         nn_bag = bag_at(sub + 2 * G);
       }
-      cp_async_wait<0>();
+      if (!TMA) {
+        cp_async_wait<0>();
+      } else if (nrows) {
+        if (!mbar_wait(mbar, phase, p.spin_max)) {
+          // the copies did not land in time: reported, and waited for once
+          // more before the slots are read or written again
+          if (g.lane == 0) raise_error(p.st, p.mirror, kErrTimeout);
+          mbar_wait(mbar, phase, p.spin_max);
+        }
+        phase ^= 1u;
+      }
       for (int u = 0; u < pc; ++u) {
         const int t = r0 + u;
         const bool ok = (has_row >> t) & 1u;
@@ -358,16 +394,16 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
 }
 
 template <int G, int VPL>
-static cudaError_t launch_pool_t(const PoolParams& p, cudaStream_t s) {
+static cudaError_t launch_pool_t(const PoolParams& p, bool tma, cudaStream_t s) {
   const int64_t threads = p.nchunks * G;
   int64_t blocks = (threads + 255) / 256;
   if (blocks < 1) blocks = 1;
   const size_t smem = (size_t)pool_piece<G, VPL>() * VPL * 256 * sizeof(float4);
-  const cudaError_t e =
-      cudaFuncSetAttribute(pool_kernel<G, VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const auto kernel = tma ? pool_kernel<G, VPL, true> : pool_kernel<G, VPL, false>;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   LaunchScope ls("gather_pool", s);
-  return launch_pdl(pool_kernel<G, VPL>, (unsigned)blocks, 256, smem, s, p);
+  return launch_pdl(kernel, (unsigned)blocks, 256, smem, s, p);
 }
 
 int group_lanes_for(int D) {
@@ -419,6 +455,7 @@ static PoolParams pool_params(const LookupArgs& a, int64_t chunk) {
   p.counters = b->bag_counter;
   p.st = t->dstate;
   p.mirror = t->mirror_dev;
+  p.spin_max = spin_limit();
   // ceil(2^64 / B) = floor((2^64 - 1) / B) + 1 (B >= 2; 2^64 itself for B = 1)
   p.b_magic = a.B >= 2 ? ~0ULL / (uint64_t)a.B + 1 : 0;
   return p;
@@ -438,15 +475,16 @@ cudaError_t launch_pool(const LookupArgs& a, int64_t chunk, cudaStream_t s) {
   const PoolParams p = pool_params(a, chunk);
   if (p.nchunks == 0) return cudaSuccess;
   const int ncol = p.ncol;
-  if (ncol <= 1) return launch_pool_t<1, 1>(p, s);
-  if (ncol <= 2) return launch_pool_t<2, 1>(p, s);
-  if (ncol <= 4) return launch_pool_t<4, 1>(p, s);
-  if (ncol <= 8) return launch_pool_t<8, 1>(p, s);
-  if (ncol <= 16) return launch_pool_t<16, 1>(p, s);
-  if (ncol <= 32) return launch_pool_t<32, 1>(p, s);
-  if (ncol <= 64) return launch_pool_t<32, 2>(p, s);
-  if (ncol <= 128) return launch_pool_t<32, 4>(p, s);
-  return launch_pool_t<32, 8>(p, s);
+  const bool tma = a.t->rows.host_numa < 0;  // EmbeddingBlocks in device memory
+  if (ncol <= 1) return launch_pool_t<1, 1>(p, tma, s);
+  if (ncol <= 2) return launch_pool_t<2, 1>(p, tma, s);
+  if (ncol <= 4) return launch_pool_t<4, 1>(p, tma, s);
+  if (ncol <= 8) return launch_pool_t<8, 1>(p, tma, s);
+  if (ncol <= 16) return launch_pool_t<16, 1>(p, tma, s);
+  if (ncol <= 32) return launch_pool_t<32, 1>(p, tma, s);
+  if (ncol <= 64) return launch_pool_t<32, 2>(p, tma, s);
+  if (ncol <= 128) return launch_pool_t<32, 4>(p, tma, s);
+  return launch_pool_t<32, 8>(p, tma, s);
 }
 
 }  // namespace recis

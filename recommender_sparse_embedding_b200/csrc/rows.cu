@@ -52,6 +52,10 @@ extern "C" recis_status recis_table_read_rows(recis_table_t t, const int64_t* ro
     set_error("read_rows: bad arguments");
     return RECIS_ERR_INVALID_ARG;
   }
+  if (misaligned(rows, 8) || misaligned(keys_out, 8) || misaligned(emb_out, 16) || misaligned(state_out, 16)) {
+    set_error("read_rows: misaligned array (int64 arrays 8-byte, float rows 16-byte)");
+    return RECIS_ERR_INVALID_ARG;
+  }
   if (n == 0 || (!keys_out && !emb_out && !state_out)) return RECIS_OK;
   cudaStream_t s = (cudaStream_t)stream;
   // rows at or past the live count read as key -1 and zeros; the live count

@@ -552,7 +552,8 @@ __global__ void __launch_bounds__(1024) ss_tilescan_kernel(const __grid_constant
 // ------------------------------------------------------------------ scatter
 // Stable move of (ukey, occurrence) into bucket order.  Within a tile, warp w
 // holds keys w*256 .. w*256+255 (item j of lane l is key w*256 + 32j + l);
-// ranks within a warp come from match_any over the items in order, ranks
+// ranks within a warp come from the lanes sharing a bucket (ballots on its
+// bits) over the items in order, ranks
 // across warps from a prefix over per-warp bucket counters.
 __global__ void __launch_bounds__(kCountThreads) ss_scatter_kernel(const __grid_constant__ SsParams p) {
   pdl_wait();
@@ -573,14 +574,27 @@ __global__ void __launch_bounds__(kCountThreads) ss_scatter_kernel(const __grid_
   __syncthreads();
   unsigned* mine = s_wc + w * nbp;
   const unsigned lt = (1u << lane) - 1u;
+  // lanes holding the same bucket: 12 ballots on the bucket's bits (buckets
+  // are below 4095; a missing key takes 4095), all items first
+  unsigned peers[kCountItems];
 #pragma unroll
   for (int j = 0; j < kCountItems; ++j) {
-    const unsigned peers = __match_any_sync(0xffffffffu, b[j]);
-    const int leader = __ffs(peers) - 1;
+    const unsigned bb = b[j] != 0xffffffffu ? b[j] : 4095u;
+    unsigned pm = 0xffffffffu;
+#pragma unroll
+    for (int q = 0; q < 12; ++q) {
+      const unsigned bal = __ballot_sync(0xffffffffu, (bb >> q) & 1u);
+      pm &= ((bb >> q) & 1u) ? bal : ~bal;
+    }
+    peers[j] = pm;
+  }
+#pragma unroll
+  for (int j = 0; j < kCountItems; ++j) {
+    const int leader = __ffs(peers[j]) - 1;
     const unsigned before = b[j] != 0xffffffffu ? mine[b[j]] : 0u;
-    rank[j] = before + __popc(peers & lt);
+    rank[j] = before + __popc(peers[j] & lt);
     __syncwarp();
-    if (lane == leader && b[j] != 0xffffffffu) mine[b[j]] = before + __popc(peers);
+    if (lane == leader && b[j] != 0xffffffffu) mine[b[j]] = before + __popc(peers[j]);
     __syncwarp();
   }
   __syncthreads();

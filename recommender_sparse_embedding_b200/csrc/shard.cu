@@ -284,6 +284,10 @@ extern "C" recis_status recis_batch_dedup(recis_batch_t b, const int64_t* keys, 
     set_error("batch_dedup: bad arguments");
     return RECIS_ERR_INVALID_ARG;
   }
+  if (misaligned(keys, 8) || misaligned(uniq_out, 8) || misaligned(inv_out, 4) || misaligned(U_out, 8)) {
+    set_error("batch_dedup: misaligned array (int64 arrays 8-byte, inv_out 4-byte)");
+    return RECIS_ERR_INVALID_ARG;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   recis_status st = batch_ensure(b, N, 0, 4);
   if (st != RECIS_OK) return st;
@@ -334,6 +338,10 @@ extern "C" recis_status recis_partition_keys(recis_batch_t b, const int64_t* key
   if (!b || n < 0 || n >= ((int64_t)1 << 31) || G < 1 || G > kMaxOwners || !counts_out ||
       (n > 0 && (!keys || !out_keys || !out_pos))) {
     set_error("partition_keys: bad arguments (G must be in 1..256)");
+    return RECIS_ERR_INVALID_ARG;
+  }
+  if (misaligned(keys, 8) || misaligned(out_keys, 8) || misaligned(out_pos, 4) || misaligned(counts_out, 8)) {
+    set_error("partition_keys: misaligned array (int64 arrays 8-byte, out_pos 4-byte)");
     return RECIS_ERR_INVALID_ARG;
   }
   cudaStream_t s = (cudaStream_t)stream;
@@ -391,6 +399,11 @@ extern "C" recis_status recis_pool_rows(const float* rows, const int32_t* row_of
     set_error("pool_rows: bad arguments");
     return RECIS_ERR_INVALID_ARG;
   }
+  if (misaligned(rows, 16) || misaligned(pooled_out, 16) || misaligned(bag_offsets, 8) ||
+      misaligned(row_of_unique, 4) || misaligned(inv, 4)) {
+    set_error("pool_rows: misaligned array (float rows 16-byte, bag_offsets 8-byte, indices 4-byte)");
+    return RECIS_ERR_INVALID_ARG;
+  }
   const int64_t nb = (int64_t)F * B;
   if (nb == 0) return RECIS_OK;
   int64_t blocks = (nb * 32 + 255) / 256;
@@ -410,6 +423,11 @@ extern "C" recis_status recis_reduce_grad(recis_batch_t b, const int64_t* bag_of
   if (!b || b->dedup_N < 0 || F < 0 || B < 0 || D < 1 || (combiner != RECIS_SUM && combiner != RECIS_MEAN) ||
       !grad_out || (grad_pooled && !bag_offsets)) {
     set_error("reduce_grad: bad arguments, or the batch holds no recis_batch_dedup");
+    return RECIS_ERR_INVALID_ARG;
+  }
+  if (misaligned(grad_pooled, 16) || misaligned(grad_unpooled, 16) || misaligned(grad_out, 16) ||
+      misaligned(bag_offsets, 8) || misaligned(out_index, 4)) {
+    set_error("reduce_grad: misaligned array (float rows 16-byte, bag_offsets 8-byte, out_index 4-byte)");
     return RECIS_ERR_INVALID_ARG;
   }
   if (b->dedup_N == 0) return RECIS_OK;

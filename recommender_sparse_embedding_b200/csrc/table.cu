@@ -703,6 +703,10 @@ recis_status recis_feature_hash(const recis_feature_op* ops, int32_t F, const in
     set_error("feature_hash: bad F, ops or feat_offsets");
     return RECIS_ERR_INVALID_ARG;
   }
+  if (misaligned(values, 8) || misaligned(keys_out, 8)) {
+    set_error("feature_hash: values and keys_out must be 8-byte aligned");
+    return RECIS_ERR_INVALID_ARG;
+  }
   if (F == 0) return RECIS_OK;
   if (feat_offsets[0] != 0) {
     set_error("feature_hash: feat_offsets[0] must be 0");
@@ -926,6 +930,10 @@ static recis_status check_lookup_args(recis_table_t t, recis_batch_t b, const in
     set_error("N must be in [0, 2^30) and keys non-null");
     return RECIS_ERR_INVALID_ARG;
   }
+  if (misaligned(keys, 8) || misaligned(bag_offsets, 8)) {
+    set_error("keys and bag_offsets must be 8-byte aligned");
+    return RECIS_ERR_INVALID_ARG;
+  }
   if (need_bags) {
     if (F < 0 || B < 0 || (int64_t)F * B >= ((int64_t)1 << 31) ||
         (combiner != RECIS_SUM && combiner != RECIS_MEAN)) {
@@ -951,6 +959,10 @@ recis_status recis_lookup_pooled(recis_table_t t, recis_batch_t b, const int64_t
     set_error("lookup_pooled: pooled_out and unpooled_out are both null");
     return RECIS_ERR_INVALID_ARG;
   }
+  if (misaligned(pooled_out, 16) || misaligned(unpooled_out, 16)) {
+    set_error("lookup_pooled: pooled_out and unpooled_out must be 16-byte aligned");
+    return RECIS_ERR_INVALID_ARG;
+  }
   LookupArgs a{t, b, keys, N, bag_offsets, F, B, combiner, pooled_out, unpooled_out, nullptr, false};
   return lookup_impl(a, (cudaStream_t)stream);
 }
@@ -959,6 +971,10 @@ recis_status recis_table_insert(recis_table_t t, recis_batch_t b, const int64_t*
                                 int64_t* rows_out, recis_stream_t stream) {
   recis_status st = check_lookup_args(t, b, keys, N, nullptr, 0, 0, RECIS_SUM, false);
   if (st != RECIS_OK) return st;
+  if (misaligned(rows_out, 8)) {
+    set_error("table_insert: rows_out must be 8-byte aligned");
+    return RECIS_ERR_INVALID_ARG;
+  }
   LookupArgs a{t, b, keys, N, nullptr, 0, 0, RECIS_SUM, nullptr, nullptr, rows_out, true};
   st = lookup_impl(a, (cudaStream_t)stream);
   b->have_lookup = false;  // no bags: nothing to back-propagate
@@ -969,6 +985,10 @@ recis_status recis_backward_update(recis_table_t t, recis_batch_t b, const float
                                    const float* grad_unpooled, recis_stream_t stream) {
   if (!t || !b || !b->have_lookup || b->table != t) {
     set_error("backward_update: the batch holds no lookup of this table");
+    return RECIS_ERR_INVALID_ARG;
+  }
+  if (misaligned(grad_pooled, 16) || misaligned(grad_unpooled, 16)) {
+    set_error("backward_update: grad_pooled and grad_unpooled must be 16-byte aligned");
     return RECIS_ERR_INVALID_ARG;
   }
   cudaStream_t s = (cudaStream_t)stream;

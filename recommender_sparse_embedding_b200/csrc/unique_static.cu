@@ -177,6 +177,10 @@ extern "C" recis_status recis_unique_static(const int64_t* keys, int64_t N, int6
     set_error("recis_unique_static: null argument");
     return RECIS_ERR_INVALID_ARG;
   }
+  if (misaligned(keys, 8) || misaligned(uniq_out, 8) || misaligned(inv_out, 4) || misaligned(U_out, 8)) {
+    set_error("recis_unique_static: misaligned array (int64 arrays 8-byte, inv_out 4-byte)");
+    return RECIS_ERR_INVALID_ARG;
+  }
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");

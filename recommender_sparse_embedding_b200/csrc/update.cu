@@ -26,6 +26,8 @@
 //               times come from the dedup's list, spread evenly over the
 //               groups, when there are a few per group.
 // No float atomics anywhere; the result does not depend on scheduling.
+#include <algorithm>
+
 #include "segreduce.cuh"
 
 namespace recis {
@@ -54,6 +56,9 @@ struct UpdateParams {
   int2* long_segs;          // [seg_cap] long segments crossing a span end: the CTA-combined ones
                             // from the back, the others from the front
   int64_t seg_cap;
+  DevState* st;             // status word (a bounded wait that gave up)
+  HostMirror* mirror;
+  int spin_max;             // polls before a wait gives up
   const int32_t* multi_keys;  // keys seen 2 to kShortSeg times (bdev->nmulti of them), or null
   // optimiser
   float lr;        // Adagrad: lr; Adam: lr / (1 - beta1^t)
@@ -205,6 +210,29 @@ __device__ __forceinline__ void load_step_b(const UpdateParams& p, const StepA<E
   }
 }
 
+// the pooled gradient's scale of each position: 1 / bag length (mean
+// pooling), else 1
+template <int E>
+__device__ __forceinline__ void step_scales(const UpdateParams& p, const StepB<E>& b, double (&sc)[E]) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) sc[e] = (p.mean && b.src[e].y > 0) ? 1.0 / (double)b.src[e].y : 1.0;
+}
+
+// bit t (t >= 1): position t of the step lies in another segment than
+// position t - 1
+template <int G, int E>
+__device__ __forceinline__ unsigned run_starts(const GroupCtx<G>& g, const StepB<E>& b) {
+  unsigned m = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int32_t up = __shfl_up_sync(g.mask, b.seg[e], 1, G);
+    const int32_t wrap = g.bcast(b.seg[e > 0 ? e - 1 : 0], G - 1);
+    const int32_t prev = g.lane > 0 ? up : (e > 0 ? wrap : b.seg[e]);
+    m |= g.ballot(b.seg[e] != prev) << (e * G);
+  }
+  return m;
+}
+
 // bit t (t = lane + e * G): position t of the step lies in a long segment
 template <int G, int E>
 __device__ __forceinline__ unsigned long_mask(const GroupCtx<G>& g, const StepB<E>& b) {
@@ -212,11 +240,6 @@ __device__ __forceinline__ unsigned long_mask(const GroupCtx<G>& g, const StepB<
 #pragma unroll
   for (int e = 0; e < E; ++e) m |= g.ballot(b.seg[e] >= 0 && b.en[e] - b.st[e] > kShortSeg) << (e * G);
   return m;
-}
-
-__device__ __forceinline__ void cp_async16_(void* smem, const void* gmem) {
-  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
 }
 
 template <int G, int VPL>
@@ -236,18 +259,31 @@ template <int G, int VPL>
 constexpr int kPartialCtas = VPL >= 4 ? 1 : (G < 8 ? 2 : 3);
 
 // Staging: kChunk 16-byte slots per lane, PR long positions' rows at a time.
-template <int G, int VPL, bool GP, bool GU>
+__device__ __forceinline__ void cp_async16_(void* smem, const void* gmem) {
+  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+
+// TMA: the gradient rows are copied by the bulk-copy engine (gradients in
+// device memory), else by cp.async (any memory the GPU can address).
+template <int G, int VPL, bool GP, bool GU, bool TMA>
 __global__ void __launch_bounds__(256, kPartialCtas<G, VPL>) seg_partial_kernel(const __grid_constant__ UpdateParams p) {
   pdl_wait();
   constexpr int NRW = (GP && GU) ? 2 : 1;  // gradient rows per position
   constexpr int PR = kChunk / (VPL * NRW) > 0 ? kChunk / (VPL * NRW) : 1;  // positions staged at once
   constexpr int Q = SegStep<G>::Q, E = SegStep<G>::E;
   extern __shared__ float4 s_rows[];  // [groups of the CTA][kChunk][G]
+  __shared__ uint64_t s_mbar[256];     // one transaction barrier per group
   const GroupCtx<G> g;
   float4* rows = s_rows + (size_t)(threadIdx.x / G) * kChunk * G;
+  uint64_t* mbar = s_mbar + threadIdx.x / G;
   const int64_t span = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
   const int64_t p0 = span * p.span;
   if (p0 >= p.N) return;
+  if (TMA && g.lane == 0) mbar_init(mbar, 1);
+  __syncwarp(g.mask);
+  unsigned phase = 0;
+  const unsigned row_bytes = (unsigned)p.ncol * 16u;
   const int64_t p1 = p0 + p.span < p.N ? p0 + p.span : p.N;
   const int64_t D = (int64_t)p.ncol * 4;
   Acc4 acc[VPL];
@@ -286,7 +322,11 @@ __global__ void __launch_bounds__(256, kPartialCtas<G, VPL>) seg_partial_kernel(
   load_step_b<E>(p, a1, cur_b);
   load_step_a<G, E>(g, p, p0 + Q, p1, a1);
   unsigned mask = long_mask<G, E>(g, cur_b);
+  unsigned runs = run_starts<G, E>(g, cur_b);
+  double scale[E];
+  if (GP) step_scales<E>(p, cur_b, scale);
   for (int64_t base = p0; base < p1; base += Q) {
+    const int32_t first_seg = g.bcast(cur_b.seg[0], 0);
     bool ahead = false;  // next steps' loads issued
     unsigned rem = mask;
     do {
@@ -300,49 +340,82 @@ __global__ void __launch_bounds__(256, kPartialCtas<G, VPL>) seg_partial_kernel(
         }
       }
       rem &= ~piece;
-      int u = 0;
-      for (unsigned m = piece; m; m &= m - 1, ++u) {
-        const int t = __ffs(m) - 1;
-        const int e = t / G, l = t % G;
-        const int4 sv = pick(cur_b.src, e);
-        if (GP) {
-          const float* r = p.gp + (int64_t)g.bcast(sv.x, l) * D;
+      // the piece's rows into slot u = the position's rank in the piece
+      if (TMA) {
+        // each lane copies the rows of its own positions, one bulk copy per row
+        if (piece) {
+          __syncwarp(g.mask);  // the group has read the previous piece
+          fence_async_smem();
+          if (g.lane == 0) mbar_arrive_expect(mbar, (unsigned)__popc(piece) * NRW * row_bytes);
 #pragma unroll
-          for (int v = 0; v < VPL; ++v) {
-            const int col = g.lane + v * G;
-            if (col < p.ncol) cp_async16_(rows + ((u * NRW) * VPL + v) * G + g.lane, r + 4 * col);
+          for (int e = 0; e < E; ++e) {
+            const int t = g.lane + e * G;
+            if (t < 32 && ((piece >> t) & 1u)) {
+              const int u = __popc(piece & ((1u << t) - 1u));
+              if (GP) bulk_row(rows + (u * NRW) * VPL * G, p.gp + (int64_t)cur_b.src[e].x * D, row_bytes, mbar);
+              if (GU)
+                bulk_row(rows + (u * NRW + (GP ? 1 : 0)) * VPL * G, p.gu + (int64_t)cur_b.src[e].z * D,
+                         row_bytes, mbar);
+            }
           }
         }
-        if (GU) {
-          const float* r = p.gu + (int64_t)g.bcast(sv.z, l) * D;
+      } else {
+        // 16 bytes per lane and row, by cp.async
+        int u = 0;
+        for (unsigned m = piece; m; m &= m - 1, ++u) {
+          const int t = __ffs(m) - 1;
+          const int e = t / G, l = t % G;
+          const int4 sv = pick(cur_b.src, e);
+          if (GP) {
+            const float* r = p.gp + (int64_t)g.bcast(sv.x, l) * D;
 #pragma unroll
-          for (int v = 0; v < VPL; ++v) {
-            const int col = g.lane + v * G;
-            if (col < p.ncol)
-              cp_async16_(rows + ((u * NRW + (GP ? 1 : 0)) * VPL + v) * G + g.lane, r + 4 * col);
+            for (int v = 0; v < VPL; ++v) {
+              const int col = g.lane + v * G;
+              if (col < p.ncol) cp_async16_(rows + ((u * NRW) * VPL + v) * G + g.lane, r + 4 * col);
+            }
+          }
+          if (GU) {
+            const float* r = p.gu + (int64_t)g.bcast(sv.z, l) * D;
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+              const int col = g.lane + v * G;
+              if (col < p.ncol)
+                cp_async16_(rows + ((u * NRW + (GP ? 1 : 0)) * VPL + v) * G + g.lane, r + 4 * col);
+            }
           }
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
       }
-      asm volatile("cp.async.commit_group;" ::: "memory");
       if (!ahead) {
         load_step_b<E>(p, a1, nxt_b);
         load_step_a<G, E>(g, p, base + 2 * Q, p1, a2);
         ahead = true;
       }
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      if (!TMA) {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      } else if (piece) {
+        if (!mbar_wait(mbar, phase, p.spin_max)) {
+          // the copies did not land in time: reported, and waited for once
+          // more before the slots are read or written again
+          if (g.lane == 0) raise_error(p.st, p.mirror, kErrTimeout);
+          mbar_wait(mbar, phase, p.spin_max);
+        }
+        phase ^= 1u;
+      }
       // the piece's positions in order, one segment run at a time
-      u = 0;
+      int u = 0;
       for (unsigned m = piece; m; m &= m - 1, ++u) {
         const int t = __ffs(m) - 1;
         const int e = t / G, l = t % G;
-        const int32_t sg = g.bcast(pick(cur_b.seg, e), l);
-        if (sg != cur) {
+        // a new segment run: the step's first position in another segment
+        // than the last one added, or a segment start within the step
+        if (t == 0 ? first_seg != cur : ((runs >> t) & 1u) != 0u) {
           if (cur >= 0) flush();
-          cur = sg;
+          cur = g.bcast(pick(cur_b.seg, e), l);
           cst = g.bcast(pick(cur_b.st, e), l);
           cen = g.bcast(pick(cur_b.en, e), l);
         }
-        const double sc = (GP && p.mean) ? 1.0 / (double)g.bcast(pick(cur_b.src, e).y, l) : 1.0;
+        const double sc = (GP && p.mean) ? g.bcast(pick(scale, e), l) : 1.0;
 #pragma unroll
         for (int v = 0; v < VPL; ++v) {
           const int col = g.lane + v * G;
@@ -361,6 +434,8 @@ __global__ void __launch_bounds__(256, kPartialCtas<G, VPL>) seg_partial_kernel(
     cur_b = nxt_b;
     a1 = a2;
     mask = long_mask<G, E>(g, cur_b);
+    runs = run_starts<G, E>(g, cur_b);
+    if (GP) step_scales<E>(p, cur_b, scale);
   }
   if (cur >= 0) flush();
   pdl_trigger();
@@ -635,12 +710,15 @@ __device__ __noinline__ void update_listed(const UpdateParams& p, int64_t gid, i
 // Pipeline depth: 4 when each group walks many keys (long-sequence batches),
 // 2 otherwise (measured: 3 or 4 keys deep, or a fourth CTA per SM, only
 // lengthen every request on the 26-feature step).
-template <int G, int VPL, bool ADAM, bool GP, bool GU, int S>
+template <int G, int VPL, bool ADAM, bool GP, bool GU, int S, bool TMA>
 __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constant__ UpdateParams p) {
   pdl_wait();
   constexpr int NR = ADAM ? 3 : 2;             // row slices: emb, state(s)
   constexpr int NS = NR * VPL + VPL;           // staged float4 per thread per stage
-  extern __shared__ float4 s_stage[];          // [S][NS][blockDim], then [S][groups] keys
+  // [S][NS][blockDim] float4 (TMA: [S][groups][NS * G], each row contiguous
+  // followed by the gradient row), then [S][groups] keys, then (TMA)
+  // [S][groups] transaction barriers
+  extern __shared__ float4 s_stage[];
   const GroupCtx<G> g;
   const int tid = threadIdx.x, nt = blockDim.x;
   const int grp = tid / G, ngrp = nt / G;
@@ -659,14 +737,47 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
   auto is_listed = [&](const KeyIdx& k) { return listed && k.s1 - k.s0 > 1 && k.s1 - k.s0 <= kShortSeg; };
   if (u0 >= U) return;
   KeyIdx* s_keys = reinterpret_cast<KeyIdx*>(s_stage + S * NS * nt);
+  uint64_t* s_mbar = reinterpret_cast<uint64_t*>(s_keys + S * ngrp);
   auto key_slot = [&](int st) -> KeyIdx* { return s_keys + st * ngrp + grp; };
-  auto slot = [&](int stage, int sl) -> float4* { return s_stage + ((stage * NS + sl) * nt + tid); };
+  auto mbar = [&](int st) -> uint64_t* { return s_mbar + st * ngrp + grp; };
+  // this lane's 16-byte column of row slice sl (the gradient row: sl = NR * VPL)
+  auto slot = [&](int stage, int sl) -> float4* {
+    if (TMA) {
+      float4* region = s_stage + (size_t)(stage * ngrp + grp) * NS * G;
+      const int r = sl / VPL, v = sl % VPL;
+      return region + (r < NR ? r * p.ncol : NR * VPL * G) + g.lane + v * G;
+    }
+    return s_stage + ((stage * NS + sl) * nt + tid);
+  };
+  const int stride = TMA ? G : nt;  // between a lane's columns v and v + 1
+  const unsigned row_bytes = (unsigned)p.row_floats * 4u;
+  if (TMA) {
+    if (g.lane == 0)
+      for (int st = 0; st < S; ++st) mbar_init(mbar(st), 1);
+    __syncwarp(g.mask);
+  }
   auto issue = [&](int stage, const KeyIdx& k) {
-    if (g.lane == 0) *key_slot(stage) = k;
-    if (k.row < 0 || is_listed(k)) return;
-    const float* base = p.row_data + (int64_t)k.row * p.row_floats;
+    const bool copy = k.row >= 0 && !is_listed(k);
     const bool stage_grad = GP && !GU && k.s1 - k.s0 == 1;
+    const float* base = p.row_data + (int64_t)(k.row < 0 ? 0 : k.row) * p.row_floats;
     const float* gsrc_row = p.gp + (int64_t)k.first.x * D;
+    if (TMA) {
+      // the whole row [emb | state] and a singleton's gradient row by the
+      // bulk-copy engine, one instruction each; one barrier phase per issue
+      if (g.lane == 0) {
+        *key_slot(stage) = k;
+        fence_async_smem();
+        mbar_arrive_expect(mbar(stage), copy ? row_bytes + (stage_grad ? (unsigned)D * 4u : 0u) : 0u);
+        if (copy) {
+          float4* region = s_stage + (size_t)(stage * ngrp + grp) * NS * G;
+          bulk_row(region, base, row_bytes, mbar(stage));
+          if (stage_grad) bulk_row(region + NR * VPL * G, gsrc_row, (unsigned)D * 4u, mbar(stage));
+        }
+      }
+      return;
+    }
+    if (g.lane == 0) *key_slot(stage) = k;
+    if (!copy) return;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       const int col = g.lane + v * G;
@@ -684,23 +795,32 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
 #pragma unroll
   for (int k = 0; k < S - 1; ++k) {
     issue(k, idx_of(k));
-    cp_async_commit();
+    if (!TMA) cp_async_commit();
   }
   KeyIdx pre = idx_of(S - 1);
   for (int64_t k = 0; u0 + k * groups < U; ++k) {
     __syncwarp(g.mask);  // every lane is done with the slot about to be reused
     issue((int)((k + S - 1) % S), pre);
-    cp_async_commit();
+    if (!TMA) cp_async_commit();
     pre = idx_of(k + S);
     __syncwarp(g.mask);
     const int stage = (int)(k % S);
     const KeyIdx cur = *key_slot(stage);
     const bool staged_grad = GP && !GU && cur.s1 - cur.s0 == 1;
     float4 grad[VPL];
-    cp_async_wait<S - 1>();
+    if (TMA) {
+      // the (k / S)-th use of this stage's barrier
+      const unsigned parity = (unsigned)((k / S) & 1);
+      if (!mbar_wait(mbar(stage), parity, p.spin_max)) {
+        if (g.lane == 0) raise_error(p.st, p.mirror, kErrTimeout);
+        mbar_wait(mbar(stage), parity, p.spin_max);
+      }
+    } else {
+      cp_async_wait<S - 1>();
+    }
     if (is_listed(cur)) continue;  // updated above
     key_grad<G, VPL, GP, GU>(g, p, cur.s0, cur.s1, cur.first,
-                             staged_grad ? slot(stage, NR * VPL) : nullptr, nt, grad);
+                             staged_grad ? slot(stage, NR * VPL) : nullptr, stride, grad);
     if (cur.row >= 0) {
       RowRegs<VPL, ADAM> r;
 #pragma unroll
@@ -759,18 +879,21 @@ static cudaError_t smem_attr(K kernel, size_t smem, bool (&done)[64]) {
 }
 
 template <int G, int VPL, bool GP, bool GU>
-static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t ucap, cudaStream_t s) {
+static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t ucap, bool tma, bool rows_tma,
+                                   cudaStream_t s) {
   {
     // one lane group per span; one staging slot per position, row and lane
     constexpr size_t smem = (size_t)256 * kChunk * sizeof(float4);
-    static bool attr[64] = {false};
-    cudaError_t e = smem_attr(seg_partial_kernel<G, VPL, GP, GU>, smem, attr);
+    static bool attr[64] = {false}, attr_t[64] = {false};
+    cudaError_t e = tma ? smem_attr(seg_partial_kernel<G, VPL, GP, GU, true>, smem, attr_t)
+                        : smem_attr(seg_partial_kernel<G, VPL, GP, GU, false>, smem, attr);
     if (e != cudaSuccess) return e;
     const int64_t spans = (p.N + p.span - 1) / p.span;
-    const int64_t blocks = (spans * G + 255) / 256;
+    const unsigned blocks = (unsigned)std::max<int64_t>(1, (spans * G + 255) / 256);
     {
       LaunchScope ls("seg_partial", s);
-      e = launch_pdl(seg_partial_kernel<G, VPL, GP, GU>, (unsigned)(blocks < 1 ? 1 : blocks), 256, smem, s, p);
+      e = tma ? launch_pdl(seg_partial_kernel<G, VPL, GP, GU, true>, blocks, 256, smem, s, p)
+              : launch_pdl(seg_partial_kernel<G, VPL, GP, GU, false>, blocks, 256, smem, s, p);
       if (e != cudaSuccess) return e;
     }
     constexpr size_t csmem = (size_t)256 * VPL * sizeof(Acc4);
@@ -793,17 +916,29 @@ static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t uca
     const bool deep = ucap / (blocks * (256 / G)) >= 64;
     const int S = deep ? 4 : 2;
     const int ns = ((adam ? 3 : 2) * VPL + VPL);
-    const size_t smem = (size_t)S * ns * 256 * sizeof(float4) + (size_t)S * (256 / G) * sizeof(KeyIdx);
+    const size_t smem = (size_t)S * ns * 256 * sizeof(float4) + (size_t)S * (256 / G) * sizeof(KeyIdx) +
+                        (rows_tma ? (size_t)S * (256 / G) * sizeof(uint64_t) : 0);
     cudaError_t e;
     auto go = [&](auto kernel) -> cudaError_t {
       cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (err != cudaSuccess) return err;
       return launch_pdl(kernel, (unsigned)blocks, 256, smem, s, p);
     };
-    if (adam)
-      e = deep ? go(row_update_kernel<G, VPL, true, GP, GU, 4>) : go(row_update_kernel<G, VPL, true, GP, GU, 2>);
-    else
-      e = deep ? go(row_update_kernel<G, VPL, false, GP, GU, 4>) : go(row_update_kernel<G, VPL, false, GP, GU, 2>);
+    if (rows_tma) {
+      if (adam)
+        e = deep ? go(row_update_kernel<G, VPL, true, GP, GU, 4, true>)
+                 : go(row_update_kernel<G, VPL, true, GP, GU, 2, true>);
+      else
+        e = deep ? go(row_update_kernel<G, VPL, false, GP, GU, 4, true>)
+                 : go(row_update_kernel<G, VPL, false, GP, GU, 2, true>);
+    } else {
+      if (adam)
+        e = deep ? go(row_update_kernel<G, VPL, true, GP, GU, 4, false>)
+                 : go(row_update_kernel<G, VPL, true, GP, GU, 2, false>);
+      else
+        e = deep ? go(row_update_kernel<G, VPL, false, GP, GU, 4, false>)
+                 : go(row_update_kernel<G, VPL, false, GP, GU, 2, false>);
+    }
     if (e != cudaSuccess) return e;
   } else {
     if (adam)
@@ -815,11 +950,25 @@ static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t uca
 }
 
 template <int G, int VPL>
-static cudaError_t launch_update_t(const UpdateParams& p, bool adam, int64_t ucap, cudaStream_t s) {
-  if (p.gp && p.gu) return launch_update_g<G, VPL, true, true>(p, adam, ucap, s);
-  if (p.gp) return launch_update_g<G, VPL, true, false>(p, adam, ucap, s);
-  if (p.gu) return launch_update_g<G, VPL, false, true>(p, adam, ucap, s);
-  return launch_update_g<G, VPL, false, false>(p, adam, ucap, s);  // touched rows, zero gradient
+static cudaError_t launch_update_t(const UpdateParams& p, bool adam, int64_t ucap, bool tma, bool rows_tma,
+                                   cudaStream_t s) {
+  if (p.gp && p.gu) return launch_update_g<G, VPL, true, true>(p, adam, ucap, tma, rows_tma, s);
+  if (p.gp) return launch_update_g<G, VPL, true, false>(p, adam, ucap, tma, rows_tma, s);
+  if (p.gu) return launch_update_g<G, VPL, false, true>(p, adam, ucap, tma, rows_tma, s);
+  return launch_update_g<G, VPL, false, false>(p, adam, ucap, tma, rows_tma, s);  // touched rows, zero gradient
+}
+
+// device memory of this GPU's own address space (allocations and VMM
+// mappings of device memory): the bulk-copy engine reads it; other memory
+// (host-mapped, managed) takes the cp.async path
+static bool device_memory(const void* ptr) {
+  if (!ptr) return true;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice;
 }
 
 cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pooled,
@@ -846,6 +995,9 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   p.partials = b->partials;
   p.long_segs = b->long_segs;
   p.seg_cap = b->capSegs;
+  p.st = t->dstate;
+  p.mirror = t->mirror_dev;
+  p.spin_max = spin_limit();
   p.lr = lr_t;
   p.eps = (float)t->cfg.eps;
   p.beta1 = (float)t->cfg.beta1;
@@ -856,16 +1008,20 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   if (p.N == 0) return cudaSuccess;
   const bool adam = t->cfg.optimizer == RECIS_ADAM;
   const int64_t ucap = b->N;  // U <= N; groups past U return at once
+  // bulk copies for gradients in device memory, and for rows too when the
+  // EmbeddingBlocks are device memory
+  const bool tma = device_memory(grad_pooled) && device_memory(grad_unpooled);
+  const bool rows_tma = tma && t->rows.host_numa < 0;
   const int ncol = p.ncol;
-  if (ncol <= 1) return launch_update_t<1, 1>(p, adam, ucap, s);
-  if (ncol <= 2) return launch_update_t<2, 1>(p, adam, ucap, s);
-  if (ncol <= 4) return launch_update_t<4, 1>(p, adam, ucap, s);
-  if (ncol <= 8) return launch_update_t<8, 1>(p, adam, ucap, s);
-  if (ncol <= 16) return launch_update_t<16, 1>(p, adam, ucap, s);
-  if (ncol <= 32) return launch_update_t<32, 1>(p, adam, ucap, s);
-  if (ncol <= 64) return launch_update_t<32, 2>(p, adam, ucap, s);
-  if (ncol <= 128) return launch_update_t<32, 4>(p, adam, ucap, s);
-  return launch_update_t<32, 8>(p, adam, ucap, s);
+  if (ncol <= 1) return launch_update_t<1, 1>(p, adam, ucap, tma, rows_tma, s);
+  if (ncol <= 2) return launch_update_t<2, 1>(p, adam, ucap, tma, rows_tma, s);
+  if (ncol <= 4) return launch_update_t<4, 1>(p, adam, ucap, tma, rows_tma, s);
+  if (ncol <= 8) return launch_update_t<8, 1>(p, adam, ucap, tma, rows_tma, s);
+  if (ncol <= 16) return launch_update_t<16, 1>(p, adam, ucap, tma, rows_tma, s);
+  if (ncol <= 32) return launch_update_t<32, 1>(p, adam, ucap, tma, rows_tma, s);
+  if (ncol <= 64) return launch_update_t<32, 2>(p, adam, ucap, tma, rows_tma, s);
+  if (ncol <= 128) return launch_update_t<32, 4>(p, adam, ucap, tma, rows_tma, s);
+  return launch_update_t<32, 8>(p, adam, ucap, tma, rows_tma, s);
 }
 
 }  // namespace recis

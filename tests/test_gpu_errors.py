@@ -146,3 +146,33 @@ def test_bounded_wait_gives_up_and_is_reported(R):
     assert u == len(ref)
     assert np.array_equal(uniq[:u].cpu().numpy(), ref)
     assert np.array_equal(inv.cpu().numpy(), ref_inv)
+
+
+def test_misaligned_pointers_rejected_on_the_host(R):
+    # vector loads and row copies need aligned arrays: the entry points
+    # refuse a misaligned pointer before any work is queued, and the table
+    # then works as before
+    L = R.load()
+    spec = W.TableSpec("t", [0], 16, "adagrad", 0.05, "sum", pooled=True, init_seed=3)
+    p = Pair(R, spec)
+    N, B, D = 64, 8, 16
+    keys = torch.arange(1, N + 2, dtype=torch.int64, device=DEV)  # one spare element to shift into
+    bo = torch.linspace(0, N, B + 1, device=DEV).to(torch.int64)
+    pooled = torch.empty((B * D + 4,), dtype=torch.float32, device=DEV)
+    s = None  # the legacy default stream
+    bad_keys = keys.data_ptr() + 4
+    assert L.recis_lookup_pooled(p.gpu.handle, p.batch.handle, bad_keys, N, bo.data_ptr(), 1, B, R.SUM,
+                                 pooled.data_ptr(), None, s) == R.ERR_INVALID_ARG
+    assert L.recis_lookup_pooled(p.gpu.handle, p.batch.handle, keys.data_ptr(), N, bo.data_ptr(), 1, B, R.SUM,
+                                 pooled.data_ptr() + 4, None, s) == R.ERR_INVALID_ARG
+    assert L.recis_lookup_pooled(p.gpu.handle, p.batch.handle, keys.data_ptr(), N, bo.data_ptr(), 1, B, R.SUM,
+                                 pooled.data_ptr(), None, s) == R.OK
+    grad = torch.ones((B * D + 4,), dtype=torch.float32, device=DEV)
+    assert L.recis_backward_update(p.gpu.handle, p.batch.handle, grad.data_ptr() + 8, None, s) == R.ERR_INVALID_ARG
+    assert L.recis_backward_update(p.gpu.handle, p.batch.handle, grad.data_ptr(), None, s) == R.OK
+    p.gpu.status_sync()
+    kh = keys[:N].cpu().numpy()
+    p.ora.lookup(kh, bo.cpu().numpy(), 1, B, p.combiner_o)
+    p.ora.backward_update(np.ones((B, 1, D), np.float32))
+    compare_tables(p, "after the refused calls")
+    p.close()

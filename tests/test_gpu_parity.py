@@ -276,6 +276,59 @@ def test_long_segments_over_many_spans(R, D, opt, comb, unpooled):
     _single(R, keys, lengths, D=D, opt=opt, comb=comb, unpooled=unpooled, grad_signed=True)
 
 
+@pytest.mark.parametrize("N", [50_000, 1_700_000])
+def test_new_rows_bit_exact(R, N):
+    # fresh rows (seeded hash of the key; optimiser state initial) equal the
+    # oracle's bit for bit, on the sample-sort path and on the radix path
+    rng = np.random.default_rng(N)
+    keys = rng.integers(-(1 << 62), 1 << 62, size=N)
+    keys[keys == -1] = 7
+    spec = W.TableSpec("t", [0], 8, "adagrad", 0.05, "sum", pooled=True, init_seed=17)
+    p = Pair(R, spec, init_acc=0.125)
+    bo = np.array([0, N], np.int64)
+    pooled = torch.empty((1, 1, 8), dtype=torch.float32, device=DEV)
+    p.gpu.lookup_pooled(p.batch, torch.from_numpy(keys).to(DEV), torch.from_numpy(bo).to(DEV), 1, 1,
+                        p.combiner_r, pooled)
+    p.ora.lookup(keys, bo, 1, 1, p.combiner_o)
+    p.gpu.status_sync()
+    gk, ge, gs, _ = p.gpu.export()
+    ok, oe, os_ = p.ora.export()
+    assert np.array_equal(gk, ok)
+    assert np.array_equal(ge, oe)
+    assert np.array_equal(gs, os_)
+    p.close()
+
+
+def test_gradients_in_pinned_host_memory(R):
+    # gradients the GPU reads from pinned host memory (not device memory):
+    # the backward gathers them with cp.async instead of the bulk-copy engine
+    rng = np.random.default_rng(31)
+    N, B, D = 40_000, 5_000, 32
+    keys = np.concatenate([np.full(3_000, 42, np.int64), rng.integers(0, 1 << 40, size=N - 3_000)])
+    keys = keys[rng.permutation(N)]
+    bo = np.linspace(0, N, B + 1).astype(np.int64)
+    spec = W.TableSpec("t", [0], D, "adam", 0.05, "mean", pooled=True, unpooled=True, init_seed=8)
+    p = Pair(R, spec)
+    k_dev, bo_dev = torch.from_numpy(keys).to(DEV), torch.from_numpy(bo).to(DEV)
+    for step in range(2):
+        pooled = torch.empty((B, 1, D), dtype=torch.float32, device=DEV)
+        unp = torch.empty((N, D), dtype=torch.float32, device=DEV)
+        p.gpu.lookup_pooled(p.batch, k_dev, bo_dev, 1, B, p.combiner_r, pooled, unp)
+        p.ora.lookup(keys, bo, 1, B, p.combiner_o, unpooled=True)
+        gp = W.make_grad((B, 1, D), 70 + step, signed=True)
+        gu = W.make_grad((N, D), 80 + step, signed=True)
+        gp_h = torch.from_numpy(gp).pin_memory()
+        gu_h = torch.from_numpy(gu).pin_memory()
+        # the binding takes CUDA tensors only; the C ABI takes any address the GPU can read
+        assert R.load().recis_backward_update(p.gpu.handle, p.batch.handle, gp_h.data_ptr(), gu_h.data_ptr(),
+                                              None) == R.OK
+        torch.cuda.synchronize()
+        p.ora.backward_update(gp, gu)
+        p.gpu.status_sync()
+        compare_tables(p, f"step {step}")
+    p.close()
+
+
 def test_all_new_then_all_old(R):
     keys = np.arange(50_000, dtype=np.int64) * 1_000_003
     _single(R, keys[::-1].copy(), np.ones(50_000, np.int64), D=8, steps=3)

@@ -182,6 +182,21 @@ def test_init_range_granularity_and_independence():
     assert np.all(t4.export()[2] == np.float32(0.25))
 
 
+def test_init_row_rebuilt_from_the_hash():
+    # a fresh row rebuilt value by value from the pinned hash: seed mixed into
+    # the key, one hash per column, the top 24 bits as a uniform on [0, 1)
+    D, seed = 8, 0x1234_5678_9ABC_DEF0
+    t = O.Table(D, O.ADAM, 0.1, init_seed=seed)
+    keys = np.array([0, 1, -2, 123456789, -(1 << 62), (1 << 62) + 5], np.int64)  # -1 is reserved
+    t.lookup(keys, np.array([0, len(keys)]), 1, 1)
+    k, emb, _ = t.export()
+    two_s = 2.0 * float(np.float32(1.0 / math.sqrt(D)))
+    for key, row in zip(k.tolist(), emb):
+        base = O.hash64((key & M64) ^ seed)
+        want = [np.float32(((O.hash64((base + j) & M64) >> 40) / 2.0**24 - 0.5) * two_s) for j in range(D)]
+        assert np.array_equal(row, np.array(want, np.float32))
+
+
 # ---------------------------------------------------------------- pooling / grad
 def _dense(t):
     k, emb, st = t.export()
