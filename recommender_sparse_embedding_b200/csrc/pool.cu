@@ -145,10 +145,11 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
   struct Ids {
     int row, spos, seg;
   };
+  int lim = p1;  // positions below lim are walked (the bag walk moves it to a bag end)
   auto resolve = [&](int sub) {
     Ids r{-1, 0, 0};
     const int q = sub + g.lane;
-    if (q < p1) {
+    if (q < lim) {
       r.seg = __ldg(p.inv + q);
       r.spos = (int)__ldg(p.spos + q);
       const int64_t pr = p.pocc ? __ldcg(p.pocc + q) : -2;
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
   auto bag_at = [&](int sub) {
     Bag r{0, 0, 0};
     const int q = sub + g.lane;
-    if (q < p1) {
+    if (q < lim) {
       int j = __ldg(p.bag_of + q);
       if (j < 0 || j >= nbags) j = 0;  // only with malformed bag offsets (reported by the preparation)
       r.j = j;
@@ -286,10 +287,33 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
   // chunk.  The sub-block's rows are copied into shared memory by cp.async,
   // PR rows per lane at once (one round trip), while the sub-block after the
   // next one is resolved; then they are added in position order.
+  // Bags of at most C/2 occurrences are never cut: the chunk walks from the
+  // first bag that starts in it to the end of the last one that starts in
+  // it (a bag crossing the chunk's start belongs to the chunk before);
+  // longer bags are cut at chunk ends and combined from partials.  (Whole
+  // bags of up to 2C made the chunks' work too uneven: slower on bags of 1
+  // to 100 occurrences.)
+  const int lcap = C / 2;
+  int q0 = p0, q1 = p1;
+  {
+    const int hi0 = (int)p.offs[j0 + 1];
+    if (cur_start < p0 && hi0 - cur_start <= lcap) q0 = hi0;
+    if (p1 < N) {
+      int j1 = p.chunk_bag[chunk + 1];
+      if (j1 < 0 || j1 >= nbags) j1 = 0;  // only with malformed offsets (reported above)
+      const int lo1 = (int)p.offs[j1], hi1 = (int)p.offs[j1 + 1];
+      if (lo1 < p1 && hi1 - lo1 <= lcap && hi1 <= N) q1 = hi1;
+    }
+  }
+  if (q0 >= q1) {
+    pdl_trigger();
+    return;
+  }
+  lim = q1;
   auto flush_bag = [&](int j, int lo, int hi) {
     if (!(lo >= 0 && lo < hi && hi <= N)) {  // malformed bag offsets
       if (g.lane == 0) raise_error(p.st, p.mirror, kErrBadOffsets);
-    } else if (lo >= p0 && hi <= p1) {
+    } else if (lo >= q0 && hi <= q1) {
       store_bag(j, hi - lo);
     } else if (combine_split<G, VPL>(g, acc, p.partials, p.counters, j, chunk, lo <= p0, lo, hi, C,
                                      ncol)) {
@@ -300,13 +324,13 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
   };
   auto emit = [&](int sub, const Ids& ids, const Bag& bg) {
     const int q = sub + g.lane;
-    if (q < p1) {
+    if (q < q1) {
       const int f = div_b(p, bg.j);
       const int4 src = make_int4((bg.j - f * B) * F + f, bg.hi - bg.lo, q, 0);
       p.gsrc[ids.spos] = src;
       p.gfirst[ids.seg] = src;
     }
-    return g.ballot(q < p1 && (q + 1 == bg.hi || q + 1 == p1));
+    return g.ballot(q < q1 && (q + 1 == bg.hi || q + 1 == q1));
   };
   constexpr int PR = pool_piece<G, VPL>();  // rows per lane staged at once
   float4* stage = s_ring + (size_t)(threadIdx.x / G) * PR * VPL * G;
@@ -318,12 +342,12 @@ __global__ void __launch_bounds__(256, VPL == 1 ? 3 : (VPL == 2 ? 2 : 1))
     if (g.lane == 0) mbar_init(mbar, 1);
     __syncwarp(g.mask);
   }
-  Ids cur_ids = ids0, nxt_ids = resolve(p0 + G);
-  Bag cur_bag = bag_at(p0), nxt_bag = bag_at(p0 + G);
-  for (int sub = p0; sub < p1; sub += G) {
+  Ids cur_ids = (q0 == p0 && q1 == p1) ? ids0 : resolve(q0), nxt_ids = resolve(q0 + G);
+  Bag cur_bag = bag_at(q0), nxt_bag = bag_at(q0 + G);
+  for (int sub = q0; sub < q1; sub += G) {
     const unsigned ends = emit(sub, cur_ids, cur_bag);
     const unsigned has_row = g.ballot(cur_ids.row >= 0);
-    const int cnt = p1 - sub < G ? p1 - sub : G;
+    const int cnt = q1 - sub < G ? q1 - sub : G;
     Ids nn_ids{-1, 0, 0};
     Bag nn_bag{0, 0, 0};
     for (int r0 = 0; r0 < cnt; r0 += PR) {

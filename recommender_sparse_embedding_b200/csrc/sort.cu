@@ -133,7 +133,10 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int64_t* __restric
   }
 }
 
-__global__ void __launch_bounds__(kSortBlock) sort_pass_kernel(
+// four CTAs per SM (64 registers a thread): 11 % faster on the 32.8M-key
+// step than three with 80 registers, the look-back waits of more tiles
+// overlapping
+__global__ void __launch_bounds__(kSortBlock, 4) sort_pass_kernel(
     int P, const int64_t* __restrict__ in_keys, uint64_t* kb0, uint64_t* kb1, uint32_t* vb0,
     uint32_t* vb1, int64_t N, SortCtl* ctl, unsigned long long* lookback, uint32_t epoch,
     DevState* st, HostMirror* mirror, int spin_max) {

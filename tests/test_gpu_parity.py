@@ -329,6 +329,20 @@ def test_gradients_in_pinned_host_memory(R):
     p.close()
 
 
+@pytest.mark.parametrize("comb", ["sum", "mean"])
+def test_bag_lengths_around_the_pool_chunk(R, comb):
+    # about 330K occurrences of D = 64: pool chunks of 32 positions; bags of
+    # 1 to 100 occurrences, many one shorter or longer than half a chunk, a
+    # chunk or two, so bags cross chunk ends whole (up to half a chunk long)
+    # or are cut into pieces
+    rng = np.random.default_rng(41)
+    lengths = rng.choice([1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 100], size=9_000)
+    N = int(lengths.sum())
+    assert 227_500 <= N < 454_000  # chunks of 32 positions for this N and D
+    keys = np.minimum(rng.zipf(1.2, size=N), 1 << 40).astype(np.int64) * 7_919
+    _single(R, keys, lengths, D=64, opt="adam", comb=comb, unpooled=True, grad_signed=True)
+
+
 def test_all_new_then_all_old(R):
     keys = np.arange(50_000, dtype=np.int64) * 1_000_003
     _single(R, keys[::-1].copy(), np.ones(50_000, np.int64), D=8, steps=3)
