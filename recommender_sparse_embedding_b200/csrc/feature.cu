@@ -4,7 +4,8 @@
 // One launch transforms up to kFeatPerLaunch features: every value finds its
 // feature by a binary search over the offsets held in the kernel's parameter
 // space, then applies bucketize or hash -> mod, then the feature tag.  The
-// kernel streams 16 bytes per value (8 in, 8 out).
+// kernel streams 16 bytes per value (8 in, 8 out), four values per thread
+// in flight.
 #include "internal.h"
 
 namespace recis {
@@ -29,47 +30,58 @@ struct FeatParams {
   FeatOpDev ops[kFeatPerLaunch];
 };
 
+constexpr int kFeatItems = 4;  // values per thread per round, all loaded before any is transformed
+
+// the transform of value x of feature op
+__device__ __forceinline__ int64_t feature_key(const FeatOpDev& op, int64_t x, int* status) {
+  uint64_t v;
+  if (op.flags & RECIS_BUCKETIZE) {
+    int l = 0, r = op.n_bound;  // count of boundaries <= x
+    while (l < r) {
+      const int m = (l + r) >> 1;
+      if (__ldg(op.bounds + m) <= x) l = m + 1; else r = m;
+    }
+    v = (uint64_t)l;
+  } else {
+    v = (uint64_t)x;
+    if (op.flags & RECIS_HASH) v = mix64(v ^ op.seed);
+    if (op.flags & RECIS_MOD) v = (op.flags & kModPow2) ? (v & (op.mod - 1)) : (v % op.mod);
+  }
+  if (!(op.flags & RECIS_TAG)) return (int64_t)v;
+  if (v >= op.limit) {
+    atomicOr(status, kErrTagOverflow);
+    return kEmptyKey;
+  }
+  return (int64_t)(op.tag_bits | v);
+}
+
 __global__ void __launch_bounds__(256) feature_hash_kernel(const __grid_constant__ FeatParams p,
                                                            const int64_t* __restrict__ values,
                                                            int64_t* __restrict__ keys,
                                                            int* __restrict__ status) {
   pdl_wait();
   const int64_t lo = p.offs[0], hi = p.offs[p.F];
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = lo + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < hi; i += stride) {
-    // feature of value i: last f with offs[f] <= i (and offs[f+1] > i)
-    int a = 0, b = p.F;  // invariant: offs[a] <= i < offs[b]
-    while (b - a > 1) {
-      const int m = (a + b) >> 1;
-      if (p.offs[m] <= i) a = m; else b = m;
+  constexpr int64_t kRound = 256 * kFeatItems;
+  const int64_t stride = (int64_t)gridDim.x * kRound;
+  for (int64_t base = lo + (int64_t)blockIdx.x * kRound + threadIdx.x; base < hi; base += stride) {
+    int64_t x[kFeatItems];
+#pragma unroll
+    for (int j = 0; j < kFeatItems; ++j) {
+      const int64_t i = base + j * 256;
+      x[j] = i < hi ? __ldcs(values + i) : 0;
     }
-    const FeatOpDev& op = p.ops[a];
-    const int64_t x = values[i];
-    uint64_t v;
-    if (op.flags & RECIS_BUCKETIZE) {
-      int l = 0, r = op.n_bound;  // count of boundaries <= x
-      while (l < r) {
-        const int m = (l + r) >> 1;
-        if (__ldg(op.bounds + m) <= x) l = m + 1; else r = m;
+#pragma unroll
+    for (int j = 0; j < kFeatItems; ++j) {
+      const int64_t i = base + j * 256;
+      if (i >= hi) break;
+      // feature of value i: last f with offs[f] <= i (and offs[f+1] > i)
+      int a = 0, b = p.F;  // invariant: offs[a] <= i < offs[b]
+      while (b - a > 1) {
+        const int m = (a + b) >> 1;
+        if (p.offs[m] <= i) a = m; else b = m;
       }
-      v = (uint64_t)l;
-    } else {
-      v = (uint64_t)x;
-      if (op.flags & RECIS_HASH) v = mix64(v ^ op.seed);
-      if (op.flags & RECIS_MOD) v = (op.flags & kModPow2) ? (v & (op.mod - 1)) : (v % op.mod);
+      __stcs(keys + i, feature_key(p.ops[a], x[j], status));
     }
-    int64_t key;
-    if (op.flags & RECIS_TAG) {
-      if (v >= op.limit) {
-        atomicOr(status, kErrTagOverflow);
-        key = kEmptyKey;
-      } else {
-        key = (int64_t)(op.tag_bits | v);
-      }
-    } else {
-      key = (int64_t)v;
-    }
-    keys[i] = key;
   }
   pdl_trigger();
 }
@@ -97,7 +109,7 @@ cudaError_t launch_feature_hash(const recis_feature_op* ops, int F, const int64_
     }
     const int64_t n = p.offs[nf] - p.offs[0];
     if (n <= 0) continue;
-    int64_t blocks = (n + 255) / 256;
+    int64_t blocks = (n + 256 * kFeatItems - 1) / (256 * kFeatItems);
     const int64_t cap = (int64_t)kSMs * 8;
     if (blocks > cap) blocks = cap;
     LaunchScope ls("feature_hash", s);

@@ -331,10 +331,11 @@ __global__ void __launch_bounds__(256, kPartialCtas<G, VPL>) seg_partial_kernel(
     unsigned rem = mask;
     do {
       // the next PR long positions of the step: rows into shared memory
-      unsigned piece = 0;
-      {
+      unsigned piece = rem;  // a step's positions fit in one piece when PR >= Q
+      if (PR < Q && __popc(rem) > PR) {
+        piece = 0;
         unsigned r = rem;
-        for (int u = 0; u < PR && r; ++u) {
+        for (int u = 0; u < PR; ++u) {
           piece |= r & (0u - r);
           r &= r - 1;
         }
