@@ -656,11 +656,26 @@ def measure(w: W.Workload, args, R, dist, world: int, rank: int, dev, headline: 
                         "note": ("algorithmic bytes of the row / its kernels' event time"
                                  if len(members) > 1 else
                                  "algorithmic bytes per launch / CUDA-event time per launch")}
+        # actual DRAM traffic (ncu capture) of the kernels that have one:
+        # per kernel, and over those kernels' share of the step
         l2 = {}
-        for k in kern:
-            _, hit, _n = _traffic(w.name, k, Nm)
+        dram_b = dram_t = 0.0
+        for k, v in prof.items():
+            lps = v[0] / prof_steps  # launches per step
+            tb, hit, _n = _traffic(w.name, k, Nm / max(lps, 1e-9))
             if hit is not None:
                 l2[k] = hit
+            if tb is not None:
+                kern[k]["dram_bytes_per_launch"] = tb
+                kern[k]["dram_gbs"] = tb / (kern[k]["avg_us"] * 1e-6) / 1e9
+                kern[k]["dram_frac"] = kern[k]["dram_gbs"] / peak
+                dram_b += tb * lps
+                dram_t += kern[k]["avg_us"] * 1e-6 * lps
+        dram = ({"gbs": dram_b / dram_t / 1e9, "frac": dram_b / dram_t / 1e9 / peak,
+                 "kernels": sorted(k for k in kern if "dram_gbs" in kern[k]),
+                 "share_of_step_kernel_time": dram_t / (sum(v[1] for v in prof.values()) / prof_steps / 1e3),
+                 "note": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of these kernels "
+                         "(profiles/traffic.json) / their CUDA-event time"} if dram_t > 0 else None)
         step_alg = sum(alg.values()) - alg["feature_hash"] + 16 * Nm
         step_s = dev_ms / args.steps / 1e3
         rec = {
@@ -680,6 +695,7 @@ def measure(w: W.Workload, args, R, dist, world: int, rank: int, dev, headline: 
             "step_alg_gbs": step_alg / step_s / 1e9,
             "step_frac_of_peak": step_alg / step_s / 1e9 / peak,
             "l2_hit_rate_pct": l2 or None,
+            "dram_achieved": dram,
             "e2e": {"value": e2e_value, "unit": "IDs/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h,
                     "note": "torch copies of pinned host buffers around the library's "
@@ -738,7 +754,8 @@ def run_gpu(args):
         if r is not None:
             keep = ("value", "unit", "ms_per_step", "ms_per_step_p50", "ms_per_step_p90", "config",
                     "roofline", "step_alg_bytes", "step_alg_gbs", "step_frac_of_peak",
-                    "l2_hit_rate_pct", "e2e", "gpu_launches", "kernels", "clocks", "cpu_baseline")
+                    "l2_hit_rate_pct", "dram_achieved", "e2e", "gpu_launches", "kernels", "clocks",
+                    "cpu_baseline")
             sub_recs[name] = {k: r[k] for k in keep if k in r}
     if rank == 0:
         if sub_recs:
