@@ -30,6 +30,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -281,11 +282,20 @@ class Clocks:
         return out
 
 
+def _code_only(text: str) -> str:
+    """Source text without // and /* */ comments and blank lines: what a
+    capture depends on (a comment edit leaves the kernels as they were)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
 def _files_sha(files):
+    """sha256 of the code (comments dropped) of a kernel's source files."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()
 
 

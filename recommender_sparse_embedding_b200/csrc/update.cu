@@ -135,7 +135,8 @@ __device__ __forceinline__ void add_terms(const GroupCtx<G>& g, const UpdatePara
 // of step k, the segment bounds of step k+1 and the segments and gradient
 // sources of step k+2.  A position is long when its segment is; the
 // gradient rows of a step's long positions are copied into shared memory by
-// cp.async, up to PR positions at once (one slot per position, row and
+// bulk copies (cp.async when the gradients are not device memory), up to
+// PR positions at once (one slot per position, row and
 // lane), then added in position order into one fp64 sum per segment run.
 // A run's sum is
 //   - the segment's gradient, rounded once and stored in gbuf at row
@@ -702,11 +703,13 @@ __device__ __noinline__ void update_listed(const UpdateParams& p, int64_t gid, i
 // A persistent grid of G-lane groups walks the unique keys u = gid, gid +
 // groups, ... (U from the lookup), S keys deep: while key u is
 // updated, the next S-1 keys' rows [emb | state] (and a singleton's
-// pooled gradient row) are in flight into shared memory by cp.async, and the
-// key after those has its indices loaded.  Each lane copies and reads back
-// only its own 16-byte columns, so a lane's own wait is enough for the data;
-// a key's indices are shared by the group through shared memory (written by
-// its lane 0, read after __syncwarp).  Other keys' gradients (repeated keys,
+// pooled gradient row) are in flight into shared memory, and the key after
+// those has its indices loaded.  TMA: the group's lane 0 copies each row with
+// one bulk copy on the stage's transaction barrier, which every lane waits
+// on.  Otherwise each lane copies (cp.async) and reads back only its own
+// 16-byte columns, so a lane's own wait is enough for the data.  A key's
+// indices are shared by the group through shared memory (written by its
+// lane 0, read after __syncwarp).  Other keys' gradients (repeated keys,
 // long segments, unpooled gradients) are gathered while the key is updated.
 // Pipeline depth: 4 when each group walks many keys (long-sequence batches),
 // 2 otherwise (measured: 3 or 4 keys deep, or a fourth CTA per SM, only
