@@ -236,8 +236,14 @@ recis_status recis_lookup_pooled(recis_table_t t, recis_batch_t b, const int64_t
  * optimiser state beside the parameters).  g(u) = sum over occurrences of
  * key u of grad_pooled[b][f] (x 1/length for MEAN) + grad_unpooled[i], then one
  * Adagrad or Adam step on every row touched by the lookup (Adam: the table's
- * step counter advances by one per call).  grad_pooled: device [B][F][D] or
- * NULL; grad_unpooled: device [N][D] or NULL (NULL = zero gradient). */
+ * step counter advances by one per call).  grad_pooled: [B][F][D] or NULL;
+ * grad_unpooled: [N][D] or NULL (NULL = zero gradient); 16-byte aligned,
+ * unchanged until the call's work has finished.  They are normally device
+ * memory (gathered by the bulk-copy engine); any memory the GPU can read
+ * (host-mapped pinned memory, managed memory) is accepted and gathered with
+ * per-thread copies instead.  A gradient of several occurrences is summed in
+ * fp64 in a fixed order and rounded once, so results do not depend on
+ * scheduling. */
 recis_status recis_backward_update(recis_table_t t, recis_batch_t b, const float* grad_pooled,
                                    const float* grad_unpooled, recis_stream_t stream);
 
