@@ -609,11 +609,13 @@ __device__ __forceinline__ void apply_update(const GroupCtx<G>& g, const UpdateP
 // segment's sum is read from gbuf.
 // Gradient of key (s0, s1, first) into acc: a singleton's one term (its
 // pooled gradient row already staged in shared memory when staged != null),
-// a long segment's sum from gbuf, else the terms gathered here.
+// a long segment's sum from gbuf, else the terms gathered here (the first G
+// positions' source records already loaded into rec0 when have0).
 template <int G, int VPL, bool GP, bool GU>
 __device__ __forceinline__ void key_grad(const GroupCtx<G>& g, const UpdateParams& p, int32_t s0,
                                          int32_t s1, int4 first, const float4* staged, int stride,
-                                         float4 (&out)[VPL]) {
+                                         float4 (&out)[VPL], int4 rec0 = make_int4(0, 1, 0, 0),
+                                         bool have0 = false) {
   const int64_t D = (int64_t)p.ncol * 4;
   const int len = s1 - s0;
   constexpr int K = kRowsInFlight<VPL, GP && GU>;
@@ -650,7 +652,10 @@ __device__ __forceinline__ void key_grad(const GroupCtx<G>& g, const UpdateParam
     for (int base = 0; base < len; base += G) {
       const int m = len - base < G ? len - base : G;
       Src s{0, 0, 1.0};
-      if (g.lane < m) s = make_src(p, __ldg(p.gsrc + s0 + base + g.lane));
+      if (base == 0 && have0)
+        s = make_src(p, rec0);  // lanes >= m hold {0, 1, 0, 0}: the same unused source
+      else if (g.lane < m)
+        s = make_src(p, __ldg(p.gsrc + s0 + base + g.lane));
       for (int k0 = 0; k0 < m; k0 += K)
         add_terms<G, VPL, K, GP, GU>(g, p, s, k0, m - k0 < K ? m - k0 : K, acc);
     }
@@ -666,6 +671,8 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// a hint: the 128-byte line holding a into L2
+__device__ __forceinline__ void prefetch_l2(const void* a) { asm volatile("prefetch.global.L2 [%0];" ::"l"(a)); }
 
 // Indices of one key: segment bounds, row offset (positions and rows fit in
 // 32 bits: N < 2^31, rows < 2^31) and the source of one of its occurrences.
@@ -714,8 +721,17 @@ __device__ __noinline__ void update_listed(const UpdateParams& p, int64_t gid, i
 // Pipeline depth: 4 when each group walks many keys (long-sequence batches),
 // 2 otherwise (measured: 3 or 4 keys deep, or a fourth CTA per SM, only
 // lengthen every request on the 26-feature step).
-template <int G, int VPL, bool ADAM, bool GP, bool GU, int S, bool TMA>
+// AHEAD (S >= 3, gradients in device memory and too large for L2, keys seen
+// 2 to kShortSeg times not listed): their gathers run ahead of the walk too.
+// While key k is updated, the source records of key k+2's first G positions
+// are loaded (one per lane) and, with key k+1's records in hand, key k+1's
+// gradient rows are prefetched into L2, so that its gather starts from
+// registers and L2 instead of two dependent DRAM round trips (measured on
+// the large-table step: 3.32 -> 2.92 ms; where the gradients sit in L2 the
+// extra work only costs).
+template <int G, int VPL, bool ADAM, bool GP, bool GU, int S, bool TMA, bool AHEAD = false>
 __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constant__ UpdateParams p) {
+  static_assert(!AHEAD || (S >= 3 && TMA), "look-ahead needs key k+2 issued and device-memory gradients");
   pdl_wait();
   constexpr int NR = ADAM ? 3 : 2;             // row slices: emb, state(s)
   constexpr int NS = NR * VPL + VPL;           // staged float4 per thread per stage
@@ -796,6 +812,23 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
     const int64_t uk = u0 + k * groups;
     return uk < U ? key_idx(p, uk) : KeyIdx{0, 1, -1, 0, make_int4(0, 1, 0, 0)};
   };
+  auto gathers = [&](const KeyIdx& k) { return k.s1 - k.s0 > 1 && k.s1 - k.s0 <= kShortSeg && !is_listed(k); };
+  auto load_rec = [&](const KeyIdx& k) -> int4 {
+    return gathers(k) && g.lane < k.s1 - k.s0 ? __ldg(p.gsrc + k.s0 + g.lane) : make_int4(0, 1, 0, 0);
+  };
+  auto prefetch_rows = [&](const KeyIdx& k, int4 rec) {
+    if (k.row < 0 || !gathers(k) || g.lane >= k.s1 - k.s0) return;
+    for (int off = 0; off < D * 4; off += 128) {
+      if (GP) prefetch_l2(p.gp + (int64_t)rec.x * D + off / 4);
+      if (GU) prefetch_l2(p.gu + (int64_t)rec.z * D + off / 4);
+    }
+  };
+  // AHEAD: the source records of key k (rec_cur) and of key k+1 (rec_nxt)
+  int4 rec_cur = make_int4(0, 1, 0, 0), rec_nxt = make_int4(0, 1, 0, 0);
+  if constexpr (AHEAD) {
+    rec_cur = load_rec(idx_of(0));
+    rec_nxt = load_rec(idx_of(1));
+  }
 #pragma unroll
   for (int k = 0; k < S - 1; ++k) {
     issue(k, idx_of(k));
@@ -811,6 +844,13 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
     const int stage = (int)(k % S);
     const KeyIdx cur = *key_slot(stage);
     const bool staged_grad = GP && !GU && cur.s1 - cur.s0 == 1;
+    const int4 rec = rec_cur;
+    if constexpr (AHEAD) {
+      // keys k+1 and k+2 sit in their stages' slots (issued S-1 keys ahead)
+      rec_cur = rec_nxt;
+      prefetch_rows(*key_slot((int)((k + 1) % S)), rec_cur);
+      rec_nxt = load_rec(*key_slot((int)((k + 2) % S)));
+    }
     float4 grad[VPL];
     if (TMA) {
       // the (k / S)-th use of this stage's barrier
@@ -824,7 +864,7 @@ __global__ void __launch_bounds__(256, 3) row_update_kernel(const __grid_constan
     }
     if (is_listed(cur)) continue;  // updated above
     key_grad<G, VPL, GP, GU>(g, p, cur.s0, cur.s1, cur.first,
-                             staged_grad ? slot(stage, NR * VPL) : nullptr, stride, grad);
+                             staged_grad ? slot(stage, NR * VPL) : nullptr, stride, grad, rec, AHEAD && gathers(cur));
     if (cur.row >= 0) {
       RowRegs<VPL, ADAM> r;
 #pragma unroll
@@ -862,6 +902,9 @@ __global__ void __launch_bounds__(256, 2) row_update_wide_kernel(const __grid_co
 // ------------------------------------------------------------------ host
 int group_lanes_for(int D);
 
+// gradient bytes above which the row update prefetches gathers (half of L2)
+constexpr int64_t kAheadGradBytes = 64ll << 20;
+
 // seg_reduce span: kChunk * 2^k positions (at most 8 steps), as long as 16K
 // lane groups remain to fill the GPU
 int64_t update_chunk_for(int64_t N, int) {
@@ -884,7 +927,7 @@ static cudaError_t smem_attr(K kernel, size_t smem, bool (&done)[64]) {
 
 template <int G, int VPL, bool GP, bool GU>
 static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t ucap, bool tma, bool rows_tma,
-                                   cudaStream_t s) {
+                                   bool ahead_ok, cudaStream_t s) {
   {
     // one lane group per span; one staging slot per position, row and lane
     constexpr size_t smem = (size_t)256 * kChunk * sizeof(float4);
@@ -918,6 +961,7 @@ static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t uca
   if constexpr (VPL == 1) {
     // keys per group decide the depth (U <= ucap)
     const bool deep = ucap / (blocks * (256 / G)) >= 64;
+    const bool ahead = deep && rows_tma && ahead_ok;
     const int S = deep ? 4 : 2;
     const int ns = ((adam ? 3 : 2) * VPL + VPL);
     const size_t smem = (size_t)S * ns * 256 * sizeof(float4) + (size_t)S * (256 / G) * sizeof(KeyIdx) +
@@ -930,11 +974,13 @@ static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t uca
     };
     if (rows_tma) {
       if (adam)
-        e = deep ? go(row_update_kernel<G, VPL, true, GP, GU, 4, true>)
-                 : go(row_update_kernel<G, VPL, true, GP, GU, 2, true>);
+        e = ahead  ? go(row_update_kernel<G, VPL, true, GP, GU, 4, true, true>)
+            : deep ? go(row_update_kernel<G, VPL, true, GP, GU, 4, true>)
+                   : go(row_update_kernel<G, VPL, true, GP, GU, 2, true>);
       else
-        e = deep ? go(row_update_kernel<G, VPL, false, GP, GU, 4, true>)
-                 : go(row_update_kernel<G, VPL, false, GP, GU, 2, true>);
+        e = ahead  ? go(row_update_kernel<G, VPL, false, GP, GU, 4, true, true>)
+            : deep ? go(row_update_kernel<G, VPL, false, GP, GU, 4, true>)
+                   : go(row_update_kernel<G, VPL, false, GP, GU, 2, true>);
     } else {
       if (adam)
         e = deep ? go(row_update_kernel<G, VPL, true, GP, GU, 4, false>)
@@ -955,11 +1001,11 @@ static cudaError_t launch_update_g(const UpdateParams& p, bool adam, int64_t uca
 
 template <int G, int VPL>
 static cudaError_t launch_update_t(const UpdateParams& p, bool adam, int64_t ucap, bool tma, bool rows_tma,
-                                   cudaStream_t s) {
-  if (p.gp && p.gu) return launch_update_g<G, VPL, true, true>(p, adam, ucap, tma, rows_tma, s);
-  if (p.gp) return launch_update_g<G, VPL, true, false>(p, adam, ucap, tma, rows_tma, s);
-  if (p.gu) return launch_update_g<G, VPL, false, true>(p, adam, ucap, tma, rows_tma, s);
-  return launch_update_g<G, VPL, false, false>(p, adam, ucap, tma, rows_tma, s);  // touched rows, zero gradient
+                                   bool ahead_ok, cudaStream_t s) {
+  if (p.gp && p.gu) return launch_update_g<G, VPL, true, true>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  if (p.gp) return launch_update_g<G, VPL, true, false>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  if (p.gu) return launch_update_g<G, VPL, false, true>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  return launch_update_g<G, VPL, false, false>(p, adam, ucap, tma, rows_tma, ahead_ok, s);  // touched rows, zero gradient
 }
 
 // device memory of this GPU's own address space (allocations and VMM
@@ -1016,16 +1062,21 @@ cudaError_t launch_update(recis_table* t, recis_batch* b, const float* grad_pool
   // EmbeddingBlocks are device memory
   const bool tma = device_memory(grad_pooled) && device_memory(grad_unpooled);
   const bool rows_tma = tma && t->rows.host_numa < 0;
+  // the row update gathers ahead when the keys seen a few times are not
+  // listed and the gradients are too large to stay in L2
+  const int64_t grad_bytes = (grad_pooled ? (int64_t)b->F * b->B * t->D * 4 : 0) +
+                             (grad_unpooled ? b->N * t->D * 4 : 0);
+  const bool ahead_ok = p.multi_keys == nullptr && grad_bytes > kAheadGradBytes;
   const int ncol = p.ncol;
-  if (ncol <= 1) return launch_update_t<1, 1>(p, adam, ucap, tma, rows_tma, s);
-  if (ncol <= 2) return launch_update_t<2, 1>(p, adam, ucap, tma, rows_tma, s);
-  if (ncol <= 4) return launch_update_t<4, 1>(p, adam, ucap, tma, rows_tma, s);
-  if (ncol <= 8) return launch_update_t<8, 1>(p, adam, ucap, tma, rows_tma, s);
-  if (ncol <= 16) return launch_update_t<16, 1>(p, adam, ucap, tma, rows_tma, s);
-  if (ncol <= 32) return launch_update_t<32, 1>(p, adam, ucap, tma, rows_tma, s);
-  if (ncol <= 64) return launch_update_t<32, 2>(p, adam, ucap, tma, rows_tma, s);
-  if (ncol <= 128) return launch_update_t<32, 4>(p, adam, ucap, tma, rows_tma, s);
-  return launch_update_t<32, 8>(p, adam, ucap, tma, rows_tma, s);
+  if (ncol <= 1) return launch_update_t<1, 1>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  if (ncol <= 2) return launch_update_t<2, 1>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  if (ncol <= 4) return launch_update_t<4, 1>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  if (ncol <= 8) return launch_update_t<8, 1>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  if (ncol <= 16) return launch_update_t<16, 1>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  if (ncol <= 32) return launch_update_t<32, 1>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  if (ncol <= 64) return launch_update_t<32, 2>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  if (ncol <= 128) return launch_update_t<32, 4>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
+  return launch_update_t<32, 8>(p, adam, ucap, tma, rows_tma, ahead_ok, s);
 }
 
 }  // namespace recis
