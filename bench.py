@@ -149,8 +149,9 @@ def _oracle_sample(w: W.Workload):
                         f"pre-filled with {len(live)} live keys (1/{s} of the live set)")
 
 
-def _oracle_rate(w: W.Workload, budget_s: float, nbatch: int = 2):
-    """The CPU oracle (single thread) on steps of the workload for ~budget_s."""
+def _oracle_rate(w: W.Workload, budget_s: float, nbatch: int = 2, n_steps: int = 0, n_warm: int = 0):
+    """The CPU oracle (single thread) on steps of the workload for ~budget_s,
+    or, when n_steps > 0, on exactly n_warm untimed and n_steps timed steps."""
     import oracle as O
     ws, live, what = _oracle_sample(w)
     batches = []
@@ -168,9 +169,9 @@ def _oracle_rate(w: W.Workload, budget_s: float, nbatch: int = 2):
                 tab.lookup(k, np.arange(len(k) + 1, dtype=np.int64), 1, len(k), pooled=False)
     n_ids, steps, t0 = 0, 0, time.perf_counter()
     times = []
-    while True:
-        b, grads = batches[steps % len(batches)]
-        vals = b.values if live is None else W.with_fresh_ids(ws, b, 200 + steps)
+    for j in range(n_warm + n_steps if n_steps > 0 else 1 << 62):
+        b, grads = batches[j % len(batches)]
+        vals = b.values if live is None else W.with_fresh_ids(ws, b, 200 + j)
         s0 = time.perf_counter()
         keys = O.feature_hash(ops, vals, b.feat_offsets)
         for t, tab, (gp, gu) in zip(ws.tables, tabs, grads):
@@ -179,10 +180,12 @@ def _oracle_rate(w: W.Workload, budget_s: float, nbatch: int = 2):
                        O.SUM if t.combiner == "sum" else O.MEAN, pooled=t.pooled,
                        unpooled=t.unpooled)
             tab.backward_update(gp, gu)
+        if j < n_warm:
+            continue  # untimed warm-up step
         times.append(time.perf_counter() - s0)
         n_ids += len(vals)
         steps += 1
-        if time.perf_counter() - t0 >= budget_s:
+        if n_steps == 0 and time.perf_counter() - t0 >= budget_s:
             break
     el = sum(times)
     return {"value": n_ids / el, "unit": "IDs/s", "cores": 1, "kind": "oracle", "host": _host_cpu(),
@@ -196,9 +199,9 @@ def run_reference(args):
     if rank != 0:
         return
     w = W.WORKLOADS[args.workload]
-    if args.warmup > 0:
-        _oracle_rate(w, 0.0, nbatch=1)  # one untimed step
-    res = _oracle_rate(w, max(5.0, 2.0 * args.steps) if args.steps < 60 else 120.0)
+    # exactly W untimed and K timed steps, each a bounded sample of the
+    # workload (the large table's at 1/16 scale: about a second of CPU work)
+    res = _oracle_rate(w, 0.0, n_steps=max(1, args.steps), n_warm=max(0, args.warmup))
     line = {"impl": "reference", "metric": METRIC, "value": res["value"], "unit": "IDs/s",
             "n_gpus": args.gpus, "steps": res["steps"], "warmup": args.warmup,
             "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",

@@ -58,3 +58,18 @@ def test_algorithmic_bytes_of_each_row():
     assert a["dedup"] == 8 * N + 4 * N + 16 * U + 16 * U + 4 * D * (1 + s) * n_new
     assert a["gather_pool"] == 4 * D * U + 4 * D * bags + 8 * bags
     assert a["backward"] == 4 * D * bags + 2 * 4 * D * (1 + s) * U
+
+
+def test_reference_arm_times_exactly_k_steps_after_w_warmups():
+    # the reference arm (the CPU oracle) prints one line of exactly K timed
+    # steps; the tiny workload keeps it to a second
+    import subprocess
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "3", "--warmup", "2"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 2
+    assert line["value"] > 0 and line["cpu_baseline"]["sample"].startswith("3 ")
+    assert line["e2e"] == {"value": line["value"], "unit": "IDs/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
