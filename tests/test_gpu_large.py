@@ -5,7 +5,8 @@ full large-table workload.
   LSD radix dedup and is compared with the oracle element by element.
 - A 1.8M-occurrence batch of 300,000 bags at D = 64 (pooled gradients of
   77 MB, more than the row update keeps in L2) takes the row update that
-  gathers the keys seen 2 to 16 times ahead of its walk; compared element by
+  gathers the keys seen 2 to 16 times ahead of its walk, with pooled
+  gradients only and with pooled and unpooled ones; compared element by
   element over two Adam steps with signed gradients.
 - The large-table workload at full size (50M pre-inserted keys, 65536 x 100
   bags of geometric length, 32.8M occurrences, two steps) is too large for the
@@ -73,7 +74,8 @@ def test_radix_path_parity(R):
     p.close()
 
 
-def test_gather_ahead_parity(R):
+@pytest.mark.parametrize("unpooled", [False, True], ids=["pooled", "pooled+unpooled"])
+def test_gather_ahead_parity(R, unpooled):
     rng = np.random.default_rng(37)
     B, D = 300_000, 64
     lengths = rng.integers(1, 12, size=B).astype(np.int64)  # ~1.8M occurrences
@@ -86,14 +88,15 @@ def test_gather_ahead_parity(R):
     keys = rng.integers(0, 1_000_000, size=N).astype(np.int64) * 104729 + 11
     hot = rng.random(N) < 0.03
     keys[hot] = rng.integers(0, 64, size=int(hot.sum())) * 104729 + 11
-    spec = W.TableSpec("t", [0], D, "adam", 0.01, "sum", pooled=True, init_seed=29)
+    spec = W.TableSpec("t", [0], D, "adam", 0.01, "sum", pooled=True, unpooled=unpooled, init_seed=29)
     p = Pair(R, spec)
     k_dev = torch.from_numpy(keys).to(DEV)
     bo_dev = torch.from_numpy(bo).to(DEV)
     for step in range(2):
         pooled = torch.empty((B, 1, D), dtype=torch.float32, device=DEV)
-        p.gpu.lookup_pooled(p.batch, k_dev, bo_dev, 1, B, R.SUM, pooled)
-        r = p.ora.lookup(keys, bo, 1, B, O.SUM)
+        unp = torch.empty((N, D), dtype=torch.float32, device=DEV) if unpooled else None
+        p.gpu.lookup_pooled(p.batch, k_dev, bo_dev, 1, B, R.SUM, pooled, unp)
+        r = p.ora.lookup(keys, bo, 1, B, O.SUM, pooled=True, unpooled=unpooled)
         uq, inv, rows, n_new = p.batch.get_unique(N)
         assert np.array_equal(uq.cpu().numpy(), r.uniq)
         assert np.array_equal(inv.cpu().numpy(), r.inv)
@@ -102,9 +105,13 @@ def test_gather_ahead_parity(R):
         cnt = np.bincount(r.inv, minlength=len(r.uniq))
         assert ((cnt >= 2) & (cnt <= 16)).sum() > 100_000 and (cnt > 16).sum() == 64
         close(pooled.cpu().numpy(), r.pooled, f"pooled step {step}")
+        if unpooled:
+            close(unp.cpu().numpy(), r.unpooled, f"unpooled step {step}")
         gp = W.make_grad((B, 1, D), 90 + step, signed=True)
-        p.gpu.backward_update(p.batch, torch.from_numpy(gp).to(DEV))
-        p.ora.backward_update(gp)
+        gu = W.make_grad((N, D), 95 + step, signed=True) if unpooled else None
+        p.gpu.backward_update(p.batch, torch.from_numpy(gp).to(DEV),
+                              None if gu is None else torch.from_numpy(gu).to(DEV))
+        p.ora.backward_update(gp, gu)
         p.gpu.status_sync()
         compare_tables(p, f"step {step}")
     p.close()
