@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SO = os.path.join(_HERE, "liboracle.so")
 
 OK, INVALID_ARG, RESERVED_KEY = 0, 1, 2
-BUCKETIZE, HASH, MOD, TAG = 1, 2, 4, 8
+BUCKETIZE, HASH, MOD, TAG, FLOAT = 1, 2, 4, 8, 16
 ADAGRAD, ADAM = 0, 1
 SUM, MEAN = 0, 1
 
@@ -118,7 +118,9 @@ def hash64(x: int) -> int:
 
 @dataclass
 class FeatureOp:
-    """One feature's transform: flags from {BUCKETIZE, HASH, MOD, TAG}."""
+    """One feature's transform: flags from {BUCKETIZE, HASH, MOD, TAG, FLOAT}.
+    With BUCKETIZE | FLOAT the boundaries are floats and the values are
+    float64 bit patterns held in the int64 array."""
     flags: int = 0
     hash_seed: int = 0
     mod: int = 0
@@ -134,7 +136,10 @@ def feature_hash(ops: Sequence[FeatureOp], values: np.ndarray, feat_offsets: np.
     arr = (_FeatureOp * max(F, 1))()
     keep = []
     for f, op in enumerate(ops):
-        b = np.ascontiguousarray(np.asarray(op.boundaries, dtype=np.int64))
+        if op.flags & FLOAT:
+            b = np.ascontiguousarray(np.asarray(op.boundaries, dtype=np.float64)).view(np.int64)
+        else:
+            b = np.ascontiguousarray(np.asarray(op.boundaries, dtype=np.int64))
         keep.append(b)
         arr[f].flags = op.flags
         arr[f].n_bound = len(b)

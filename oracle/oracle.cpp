@@ -81,7 +81,10 @@ extern "C" uint64_t orc_hash64(uint64_t x) { return H(x); }
 
 // Feature transform (README, Core architecture, Feature Engine: Hash / Mod /
 // Bucketize).  Per value x of feature f:
-//   BUCKETIZE: v = number of boundaries <= x  (reading: upper-bound index)
+//   BUCKETIZE: v = number of boundaries <= x  (reading: upper-bound index);
+//              FLOAT: x and the boundaries are binary64 values stored as
+//              their bit patterns, compared as doubles (a NaN x is above no
+//              boundary: v = 0)
 //   else     : v = (uint64)x; HASH: v = H(v ^ seed); MOD: v = v % mod
 //   TAG      : v must be < 2^shift; key = (tag << shift) | v
 // Reading for TAG: merged tables (Distributed optimisation, "parameter
@@ -94,6 +97,7 @@ extern "C" int orc_feature_hash(const orc_feature_op* ops, int32_t F, const int6
     if ((op.flags & ORC_BUCKETIZE) && (op.flags & (ORC_HASH | ORC_MOD))) return ORC_INVALID_ARG;
     if ((op.flags & ORC_MOD) && op.mod == 0) return ORC_INVALID_ARG;
     if ((op.flags & ORC_BUCKETIZE) && op.n_bound < 0) return ORC_INVALID_ARG;
+    if ((op.flags & ORC_FLOAT) && !(op.flags & ORC_BUCKETIZE)) return ORC_INVALID_ARG;
     if (op.flags & ORC_TAG) {
       if (op.tag_shift < 1 || op.tag_shift > 62) return ORC_INVALID_ARG;
       if (op.tag >= (1ULL << (63 - op.tag_shift))) return ORC_INVALID_ARG;
@@ -102,7 +106,17 @@ extern "C" int orc_feature_hash(const orc_feature_op* ops, int32_t F, const int6
     for (int64_t i = feat_offsets[f]; i < feat_offsets[f + 1]; ++i) {
       const int64_t x = values[i];
       uint64_t v;
-      if (op.flags & ORC_BUCKETIZE) {
+      if ((op.flags & ORC_BUCKETIZE) && (op.flags & ORC_FLOAT)) {
+        double xd;
+        std::memcpy(&xd, &x, sizeof xd);
+        int64_t c = 0;
+        for (int32_t k = 0; k < op.n_bound; ++k) {
+          double bd;
+          std::memcpy(&bd, &op.boundaries[k], sizeof bd);
+          if (bd <= xd) ++c;
+        }
+        v = (uint64_t)c;
+      } else if (op.flags & ORC_BUCKETIZE) {
         int64_t c = 0;
         for (int32_t k = 0; k < op.n_bound; ++k)
           if (op.boundaries[k] <= x) ++c;

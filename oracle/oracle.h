@@ -36,6 +36,7 @@ extern "C" {
 #define ORC_HASH 2u
 #define ORC_MOD 4u
 #define ORC_TAG 8u
+#define ORC_FLOAT 16u /* with ORC_BUCKETIZE: values and boundaries are IEEE binary64 bit patterns */
 
 typedef struct {
   uint32_t flags;
@@ -45,7 +46,7 @@ typedef struct {
   uint64_t tag;               /* feature tag written above tag_shift */
   int32_t tag_shift;          /* bit position of the tag, 1..62 */
   int32_t pad_;
-  const int64_t* boundaries;  /* host, sorted ascending, n_bound entries */
+  const int64_t* boundaries;  /* host, sorted ascending, n_bound entries (binary64 bits with ORC_FLOAT) */
 } orc_feature_op;
 
 #define ORC_ADAGRAD 0

@@ -94,6 +94,36 @@ def test_bucketize_is_numpy_searchsorted_right():
         O.feature_hash([O.FeatureOp(flags=O.BUCKETIZE | O.HASH)], x, np.array([0, len(x)]))
 
 
+def test_float_bucketize_hand_worked_values():
+    # boundaries -1.5, 0, 2.25, 1e300: the count of boundaries <= x, compared
+    # as doubles (-0.0 equals 0.0; a NaN is above no boundary)
+    b = [-1.5, 0.0, 2.25, 1e300]
+    xs = np.array([-np.inf, -1.5, -1.4999, -0.0, 0.0, 5e-324, 2.25, 3.0, 1e300, np.inf, np.nan,
+                   -np.nan], dtype=np.float64)
+    want = [0, 1, 1, 2, 2, 2, 3, 3, 4, 4, 0, 0]
+    ops = [O.FeatureOp(flags=O.BUCKETIZE | O.FLOAT | O.TAG, tag=3, tag_shift=48, boundaries=b)]
+    k = O.feature_hash(ops, xs.view(np.int64), np.array([0, len(xs)]))
+    assert (k & ((1 << 48) - 1)).tolist() == want
+    assert np.all(k >> 48 == 3)
+    # FLOAT without BUCKETIZE is not an op
+    with pytest.raises(O.OracleError):
+        O.feature_hash([O.FeatureOp(flags=O.FLOAT)], xs.view(np.int64), np.array([0, len(xs)]))
+
+
+def test_float_bucketize_is_numpy_searchsorted_right():
+    rng = np.random.default_rng(5)
+    b = np.unique(np.round(rng.normal(size=63), 2))
+    x = np.round(rng.normal(scale=1.5, size=6000), 2)  # many values equal to boundaries
+    x[:len(b)] = b
+    ops = [O.FeatureOp(flags=O.BUCKETIZE | O.FLOAT, boundaries=b.tolist()),
+           O.FeatureOp(flags=O.BUCKETIZE, boundaries=[-3, 0, 7])]
+    ints = np.arange(-5, 10, dtype=np.int64)
+    vals = np.concatenate([x.view(np.int64), ints])
+    k = O.feature_hash(ops, vals, np.array([0, len(x), len(vals)]))
+    assert np.array_equal(k[:len(x)], np.searchsorted(b, x, side="right"))
+    assert np.array_equal(k[len(x):], np.searchsorted(np.array([-3, 0, 7]), ints, side="right"))
+
+
 # ---------------------------------------------------------------- dedup / IDMap
 def _tiny_batch(seed=0, B=64):
     w = W.WORKLOADS["tiny"].scaled(B)
