@@ -64,14 +64,19 @@ typedef enum {
 /* Feature-op flags (README, Core architecture > Feature Engine: "Hash / Mod /
  * Bucketize").  Per value x of a feature, in this order:
  *   BUCKETIZE: v = number of boundaries <= x (boundaries sorted ascending);
+ *              with FLOAT, x and the boundaries are IEEE-754 binary64 values
+ *              stored as their bit patterns in the int64 words and compared
+ *              as doubles (-0.0 equals 0.0; a NaN x is above no boundary,
+ *              v = 0; the boundaries must hold no NaN);
  *   otherwise: v = (uint64)x; HASH: v = H(v ^ hash_seed); MOD: v = v % mod;
  *   TAG      : v must be < 2^tag_shift, key = (tag << tag_shift) | v.
  * H is the SplitMix64 finaliser (Steele, Lea & Flood, OOPSLA 2014).
- * BUCKETIZE cannot be combined with HASH or MOD. */
+ * BUCKETIZE cannot be combined with HASH or MOD; FLOAT needs BUCKETIZE. */
 #define RECIS_BUCKETIZE 1u
 #define RECIS_HASH 2u
 #define RECIS_MOD 4u
 #define RECIS_TAG 8u
+#define RECIS_FLOAT 16u
 
 typedef struct {
   uint32_t flags;
@@ -81,7 +86,8 @@ typedef struct {
   uint64_t tag;               /* < 2^(63 - tag_shift) */
   int32_t tag_shift;          /* 1..62 */
   int32_t reserved_;
-  const int64_t* boundaries;  /* DEVICE pointer, n_bound int64, sorted ascending */
+  const int64_t* boundaries;  /* DEVICE pointer, n_bound int64 (binary64 bit patterns with
+                                 FLOAT), sorted ascending, 8-byte aligned */
 } recis_feature_op;
 
 /* Fused feature transform of F features in one launch.

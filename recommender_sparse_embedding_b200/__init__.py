@@ -6,6 +6,6 @@ Adam row update) runs in librecis.so, built from csrc/ by build.build().  This
 package is its thin ctypes binding (recis.py); PyTorch provides device memory
 and streams only.
 """
-from .recis import (ADAGRAD, ADAM, BUCKETIZE, ERR_INVALID_ARG, HASH, MEAN, MOD, OK, SUM, TAG,  # noqa: F401
+from .recis import (ADAGRAD, ADAM, BUCKETIZE, ERR_INVALID_ARG, FLOAT, HASH, MEAN, MOD, OK, SUM, TAG,  # noqa: F401
                     Batch, Feature, RecisError, Table, feature_hash, feature_status_sync, launch_count,
                     load, profile_collect, profile_enable)

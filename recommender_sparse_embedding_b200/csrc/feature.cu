@@ -3,7 +3,8 @@
 //
 // One launch transforms up to kFeatPerLaunch features: every value finds its
 // feature by a binary search over the offsets held in the kernel's parameter
-// space, then applies bucketize or hash -> mod, then the feature tag.  The
+// space, then applies bucketize (of int64 or, with RECIS_FLOAT, of float64
+// values) or hash -> mod, then the feature tag.  The
 // kernel streams 16 bytes per value (8 in, 8 out), four values per thread
 // in flight.
 #include "internal.h"
@@ -36,10 +37,15 @@ constexpr int kFeatItems = 4;  // values per thread per round, all loaded before
 __device__ __forceinline__ int64_t feature_key(const FeatOpDev& op, int64_t x, int* status) {
   uint64_t v;
   if (op.flags & RECIS_BUCKETIZE) {
-    int l = 0, r = op.n_bound;  // count of boundaries <= x
+    // count of boundaries <= x: the boundaries are sorted, so the ones <= x
+    // come first (a NaN x, as a double, compares below none of them: 0)
+    const bool fl = (op.flags & RECIS_FLOAT) != 0;
+    const double xd = __longlong_as_double(x);
+    int l = 0, r = op.n_bound;
     while (l < r) {
       const int m = (l + r) >> 1;
-      if (__ldg(op.bounds + m) <= x) l = m + 1; else r = m;
+      const int64_t bm = __ldg(op.bounds + m);
+      if (fl ? __longlong_as_double(bm) <= xd : bm <= x) l = m + 1; else r = m;
     }
     v = (uint64_t)l;
   } else {

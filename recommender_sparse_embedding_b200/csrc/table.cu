@@ -718,8 +718,10 @@ recis_status recis_feature_hash(const recis_feature_op* ops, int32_t F, const in
       set_error("feature_hash: feat_offsets must be non-decreasing");
       return RECIS_ERR_INVALID_ARG;
     }
-    if ((o.flags & ~(RECIS_BUCKETIZE | RECIS_HASH | RECIS_MOD | RECIS_TAG)) ||
+    if ((o.flags & ~(RECIS_BUCKETIZE | RECIS_HASH | RECIS_MOD | RECIS_TAG | RECIS_FLOAT)) ||
         ((o.flags & RECIS_BUCKETIZE) && (o.flags & (RECIS_HASH | RECIS_MOD))) ||
+        ((o.flags & RECIS_FLOAT) && !(o.flags & RECIS_BUCKETIZE)) ||
+        ((o.flags & RECIS_BUCKETIZE) && o.n_bound > 0 && misaligned(o.boundaries, 8)) ||
         ((o.flags & RECIS_MOD) && o.mod == 0) ||
         ((o.flags & RECIS_BUCKETIZE) && (o.n_bound < 0 || (o.n_bound > 0 && !o.boundaries))) ||
         ((o.flags & RECIS_TAG) &&

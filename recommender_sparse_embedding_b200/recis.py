@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "librecis.so")
 OK = 0
 ERR_INVALID_ARG, ERR_OOM, ERR_TABLE_FULL, ERR_RESERVED_KEY, ERR_CUDA, ERR_TIMEOUT, ERR_NO_DEVICE = (
     1, 2, 3, 4, 5, 6, 7)
-BUCKETIZE, HASH, MOD, TAG = 1, 2, 4, 8
+BUCKETIZE, HASH, MOD, TAG, FLOAT = 1, 2, 4, 8, 16
 ADAGRAD, ADAM = 0, 1
 SUM, MEAN = 0, 1
 PLACE_BLOCKS_HOST, PLACE_IDMAP_HOST = 1, 2
@@ -167,13 +167,15 @@ def _stream(stream: Optional[torch.cuda.Stream]) -> int:
 
 @dataclass
 class Feature:
-    """One feature's transform (flags from BUCKETIZE, HASH, MOD, TAG)."""
+    """One feature's transform (flags from BUCKETIZE, HASH, MOD, TAG, FLOAT).
+    BUCKETIZE | FLOAT: float64 boundaries, and the feature's values are
+    float64 bit patterns in the int64 values tensor (x.view(torch.int64))."""
     flags: int = 0
     hash_seed: int = 0
     mod: int = 0
     tag: int = 0
     tag_shift: int = 48
-    boundaries: Optional[torch.Tensor] = None  # device int64, sorted
+    boundaries: Optional[torch.Tensor] = None  # device int64 (float64 with FLOAT), sorted
 
 
 def feature_hash(features: Sequence[Feature], values: torch.Tensor, feat_offsets: Sequence[int],
@@ -190,7 +192,7 @@ def feature_hash(features: Sequence[Feature], values: torch.Tensor, feat_offsets
         ops[f].tag_shift = ft.tag_shift
         if ft.boundaries is not None:
             ops[f].n_bound = ft.boundaries.numel()
-            ops[f].boundaries = _dev(ft.boundaries, torch.int64)
+            ops[f].boundaries = _dev(ft.boundaries, torch.float64 if ft.flags & FLOAT else torch.int64)
     offs = (ctypes.c_int64 * (F + 1))(*[int(x) for x in feat_offsets])
     if keys_out is None:
         keys_out = torch.empty_like(values)

@@ -64,6 +64,42 @@ def test_feature_hash_all_op_kinds(R):
     assert np.array_equal(got, ref)
 
 
+def test_feature_bucketize_float_values(R):
+    # float64 features (values as bit patterns in the int64 array) beside
+    # int64 ones in one launch: random doubles with many equal to a
+    # boundary, infinities, signed zeros, NaNs and denormals
+    rng = np.random.default_rng(9)
+    F = 140  # more features than one launch takes
+    lens = rng.integers(0, 300, size=F)
+    lens[3] = 0
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    N = int(offs[-1])
+    fb = np.unique(np.round(rng.normal(size=40), 2))
+    fb[0] = -np.inf  # a boundary every value but NaN passes
+    x = np.round(rng.normal(scale=1.5, size=N), 2)
+    x[::7] = rng.choice(fb[1:], size=len(x[::7]))
+    special = np.array([np.inf, -np.inf, 0.0, -0.0, np.nan, -np.nan, 5e-324, -5e-324, 1e308, -1e308])
+    x[::11] = rng.choice(special, size=len(x[::11]))
+    ib = np.unique(rng.integers(-40, 40, size=9)).astype(np.int64)
+    vals = x.view(np.int64).copy()
+    rf, of = [], []
+    for f in range(F):
+        if f % 3 == 2:  # an int64 bucketize feature: its own values
+            lo, hi = offs[f], offs[f + 1]
+            vals[lo:hi] = rng.integers(-50, 50, size=hi - lo)
+            spec = dict(flags=W.BUCKETIZE | W.TAG, tag=f, tag_shift=48)
+            rf.append(R.Feature(boundaries=torch.from_numpy(ib).to(DEV), **spec))
+            of.append(O.FeatureOp(boundaries=ib.tolist(), **spec))
+        else:
+            spec = dict(flags=W.BUCKETIZE | W.FLOAT | (W.TAG if f % 3 else 0), tag=f, tag_shift=48)
+            rf.append(R.Feature(boundaries=torch.from_numpy(fb).to(DEV), **spec))
+            of.append(O.FeatureOp(boundaries=fb.tolist(), **spec))
+    got = R.feature_hash(rf, torch.from_numpy(vals).to(DEV), offs.tolist()).cpu().numpy()
+    R.feature_status_sync()
+    ref = O.feature_hash(of, vals, offs)
+    assert np.array_equal(got, ref)
+
+
 def test_feature_hash_tag_overflow_is_reported(R):
     vals = torch.tensor([1, 2, 300, 4], dtype=torch.int64, device=DEV)
     R.feature_hash([R.Feature(flags=R.TAG, tag=1, tag_shift=8)], vals, [0, 4])

@@ -25,7 +25,7 @@ from typing import List, Optional, Sequence
 
 import numpy as np
 
-BUCKETIZE, HASH, MOD, TAG = 1, 2, 4, 8
+BUCKETIZE, HASH, MOD, TAG, FLOAT = 1, 2, 4, 8, 16
 _M64 = np.uint64(0xFFFFFFFFFFFFFFFF)
 
 
