@@ -2,9 +2,10 @@
 
 It serves callers that cannot allocate device memory (a framework memory pool
 that forbids foreign cudaMalloc calls, graph recording with allocation
-disabled, fixed device-memory budgets).  Its output must equal the dedup of the
-regular path (recis_lookup_pooled + recis_batch_get_unique) on the same keys,
-bit for bit, on consecutive calls that share its static scratch.  This file
+disabled, fixed device-memory budgets).  Its output must equal
+numpy.unique(return_inverse=True) of the keys and the dedup of the regular
+path (recis_lookup_pooled + recis_batch_get_unique) on the same keys, bit for
+bit, on consecutive calls that share its static scratch.  This file
 sorts last so that a run stopping at the first failure has run every other
 test first.
 """
@@ -64,7 +65,10 @@ def test_unique_static_matches_regular_dedup_on_two_calls():
         assert u == len(ref_uniq)
         assert np.array_equal(uniq[:u].cpu().numpy(), ref_uniq)
         assert np.array_equal(inv.cpu().numpy(), ref_inv)
-        assert np.array_equal(ref_uniq, np.unique(keys_np))
+        # and directly against the definition (numpy's unique with inverse)
+        np_uniq, np_inv = np.unique(keys_np, return_inverse=True)
+        assert np.array_equal(uniq[:u].cpu().numpy(), np_uniq)
+        assert np.array_equal(inv.cpu().numpy(), np_inv.reshape(-1))
 
 
 def test_unique_static_rejects_oversized_input():
