@@ -116,14 +116,19 @@ def batch(rank, step, B=48, n_ids=300):
     return keys, bo, g
 
 
-def reference(world, steps, combiner=O.SUM, optimizer=O.ADAM):
+def bags_of(rank, empty_rank=-1):
+    """Bags of a rank's batch: none for the rank that sends nothing."""
+    return 0 if rank == empty_rank else 48
+
+
+def reference(world, steps, combiner=O.SUM, optimizer=O.ADAM, empty_rank=-1):
     """The unsharded table: every step, all ranks' bags as one batch."""
     t = O.Table(D, optimizer, 0.01, init_seed=5)
     pooled = []
     for step in range(steps):
         ks, bos, gs = [], [np.zeros(1, np.int64)], []
         for r in range(world):
-            k, bo, g = batch(r, step)
+            k, bo, g = batch(r, step, B=bags_of(r, empty_rank))
             bos.append(bo[1:] + sum(len(x) for x in ks))
             ks.append(k)
             gs.append(g)

@@ -1,8 +1,9 @@
 """The sharded-table protocol (dedup, partition by owner, all-to-all of keys,
-rows and gradients) on two gloo ranks on CPU, each rank's arithmetic done by
-the numpy/oracle engine, against one unsharded oracle table fed both ranks'
-bags as one batch: pooled rows every step and the final state of every key
-(the union of the two shards) within the usual tolerance."""
+rows and gradients) on gloo ranks on CPU (two ranks; three with one rank
+that has no bags but still owns a shard and serves the others), each rank's
+arithmetic done by the numpy/oracle engine, against one unsharded oracle
+table fed all ranks' bags as one batch: pooled rows every step and the final
+state of every key (the union of the shards) within the usual tolerance."""
 import os
 import socket
 import sys
@@ -23,7 +24,7 @@ def _free_port():
     return p
 
 
-def _rank(rank, world, port, out_dir, combiner):
+def _rank(rank, world, port, out_dir, combiner, empty_rank):
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     import torch
@@ -39,7 +40,7 @@ def _rank(rank, world, port, out_dir, combiner):
         st = ShardedTable(S.D, 1, 0.01, engine=S.OracleEngine(), salt=S.SALT)
         pooled = []
         for step in range(STEPS):
-            k, bo, g = S.batch(rank, step)
+            k, bo, g = S.batch(rank, step, B=S.bags_of(rank, empty_rank))
             out = st.lookup_pooled(torch.from_numpy(k), torch.from_numpy(bo), 1, len(bo) - 1, combiner)
             pooled.append(out.numpy())
             st.backward_update(torch.from_numpy(g))
@@ -50,13 +51,13 @@ def _rank(rank, world, port, out_dir, combiner):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("combiner", [0, 1])
-def test_two_gloo_ranks_match_the_unsharded_table(tmp_path, combiner):
+@pytest.mark.parametrize("world,combiner,empty_rank", [(2, 0, -1), (2, 1, -1), (3, 0, 1)],
+                         ids=["2 ranks sum", "2 ranks mean", "3 ranks, rank 1 without bags"])
+def test_gloo_ranks_match_the_unsharded_table(tmp_path, world, combiner, empty_rank):
     import shard_util as S
-    world = 2
-    mp.start_processes(_rank, args=(world, _free_port(), str(tmp_path), combiner), nprocs=world,
-                       start_method="spawn")
-    ref, ref_pooled = S.reference(world, STEPS, combiner=combiner)
+    mp.start_processes(_rank, args=(world, _free_port(), str(tmp_path), combiner, empty_rank),
+                       nprocs=world, start_method="spawn")
+    ref, ref_pooled = S.reference(world, STEPS, combiner=combiner, empty_rank=empty_rank)
     rk, re, rs = ref.export()
     where = {int(k): i for i, k in enumerate(rk)}
     seen = 0
